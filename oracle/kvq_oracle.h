@@ -1,0 +1,117 @@
+/*
+ * CPU oracle for quantized-KV decode attention -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, obviously-correct restatement of what the decode path computes,
+ * written from the method's description and kept independent of the CUDA
+ * library: it shares no header, helper, table or constant with it.  Only the
+ * tests, the smoke check and the benchmark's CPU-baseline leg may call it.
+ *
+ * Sources (page title, section):
+ *  - "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches"
+ *    (paperlayer.ai summary of arXiv 2610.09827): Sec. 1 (Hadamard rotation,
+ *    channel 0 in BF16, paired transforms that preserve q.k), Sec. 3.2
+ *    (dynamic query-channel pruning with one shared mask), Sec. 3.3 (asymmetric
+ *    per-token INT2 keys, channel-major key rows), Sec. 3.4 (one global softmax
+ *    over segments), App. B.2 (per-token asymmetric values), App. C.2 (group-L2
+ *    query energy summed over the GQA group), App. C.3 (channel 0 outside the
+ *    range estimate).
+ *  - "TurboQuant on Quantized Models ..." (tq-kv, Zenodo abstract): scoring
+ *    without key decompression; incremental cache append.
+ *  - "Statistical Inference and Quality Measures of KV Cache Quantisations
+ *    Inspired by TurboQuant" (gist.science explainer), scheme KQV: WHT + plain
+ *    n-bit scalar quantization of keys.
+ *  - "CASK-Q" (decentralizedcompute.company), Method: scalar codes + FP16
+ *    scales as the stored format.
+ *
+ * Precision: FWHT in fp64 (natural Sylvester order), rotated values rounded
+ * to fp32; quantization in fp32 with IEEE round-half-to-even; dequantization,
+ * channel energies, scores and softmax in fp64.
+ */
+#ifndef KVQ_ORACLE_H
+#define KVQ_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Packed cache as the oracle writes it (host memory, oracle-owned layout code). */
+typedef struct {
+  int32_t batch, kv_heads, head_dim, capacity;
+  int32_t k_bits, v_bits; /* 2 or 4 */
+  int32_t rotate_k, keep_ch0;
+  uint8_t* k_codes;   /* [B][Hkv][d/4][cap] x (4*k_bits/8) bytes          */
+  uint16_t* k_scales; /* [B][Hkv][d/32][cap] x {fp16 scale, fp16 zero}      */
+  uint16_t* k_ch0;    /* [B][Hkv][cap] bf16, or NULL                        */
+  uint8_t* v_codes;   /* [B][Hkv][cap][d*v_bits/8]                          */
+  uint16_t* v_scales; /* [B][Hkv][cap][d/32] x {fp16 scale, fp16 zero}      */
+} orc_cache;
+
+typedef struct {
+  int64_t k_elems, v_elems;     /* quantized elements written            */
+  int64_t k_exempt, v_exempt;   /* elements within the near-tie window     */
+  int64_t k_clamped, v_clamped; /* codes clamped into [0, L]               */
+  int64_t groups_exempt;        /* groups whose fp16 scale/zero is near a tie */
+} orc_stats;
+
+/* in-place unnormalized Walsh-Hadamard butterflies, natural order, fp64 */
+void orc_fwht(double* x, int32_t d);
+/* out = fp32(FWHT(x) * (1/sqrt(d))) */
+void orc_rotate(const float* x, int32_t d, float* out);
+
+/* IEEE binary16 / bfloat16 round-to-nearest-even from fp32, and widening */
+uint16_t orc_half_rn(float x);
+double orc_half_value(uint16_t h);
+uint16_t orc_bf16_rn(float x);
+double orc_bf16_value(uint16_t h);
+
+/*
+ * Asymmetric quantization of one group of n values.  include[i] == 0 leaves
+ * element i out of the range estimate and gives it code 0.  Writes fp16
+ * scale/zero bits and codes; exempt[i] (may be NULL) flags near-tie elements;
+ * returns 1 if the group's scale or zero is within the fp16 tie window.
+ */
+int32_t orc_quantize_group(const float* x, const uint8_t* include, int32_t n, int32_t bits, uint16_t* s16,
+                           uint16_t* z16, uint8_t* codes, uint8_t* exempt, int64_t* clamped);
+
+/*
+ * Quantize k_new/v_new ([B][Hkv][n_new][d] fp32 values) and write them at
+ * tokens [offset, offset+n_new) of the cache.  k_row_exempt / v_row_exempt
+ * ([B][Hkv][n_new], may be NULL) flag rows holding any exempt element.
+ * Returns 0, or -1 on bad arguments.
+ */
+int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float* v_new, int32_t n_new,
+                            int32_t offset, orc_stats* stats, uint8_t* k_row_exempt, uint8_t* v_row_exempt);
+
+/* unpack the d codes of token n of (b, h): which = 0 for K, 1 for V */
+void orc_unpack_codes(const orc_cache* c, int32_t b, int32_t h, int32_t n, int32_t which, uint8_t* codes);
+
+/* dequantized K and V rows [n][d] of (b, h), tokens n0..n0+n-1, fp64 */
+void orc_dequantize(const orc_cache* c, int32_t b, int32_t h, int32_t n0, int32_t n, double* khat, double* vhat);
+
+/*
+ * Channel selection: per (b, kv head) keep the `keep` channel groups of 4
+ * with the largest query energy summed over the GQA group.  q is
+ * [B][Hq][d] fp32 values (un-rotated; rotated here when rotate != 0).
+ * mask[b*Hkv + h] bit p set = group p kept.  energy (may be NULL) receives
+ * [B][Hkv][d/4] fp64 energies.
+ */
+void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t rotate, int32_t keep,
+                uint32_t* mask, double* energy);
+
+/*
+ * Decode attention over the oracle cache for rows r = b*Hq + hq listed in
+ * `rows` (all B*Hq rows when rows == NULL).  q as in orc_select; lens[b]
+ * tokens of sequence b; mask NULL = all channels.  out[r][d] fp64 (row-major
+ * in the order of `rows`).
+ */
+void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t* lens, const uint32_t* mask,
+                   double scale, const int32_t* rows, int32_t nrows, double* out);
+
+/* (T q) . (T^{-T} k) in fp64 for a d x d row-major invertible T; returns NaN if T is singular */
+double orc_dual_score(const double* T, int32_t d, const double* q, const double* k);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

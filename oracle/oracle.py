@@ -1,0 +1,190 @@
+"""ctypes wrapper of the C++ oracle (``kvq_oracle.cpp``) -- test infrastructure only.
+
+Arrays cross as numpy buffers; bf16 inputs are widened to fp32 (exactly)
+before they reach the oracle.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build_oracle
+
+_lib = None
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+
+
+class OrcCache(ctypes.Structure):
+    _fields_ = [("batch", _I32), ("kv_heads", _I32), ("head_dim", _I32), ("capacity", _I32),
+                ("k_bits", _I32), ("v_bits", _I32), ("rotate_k", _I32), ("keep_ch0", _I32),
+                ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P)]
+
+
+class OrcStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in
+                ("k_elems", "v_elems", "k_exempt", "v_exempt", "k_clamped", "v_clamped", "groups_exempt")]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        so = build_oracle.build()
+        L = ctypes.CDLL(so)
+        L.orc_fwht.argtypes = [_P, _I32]
+        L.orc_rotate.argtypes = [_P, _I32, _P]
+        L.orc_half_rn.argtypes = [ctypes.c_float]
+        L.orc_half_rn.restype = ctypes.c_uint16
+        L.orc_half_value.argtypes = [ctypes.c_uint16]
+        L.orc_half_value.restype = ctypes.c_double
+        L.orc_bf16_rn.argtypes = [ctypes.c_float]
+        L.orc_bf16_rn.restype = ctypes.c_uint16
+        L.orc_bf16_value.argtypes = [ctypes.c_uint16]
+        L.orc_bf16_value.restype = ctypes.c_double
+        L.orc_quantize_group.argtypes = [_P, _P, _I32, _I32, _P, _P, _P, _P, _P]
+        L.orc_quantize_group.restype = _I32
+        L.orc_quantize_append.argtypes = [ctypes.POINTER(OrcCache), _P, _P, _I32, _I32, ctypes.POINTER(OrcStats),
+                                          _P, _P]
+        L.orc_quantize_append.restype = _I32
+        L.orc_unpack_codes.argtypes = [ctypes.POINTER(OrcCache), _I32, _I32, _I32, _I32, _P]
+        L.orc_dequantize.argtypes = [ctypes.POINTER(OrcCache), _I32, _I32, _I32, _I32, _P, _P]
+        L.orc_select.argtypes = [_P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P]
+        L.orc_attention.argtypes = [ctypes.POINTER(OrcCache), _P, _I32, _P, _P, ctypes.c_double, _P, _I32, _P]
+        L.orc_dual_score.argtypes = [_P, _I32, _P, _P]
+        L.orc_dual_score.restype = ctypes.c_double
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def as_f32(x: np.ndarray) -> np.ndarray:
+    """fp32 values of an input array (bf16 bit patterns as uint16, or fp32)."""
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray((x.astype(np.uint32) << 16).view(np.float32))
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def fwht(x: np.ndarray) -> np.ndarray:
+    """Unnormalized fp64 Walsh-Hadamard butterflies (natural order)."""
+    y = np.ascontiguousarray(x, dtype=np.float64).copy()
+    lib().orc_fwht(_p(y), y.size)
+    return y
+
+
+def rotate(x: np.ndarray) -> np.ndarray:
+    """fp32(FWHT(x)/sqrt(d)) of one row."""
+    xi = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(xi)
+    lib().orc_rotate(_p(xi), xi.size, _p(out))
+    return out
+
+
+def half_rn(x: float) -> int:
+    return lib().orc_half_rn(float(x))
+
+
+def half_value(h: int) -> float:
+    return lib().orc_half_value(int(h))
+
+
+def bf16_rn(x: float) -> int:
+    return lib().orc_bf16_rn(float(x))
+
+
+def bf16_value(h: int) -> float:
+    return lib().orc_bf16_value(int(h))
+
+
+def quantize_group(x, bits: int, include=None):
+    """-> (s16 bits, z16 bits, codes, exempt flags, group_exempt, clamped count)"""
+    xi = np.ascontiguousarray(x, dtype=np.float32)
+    n = xi.size
+    inc = None if include is None else np.ascontiguousarray(include, dtype=np.uint8)
+    s = ctypes.c_uint16()
+    z = ctypes.c_uint16()
+    codes = np.zeros(n, np.uint8)
+    ex = np.zeros(n, np.uint8)
+    clamped = ctypes.c_int64(0)
+    gex = lib().orc_quantize_group(_p(xi), _p(inc), n, bits, ctypes.byref(s), ctypes.byref(z), _p(codes), _p(ex),
+                                   ctypes.byref(clamped))
+    return s.value, z.value, codes, ex, gex, clamped.value
+
+
+class Cache:
+    """Host copy of the packed cache, written by the oracle."""
+
+    def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0):
+        self.B, self.Hkv, self.d, self.capacity = B, Hkv, d, capacity
+        self.k_bits, self.v_bits, self.rotate_k, self.keep_ch0 = k_bits, v_bits, rotate_k, keep_ch0
+        self.k_codes = np.zeros(B * Hkv * (d // 4) * capacity * (4 * k_bits // 8), np.uint8)
+        self.k_scales = np.zeros(B * Hkv * (d // 32) * capacity * 2, np.uint16)
+        self.k_ch0 = np.zeros(B * Hkv * capacity, np.uint16) if keep_ch0 else None
+        self.v_codes = np.zeros(B * Hkv * capacity * (d * v_bits // 8), np.uint8)
+        self.v_scales = np.zeros(B * Hkv * capacity * (d // 32) * 2, np.uint16)
+        self.struct = OrcCache(B, Hkv, d, capacity, k_bits, v_bits, rotate_k, keep_ch0, _p(self.k_codes),
+                               _p(self.k_scales), _p(self.k_ch0), _p(self.v_codes), _p(self.v_scales))
+
+    def append(self, k_new: np.ndarray, v_new: np.ndarray, offset: int, want_exempt: bool = False):
+        """k_new, v_new: [B][Hkv][n][d] (bf16 as uint16, or fp32)."""
+        k = as_f32(k_new)
+        v = as_f32(v_new)
+        n_new = k.shape[2]
+        st = OrcStats()
+        kex = np.zeros(self.B * self.Hkv * n_new, np.uint8) if want_exempt else None
+        vex = np.zeros(self.B * self.Hkv * n_new, np.uint8) if want_exempt else None
+        rc = lib().orc_quantize_append(ctypes.byref(self.struct), _p(k), _p(v), n_new, offset, ctypes.byref(st),
+                                       _p(kex), _p(vex))
+        if rc != 0:
+            raise ValueError("oracle rejected append arguments")
+        stats = {f: getattr(st, f) for f, _ in OrcStats._fields_}
+        if want_exempt:
+            stats["k_row_exempt"] = kex.reshape(self.B, self.Hkv, n_new)
+            stats["v_row_exempt"] = vex.reshape(self.B, self.Hkv, n_new)
+        return stats
+
+    def unpack(self, b, h, n, which):
+        out = np.zeros(self.d, np.uint8)
+        lib().orc_unpack_codes(ctypes.byref(self.struct), b, h, n, which, _p(out))
+        return out
+
+    def dequantize(self, b, h, n0, n):
+        kh = np.zeros((n, self.d), np.float64)
+        vh = np.zeros((n, self.d), np.float64)
+        lib().orc_dequantize(ctypes.byref(self.struct), b, h, n0, n, _p(kh), _p(vh))
+        return kh, vh
+
+    def attention(self, q: np.ndarray, lens: np.ndarray, mask: np.ndarray | None, scale: float,
+                  rows: np.ndarray | None = None) -> np.ndarray:
+        """q: [B][Hq][d]; returns [nrows][d] fp64 (all B*Hq rows when rows is None)."""
+        qf = as_f32(q)
+        Hq = qf.shape[1]
+        ln = np.ascontiguousarray(lens, dtype=np.int32)
+        mk = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint32)
+        rw = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+        n = self.B * Hq if rw is None else rw.size
+        out = np.zeros((n, self.d), np.float64)
+        lib().orc_attention(ctypes.byref(self.struct), _p(qf), Hq, _p(ln), _p(mk), float(scale), _p(rw),
+                            0 if rw is None else rw.size, _p(out))
+        return out
+
+
+def select(q: np.ndarray, Hkv: int, rotate: int, keep: int):
+    """-> (mask [B][Hkv] uint32, energy [B][Hkv][d/4] fp64)"""
+    qf = as_f32(q)
+    B, Hq, d = qf.shape
+    mask = np.zeros((B, Hkv), np.uint32)
+    energy = np.zeros((B, Hkv, d // 4), np.float64)
+    lib().orc_select(_p(qf), B, Hq, Hkv, d, rotate, keep, _p(mask), _p(energy))
+    return mask, energy
+
+
+def dual_score(T: np.ndarray, q: np.ndarray, k: np.ndarray) -> float:
+    Tc = np.ascontiguousarray(T, dtype=np.float64)
+    qc = np.ascontiguousarray(q, dtype=np.float64)
+    kc = np.ascontiguousarray(k, dtype=np.float64)
+    return lib().orc_dual_score(_p(Tc), Tc.shape[0], _p(qc), _p(kc))

@@ -1,0 +1,48 @@
+"""The five synthetic workloads of the quantized-KV decode path.
+
+Each names its shapes, code widths and flags; inputs are drawn by
+``synth.Synth`` with seed ``base_seed + id``.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+
+@dataclass(frozen=True)
+class Workload:
+    id: int
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    T: int              # tokens drawn per sequence (= tokens appended)
+    capacity: int       # cache capacity in tokens
+    offset: int         # first token written by the append
+    fmt: str            # "f32" or "bf16" inputs
+    k_bits: int
+    v_bits: int
+    rotate_k: int
+    keep_ch0: int
+    keep_groups: int    # channel groups of 4 kept by the query-channel pruning (32 = none)
+    len_range: tuple | None = None  # per-sequence lengths U[lo, hi] (ragged), else all T
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+
+WORKLOADS = [
+    Workload(0, "tiny_int4", 1, 1, 1, 128, 1024, 1024, 0, "f32", 4, 4, 1, 0, 32),
+    Workload(1, "gqa_int4_b8_h32x8_n32k", 8, 32, 8, 128, 32768, 32768, 0, "bf16", 4, 4, 1, 0, 32),
+    Workload(2, "dualqk_int2_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16", 2, 2, 1, 1, 19),
+    Workload(3, "append_b16_h8_t4096_at8192", 16, 8, 8, 128, 4096, 12288, 8192, "bf16", 4, 2, 1, 0, 32),
+    Workload(4, "ragged_b64_h64x8_n1k16k_keep24", 64, 64, 8, 128, 16384, 16384, 0, "bf16", 4, 2, 1, 1, 24,
+             (1024, 16384)),
+]
+
+BASE_SEED = 0
+
+
+def by_id(i: int) -> Workload:
+    return WORKLOADS[i]
