@@ -1,0 +1,174 @@
+/*
+ * kvq -- decode attention over a low-bit quantized KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every entry point takes plain pointers and sizes; device pointers
+ * are CUDA global memory owned by the caller (the library never allocates or
+ * frees them), host pointers are ordinary (preferably pinned) host memory.
+ * All GPU work is enqueued asynchronously on the CUDA stream passed as
+ * `stream` (a cudaStream_t cast to void*; NULL = legacy default stream).
+ * Arguments are checked on the host before anything is launched; a rejected
+ * call returns a non-zero kvq_status and enqueues nothing.  No C++ exception
+ * crosses this boundary.  KVQ_ERR_CUDA reports a launch or copy error
+ * reported by the CUDA runtime at enqueue time.
+ *
+ * Method sources (page title, section):
+ *  [DQK] "Dual-QK: Sharp Queries and Flat Keys for Prunable 2-bit KV Caches"
+ *        (paperlayer.ai summary of arXiv 2610.09827)
+ *  [TQ]  "TurboQuant on Quantized Models: Solving Compound Quantization Error
+ *        with Pre-RoPE Compression and KV Compaction" (tq-kv, Zenodo abstract)
+ *  [SIQ] "Statistical Inference and Quality Measures of KV Cache Quantisations
+ *        Inspired by TurboQuant" (gist.science explainer), scheme KQV
+ *  [CQ]  "CASK-Q" (decentralizedcompute.company), Method
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned pointer, bad flag   */
+  KVQ_ERR_UNSUPPORTED = 2, /* a valid configuration this build does not implement          */
+  KVQ_ERR_CAPACITY = 3,    /* offset + n_new > capacity, or max_len > capacity             */
+  KVQ_ERR_WORKSPACE = 4,   /* workspace smaller than the matching *_workspace_bytes query */
+  KVQ_ERR_CUDA = 5         /* the CUDA runtime reported an error when enqueuing            */
+} kvq_status;
+
+typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1, KVQ_F16 = 2 } kvq_dtype;
+
+/*
+ * Packed cache descriptor.  Shapes: B = batch, H = kv_heads, d = head_dim,
+ * N = capacity (tokens), g = 32 (group_size), P = 4 (prune_granule).
+ * Supported: d = 128, g = 32, P = 4, k_bits, v_bits in {2, 4},
+ * N a multiple of 64, every pointer 16-byte aligned.
+ *
+ * Byte layout (all little-endian; ownership: caller-allocated device memory
+ * of the sizes kvq_cache_sizes reports):
+ *  k_codes  [B][H][d/P][N] words of P*k_bits bits (uint16 for INT4, uint8 for
+ *           INT2): one row per group of 4 channels, channel-major, so a decode
+ *           step reads only the rows it keeps [DQK Sec. 3.3].  Channel
+ *           4p+i of token n sits in bits [i*k_bits, (i+1)*k_bits) of word
+ *           (p, n).
+ *  k_scales [B][H][d/g][N] x {fp16 scale, fp16 zero} (4 bytes).
+ *  k_ch0    [B][H][N] bf16, channel 0 of the rotated key (only when keep_ch0;
+ *           NULL otherwise); code slot 0 of such keys is written as 0 and
+ *           channel 0 is outside group 0's range [DQK Sec. 1, Sec. 3.3, App. C.3].
+ *  v_codes  [B][H][N][d*v_bits/8] bytes, token-major; channel c at byte
+ *           c*v_bits/8, bits ((c mod (8/v_bits))*v_bits ...).
+ *  v_scales [B][H][N][d/g] x {fp16 scale, fp16 zero}.
+ * Dequantized element: x = scale * code + zero [DQK Sec. 3.3, App. B.2; CQ].
+ */
+typedef struct {
+  int32_t batch, kv_heads, head_dim, capacity;
+  int32_t k_bits, v_bits, group_size, prune_granule;
+  int32_t rotate_k; /* 1: keys (and queries) pass through the orthonormal Walsh-Hadamard transform */
+  int32_t keep_ch0; /* 1: rotated channel 0 of each key is kept in bf16, unquantized               */
+  void* k_codes;
+  void* k_scales;
+  void* k_ch0;
+  void* v_codes;
+  void* v_scales;
+} kvq_cache;
+
+/*
+ * Sizes in bytes of the five cache arrays, in the order k_codes, k_scales,
+ * k_ch0 (0 unless keep_ch0), v_codes, v_scales.  Pointer fields are ignored.
+ */
+KVQ_API kvq_status kvq_cache_sizes(const kvq_cache* cache, size_t bytes_out[5]);
+
+/*
+ * Quantize and append n_new tokens per (sequence, kv head) at token positions
+ * [offset, offset + n_new) of the cache; no other token is read or written,
+ * so earlier tokens are never re-quantized (incremental cache [TQ]).
+ *  k_new, v_new: device [B][H][n_new][d] of `dtype`.
+ * Keys: x = H_d k / sqrt(d) when rotate_k (fp64 butterflies in natural
+ * Sylvester order, rounded to fp32) [DQK Sec. 1; SIQ KQV; TQ]; channel 0 to
+ * bf16 when keep_ch0; then per token and per 32-channel group
+ * scale = fp16((max - min) / L), zero = fp16(min), L = 2^bits - 1,
+ * code = clamp(round_half_even((x - zero) / scale), 0, L) with IEEE fp32
+ * subtract and divide [DQK Sec. 3.3].  Values: same quantizer, no rotation
+ * [DQK App. B.2].  n_new == 0 is a no-op.
+ */
+KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new,
+                                       kvq_dtype dtype, int32_t n_new, int32_t offset, void* stream);
+
+/*
+ * Dynamic query-channel pruning [DQK Sec. 3.2, App. C.2]: for each
+ * (sequence b, kv head h) the energy of channel group p is
+ * E[p] = sum over the G = q_heads/kv_heads query heads of head h and the 4
+ * channels of group p of q_rot^2 (fp64, heads outer, channels inner);
+ * the keep_groups largest energies are kept, equal energies keeping the
+ * lower p.  mask_out[b*H + h] (device uint32) gets bit p set for a kept group.
+ *  q: device [B][q_heads][d] of `dtype`, un-rotated (rotated here when
+ *  rotate_k).  Query head j belongs to kv head j / G.  keep_groups in [1, 32].
+ */
+KVQ_API kvq_status kvq_select_channels(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                       int32_t keep_groups, uint32_t* mask_out, void* stream);
+
+/* Tokens per sequence split that kvq_decode_attention uses for these sizes (> 0), or 0 on bad arguments. */
+KVQ_API int32_t kvq_decode_split_tokens(const kvq_cache* cache, int32_t q_heads, int32_t max_len);
+
+/* Device workspace bytes kvq_decode_attention needs for these sizes (0 on bad arguments). */
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_heads, int32_t max_len);
+
+/*
+ * Fused decode attention over the packed cache [DQK Sec. 3.2-3.4; TQ].
+ * For each sequence b and query head j (kv head h = j / G):
+ *  s_n = softmax_scale * sum over kept channels c of q_rot[c] * k_hat_n[c],
+ *  o = sum_n softmax(s)_n * v_hat_n over n < seq_lens[b],
+ * scored directly from the key codes (no dequantized key is written):
+ * per group, scale * (q . codes) + zero * sum(q), plus q_rot[0] * k_ch0 when
+ * channel 0 is kept.  The sequence is cut into splits; each split keeps a
+ * running max and sum, and a combine pass merges them into one softmax
+ * over the whole sequence [DQK Sec. 3.4].
+ *  q:        device [B][q_heads][d] of `dtype`, un-rotated.
+ *  seq_lens: device int32 [B]; entries are clamped to [0, max_len]; a
+ *            sequence of length 0 gets a zero output.
+ *  max_len:  host bound on seq_lens, 0 <= max_len <= capacity; sizes the grid.
+ *  mask:     device uint32 [B][H] from kvq_select_channels, or NULL = every
+ *            channel group.
+ *  out:      device fp32 [B][q_heads][d].
+ *  workspace: device scratch of at least kvq_decode_workspace_bytes bytes,
+ *            owned by the caller; not read by later calls.
+ */
+KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                        const int32_t* seq_lens, int32_t max_len, const uint32_t* mask,
+                                        float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+
+/* Device workspace bytes kvq_decode_step_host needs (0 on bad arguments). */
+KVQ_API size_t kvq_decode_step_workspace_bytes(const kvq_cache* cache, kvq_dtype dtype, int32_t q_heads,
+                                               int32_t max_len);
+
+/*
+ * One decode step from host buffers: copies q_host ([B][q_heads][d] of
+ * `dtype`) into the device workspace, runs kvq_select_channels when
+ * keep_groups < 32, then kvq_decode_attention, and copies the fp32 output to
+ * out_host ([B][q_heads][d]).  Everything is enqueued on `stream`; out_host
+ * is valid once the stream has been synchronized.  Host buffers should be
+ * page-locked for the copies to run asynchronously.
+ */
+KVQ_API kvq_status kvq_decode_step_host(const kvq_cache* cache, const void* q_host, kvq_dtype dtype,
+                                        int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
+                                        int32_t keep_groups, float softmax_scale, float* out_host,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Static description of a status code. */
+KVQ_API const char* kvq_status_string(kvq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

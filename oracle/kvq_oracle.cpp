@@ -157,6 +157,10 @@ int32_t orc_quantize_group(const float* x, const uint8_t* include, int32_t n, in
       if (x[i] < mn) mn = x[i];
       if (x[i] > mx) mx = x[i];
     }
+  // -0 and +0 compare equal; the extremes are taken as +0 so that the stored
+  // scale and zero do not depend on which of the two came first.
+  mn = mn + 0.0f;
+  mx = mx + 0.0f;
   // scale = (max - min) / L and zero = min, both computed in fp32 and stored
   // as fp16; values beyond the fp16 range saturate at +-65504.
   float range = mx - mn;

@@ -205,3 +205,9 @@ def test_tie_window_flags_exact_midpoints():
     # (x - z)/s = 0.5 exactly -> exempt
     _, _, _, ex, _, _ = orc.quantize_group(np.array([0, 0.5, 1, 3], np.float32), 2)
     assert list(ex) == [0, 1, 0, 0]
+
+
+def test_signed_zero_extremes_are_canonical():
+    a = orc.quantize_group(np.array([-0.0, 0.0, 0.0, -0.0], np.float32), 2)
+    b = orc.quantize_group(np.array([0.0, -0.0, -0.0, 0.0], np.float32), 2)
+    assert a[0] == b[0] == 0 and a[1] == b[1] == 0
