@@ -147,6 +147,28 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, k
                                         float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                                         void* stream);
 
+/*
+ * The two halves of kvq_decode_attention, for callers that time them apart or
+ * move the per-split partials elsewhere before combining them (the partials
+ * are exactly what a sequence-sharded deployment would exchange).
+ * kvq_decode_partials runs the split kernel only and writes, in `workspace`:
+ *   acc [B][q_heads][S][d] fp32 at byte 0, the unnormalized sum of
+ *       p * v_hat over split s of each (sequence, query head);
+ *   ml  [B][q_heads][S] x {max, sum} fp32 pairs at byte
+ *       round_up(B*q_heads*S*d*4, 256): the split's running max of the scores
+ *       in base-2 units (score * log2(e)) and its sum of 2^(score - max);
+ * S = ceil(max_len / kvq_decode_split_tokens(...)).  Splits at or beyond a
+ * sequence's length are not written.  kvq_decode_combine reads them back
+ * (same cache, q_heads, seq_lens and max_len) and writes `out` [B][q_heads][d].
+ * Argument rules and statuses are those of kvq_decode_attention.
+ */
+KVQ_API kvq_status kvq_decode_partials(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                       const int32_t* seq_lens, int32_t max_len, const uint32_t* mask,
+                                       float softmax_scale, void* workspace, size_t workspace_bytes, void* stream);
+KVQ_API kvq_status kvq_decode_combine(const kvq_cache* cache, int32_t q_heads, const int32_t* seq_lens,
+                                      int32_t max_len, float* out, const void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
 /* Device workspace bytes kvq_decode_step_host needs (0 on bad arguments). */
 KVQ_API size_t kvq_decode_step_workspace_bytes(const kvq_cache* cache, kvq_dtype dtype, int32_t q_heads,
                                                int32_t max_len);

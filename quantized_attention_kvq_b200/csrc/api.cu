@@ -1,0 +1,308 @@
+// C ABI of libkvq: argument checks, split planning, workspace carving and
+// kernel launches.  Every check happens on the host before anything is
+// enqueued; no exception leaves this file.
+#include <cmath>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kSMs = 148;            // B200
+constexpr long kTargetCtas = 8L * kSMs;  // split CTAs aimed at for a full-length batch
+constexpr size_t kAlign = 256;
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t dtype_size(kvq_dtype t) { return t == KVQ_F32 ? 4 : 2; }
+inline bool dtype_ok(int t) { return t == KVQ_F32 || t == KVQ_BF16 || t == KVQ_F16; }
+
+// Shape/flag checks that do not look at pointers.
+kvq_status check_shape(const kvq_cache* c) {
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->kv_heads < 1 || c->capacity < 1 || c->head_dim < 1) return KVQ_ERR_INVALID_ARG;
+  if ((c->rotate_k != 0 && c->rotate_k != 1) || (c->keep_ch0 != 0 && c->keep_ch0 != 1)) return KVQ_ERR_INVALID_ARG;
+  if (c->head_dim != kHeadDim || c->group_size != kGroup || c->prune_granule != kGranule) return KVQ_ERR_UNSUPPORTED;
+  if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return KVQ_ERR_UNSUPPORTED;
+  if (c->capacity % 64 != 0) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+kvq_status check_cache(const kvq_cache* c) {
+  kvq_status st = check_shape(c);
+  if (st != KVQ_OK) return st;
+  if (!c->k_codes || !c->k_scales || !c->v_codes || !c->v_scales || (c->keep_ch0 && !c->k_ch0))
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(c->k_codes) || !aligned16(c->k_scales) || !aligned16(c->v_codes) || !aligned16(c->v_scales) ||
+      (c->keep_ch0 && !aligned16(c->k_ch0)))
+    return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+kvq_status check_heads(const kvq_cache* c, int32_t q_heads) {
+  if (q_heads < 1 || q_heads % c->kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  return KVQ_OK;
+}
+
+bool decode_g_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+
+CacheView view(const kvq_cache* c) {
+  CacheView v;
+  v.B = c->batch;
+  v.H = c->kv_heads;
+  v.cap = c->capacity;
+  v.k_bits = c->k_bits;
+  v.v_bits = c->v_bits;
+  v.rotate = c->rotate_k;
+  v.keep_ch0 = c->keep_ch0;
+  v.kc = static_cast<uint8_t*>(c->k_codes);
+  v.ks = static_cast<__half2*>(c->k_scales);
+  v.k0 = static_cast<__nv_bfloat16*>(c->k_ch0);
+  v.vc = static_cast<uint8_t*>(c->v_codes);
+  v.vs = static_cast<__half2*>(c->v_scales);
+  return v;
+}
+
+double inv_sqrt_d() { return 1.0 / std::sqrt((double)kHeadDim); }
+
+// Tokens per split: a multiple of the 128-token tile chosen so that a batch
+// of full-length sequences yields about kTargetCtas split CTAs.
+int32_t plan_split_tokens(int B, int H, int max_len) {
+  if (max_len <= kDecodeTile) return kDecodeTile;
+  const long units = (long)B * H;
+  const long splits = (kTargetCtas + units - 1) / units;
+  long s = (max_len + splits - 1) / splits;
+  s = (long)round_up((size_t)s, kDecodeTile);
+  if (s < 2 * kDecodeTile) s = 2 * kDecodeTile;
+  return (int32_t)s;
+}
+
+struct DecodePlan {
+  int32_t split_tokens, max_splits;
+  size_t acc_bytes, ml_offset, bytes;
+};
+
+DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
+  DecodePlan p;
+  p.split_tokens = plan_split_tokens(c->batch, c->kv_heads, max_len);
+  p.max_splits = (max_len + p.split_tokens - 1) / p.split_tokens;
+  const size_t units = (size_t)c->batch * q_heads * (size_t)p.max_splits;
+  p.acc_bytes = units * kHeadDim * sizeof(float);
+  p.ml_offset = round_up(p.acc_bytes, kAlign);
+  p.bytes = p.ml_offset + round_up(units * sizeof(float2), kAlign);
+  if (p.bytes == 0) p.bytes = kAlign;
+  return p;
+}
+
+kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+// which halves of the decode to enqueue
+enum { kRunSplit = 1, kRunCombine = 2 };
+
+kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                          const int32_t* seq_lens, int32_t max_len, const uint32_t* mask, float softmax_scale,
+                          float* out, void* workspace, const DecodePlan& plan, cudaStream_t s,
+                          int parts = kRunSplit | kRunCombine) {
+  DecodeArgs a;
+  a.c = view(c);
+  a.q = q;
+  a.dtype = dtype;
+  a.Hq = q_heads;
+  a.seq_lens = seq_lens;
+  a.max_len = max_len;
+  a.mask = mask;
+  a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);  // log2(e)
+  a.inv_sqrt_d = inv_sqrt_d();
+  a.split_tokens = plan.split_tokens;
+  a.max_splits = plan.max_splits;
+  a.part_acc = static_cast<float*>(workspace);
+  a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
+  a.out = out;
+  if ((parts & kRunSplit) && plan.max_splits > 0) {
+    kvq_status st = cuda_status(launch_decode_split(a, s));
+    if (st != KVQ_OK) return st;
+  }
+  if (parts & kRunCombine) return cuda_status(launch_combine(a, s));
+  return KVQ_OK;
+}
+
+kvq_status check_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                        const int32_t* seq_lens, int32_t max_len, float softmax_scale, const void* out,
+                        const void* workspace, size_t workspace_bytes, bool need_q) {
+  kvq_status st = check_cache(c);
+  if (st != KVQ_OK) return st;
+  if ((st = check_heads(c, q_heads)) != KVQ_OK) return st;
+  if (!dtype_ok(dtype) || (need_q && (!q || !aligned16(q))) || !seq_lens || !out || !workspace ||
+      !aligned16(workspace))
+    return KVQ_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  if (max_len < 0) return KVQ_ERR_INVALID_ARG;
+  if (max_len > c->capacity) return KVQ_ERR_CAPACITY;
+  if (!decode_g_supported(q_heads / c->kv_heads)) return KVQ_ERR_UNSUPPORTED;
+  if (workspace_bytes < plan_decode(c, q_heads, max_len).bytes) return KVQ_ERR_WORKSPACE;
+  return KVQ_OK;
+}
+
+}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+KVQ_API kvq_status kvq_cache_sizes(const kvq_cache* c, size_t bytes_out[5]) {
+  kvq_status st = check_shape(c);
+  if (st != KVQ_OK) return st;
+  if (!bytes_out) return KVQ_ERR_INVALID_ARG;
+  const size_t rows = (size_t)c->batch * c->kv_heads * (size_t)c->capacity;
+  bytes_out[0] = rows * kPruneGroups * (c->k_bits == 4 ? 2 : 1);
+  bytes_out[1] = rows * kGroups * 4;
+  bytes_out[2] = c->keep_ch0 ? rows * 2 : 0;
+  bytes_out[3] = rows * (kHeadDim * c->v_bits / 8);
+  bytes_out[4] = rows * kGroups * 4;
+  return KVQ_OK;
+}
+
+KVQ_API kvq_status kvq_quantize_append(const kvq_cache* c, const void* k_new, const void* v_new, kvq_dtype dtype,
+                                       int32_t n_new, int32_t offset, void* stream) {
+  kvq_status st = check_cache(c);
+  if (st != KVQ_OK) return st;
+  if (!dtype_ok(dtype) || n_new < 0 || offset < 0) return KVQ_ERR_INVALID_ARG;
+  if ((int64_t)offset + n_new > c->capacity) return KVQ_ERR_CAPACITY;
+  if (n_new == 0) return KVQ_OK;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
+  AppendArgs a;
+  a.c = view(c);
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.dtype = dtype;
+  a.n_new = n_new;
+  a.offset = offset;
+  a.inv_sqrt_d = inv_sqrt_d();
+  return cuda_status(launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
+KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                       int32_t keep_groups, uint32_t* mask_out, void* stream) {
+  kvq_status st = check_shape(c);
+  if (st != KVQ_OK) return st;
+  if ((st = check_heads(c, q_heads)) != KVQ_OK) return st;
+  if (!dtype_ok(dtype) || !q || !mask_out || !aligned16(q)) return KVQ_ERR_INVALID_ARG;
+  if (keep_groups < 1 || keep_groups > kPruneGroups) return KVQ_ERR_INVALID_ARG;
+  if (q_heads / c->kv_heads > 64) return KVQ_ERR_UNSUPPORTED;
+  SelectArgs a;
+  a.q = q;
+  a.dtype = dtype;
+  a.B = c->batch;
+  a.Hq = q_heads;
+  a.H = c->kv_heads;
+  a.rotate = c->rotate_k;
+  a.keep = keep_groups;
+  a.inv_sqrt_d = inv_sqrt_d();
+  a.mask = mask_out;
+  return cuda_status(launch_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+KVQ_API int32_t kvq_decode_split_tokens(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
+  if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK) return 0;
+  if (max_len < 0 || max_len > c->capacity) return 0;
+  return plan_split_tokens(c->batch, c->kv_heads, max_len);
+}
+
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
+  if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK) return 0;
+  if (max_len < 0 || max_len > c->capacity) return 0;
+  return plan_decode(c, q_heads, max_len).bytes;
+}
+
+KVQ_API kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                        const int32_t* seq_lens, int32_t max_len, const uint32_t* mask,
+                                        float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+  kvq_status st = check_decode(c, q, dtype, q_heads, seq_lens, max_len, softmax_scale, out, workspace,
+                               workspace_bytes, true);
+  if (st != KVQ_OK) return st;
+  return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, out, workspace,
+                        plan_decode(c, q_heads, max_len), static_cast<cudaStream_t>(stream));
+}
+
+KVQ_API kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                       const int32_t* seq_lens, int32_t max_len, const uint32_t* mask,
+                                       float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  kvq_status st = check_decode(c, q, dtype, q_heads, seq_lens, max_len, softmax_scale, workspace, workspace,
+                               workspace_bytes, true);
+  if (st != KVQ_OK) return st;
+  return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, nullptr, workspace,
+                        plan_decode(c, q_heads, max_len), static_cast<cudaStream_t>(stream), kRunSplit);
+}
+
+KVQ_API kvq_status kvq_decode_combine(const kvq_cache* c, int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
+                                      float* out, const void* workspace, size_t workspace_bytes, void* stream) {
+  kvq_status st = check_decode(c, nullptr, KVQ_F32, q_heads, seq_lens, max_len, 1.0f, out, workspace,
+                               workspace_bytes, false);
+  if (st != KVQ_OK) return st;
+  return enqueue_decode(c, nullptr, KVQ_F32, q_heads, seq_lens, max_len, nullptr, 1.0f, out,
+                        const_cast<void*>(workspace), plan_decode(c, q_heads, max_len),
+                        static_cast<cudaStream_t>(stream), kRunCombine);
+}
+
+KVQ_API size_t kvq_decode_step_workspace_bytes(const kvq_cache* c, kvq_dtype dtype, int32_t q_heads,
+                                               int32_t max_len) {
+  if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK || !dtype_ok(dtype)) return 0;
+  if (max_len < 0 || max_len > c->capacity) return 0;
+  const size_t qb = (size_t)c->batch * q_heads * kHeadDim * dtype_size(dtype);
+  const size_t mb = (size_t)c->batch * c->kv_heads * sizeof(uint32_t);
+  const size_t ob = (size_t)c->batch * q_heads * kHeadDim * sizeof(float);
+  return round_up(qb, kAlign) + round_up(mb, kAlign) + round_up(ob, kAlign) + plan_decode(c, q_heads, max_len).bytes;
+}
+
+KVQ_API kvq_status kvq_decode_step_host(const kvq_cache* c, const void* q_host, kvq_dtype dtype, int32_t q_heads,
+                                        const int32_t* seq_lens, int32_t max_len, int32_t keep_groups,
+                                        float softmax_scale, float* out_host, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  kvq_status st = check_cache(c);
+  if (st != KVQ_OK) return st;
+  if ((st = check_heads(c, q_heads)) != KVQ_OK) return st;
+  if (!dtype_ok(dtype) || !q_host || !out_host || !seq_lens || !workspace || !aligned16(workspace))
+    return KVQ_ERR_INVALID_ARG;
+  if (keep_groups < 1 || keep_groups > kPruneGroups || !std::isfinite(softmax_scale) || max_len < 0)
+    return KVQ_ERR_INVALID_ARG;
+  if (max_len > c->capacity) return KVQ_ERR_CAPACITY;
+  if (!decode_g_supported(q_heads / c->kv_heads)) return KVQ_ERR_UNSUPPORTED;
+  if (workspace_bytes < kvq_decode_step_workspace_bytes(c, dtype, q_heads, max_len)) return KVQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const size_t qb = (size_t)c->batch * q_heads * kHeadDim * dtype_size(dtype);
+  const size_t mb = (size_t)c->batch * c->kv_heads * sizeof(uint32_t);
+  const size_t ob = (size_t)c->batch * q_heads * kHeadDim * sizeof(float);
+  void* q_dev = ws;
+  uint32_t* mask_dev = reinterpret_cast<uint32_t*>(ws + round_up(qb, kAlign));
+  float* out_dev = reinterpret_cast<float*>(ws + round_up(qb, kAlign) + round_up(mb, kAlign));
+  void* dec_ws = ws + round_up(qb, kAlign) + round_up(mb, kAlign) + round_up(ob, kAlign);
+  if ((st = cuda_status(cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s))) != KVQ_OK) return st;
+  const uint32_t* mask = nullptr;
+  if (keep_groups < kPruneGroups) {
+    st = kvq_select_channels(c, q_dev, dtype, q_heads, keep_groups, mask_dev, stream);
+    if (st != KVQ_OK) return st;
+    mask = mask_dev;
+  }
+  const DecodePlan plan = plan_decode(c, q_heads, max_len);
+  st = enqueue_decode(c, q_dev, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, out_dev, dec_ws, plan, s);
+  if (st != KVQ_OK) return st;
+  return cuda_status(cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s));
+}
+
+KVQ_API const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
+    case KVQ_ERR_WORKSPACE: return "workspace too small";
+    case KVQ_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

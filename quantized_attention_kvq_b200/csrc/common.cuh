@@ -1,0 +1,136 @@
+// Internal helpers shared by the kvq kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kGroup = 32;         // channels per quantization group
+constexpr int kGroups = kHeadDim / kGroup;      // 4
+constexpr int kGranule = 4;        // channels per pruning group
+constexpr int kPruneGroups = kHeadDim / kGranule;  // 32
+constexpr int kDecodeTile = 128;   // tokens per decode tile; split lengths are multiples of it
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// ---------------------------------------------------------------- loads
+// Four consecutive input elements as fp32 (exact widening).
+__device__ __forceinline__ void load4(const float* p, float f[4]) {
+  float4 v = *reinterpret_cast<const float4*>(p);
+  f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+__device__ __forceinline__ void load4(const __nv_bfloat16* p, float f[4]) {
+  uint2 v = *reinterpret_cast<const uint2*>(p);
+  f[0] = __uint_as_float(v.x << 16);
+  f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  f[2] = __uint_as_float(v.y << 16);
+  f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ void load4(const __half* p, float f[4]) {
+  uint2 v = *reinterpret_cast<const uint2*>(p);
+  __half2 a = *reinterpret_cast<__half2*>(&v.x), b = *reinterpret_cast<__half2*>(&v.y);
+  float2 fa = __half22float2(a), fb = __half22float2(b);
+  f[0] = fa.x; f[1] = fa.y; f[2] = fb.x; f[3] = fb.y;
+}
+
+// ---------------------------------------------------------------- rotation
+// Orthonormal Walsh-Hadamard transform of one 128-channel row held by a warp,
+// lane l owning channels 4l..4l+3.  Butterflies in fp64, natural Sylvester
+// order (stage h pairs channel i with i+h, i & h == 0, -> (a+b, a-b)), then one
+// fp64 multiply by 1/sqrt(128) and a round to fp32.  Every fp64 add of bf16 or
+// fp32 inputs is IEEE-rounded in the same order on every lane, so the fp32
+// result is reproducible bit for bit.
+__device__ __forceinline__ void rotate_row_warp(float x[4], double inv_sqrt_d, int lane) {
+  double v0 = x[0], v1 = x[1], v2 = x[2], v3 = x[3];
+  // h = 1: (0,1), (2,3)
+  double a0 = __dadd_rn(v0, v1), a1 = __dsub_rn(v0, v1);
+  double a2 = __dadd_rn(v2, v3), a3 = __dsub_rn(v2, v3);
+  // h = 2: (0,2), (1,3)
+  v0 = __dadd_rn(a0, a2); v2 = __dsub_rn(a0, a2);
+  v1 = __dadd_rn(a1, a3); v3 = __dsub_rn(a1, a3);
+  // h = 4 .. 64: partner lane l ^ m; the lower lane keeps a+b, the upper a-b
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+    double o0 = __shfl_xor_sync(kFull, v0, m), o1 = __shfl_xor_sync(kFull, v1, m);
+    double o2 = __shfl_xor_sync(kFull, v2, m), o3 = __shfl_xor_sync(kFull, v3, m);
+    v0 = upper ? __dsub_rn(o0, v0) : __dadd_rn(v0, o0);
+    v1 = upper ? __dsub_rn(o1, v1) : __dadd_rn(v1, o1);
+    v2 = upper ? __dsub_rn(o2, v2) : __dadd_rn(v2, o2);
+    v3 = upper ? __dsub_rn(o3, v3) : __dadd_rn(v3, o3);
+  }
+  x[0] = __double2float_rn(__dmul_rn(v0, inv_sqrt_d));
+  x[1] = __double2float_rn(__dmul_rn(v1, inv_sqrt_d));
+  x[2] = __double2float_rn(__dmul_rn(v2, inv_sqrt_d));
+  x[3] = __double2float_rn(__dmul_rn(v3, inv_sqrt_d));
+}
+
+// Load one 128-channel row (4 channels per lane) and optionally rotate it.
+template <typename In>
+__device__ __forceinline__ void load_row_warp(const In* row, bool rotate, double inv_sqrt_d, int lane, float x[4]) {
+  load4(row + 4 * lane, x);
+  if (rotate) rotate_row_warp(x, inv_sqrt_d, lane);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+  return v;
+}
+
+// ---------------------------------------------------------------- launch plumbing
+struct CacheView {
+  int B, H, cap, k_bits, v_bits, rotate, keep_ch0;
+  uint8_t* kc;
+  __half2* ks;
+  __nv_bfloat16* k0;
+  uint8_t* vc;
+  __half2* vs;
+};
+
+struct AppendArgs {
+  CacheView c;
+  const void* k_new;
+  const void* v_new;
+  int dtype, n_new, offset;
+  double inv_sqrt_d;
+};
+
+struct SelectArgs {
+  const void* q;
+  int dtype, B, Hq, H, rotate, keep;
+  double inv_sqrt_d;
+  uint32_t* mask;
+};
+
+struct DecodeArgs {
+  CacheView c;
+  const void* q;
+  int dtype, Hq;
+  const int32_t* seq_lens;
+  int max_len;
+  const uint32_t* mask;
+  float scale_log2;  // softmax_scale * log2(e): scores live in the exp2 domain
+  double inv_sqrt_d;
+  int split_tokens, max_splits;
+  float* part_acc;  // [B][Hq][max_splits][128]
+  float2* part_ml;  // [B][Hq][max_splits] (running max, running sum)
+  float* out;       // [B][Hq][128]
+};
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
+cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace kvq

@@ -1,0 +1,84 @@
+"""Helpers shared by the GPU parity tests: upload seeded inputs, run the CUDA
+path through the C ABI, run the oracle on the same host arrays, compare."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from oracle import oracle as orc
+from quantized_attention_kvq_b200 import native, synth
+
+ATOL_REL = 2e-3  # max|o_gpu - o_ref| <= 2e-3 * max|o_ref|
+TIE_BUDGET = 1e-5  # exempt (near-tie) elements allowed per element quantized
+
+
+def to_device(a: np.ndarray, fmt: str) -> torch.Tensor:
+    if fmt == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    if fmt == "f16":
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float16)).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def host_f32(a: np.ndarray, fmt: str) -> np.ndarray:
+    """fp32 values the device receives for a host input array."""
+    if fmt == "bf16":
+        return synth.bf16_to_f32(a)
+    if fmt == "f16":
+        return np.ascontiguousarray(a, dtype=np.float16).astype(np.float32)
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def gpu_arrays(cache: native.KVQCache) -> dict:
+    out = {"k_codes": cache.k_codes, "k_scales": cache.k_scales, "v_codes": cache.v_codes,
+           "v_scales": cache.v_scales}
+    if cache.k_ch0 is not None:
+        out["k_ch0"] = cache.k_ch0
+    return {k: v.cpu().numpy() for k, v in out.items()}
+
+
+def oracle_arrays(c: orc.Cache) -> dict:
+    out = {"k_codes": c.k_codes, "k_scales": c.k_scales.view(np.uint8), "v_codes": c.v_codes,
+           "v_scales": c.v_scales.view(np.uint8)}
+    if c.k_ch0 is not None:
+        out["k_ch0"] = c.k_ch0.view(np.uint8)
+    return out
+
+
+def compare_cache_bytes(gpu: dict, ref: dict, stats: dict | None = None):
+    """Bit-exact comparison; mismatches are allowed only where the oracle counted
+    a near-tie, and the exempt count must stay within TIE_BUDGET of the elements."""
+    mismatched = {}
+    for name, r in ref.items():
+        g = gpu[name]
+        assert g.shape == r.shape, (name, g.shape, r.shape)
+        bad = np.count_nonzero(g != r)
+        if bad:
+            mismatched[name] = bad
+    if stats is not None:
+        elems = stats["k_elems"] + stats["v_elems"]
+        exempt = stats["k_exempt"] + stats["v_exempt"]
+        assert exempt <= TIE_BUDGET * max(elems, 1) + 1, (exempt, elems)
+        if mismatched:
+            total_bad = sum(mismatched.values())
+            assert total_bad <= exempt * 4 + 8 * stats["groups_exempt"], (mismatched, stats)
+    else:
+        assert not mismatched, mismatched
+    return mismatched
+
+
+def assert_close_output(o_gpu: np.ndarray, o_ref: np.ndarray, what: str = ""):
+    ref_max = np.abs(o_ref).max()
+    err = np.abs(o_gpu.astype(np.float64) - o_ref).max()
+    assert err <= ATOL_REL * ref_max, f"{what}: max err {err:.3e} > {ATOL_REL} * {ref_max:.3e}"
+    return err / max(ref_max, 1e-300)
+
+
+def mask_u32(mask_t: torch.Tensor) -> np.ndarray:
+    return mask_t.cpu().numpy().view(np.uint32)
+
+
+def softmax_scale() -> float:
+    return 1.0 / math.sqrt(128)

@@ -1,0 +1,148 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads and exports
+every entry point include/kvq.h declares, sizes and plans follow the layout,
+and bad arguments are rejected with the documented status before anything is
+enqueued.  Every call here fails validation or is a pure host query, so no
+kernel is ever launched with the placeholder pointers used below."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_attention_kvq_b200 import native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x100000  # 16-byte-aligned placeholder; only reaches calls that are rejected
+
+
+@pytest.fixture(scope="module")
+def L():
+    from quantized_attention_kvq_b200 import build
+    build.build_kvq()
+    return native.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]+?\b(kvq_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    declared = header_functions()
+    assert len(declared) >= 9
+    assert sorted(native.SYMBOLS) == declared
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def desc(**kw):
+    d = native.describe(kw.pop("B", 2), kw.pop("H", 2), kw.pop("cap", 256), kw.pop("kb", 4), kw.pop("vb", 2),
+                        kw.pop("rot", 1), kw.pop("ch0", 1))
+    for k, v in kw.items():
+        setattr(d, k, v)
+    for f in ("k_codes", "k_scales", "k_ch0", "v_codes", "v_scales"):
+        if getattr(d, f) is None:
+            setattr(d, f, FAKE)
+    return d
+
+
+def test_cache_sizes_follow_layout(L):
+    d = native.describe(3, 5, 128, 4, 2, 1, 1)
+    assert native.cache_sizes(d) == [3 * 5 * 128 * 32 * 2, 3 * 5 * 128 * 16, 3 * 5 * 128 * 2,
+                                     3 * 5 * 128 * 32, 3 * 5 * 128 * 16]
+    d = native.describe(1, 1, 64, 2, 4, 0, 0)
+    assert native.cache_sizes(d) == [64 * 32, 64 * 16, 0, 64 * 64, 64 * 16]
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 64, native.KVQ_ERR_UNSUPPORTED), ("k_bits", 3, native.KVQ_ERR_UNSUPPORTED),
+    ("v_bits", 8, native.KVQ_ERR_UNSUPPORTED), ("capacity", 100, native.KVQ_ERR_UNSUPPORTED),
+    ("group_size", 64, native.KVQ_ERR_UNSUPPORTED), ("prune_granule", 8, native.KVQ_ERR_UNSUPPORTED),
+    ("batch", 0, native.KVQ_ERR_INVALID_ARG), ("rotate_k", 2, native.KVQ_ERR_INVALID_ARG),
+    ("k_codes", 0, native.KVQ_ERR_INVALID_ARG), ("k_ch0", 0, native.KVQ_ERR_INVALID_ARG),
+    ("v_scales", FAKE + 4, native.KVQ_ERR_INVALID_ARG),
+])
+def test_bad_cache_rejected(L, field, value, status):
+    d = desc()
+    setattr(d, field, value)
+    rc = L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 0, None)
+    assert rc == status
+
+
+def test_append_argument_checks(L):
+    d = desc()
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 200, 100, None) == \
+        native.KVQ_ERR_CAPACITY
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, -1, 0, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, 7, 4, 0, None) == native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_append(ctypes.byref(d), None, FAKE, native.KVQ_BF16, 4, 0, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE + 2, FAKE, native.KVQ_BF16, 4, 0, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    # zero new tokens is an accepted no-op that enqueues nothing
+    assert L.kvq_quantize_append(ctypes.byref(d), None, None, native.KVQ_BF16, 0, 256, None) == native.KVQ_OK
+    assert L.kvq_quantize_append(None, FAKE, FAKE, native.KVQ_BF16, 4, 0, None) == native.KVQ_ERR_INVALID_ARG
+
+
+def test_select_argument_checks(L):
+    d = desc()
+    for keep in (0, 33):
+        assert L.kvq_select_channels(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, keep, FAKE, None) == \
+            native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_select_channels(ctypes.byref(d), FAKE, native.KVQ_BF16, 7, 4, FAKE, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_select_channels(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, 4, None, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_select_channels(ctypes.byref(d), FAKE, native.KVQ_BF16, 2 * 128, 4, FAKE, None) == \
+        native.KVQ_ERR_UNSUPPORTED
+
+
+def test_decode_argument_checks(L):
+    d = desc()
+    ws = L.kvq_decode_workspace_bytes(ctypes.byref(d), 8, 256)
+    assert ws > 0
+
+    def call(q_heads=8, max_len=256, ws_bytes=ws, scale=0.088, wsp=FAKE, lens=FAKE):
+        return L.kvq_decode_attention(ctypes.byref(d), FAKE, native.KVQ_BF16, q_heads, lens, max_len, None,
+                                      scale, FAKE, wsp, ws_bytes, None)
+    assert call(ws_bytes=ws - 1) == native.KVQ_ERR_WORKSPACE
+    assert call(max_len=257) == native.KVQ_ERR_CAPACITY
+    assert call(max_len=-1) == native.KVQ_ERR_INVALID_ARG
+    assert call(q_heads=7) == native.KVQ_ERR_INVALID_ARG
+    assert call(q_heads=6) == native.KVQ_ERR_UNSUPPORTED  # G = 3 not built
+    assert call(q_heads=2 * 32) == native.KVQ_ERR_UNSUPPORTED  # G = 32 not built
+    assert call(scale=float("nan")) == native.KVQ_ERR_INVALID_ARG
+    assert call(wsp=None) == native.KVQ_ERR_INVALID_ARG
+    assert call(lens=None) == native.KVQ_ERR_INVALID_ARG
+    assert call(wsp=FAKE + 8) == native.KVQ_ERR_INVALID_ARG
+
+
+def test_decode_step_host_argument_checks(L):
+    d = desc()
+    ws = L.kvq_decode_step_workspace_bytes(ctypes.byref(d), native.KVQ_BF16, 8, 256)
+    assert ws > L.kvq_decode_workspace_bytes(ctypes.byref(d), 8, 256)
+    rc = L.kvq_decode_step_host(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, FAKE, 256, 19, 0.088, FAKE, FAKE,
+                                ws - 1, None)
+    assert rc == native.KVQ_ERR_WORKSPACE
+    rc = L.kvq_decode_step_host(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, FAKE, 256, 0, 0.088, FAKE, FAKE, ws, None)
+    assert rc == native.KVQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B,H,max_len", [(8, 8, 32768), (4, 8, 131072), (64, 8, 16384), (1, 1, 1024),
+                                         (16, 8, 12288), (2, 2, 100), (1, 1, 0), (3, 7, 4096)])
+def test_split_plan_covers_sequence(L, B, H, max_len):
+    d = native.describe(B, H, max(64, (max_len + 63) // 64 * 64), 4, 4)
+    S = L.kvq_decode_split_tokens(ctypes.byref(d), H, max_len)
+    assert S > 0 and S % 128 == 0
+    splits = (max_len + S - 1) // S
+    ws = L.kvq_decode_workspace_bytes(ctypes.byref(d), H * 2, max_len)
+    assert ws >= B * H * 2 * splits * (128 * 4 + 8)
+    if max_len >= 4096 and B * H <= 1184:
+        assert B * H * splits >= 148  # enough split CTAs to cover every SM
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert native.status_string(s)
+    assert "workspace" in native.status_string(native.KVQ_ERR_WORKSPACE)
