@@ -274,21 +274,9 @@ def run_kvq(args):
     q_np = s.q()
     cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev)
     for b in range(wl.B):  # one sequence at a time keeps host memory small
-        kb = np.stack([s.k_slice(b, h) for h in range(wl.Hkv)])[None]
-        vb = np.stack([s.v_slice(b, h) for h in range(wl.Hkv)])[None]
-        sub = native.describe(1, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0)
-        per = [x // wl.B for x in native.cache_sizes(cache.desc)]
-        sub.k_codes = cache.k_codes.data_ptr() + b * per[0]
-        sub.k_scales = cache.k_scales.data_ptr() + b * per[1]
-        sub.k_ch0 = cache.k_ch0.data_ptr() + b * per[2] if wl.keep_ch0 else None
-        sub.v_codes = cache.v_codes.data_ptr() + b * per[3]
-        sub.v_scales = cache.v_scales.data_ptr() + b * per[4]
-        kd, vd = up(kb), up(vb)
-        rc = native.lib().kvq_quantize_append(native.ctypes.byref(sub), kd.data_ptr(), vd.data_ptr(),
-                                              native.torch_dtype_code(kd.dtype), wl.T, wl.offset,
-                                              torch.cuda.current_stream().cuda_stream)
-        if rc != native.KVQ_OK:
-            raise native.KvqError(rc, "kvq_quantize_append")
+        kd = up(np.stack([s.k_slice(b, h) for h in range(wl.Hkv)]))
+        vd = up(np.stack([s.v_slice(b, h) for h in range(wl.Hkv)]))
+        cache.append_sequence(b, kd, vd, wl.offset)
         torch.cuda.synchronize()
         del kd, vd
     qd = up(q_np)

@@ -138,6 +138,27 @@ class KVQCache:
         self.desc.v_scales = _dev_ptr(self.v_scales)
         self.B, self.H, self.capacity = B, H, capacity
 
+    def sequence_desc(self, b: int) -> KvqCacheStruct:
+        """Descriptor of sequence b alone (batch 1): every cache array is [B][...]
+        with the sequence outermost, so this is a pointer offset per array."""
+        per = [x // self.B for x in cache_sizes(self.desc)]
+        d = describe(1, self.H, self.capacity, self.desc.k_bits, self.desc.v_bits, self.desc.rotate_k,
+                     self.desc.keep_ch0)
+        d.k_codes = self.desc.k_codes + b * per[0]
+        d.k_scales = self.desc.k_scales + b * per[1]
+        d.k_ch0 = self.desc.k_ch0 + b * per[2] if self.desc.keep_ch0 else None
+        d.v_codes = self.desc.v_codes + b * per[3]
+        d.v_scales = self.desc.v_scales + b * per[4]
+        return d
+
+    def append_sequence(self, b: int, k_new: torch.Tensor, v_new: torch.Tensor, offset: int, stream=None):
+        """Append [H][n_new][128] (or [1][H][n_new][128]) tokens to sequence b only."""
+        d = self.sequence_desc(b)
+        n_new = k_new.shape[-2]
+        _check(lib().kvq_quantize_append(ctypes.byref(d), _dev_ptr(k_new), _dev_ptr(v_new),
+                                         torch_dtype_code(k_new.dtype), n_new, offset, _stream(stream)),
+               "kvq_quantize_append")
+
     # -- calls --------------------------------------------------------------
     def append(self, k_new: torch.Tensor, v_new: torch.Tensor, offset: int, stream=None):
         """k_new, v_new: [B][H][n_new][128] (fp32 / bf16 / fp16) on the device."""

@@ -26,19 +26,25 @@ def draw(seed, B, Hq, H, T, fmt):
 
 
 def build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset=0, chunks=None):
+    """Append the same inputs through the C ABI and through the oracle.
+    Returns (gpu cache, oracle cache, near-tie row flags, comparison geometry)."""
     gc = native.KVQCache(B, H, cap, kb, vb, rot, ch0)
     oc = orc.Cache(B, H, 128, cap, kb, vb, rot, ch0)
     T = k.shape[2]
     chunks = chunks or [T]
+    flags = {"k": np.zeros((B, H, cap), np.uint8), "v": np.zeros((B, H, cap), np.uint8)}
+    elems = 0
     t = 0
-    stats = None
     for n in chunks:
         gc.append(to_device(k[:, :, t:t + n], fmt), to_device(v[:, :, t:t + n], fmt), offset + t)
-        st = oc.append(host_f32(k[:, :, t:t + n], fmt), host_f32(v[:, :, t:t + n], fmt), offset + t)
-        stats = st if stats is None else {key: stats[key] + st[key] for key in st}
+        st = oc.append(host_f32(k[:, :, t:t + n], fmt), host_f32(v[:, :, t:t + n], fmt), offset + t,
+                       want_exempt=True)
+        flags["k"][:, :, offset + t:offset + t + n] = st["k_row_exempt"]
+        flags["v"][:, :, offset + t:offset + t + n] = st["v_row_exempt"]
+        elems += st["k_elems"] + st["v_elems"]
         t += n
     torch.cuda.synchronize()
-    return gc, oc, stats
+    return gc, oc, flags, (cap, kb, vb, elems)
 
 
 @pytest.mark.parametrize("kb,vb,rot,ch0,fmt,T,offset,cap", [
@@ -53,20 +59,19 @@ def build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset=0, chunks=None):
 def test_append_bitexact(kb, vb, rot, ch0, fmt, T, offset, cap):
     B, H = 2, 3
     _, k, v = draw(100 + T, B, H, H, T, fmt)
-    gc, oc, stats = build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset)
-    compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), stats)
-    assert stats["k_exempt"] + stats["v_exempt"] <= 1e-5 * (stats["k_elems"] + stats["v_elems"]) + 1
+    gc, oc, flags, geom = build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset)
+    compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), flags, geom)
 
 
 def test_append_in_chunks_equals_one_append():
     B, H, T = 2, 2, 300
     _, k, v = draw(7, B, H, H, T, "bf16")
-    whole, _, _ = build_both(B, H, 320, 4, 2, 1, 1, k, v, "bf16")
-    parts, oc, stats = build_both(B, H, 320, 4, 2, 1, 1, k, v, "bf16", chunks=[1, 63, 64, 100, 72])
+    whole, _, _, _ = build_both(B, H, 320, 4, 2, 1, 1, k, v, "bf16")
+    parts, oc, flags, geom = build_both(B, H, 320, 4, 2, 1, 1, k, v, "bf16", chunks=[1, 63, 64, 100, 72])
     gw, gp = gpu_arrays(whole), gpu_arrays(parts)
     for name in gw:
         np.testing.assert_array_equal(gw[name], gp[name])
-    compare_cache_bytes(gp, oracle_arrays(oc), stats)
+    compare_cache_bytes(gp, oracle_arrays(oc), flags, geom)
 
 
 def test_append_stress_distributions():
@@ -81,8 +86,8 @@ def test_append_stress_distributions():
     for x in (heavy, low, focused):
         k = x.astype(np.float32)
         v = np.flip(k, axis=2).copy()
-        gc, oc, stats = build_both(B, H, T, 4, 2, 1, 1, k, v, "f32")
-        compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), stats)
+        gc, oc, flags, geom = build_both(B, H, T, 4, 2, 1, 1, k, v, "f32")
+        compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), flags, geom)
 
 
 @pytest.mark.parametrize("G,keep,rot,fmt", [(1, 7, 1, "f32"), (4, 19, 1, "bf16"), (8, 24, 1, "bf16"),
@@ -118,8 +123,8 @@ DECODE_CASES = [
 def test_decode_matches_oracle(case):
     B, G, H, kb, vb, rot, ch0, keep, fmt, T, lens = case
     q, k, v = draw(300 + T + G, B, G * H, H, T, fmt)
-    gc, oc, stats = build_both(B, H, T, kb, vb, rot, ch0, k, v, fmt)
-    compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), stats)
+    gc, oc, flags, geom = build_both(B, H, T, kb, vb, rot, ch0, k, v, fmt)
+    compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), flags, geom)
     qd = to_device(q, fmt)
     lens_np = np.array(lens, np.int32)
     lens_d = torch.from_numpy(lens_np).cuda()
@@ -143,7 +148,7 @@ def test_decode_matches_oracle(case):
 def test_full_mask_is_bit_identical_to_no_mask_and_split_plan_is_exact():
     B, G, H, T = 2, 4, 2, 1024
     q, k, v = draw(9, B, G * H, H, T, "bf16")
-    gc, _, _ = build_both(B, H, T, 4, 4, 1, 1, k, v, "bf16")
+    gc, _, _, _ = build_both(B, H, T, 4, 4, 1, 1, k, v, "bf16")
     qd = to_device(q, "bf16")
     lens = torch.tensor([1024, 700], dtype=torch.int32, device="cuda")
     full = torch.full((B, H), -1, dtype=torch.int32, device="cuda")
@@ -161,7 +166,7 @@ def test_full_mask_is_bit_identical_to_no_mask_and_split_plan_is_exact():
 def test_decode_step_host_matches_device_calls():
     B, G, H, T = 2, 4, 2, 512
     q, k, v = draw(13, B, G * H, H, T, "bf16")
-    gc, _, _ = build_both(B, H, T, 2, 2, 1, 1, k, v, "bf16")
+    gc, _, _, _ = build_both(B, H, T, 2, 2, 1, 1, k, v, "bf16")
     qd = to_device(q, "bf16")
     lens = torch.tensor([512, 300], dtype=torch.int32, device="cuda")
     want = gc.decode(qd, lens, T, gc.select(qd, 19)).cpu()
