@@ -169,6 +169,32 @@ KVQ_API kvq_status kvq_decode_combine(const kvq_cache* cache, int32_t q_heads, c
                                       int32_t max_len, float* out, const void* workspace, size_t workspace_bytes,
                                       void* stream);
 
+/*
+ * kvq_decode_attention without a workspace argument, for callers that cannot
+ * allocate device memory: an engine that owns every byte of device memory in
+ * its own pool and has no allocator to lend across this C boundary, or a
+ * decode loop that must never call cudaMalloc because it can synchronize the
+ * device or fail under a fixed memory budget.  The pages have no counterpart
+ * to this entry point; it is an interface convenience only.
+ *
+ * Same arguments, results and statuses as kvq_decode_attention, minus the
+ * workspace.  The per-split partials live in a fixed 16 MiB device array
+ * inside the library (every GPU that loads the library holds it until the
+ * process exits); a call whose partials would not fit, i.e. whose
+ * kvq_decode_workspace_bytes exceeds 16 MiB, returns KVQ_ERR_WORKSPACE and
+ * enqueues nothing.  The call allocates nothing.  The first call on a device
+ * looks up that array's device address (with the device current) and caches
+ * it, so make that first call before any stream capture.  Every call shares
+ * the array: calls that run concurrently on the GPU (different streams, or
+ * different host threads, without ordering between them) race on it and give
+ * undefined results.  Nothing in the array needs to start at zero: each call
+ * writes every partial it reads back.
+ */
+KVQ_API kvq_status kvq_decode_attention_static(const kvq_cache* cache, const void* q, kvq_dtype dtype,
+                                               int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
+                                               const uint32_t* mask, float softmax_scale, float* out,
+                                               void* stream);
+
 /* Device workspace bytes kvq_decode_step_host needs (0 on bad arguments). */
 KVQ_API size_t kvq_decode_step_workspace_bytes(const kvq_cache* cache, kvq_dtype dtype, int32_t q_heads,
                                                int32_t max_len);

@@ -145,6 +145,17 @@ kvq_status check_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, int3
 }
 
 }  // namespace
+
+kvq_status decode_into(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads, const int32_t* seq_lens,
+                       int32_t max_len, const uint32_t* mask, float softmax_scale, float* out, void* workspace,
+                       size_t workspace_bytes, cudaStream_t s) {
+  kvq_status st = check_decode(c, q, dtype, q_heads, seq_lens, max_len, softmax_scale, out, workspace,
+                               workspace_bytes, true);
+  if (st != KVQ_OK) return st;
+  return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, out, workspace,
+                        plan_decode(c, q_heads, max_len), s);
+}
+
 }  // namespace kvq
 
 using namespace kvq;

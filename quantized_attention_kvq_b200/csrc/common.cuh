@@ -133,4 +133,10 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 
+// Checked split decode + combine into a caller-chosen scratch buffer of
+// `workspace_bytes` bytes (the body of kvq_decode_attention).
+kvq_status decode_into(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads, const int32_t* seq_lens,
+                       int32_t max_len, const uint32_t* mask, float softmax_scale, float* out, void* workspace,
+                       size_t workspace_bytes, cudaStream_t s);
+
 }  // namespace kvq

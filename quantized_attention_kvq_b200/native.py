@@ -21,7 +21,7 @@ KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 SYMBOLS = ("kvq_cache_sizes", "kvq_quantize_append", "kvq_select_channels", "kvq_decode_split_tokens",
            "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
            "kvq_decode_step_workspace_bytes",
-           "kvq_decode_step_host", "kvq_status_string")
+           "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_status_string")
 
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -73,6 +73,8 @@ def lib():
         L.kvq_decode_step_host.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _I32, ctypes.c_float, _P, _P,
                                            ctypes.c_size_t, _P]
         L.kvq_decode_step_host.restype = ctypes.c_int
+        L.kvq_decode_attention_static.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _P, ctypes.c_float, _P, _P]
+        L.kvq_decode_attention_static.restype = ctypes.c_int
         L.kvq_status_string.argtypes = [ctypes.c_int]
         L.kvq_status_string.restype = ctypes.c_char_p
         _lib = L
