@@ -120,7 +120,8 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
   if ((parts & kRunSplit) && plan.max_splits > 0) {
-    kvq_status st = cuda_status(launch_decode_split(a, s));
+    const bool tc = decode_tc_supported(q_heads / c->kv_heads);
+    kvq_status st = cuda_status(tc ? launch_decode_split_tc(a, s) : launch_decode_split(a, s));
     if (st != KVQ_OK) return st;
   }
   if (parts & kRunCombine) return cuda_status(launch_combine(a, s));

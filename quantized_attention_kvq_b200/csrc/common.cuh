@@ -132,6 +132,9 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
+// tensor-core split decode: GQA groups of 4, 8 or 16 query heads
+bool decode_tc_supported(int g);
+cudaError_t launch_decode_split_tc(const DecodeArgs& a, cudaStream_t s);
 
 // Checked split decode + combine into a caller-chosen scratch buffer of
 // `workspace_bytes` bytes (the body of kvq_decode_attention).

@@ -1,0 +1,169 @@
+// Thin inline-PTX wrappers for the sm_100a features the tensor-core decode
+// uses: mbarriers, 1-D bulk async copies (TMA), tcgen05 tensor-memory
+// allocation, UMMA issue/commit and tensor-memory loads.  Each wrapper is one
+// PTX instruction (or a bounded loop around one).
+#pragma once
+
+#include <stdint.h>
+
+namespace kvq {
+namespace sm100 {
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_fence_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for phase `parity` of the barrier, giving up after `limit` polls (each
+// poll itself suspends for a bounded, hardware-chosen time).  Returns false on
+// give-up so the caller can flag the result instead of hanging.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t limit = 1u << 22) {
+  for (uint32_t i = 0; i < limit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// ---------------------------------------------------------------- bulk copy
+// 1-D bulk copy global -> shared, completion counted in bytes on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// generic-proxy shared-memory writes -> visible to the async proxy (UMMA operands)
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// ---------------------------------------------------------------- tensor memory
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols));
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, no swizzle: start address, leading-dim
+// byte offset (LBO), stride-dim byte offset (SBO), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Instruction descriptor for kind::f16 with f16 A/B and f32 accumulation.
+// a_mn / b_mn: operand stored MN-major (1) or K-major (0).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                        // D format: f32
+         | (0u << 7) | (0u << 10)         // A, B format: f16
+         | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+// Arrive once on `bar` when every UMMA this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// Each thread of the warp reads N consecutive 32-bit columns of its own lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_ld<2>(uint32_t taddr, uint32_t (&r)[2]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<4>(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ---------------------------------------------------------------- code -> f16
+// Eight 4-bit codes n0..n7 (n_i in bits 4i..4i+3 of x) -> exact f16 integers,
+// returned as half2 pairs (n0,n4) (n1,n5) (n2,n6) (n3,n7).  Each nibble is
+// OR-ed into the mantissa of 1024.0 (0x6400), then 1024 (or 16*1024 for the
+// high nibble of a byte, rescaled by 1/16) is subtracted; all exact in f16.
+__device__ __forceinline__ void codes4_to_f16(uint32_t x, uint32_t (&r)[4]) {
+  const uint32_t magic = 0x64006400u;
+  uint32_t a, b, c, d;
+  const uint32_t x2 = x >> 8;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(a) : "r"(x), "r"(0x000F000Fu), "r"(magic));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(b) : "r"(x), "r"(0x00F000F0u), "r"(magic));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(c) : "r"(x2), "r"(0x000F000Fu), "r"(magic));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(x2), "r"(0x00F000F0u), "r"(magic));
+  const uint32_t sub = 0x64006400u;    // (1024, 1024)
+  const uint32_t mul16 = 0x2C002C00u;  // (1/16, 1/16)
+  const uint32_t add64 = 0xD400D400u;  // (-64, -64)
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r[0]) : "r"(a), "r"(sub));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[1]) : "r"(b), "r"(mul16), "r"(add64));
+  asm("sub.f16x2 %0, %1, %2;" : "=r"(r[2]) : "r"(c), "r"(sub));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[3]) : "r"(d), "r"(mul16), "r"(add64));
+}
+
+// Sixteen 2-bit codes f0..f15 (f_i in bits 2i..2i+1) -> exact f16 integers as
+// half2 pairs (f0,f8) (f1,f9) ... (f7,f15).
+__device__ __forceinline__ void codes2_to_f16(uint32_t x, uint32_t (&r)[8]) {
+  const uint32_t magic = 0x64006400u;
+  // field k of the low byte pair sits at bit 2k of each half: value 1024 + 4^k f
+  const uint32_t mul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};  // 1, 1/4, 1/16, 1/64
+  const uint32_t add[4] = {0xE400E400u, 0xDC00DC00u, 0xD400D400u, 0xCC00CC00u};  // -1024, -256, -64, -16
+  const uint32_t xs[2] = {x, x >> 8};
+#pragma unroll
+  for (int half = 0; half < 2; ++half)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t t;
+      asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(t) : "r"(xs[half]), "r"(0x00030003u << (2 * k)), "r"(magic));
+      asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[half * 4 + k]) : "r"(t), "r"(mul[k]), "r"(add[k]));
+    }
+}
+
+}  // namespace sm100
+}  // namespace kvq
