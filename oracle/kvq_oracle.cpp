@@ -78,14 +78,20 @@ bool near_half_midpoint(float x, double rel) {
 inline size_t bh_index(const orc_cache* c, int b, int h) { return (size_t)b * c->kv_heads + h; }
 
 // --- layout: byte/element addresses of the packed cache --------------------
-// K codes: channel-major rows, one row per group of 4 channels; a token's 4
+// Keys are stored in blocks of kBlock tokens.  Within a block, K codes are
+// channel-major: one row of kBlock words per group of 4 channels; a token's 4
 // codes share one 16-bit (INT4) or 8-bit (INT2) word, channel 4p+i in bits
-// [i*bits, (i+1)*bits).
+// [i*bits, (i+1)*bits).  Key scale/zero pairs follow the same blocking with
+// one row per 32-channel group.
+constexpr int kBlock = 128;
+inline size_t n_blocks(const orc_cache* c) { return (size_t)(c->capacity + kBlock - 1) / kBlock; }
 inline size_t k_word_index(const orc_cache* c, int b, int h, int pg, int n) {
-  return (bh_index(c, b, h) * (c->head_dim / kGranule) + pg) * (size_t)c->capacity + n;
+  const size_t blk = bh_index(c, b, h) * n_blocks(c) + n / kBlock;
+  return (blk * (c->head_dim / kGranule) + pg) * kBlock + n % kBlock;
 }
 inline size_t k_scale_index(const orc_cache* c, int b, int h, int g, int n) {
-  return (bh_index(c, b, h) * (c->head_dim / kGroup) + g) * (size_t)c->capacity + n;
+  const size_t blk = bh_index(c, b, h) * n_blocks(c) + n / kBlock;
+  return (blk * (c->head_dim / kGroup) + g) * kBlock + n % kBlock;
 }
 inline size_t ch0_index(const orc_cache* c, int b, int h, int n) {
   return bh_index(c, b, h) * (size_t)c->capacity + n;

@@ -40,8 +40,8 @@ typedef struct {
   int32_t batch, kv_heads, head_dim, capacity;
   int32_t k_bits, v_bits; /* 2 or 4 */
   int32_t rotate_k, keep_ch0;
-  uint8_t* k_codes;   /* [B][Hkv][d/4][cap] x (4*k_bits/8) bytes          */
-  uint16_t* k_scales; /* [B][Hkv][d/32][cap] x {fp16 scale, fp16 zero}      */
+  uint8_t* k_codes;   /* [B][Hkv][ceil(cap/128)][d/4][128] x (4*k_bits/8) bytes     */
+  uint16_t* k_scales; /* [B][Hkv][ceil(cap/128)][d/32][128] x {fp16 scale, fp16 zero} */
   uint16_t* k_ch0;    /* [B][Hkv][cap] bf16, or NULL                        */
   uint8_t* v_codes;   /* [B][Hkv][cap][d*v_bits/8]                          */
   uint16_t* v_scales; /* [B][Hkv][cap][d/32] x {fp16 scale, fp16 zero}      */

@@ -132,14 +132,19 @@ def test_key_layout_is_channel_major_words():
         k[0, 0, 0, 32 * g:32 * g + 32] = np.arange(32) % 16
         k[0, 0, 0, 32 * g + 31] = 15  # max 15, min 0 -> scale 1, zero 0
     v = np.zeros_like(k)
-    c, _ = _cache_with(k, v, 4, 4, 0, 0, capacity=3, offset=1)
+    c, _ = _cache_with(k, v, 4, 4, 0, 0, capacity=256, offset=129)
     codes = (np.arange(d) % 32) % 16
     codes[31::32] = 15
-    words = c.k_codes.view(np.uint16).reshape(32, 3)  # [group of 4 channels][token]
+    words = c.k_codes.view(np.uint16).reshape(2, 32, 128)  # [block of 128 tokens][group of 4 channels][token]
     for p in range(32):
         want = sum(int(codes[4 * p + i]) << (4 * i) for i in range(4))
-        assert words[p, 1] == want
-        assert words[p, 0] == 0 and words[p, 2] == 0
+        assert words[1, p, 1] == want  # token 129 = block 1, position 1
+    words[1, :, 1] = 0
+    assert not words.any()
+    sc = c.k_scales.view(np.uint32).reshape(2, 4, 128)  # [block][group][token]
+    assert sc[1, :, 1].all()
+    sc[1, :, 1] = 0
+    assert not sc.any()
 
 
 def test_value_layout_is_token_major_nibbles():
@@ -160,14 +165,14 @@ def test_channel0_outlier_is_excluded_from_range():
     k[0, 0, 1, 0] = 1000.0  # outlier only in channel 0 of token 1
     v = np.zeros_like(k)
     c, _ = _cache_with(k, v, 2, 2, 0, 1)
-    sc = c.k_scales.reshape(4, 2, 2)  # [group][token][scale, zero]
+    sc = c.k_scales.reshape(4, 128, 2)  # [group][token (one block)][scale, zero]
     np.testing.assert_array_equal(sc[:, 0], sc[:, 1])
     np.testing.assert_array_equal(c.unpack(0, 0, 0, 0)[1:], c.unpack(0, 0, 1, 0)[1:])
     assert c.unpack(0, 0, 1, 0)[0] == 0
     assert orc.bf16_value(int(c.k_ch0[1])) == 1000.0
     # without the channel-0 rule the outlier widens group 0's range
     c2, _ = _cache_with(k, v, 2, 2, 0, 0)
-    assert orc.half_value(int(c2.k_scales.reshape(4, 2, 2)[0, 1, 0])) > 100
+    assert orc.half_value(int(c2.k_scales.reshape(4, 128, 2)[0, 1, 0])) > 100
 
 
 def test_channel0_keeps_rotated_value_in_bf16():
@@ -190,9 +195,9 @@ def test_append_leaves_other_tokens_untouched_and_is_incremental():
     parts.append(k[:, :, 5:], v[:, :, 5:], 5)
     for name in ("k_codes", "k_scales", "k_ch0", "v_codes", "v_scales"):
         np.testing.assert_array_equal(getattr(whole, name), getattr(parts, name))
-    # tokens 12..15 were never written
-    assert not whole.k_codes.view(np.uint16).reshape(2, 2, 32, 16)[..., 12:].any()
-    assert snap.view(np.uint16).reshape(2, 2, 32, 16)[..., :5].any()
+    # tokens 12..127 of the (single) key block were never written
+    assert not whole.k_codes.view(np.uint16).reshape(2, 2, 32, 128)[..., 12:].any()
+    assert snap.view(np.uint16).reshape(2, 2, 32, 128)[..., :5].any()
 
 
 def test_append_rejects_overflowing_offset():
