@@ -51,16 +51,18 @@ typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1, KVQ_F16 = 2 } kvq_dtype;
  * Packed cache descriptor.  Shapes: B = batch, H = kv_heads, d = head_dim,
  * N = capacity (tokens), g = 32 (group_size), P = 4 (prune_granule).
  * Supported: d = 128, g = 32, P = 4, k_bits, v_bits in {2, 4},
- * N a multiple of 64, every pointer 16-byte aligned.
+ * N a multiple of 128, every pointer 16-byte aligned.
  *
  * Byte layout (all little-endian; ownership: caller-allocated device memory
- * of the sizes kvq_cache_sizes reports):
- *  k_codes  [B][H][d/P][N] words of P*k_bits bits (uint16 for INT4, uint8 for
- *           INT2): one row per group of 4 channels, channel-major, so a decode
- *           step reads only the rows it keeps [DQK Sec. 3.3].  Channel
- *           4p+i of token n sits in bits [i*k_bits, (i+1)*k_bits) of word
- *           (p, n).
- *  k_scales [B][H][d/g][N] x {fp16 scale, fp16 zero} (4 bytes).
+ * of the sizes kvq_cache_sizes reports).  Keys are stored in blocks of 128
+ * tokens, T = N / 128 blocks per (sequence, head):
+ *  k_codes  [B][H][T][d/P][128] words of P*k_bits bits (uint16 for INT4,
+ *           uint8 for INT2): inside a block, one row per group of 4 channels
+ *           (channel-major), so a decode step reads only the rows it keeps,
+ *           and adjacent kept rows are adjacent in memory [DQK Sec. 3.3].
+ *           Channel 4p+i of token n sits in bits [i*k_bits, (i+1)*k_bits) of
+ *           word (n / 128, p, n % 128).
+ *  k_scales [B][H][T][d/g][128] x {fp16 scale, fp16 zero} (4 bytes).
  *  k_ch0    [B][H][N] bf16, channel 0 of the rotated key (only when keep_ch0;
  *           NULL otherwise); code slot 0 of such keys is written as 0 and
  *           channel 0 is outside group 0's range [DQK Sec. 1, Sec. 3.3, App. C.3].
@@ -148,18 +150,16 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, k
                                         void* stream);
 
 /*
- * The two halves of kvq_decode_attention, for callers that time them apart or
- * move the per-split partials elsewhere before combining them (the partials
- * are exactly what a sequence-sharded deployment would exchange).
- * kvq_decode_partials runs the split kernel only and writes, in `workspace`:
- *   acc [B][q_heads][S][d] fp32 at byte 0, the unnormalized sum of
- *       p * v_hat over split s of each (sequence, query head);
- *   ml  [B][q_heads][S] x {max, sum} fp32 pairs at byte
- *       round_up(B*q_heads*S*d*4, 256): the split's running max of the scores
- *       in base-2 units (score * log2(e)) and its sum of 2^(score - max);
- * S = ceil(max_len / kvq_decode_split_tokens(...)).  Splits at or beyond a
- * sequence's length are not written.  kvq_decode_combine reads them back
- * (same cache, q_heads, seq_lens and max_len) and writes `out` [B][q_heads][d].
+ * The two halves of kvq_decode_attention, for callers that time them apart
+ * or schedule the combine separately.  kvq_decode_partials runs the split
+ * decode kernel only and leaves, in `workspace`, one partial per piece of
+ * sequence it scored: the piece's running max of the scores in base-2 units
+ * (score * log2(e)), its sum of 2^(score - max), and the unnormalized sum of
+ * 2^(score - max) * v_hat per channel, for every query head.  How pieces are
+ * cut and laid out in the workspace depends on the kernel chosen for the
+ * GQA group size and is private to the library: only kvq_decode_combine,
+ * called with the same cache, q_heads, seq_lens and max_len and the same
+ * workspace, reads it back, and writes `out` [B][q_heads][d].
  * Argument rules and statuses are those of kvq_decode_attention.
  */
 KVQ_API kvq_status kvq_decode_partials(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,

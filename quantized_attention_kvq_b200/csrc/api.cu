@@ -25,7 +25,7 @@ kvq_status check_shape(const kvq_cache* c) {
   if ((c->rotate_k != 0 && c->rotate_k != 1) || (c->keep_ch0 != 0 && c->keep_ch0 != 1)) return KVQ_ERR_INVALID_ARG;
   if (c->head_dim != kHeadDim || c->group_size != kGroup || c->prune_granule != kGranule) return KVQ_ERR_UNSUPPORTED;
   if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return KVQ_ERR_UNSUPPORTED;
-  if (c->capacity % 64 != 0) return KVQ_ERR_UNSUPPORTED;
+  if (c->capacity % kKeyBlock != 0) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
 
@@ -78,16 +78,26 @@ int32_t plan_split_tokens(int B, int H, int max_len) {
   return (int32_t)s;
 }
 
+// Decode kernels: the persistent warp-specialized tensor-core kernel for GQA
+// groups of 4 or 8 query heads, the per-split tensor-core kernel for 16, the
+// CUDA-core kernel for 1 or 2.
+enum DecodePath { kPathSimt = 0, kPathTc = 1, kPathWs = 2 };
+
 struct DecodePlan {
+  int path;
   int32_t split_tokens, max_splits;
   size_t acc_bytes, ml_offset, bytes;
 };
 
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
   DecodePlan p;
+  const int g = q_heads / c->kv_heads;
+  p.path = decode_ws_supported(g) ? kPathWs : (decode_tc_supported(g) ? kPathTc : kPathSimt);
   p.split_tokens = plan_split_tokens(c->batch, c->kv_heads, max_len);
   p.max_splits = (max_len + p.split_tokens - 1) / p.split_tokens;
-  const size_t units = (size_t)c->batch * q_heads * (size_t)p.max_splits;
+  // partial rows: per (sequence, query head, split), or per (slot, query head of the group)
+  const size_t units = p.path == kPathWs ? (size_t)decode_ws_slots(c->batch, c->kv_heads) * g
+                                         : (size_t)c->batch * q_heads * (size_t)p.max_splits;
   p.acc_bytes = units * kHeadDim * sizeof(float);
   p.ml_offset = round_up(p.acc_bytes, kAlign);
   p.bytes = p.ml_offset + round_up(units * sizeof(float2), kAlign);
@@ -120,11 +130,13 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
   if ((parts & kRunSplit) && plan.max_splits > 0) {
-    const bool tc = decode_tc_supported(q_heads / c->kv_heads);
-    kvq_status st = cuda_status(tc ? launch_decode_split_tc(a, s) : launch_decode_split(a, s));
+    cudaError_t e = plan.path == kPathWs   ? launch_decode_split_ws(a, s)
+                    : plan.path == kPathTc ? launch_decode_split_tc(a, s)
+                                           : launch_decode_split(a, s);
+    kvq_status st = cuda_status(e);
     if (st != KVQ_OK) return st;
   }
-  if (parts & kRunCombine) return cuda_status(launch_combine(a, s));
+  if (parts & kRunCombine) return cuda_status(plan.path == kPathWs ? launch_combine_ws(a, s) : launch_combine(a, s));
   return KVQ_OK;
 }
 

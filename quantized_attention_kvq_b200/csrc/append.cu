@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) k_quantize_append(AppendArg
   const size_t n0 = (size_t)a.offset + t0;
   for (int i = threadIdx.x; i < kPruneGroups * ntok; i += blockDim.x) {
     const int pg = i / ntok, t = i - pg * ntok;
-    const size_t idx = (bh * kPruneGroups + pg) * c.cap + n0 + t;
+    const size_t idx = key_word_index(bh, c.cap, pg, (int)n0 + t);
     if (KB == 4)
       reinterpret_cast<uint16_t*>(c.kc)[idx] = kw[pg][t];
     else
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) k_quantize_append(AppendArg
   }
   for (int i = threadIdx.x; i < kGroups * ntok; i += blockDim.x) {
     const int g = i / ntok, t = i - g * ntok;
-    c.ks[(bh * kGroups + g) * c.cap + n0 + t] = ksz[g][t];
+    c.ks[key_scale_index(bh, c.cap, g, (int)n0 + t)] = ksz[g][t];
   }
   if (CH0)
     for (int t = threadIdx.x; t < ntok; t += blockDim.x) c.k0[bh * c.cap + n0 + t] = k0s[t];

@@ -88,6 +88,20 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// ---------------------------------------------------------------- key layout
+// Keys are stored in blocks of kKeyBlock tokens; inside a block, one row of
+// kKeyBlock code words per channel group of 4, then (separately) one row of
+// kKeyBlock (scale, zero) pairs per 32-channel group.
+constexpr int kKeyBlock = 128;
+// index of the code word of (unit bh, channel group pg, token n)
+__host__ __device__ __forceinline__ size_t key_word_index(size_t bh, int cap, int pg, int n) {
+  return (((bh * (size_t)(cap / kKeyBlock) + n / kKeyBlock) * kPruneGroups + pg) * kKeyBlock) + n % kKeyBlock;
+}
+// index of the (scale, zero) pair of (unit bh, 32-channel group g, token n)
+__host__ __device__ __forceinline__ size_t key_scale_index(size_t bh, int cap, int g, int n) {
+  return (((bh * (size_t)(cap / kKeyBlock) + n / kKeyBlock) * kGroups + g) * kKeyBlock) + n % kKeyBlock;
+}
+
 // ---------------------------------------------------------------- launch plumbing
 struct CacheView {
   int B, H, cap, k_bits, v_bits, rotate, keep_ch0;
@@ -135,6 +149,12 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 // tensor-core split decode: GQA groups of 4, 8 or 16 query heads
 bool decode_tc_supported(int g);
 cudaError_t launch_decode_split_tc(const DecodeArgs& a, cudaStream_t s);
+// persistent warp-specialized tensor-core decode (GQA groups of 4 or 8) and
+// its combine; partial slots: one per (unit + CTA), decode_ws_slots of them
+bool decode_ws_supported(int g);
+int decode_ws_slots(int B, int H);
+cudaError_t launch_decode_split_ws(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_combine_ws(const DecodeArgs& a, cudaStream_t s);
 
 // Checked split decode + combine into a caller-chosen scratch buffer of
 // `workspace_bytes` bytes (the body of kvq_decode_attention).

@@ -66,7 +66,6 @@ __global__ void __launch_bounds__(kThreads) k_decode_split_simt(DecodeArgs a) {
     o[j] = 0.0f;
   }
   constexpr uint32_t LK = (1u << KB) - 1, LV = (1u << VB) - 1;
-  const size_t krow0 = bh * kPruneGroups * (size_t)c.cap;
 
   for (int tile = start; tile < end; tile += kDecodeTile) {
     const int n = tile + tid;
@@ -84,7 +83,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_split_simt(DecodeArgs a) {
         for (int pp = 0; pp < 8; ++pp) {
           const int pg = g * 8 + pp;
           if (!((msk >> pg) & 1u)) continue;  // CTA-uniform
-          const size_t idx = krow0 + (size_t)pg * c.cap + n;
+          const size_t idx = key_word_index(bh, c.cap, pg, n);
           const uint32_t w = KB == 4 ? (uint32_t)reinterpret_cast<const uint16_t*>(c.kc)[idx] : (uint32_t)c.kc[idx];
           const float c0 = (float)(w & LK), c1 = (float)((w >> KB) & LK);
           const float c2 = (float)((w >> (2 * KB)) & LK), c3 = (float)((w >> (3 * KB)) & LK);
@@ -99,7 +98,7 @@ __global__ void __launch_bounds__(kThreads) k_decode_split_simt(DecodeArgs a) {
       for (int j = 0; j < G; ++j) sc[j] = 0.0f;
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) {
-        const float2 sz = __half22float2(c.ks[(bh * kGroups + g) * c.cap + n]);
+        const float2 sz = __half22float2(c.ks[key_scale_index(bh, c.cap, g, n)]);
 #pragma unroll
         for (int j = 0; j < G; ++j) sc[j] = fmaf(sz.x, acc[g][j], fmaf(sz.y, qsum[j][g], sc[j]));
       }

@@ -105,7 +105,7 @@ __device__ __forceinline__ void issue_tile_loads(const DecodeArgs& a, uint8_t* r
                                                  int n0, uint32_t msk) {
   using S = TcShape<G, KB, VB, CH0>;
   const CacheView& c = a.c;
-  const int ntc = min(kTile, c.cap - n0);  // a multiple of 64 (cap % 64 == 0, n0 % 128 == 0)
+  const int ntc = kTile;  // cap and n0 are multiples of the 128-token key block
   uint32_t bytes = 0;
   bytes += (uint32_t)__popc(msk) * ntc * S::KW;
   bytes += kGroups * ntc * 4;
@@ -115,10 +115,9 @@ __device__ __forceinline__ void issue_tile_loads(const DecodeArgs& a, uint8_t* r
   const uint32_t dst = smem_addr(raw);
   for (int pg = 0; pg < kPruneGroups; ++pg)
     if ((msk >> pg) & 1u)
-      bulk_g2s(dst + S::R_KC + pg * S::KROW, c.kc + ((bh * kPruneGroups + pg) * c.cap + n0) * S::KW,
-               ntc * S::KW, bar);
-  for (int g = 0; g < kGroups; ++g)
-    bulk_g2s(dst + S::R_KS + g * kTile * 4, c.ks + (bh * kGroups + g) * c.cap + n0, ntc * 4, bar);
+      bulk_g2s(dst + S::R_KC + pg * S::KROW, c.kc + key_word_index(bh, c.cap, pg, n0) * S::KW, ntc * S::KW, bar);
+  // the block's 4 scale rows are contiguous
+  bulk_g2s(dst + S::R_KS, c.ks + key_scale_index(bh, c.cap, 0, n0), kGroups * ntc * 4, bar);
   if (CH0 && (msk & 1u)) bulk_g2s(dst + S::R_K0, c.k0 + bh * c.cap + n0, ntc * 2, bar);
   bulk_g2s(dst + S::R_VC, c.vc + (bh * c.cap + n0) * S::VROW, ntc * S::VROW, bar);
   bulk_g2s(dst + S::R_VS, c.vs + (bh * c.cap + n0) * kGroups, ntc * 16, bar);

@@ -32,6 +32,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but the thread may stay suspended (not polling) for up to
+// `ns` nanoseconds while the phase is incomplete; it resumes as soon as the
+// phase completes.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for phase `parity` of the barrier, giving up after `limit` polls (each
 // poll itself suspends for a bounded, hardware-chosen time).  Returns false on
 // give-up so the caller can flag the result instead of hanging.

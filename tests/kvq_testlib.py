@@ -49,12 +49,15 @@ def oracle_arrays(c: orc.Cache) -> dict:
 
 def _token_of(name: str, byte_idx: np.ndarray, cap: int, k_bits: int, v_bits: int):
     """(bh, token) of each byte index of a packed cache array (layout of include/kvq.h)."""
+    nblk = cap // 128  # keys live in blocks of 128 tokens, rows inside a block
     if name == "k_codes":
         w = byte_idx // (2 if k_bits == 4 else 1)
-        return w // (32 * cap), w % cap
+        blk = w // (32 * 128)
+        return blk // nblk, (blk % nblk) * 128 + w % 128
     if name == "k_scales":
         i = byte_idx // 4
-        return i // (4 * cap), i % cap
+        blk = i // (4 * 128)
+        return blk // nblk, (blk % nblk) * 128 + i % 128
     if name == "k_ch0":
         i = byte_idx // 2
         return i // cap, i % cap

@@ -50,8 +50,11 @@ def test_cache_sizes_follow_layout(L):
     d = native.describe(3, 5, 128, 4, 2, 1, 1)
     assert native.cache_sizes(d) == [3 * 5 * 128 * 32 * 2, 3 * 5 * 128 * 16, 3 * 5 * 128 * 2,
                                      3 * 5 * 128 * 32, 3 * 5 * 128 * 16]
-    d = native.describe(1, 1, 64, 2, 4, 0, 0)
-    assert native.cache_sizes(d) == [64 * 32, 64 * 16, 0, 64 * 64, 64 * 16]
+    d = native.describe(1, 1, 256, 2, 4, 0, 0)
+    assert native.cache_sizes(d) == [256 * 32, 256 * 16, 0, 256 * 64, 256 * 16]
+    # keys are stored in blocks of 128 tokens: other capacities are refused
+    assert native.lib().kvq_cache_sizes(ctypes.byref(native.describe(1, 1, 192, 4, 4)),
+                                        (ctypes.c_size_t * 5)()) == native.KVQ_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("field,value,status", [
@@ -132,7 +135,7 @@ def test_decode_step_host_argument_checks(L):
 @pytest.mark.parametrize("B,H,max_len", [(8, 8, 32768), (4, 8, 131072), (64, 8, 16384), (1, 1, 1024),
                                          (16, 8, 12288), (2, 2, 100), (1, 1, 0), (3, 7, 4096)])
 def test_split_plan_covers_sequence(L, B, H, max_len):
-    d = native.describe(B, H, max(64, (max_len + 63) // 64 * 64), 4, 4)
+    d = native.describe(B, H, max(128, (max_len + 127) // 128 * 128), 4, 4)
     S = L.kvq_decode_split_tokens(ctypes.byref(d), H, max_len)
     assert S > 0 and S % 128 == 0
     splits = (max_len + S - 1) // S

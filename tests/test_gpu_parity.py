@@ -49,12 +49,12 @@ def build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset=0, chunks=None):
 
 @pytest.mark.parametrize("kb,vb,rot,ch0,fmt,T,offset,cap", [
     (4, 4, 1, 0, "f32", 200, 0, 256),
-    (4, 4, 1, 0, "bf16", 64, 64, 192),
-    (2, 2, 1, 1, "bf16", 129, 7, 192),
+    (4, 4, 1, 0, "bf16", 64, 64, 256),
+    (2, 2, 1, 1, "bf16", 129, 7, 256),
     (4, 2, 1, 1, "bf16", 65, 0, 128),
-    (2, 4, 0, 0, "f16", 33, 31, 64),
-    (4, 2, 0, 1, "f32", 1, 63, 64),
-    (2, 2, 0, 0, "bf16", 300, 100, 448),
+    (2, 4, 0, 0, "f16", 33, 31, 128),
+    (4, 2, 0, 1, "f32", 1, 127, 128),
+    (2, 2, 0, 0, "bf16", 300, 100, 512),
 ])
 def test_append_bitexact(kb, vb, rot, ch0, fmt, T, offset, cap):
     B, H = 2, 3
@@ -66,8 +66,8 @@ def test_append_bitexact(kb, vb, rot, ch0, fmt, T, offset, cap):
 def test_append_in_chunks_equals_one_append():
     B, H, T = 2, 2, 300
     _, k, v = draw(7, B, H, H, T, "bf16")
-    whole, _, _, _ = build_both(B, H, 320, 4, 2, 1, 1, k, v, "bf16")
-    parts, oc, flags, geom = build_both(B, H, 320, 4, 2, 1, 1, k, v, "bf16", chunks=[1, 63, 64, 100, 72])
+    whole, _, _, _ = build_both(B, H, 384, 4, 2, 1, 1, k, v, "bf16")
+    parts, oc, flags, geom = build_both(B, H, 384, 4, 2, 1, 1, k, v, "bf16", chunks=[1, 63, 64, 100, 72])
     gw, gp = gpu_arrays(whole), gpu_arrays(parts)
     for name in gw:
         np.testing.assert_array_equal(gw[name], gp[name])
@@ -96,7 +96,7 @@ def test_append_stress_distributions():
 def test_select_bitexact(G, keep, rot, fmt):
     B, H = 3, 2
     q, _, _ = draw(200 + G, B, G * H, H, 1, fmt)
-    gc = native.KVQCache(B, H, 64, 4, 4, rot, 0)
+    gc = native.KVQCache(B, H, 128, 4, 4, rot, 0)
     m = mask_u32(gc.select(to_device(q, fmt), keep))
     ref, _ = orc.select(host_f32(q, fmt), H, rot, keep)
     np.testing.assert_array_equal(m, ref)
@@ -104,7 +104,7 @@ def test_select_bitexact(G, keep, rot, fmt):
 
 def test_select_ties_keep_lower_groups():
     q = np.ones((1, 4, 128), np.float32)
-    gc = native.KVQCache(1, 1, 64, 4, 4, 0, 0)
+    gc = native.KVQCache(1, 1, 128, 4, 4, 0, 0)
     assert int(mask_u32(gc.select(to_device(q, "f32"), 6))[0, 0]) == 0b111111
 
 

@@ -59,10 +59,12 @@ def check_slice_bytes(got: dict, c: orc.Cache, st: dict, wl):
         if diff.size:
             # every differing byte must sit in a token the oracle flagged as a near-tie
             cap = wl.capacity
-            if name == "k_codes":
-                tok = (diff // (2 if wl.k_bits == 4 else 1)) % cap
-            elif name == "k_scales":
-                tok = (diff // 4) % cap
+            if name == "k_codes":  # [block of 128 tokens][32 channel groups][128]
+                w = diff // (2 if wl.k_bits == 4 else 1)
+                tok = (w // (32 * 128)) * 128 + w % 128
+            elif name == "k_scales":  # [block][4 groups][128]
+                i = diff // 4
+                tok = (i // (4 * 128)) * 128 + i % 128
             elif name == "k_ch0":
                 tok = (diff // 2) % cap
             elif name == "v_codes":
@@ -156,8 +158,8 @@ def test_append_workload():
     # nothing before the offset was written
     cap, off = wl.capacity, wl.offset
     kw = 2 if wl.k_bits == 4 else 1
-    kc = gc.k_codes.view(wl.B * wl.Hkv * 32, cap * kw)
-    assert not kc[:, :off * kw].any().item()
-    assert kc[:, off * kw:].any().item()
+    kc = gc.k_codes.view(wl.B * wl.Hkv, cap // 128, 32 * 128 * kw)  # key blocks of 128 tokens
+    assert not kc[:, :off // 128].any().item()
+    assert kc[:, off // 128:].any().item()
     vc = gc.v_codes.view(wl.B * wl.Hkv, cap, -1)
     assert not vc[:, :off].any().item()

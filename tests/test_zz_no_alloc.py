@@ -58,7 +58,7 @@ def test_static_scratch_matches_workspace_entry_point_twice():
 def test_static_scratch_refuses_sizes_beyond_its_array():
     # 256 sequences x 128 query heads need 256*128*(128+2)*4 bytes of partials
     # (one split each), just over the 16 MiB array
-    B, H, Hq, cap = 256, 8, 128, 64
+    B, H, Hq, cap = 256, 8, 128, 128
     cache = native.KVQCache(B, H, cap, 2, 2, 1, 0)
     need = cache.workspace_bytes(Hq, cap)
     assert need > 16 << 20
