@@ -47,8 +47,8 @@ constexpr int kConvWarps = 8;   // warps 0-3 convert key codes, warps 4-7 value 
 constexpr int kKWarps = 4;
 constexpr int kOBufs = 3;       // PV accumulators in flight (read back two tiles late)
 constexpr float kLazyMax = 8.0f;  // the running max is raised only when a score exceeds it by 2^8
-constexpr int kRing = 3;                                       // raw code stages
-constexpr int kSRing = 4;                                      // per-token scale/zero stages
+constexpr int kRing = 2;                                       // raw code stages
+constexpr int kSRing = 3;                                      // per-token scale/zero stages
 
 template <int G, int KB, int VB, bool CH0>
 struct WsShape {
@@ -67,12 +67,18 @@ struct WsShape {
   static constexpr int KROW = kTile * KW;
   static constexpr int VROW = kHeadDim * VB / 8;
   static constexpr int TILE_AB = kTile * kHeadDim * 2;  // one f16 operand tile
+  static constexpr int KW_ = KB == 4 ? 2 : 1;
+  static constexpr int RAW_BYTES_ = kPruneGroups * kTile * KW_ + kTile * (kHeadDim * VB / 8);
+  // key operand stages: three when they fit next to everything else, else two
+  static constexpr int KST = (3 * TILE_AB + 2 * TILE_AB + 4 * NS * kHeadDim + 2 * NO * kTile * 2 +
+                              kRing * RAW_BYTES_ + kSRing * (kTile * kGroups * 8 + kTile * 2) + 2048) <= 227 * 1024
+                                 ? 3 : 2;
   static constexpr int AK_OFF = 0;
-  static constexpr int AV_OFF = AK_OFF + 2 * TILE_AB;
+  static constexpr int AV_OFF = AK_OFF + KST * TILE_AB;
   static constexpr int BQ_OFF = AV_OFF + 2 * TILE_AB;
   static constexpr int BQ_HALF = NS * kHeadDim * 2;    // q hi rows, then q lo rows
   static constexpr int BQ_BYTES = 2 * BQ_HALF;
-  static constexpr int BP_OFF = BQ_OFF + 2 * BQ_BYTES;
+  static constexpr int BP_OFF = BQ_OFF + BQ_BYTES;
   static constexpr int BP_BYTES = NO * kTile * 2;
   static constexpr int RAW_OFF = BP_OFF + 2 * BP_BYTES;
   static constexpr int R_KC = 0;
@@ -85,17 +91,17 @@ struct WsShape {
   static constexpr int S_VS = S_KS + kGroups * kTile * 4;
   static constexpr int S_K0 = S_VS + kTile * kGroups * 4;
   static constexpr int SC_BYTES = S_K0 + (CH0 ? kTile * 2 : 0);
-  static constexpr int QSUM_OFF = SC_OFF + kSRing * SC_BYTES;   // [2][G][4] f32
-  static constexpr int Q0_OFF = QSUM_OFF + 2 * G * kGroups * 4; // [2][G] f32
-  static constexpr int RED_OFF = Q0_OFF + 2 * G * 4;            // [2 tiles][2 parts][4 warps][8] f32
+  static constexpr int QSUM_OFF = SC_OFF + kSRing * SC_BYTES;   // [G][4] f32
+  static constexpr int Q0_OFF = QSUM_OFF + G * kGroups * 4;     // [G] f32
+  static constexpr int RED_OFF = Q0_OFF + G * 4;                // [2 tiles][2 parts][4 warps][8] f32
   static constexpr int RED2_OFF = RED_OFF + 2 * 2 * 4 * 8 * 4;  // [2 parts][4 warps][8] f32 (segment sums)
   // segment results waiting for their last PV: [2 tile parities][2 parts] x (max[4], sum[4], zero term[4 groups][4])
   static constexpr int PEND_OFF = RED2_OFF + 2 * 4 * 8 * 4;
   static constexpr int PEND_BYTES = 2 * 2 * 24 * 4;
   static constexpr int BAR_OFF = PEND_OFF + PEND_BYTES;
-  // mbarriers: full[R], empty[R], kready[2], vready[2], pready[2], sdone[2], pvdone[3],
+  // mbarriers: full[R], empty[R], kready[2], vready[2], pready[2], sdone[3], pvdone[3],
   // sfull[SR], sempty[SR]
-  static constexpr int NBAR = 2 * kRing + 11 + 2 * kSRing;
+  static constexpr int NBAR = 2 * kRing + 12 + 2 * kSRing;
   static constexpr int SLOT_OFF = BAR_OFF + NBAR * 8;
   static constexpr int ERR_OFF = SLOT_OFF + 4;
   static constexpr int SMEM_BYTES = ERR_OFF + 12;
@@ -231,10 +237,10 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
   auto KREADY = [&](int k) { return bar0 + 8 * (2 * kRing + k); };
   auto VREADY = [&](int k) { return bar0 + 8 * (2 * kRing + 2 + k); };
   auto PREADY = [&](int k) { return bar0 + 8 * (2 * kRing + 4 + k); };
-  auto SDONE = [&](int k) { return bar0 + 8 * (2 * kRing + 6 + k); };
-  auto PVDONE = [&](int k) { return bar0 + 8 * (2 * kRing + 8 + k); };  // k < kOBufs
-  auto SFULL = [&](int s) { return bar0 + 8 * (2 * kRing + 11 + s); };
-  auto SEMPTY = [&](int s) { return bar0 + 8 * (2 * kRing + 11 + kSRing + s); };
+  auto SDONE = [&](int k) { return bar0 + 8 * (2 * kRing + 6 + k); };   // k < KST: one per key stage
+  auto PVDONE = [&](int k) { return bar0 + 8 * (2 * kRing + 9 + k); };  // k < kOBufs
+  auto SFULL = [&](int s) { return bar0 + 8 * (2 * kRing + 12 + s); };
+  auto SEMPTY = [&](int s) { return bar0 + 8 * (2 * kRing + 12 + kSRing + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::SLOT_OFF);
   volatile int* err = reinterpret_cast<volatile int*>(smem + S::ERR_OFF);
 
@@ -251,8 +257,8 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
       mbar_init(KREADY(k), kKWarps * 32);
       mbar_init(VREADY(k), (kConvWarps - kKWarps) * 32);
       mbar_init(PREADY(k), EPI_THREADS);
-      mbar_init(SDONE(k), 1);
     }
+    for (int k = 0; k < S::KST; ++k) mbar_init(SDONE(k), 1);
     for (int k = 0; k < kOBufs; ++k) mbar_init(PVDONE(k), 1);
     *err = 0;
     mbar_fence_init();
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
     tmem_alloc(smem_addr(tmem_slot), S::TMEM_COLS);
     tmem_relinquish();
   }
-  for (int i = tid; i < 2 * S::BQ_BYTES / 16; i += S::THREADS)
+  for (int i = tid; i < S::BQ_BYTES / 16; i += S::THREADS)
     reinterpret_cast<uint4*>(smem + S::BQ_OFF)[i] = make_uint4(0, 0, 0, 0);
   tc_fence_before();
   __syncthreads();
@@ -310,12 +316,11 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
     const uint32_t idesc_o = idesc_f16_f32(kTile, S::NO, 1, 1);
     const uint32_t ak = smem_addr(smem + S::AK_OFF), av = smem_addr(smem + S::AV_OFF);
     const uint32_t bq = smem_addr(smem + S::BQ_OFF), bp = smem_addr(smem + S::BP_OFF);
-    TileIter nx = it;  // one tile ahead, for the scores
-    auto score = [&](int t, int segbuf) {
+    auto score = [&](int t) {
       ws_wait(KREADY(t & 1), (t >> 1) & 1, err);
       if (lane == 0) {
         tc_fence_after();
-        const uint32_t a0 = ak + (t & 1) * S::TILE_AB, b0 = bq + segbuf * S::BQ_BYTES;
+        const uint32_t a0 = ak + (t % S::KST) * S::TILE_AB, b0 = bq;
         // descriptors advance by 256 B (16 channels) per step: +16 in the 16-byte address field
         const uint64_t da = smem_desc(a0, 128, 2048), db = smem_desc(b0, 128, 2048);
 #pragma unroll
@@ -325,17 +330,13 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
           umma_f16(tmem + S::TM_S + (t & 1) * 4 * S::NS + g * S::NS, da + (uint64_t)(ks * 16),
                    db + (uint64_t)((part * S::BQ_HALF + ks * 256) >> 4), idesc_s, (part | s) ? 1u : 0u);
         }
-        umma_commit(SDONE(t & 1));
+        umma_commit(SDONE(t % S::KST));
       }
       __syncwarp();
     };
-    score(0, nx.seg & 1);
-    nx.next(a);
+    score(0);
     for (int t = 0; t < ntiles; ++t) {
-      if (t + 1 < ntiles) {
-        score(t + 1, nx.seg & 1);
-        nx.next(a);
-      }
+      if (t + 1 < ntiles) score(t + 1);
       ws_wait(PREADY(t & 1), (t >> 1) & 1, err);
       ws_wait(VREADY(t & 1), (t >> 1) & 1, err);
       if (lane == 0) {
@@ -358,15 +359,17 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
       const uint8_t* raw = smem + S::RAW_OFF + s * S::RAW_BYTES;
       const size_t bh = it.bh(a);
       const uint32_t msk = it.msk;
+      const int ks = t % S::KST;
       ws_wait(FULL(s), (t / kRing) & 1, err);
-      if (t >= 2) ws_wait(SDONE(k), ((t - 2) >> 1) & 1, err);  // AK[k] read by the score UMMAs of t-2
+      // AK[ks] was read by the score UMMAs of tile t - KST
+      if (t >= S::KST) ws_wait(SDONE(ks), ((t - S::KST) / S::KST) & 1, err);
       if (it.first) {
-        // query operand of the new segment: BQ (hi, lo), per-group sums and q_0
-        if (t >= 2) ws_wait(PREADY(k), ((t - 2) >> 1) & 1, err);  // segment buffer free
-        const int sb = it.seg & 1;
-        uint8_t* BQ = smem + S::BQ_OFF + sb * S::BQ_BYTES;
-        float* qsum = reinterpret_cast<float*>(smem + S::QSUM_OFF) + sb * G * kGroups;
-        float* q0s = reinterpret_cast<float*>(smem + S::Q0_OFF) + sb * G;
+        // query operand of the new segment: BQ (hi, lo), per-group sums and q_0.  The
+        // previous tile's epilogue (and so its score UMMAs) must be done with the old ones.
+        if (t >= 1) ws_wait(PREADY((t - 1) & 1), ((t - 1) >> 1) & 1, err);
+        uint8_t* BQ = smem + S::BQ_OFF;
+        float* qsum = reinterpret_cast<float*>(smem + S::QSUM_OFF);
+        float* q0s = reinterpret_cast<float*>(smem + S::Q0_OFF);
         for (int hq = warp; hq < G; hq += kKWarps) {
           const In* qrow = static_cast<const In*>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.h * G + hq) * kHeadDim;
           float x[4];
@@ -395,7 +398,7 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
       // key codes -> AK[k]: every word is read (rows of dropped groups hold stale
       // codes) and dropped groups are zeroed by a select, so the loads issue
       // back to back with no branches between them
-      uint8_t* AK = smem + S::AK_OFF + k * S::TILE_AB;
+      uint8_t* AK = smem + S::AK_OFF + ks * S::TILE_AB;
 #pragma unroll 1
       for (int hh = 0; hh < 2; ++hh) {
         if (KB == 4) {
@@ -524,7 +527,7 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
     };
 
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
-      const int k = t & 1, sb = it.seg & 1;
+      const int k = t & 1;
       const size_t bh = it.bh(a);
       const uint32_t msk = it.msk;
       const int n0 = it.i * kTile;
@@ -558,13 +561,13 @@ __global__ void __launch_bounds__(WsShape<G, KB, VB, CH0>::THREADS, 1) k_decode_
       if (CH0 && (msk & 1u)) k0v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(sc_st + S::S_K0)[j]);
       mbar_arrive(SEMPTY(ss));
 
-      ok &= ws_wait(SDONE(k), (t >> 1) & 1, err);
+      ok &= ws_wait(SDONE(t % S::KST), (t / S::KST) & 1, err);
       tc_fence_after();
       if (it.first) {
         // the segment's query sums: written by the converters before the score UMMAs of
         // this tile were issued, so visible once those completed
-        const float* qsum = reinterpret_cast<const float*>(smem + S::QSUM_OFF) + sb * G * kGroups;
-        const float* q0s = reinterpret_cast<const float*>(smem + S::Q0_OFF) + sb * G;
+        const float* qsum = reinterpret_cast<const float*>(smem + S::QSUM_OFF);
+        const float* q0s = reinterpret_cast<const float*>(smem + S::Q0_OFF);
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           q0_reg[i] = q0s[part * HH + i];
