@@ -34,7 +34,7 @@ from quantized_attention_kvq_b200 import synth, workloads  # noqa: E402
 
 DEFAULT_WORKLOAD = 1  # GQA INT4 decode, batch 8, 32/8 heads, 32768 cached tokens
 FALLBACK_HBM_GBS = 6650.0
-DECODE_SOURCES = ("decode_simt.cu", "common.cuh")
+DECODE_SOURCES = ("decode.cu", "common.cuh", "sm100.cuh")
 
 
 # ------------------------------------------------------------------ helpers

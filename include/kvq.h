@@ -54,7 +54,7 @@ typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1, KVQ_F16 = 2 } kvq_dtype;
  * N a multiple of 128, every pointer 16-byte aligned.
  *
  * Byte layout (all little-endian; ownership: caller-allocated device memory
- * of the sizes kvq_cache_sizes reports).  Keys are stored in blocks of 128
+ * of the sizes kvq_cache_sizes reports).  Codes are stored in blocks of 128
  * tokens, T = N / 128 blocks per (sequence, head):
  *  k_codes  [B][H][T][d/P][128] words of P*k_bits bits (uint16 for INT4,
  *           uint8 for INT2): inside a block, one row per group of 4 channels
@@ -66,8 +66,15 @@ typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1, KVQ_F16 = 2 } kvq_dtype;
  *  k_ch0    [B][H][N] bf16, channel 0 of the rotated key (only when keep_ch0;
  *           NULL otherwise); code slot 0 of such keys is written as 0 and
  *           channel 0 is outside group 0's range [DQK Sec. 1, Sec. 3.3, App. C.3].
- *  v_codes  [B][H][N][d*v_bits/8] bytes, token-major; channel c at byte
- *           c*v_bits/8, bits ((c mod (8/v_bits))*v_bits ...).
+ *  v_codes  [B][H][T][d][16*v_bits] bytes: inside a block, one row per
+ *           channel holding that channel's 128 codes in token order (token t
+ *           at bits ((t mod (8/v_bits)) * v_bits) of byte t / (8/v_bits) of
+ *           the row).  Each row is cut into 16-byte chunks (32 tokens for
+ *           INT4, 64 for INT2); chunk i of channel c is stored at chunk
+ *           position i XOR s(c), s(c) = (c >> 1) & 3 for INT4 and
+ *           (c >> 2) & 1 for INT2, so that the rows of 8 consecutive
+ *           channels begin in 8 different shared-memory bank groups when a
+ *           block is staged on chip.
  *  v_scales [B][H][N][d/g] x {fp16 scale, fp16 zero}.
  * Dequantized element: x = scale * code + zero [DQK Sec. 3.3, App. B.2; CQ].
  */
@@ -91,8 +98,12 @@ KVQ_API kvq_status kvq_cache_sizes(const kvq_cache* cache, size_t bytes_out[5]);
 
 /*
  * Quantize and append n_new tokens per (sequence, kv head) at token positions
- * [offset, offset + n_new) of the cache; no other token is read or written,
- * so earlier tokens are never re-quantized (incremental cache [TQ]).
+ * [offset, offset + n_new) of the cache; no other token's codes, scales or
+ * zeros change, so earlier tokens are never re-quantized (incremental cache
+ * [TQ]).  Value-code bytes that also hold tokens outside the range are read
+ * and written back with those tokens' bits unchanged, so two appends to the
+ * same sequence whose ranges touch the same 64-token window must not run
+ * concurrently (on different streams without ordering).
  *  k_new, v_new: device [B][H][n_new][d] of `dtype`.
  * Keys: x = H_d k / sqrt(d) when rotate_k (fp64 butterflies in natural
  * Sylvester order, rounded to fp32) [DQK Sec. 1; SIQ KQV; TQ]; channel 0 to
@@ -118,9 +129,6 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new
 KVQ_API kvq_status kvq_select_channels(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
                                        int32_t keep_groups, uint32_t* mask_out, void* stream);
 
-/* Tokens per sequence split that kvq_decode_attention uses for these sizes (> 0), or 0 on bad arguments. */
-KVQ_API int32_t kvq_decode_split_tokens(const kvq_cache* cache, int32_t q_heads, int32_t max_len);
-
 /* Device workspace bytes kvq_decode_attention needs for these sizes (0 on bad arguments). */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_heads, int32_t max_len);
 
@@ -131,9 +139,12 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_head
  *  o = sum_n softmax(s)_n * v_hat_n over n < seq_lens[b],
  * scored directly from the key codes (no dequantized key is written):
  * per group, scale * (q . codes) + zero * sum(q), plus q_rot[0] * k_ch0 when
- * channel 0 is kept.  The sequence is cut into splits; each split keeps a
- * running max and sum, and a combine pass merges them into one softmax
- * over the whole sequence [DQK Sec. 3.4].
+ * channel 0 is kept.  Sequences are cut into 128-token tiles and the tiles
+ * of all (sequence, kv head) pairs are spread evenly over the GPU's SMs, so a
+ * sequence may be split between several of them; each piece keeps a running
+ * max and sum, and a combine pass merges the pieces into one softmax over the
+ * whole sequence [DQK Sec. 3.4].  Supported GQA group sizes
+ * G = q_heads / kv_heads: 1, 2, 4, 8, 16 (others: KVQ_ERR_UNSUPPORTED).
  *  q:        device [B][q_heads][d] of `dtype`, un-rotated.
  *  seq_lens: device int32 [B]; entries are clamped to [0, max_len]; a
  *            sequence of length 0 gets a zero output.
@@ -156,10 +167,10 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* cache, const void* q, k
  * sequence it scored: the piece's running max of the scores in base-2 units
  * (score * log2(e)), its sum of 2^(score - max), and the unnormalized sum of
  * 2^(score - max) * v_hat per channel, for every query head.  How pieces are
- * cut and laid out in the workspace depends on the kernel chosen for the
- * GQA group size and is private to the library: only kvq_decode_combine,
- * called with the same cache, q_heads, seq_lens and max_len and the same
- * workspace, reads it back, and writes `out` [B][q_heads][d].
+ * cut and laid out in the workspace is private to the library: only
+ * kvq_decode_combine, called with the same cache, q_heads, seq_lens and
+ * max_len and the same workspace, reads it back, and writes `out`
+ * [B][q_heads][d].
  * Argument rules and statuses are those of kvq_decode_attention.
  */
 KVQ_API kvq_status kvq_decode_partials(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,

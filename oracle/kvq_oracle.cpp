@@ -96,10 +96,25 @@ inline size_t k_scale_index(const orc_cache* c, int b, int h, int g, int n) {
 inline size_t ch0_index(const orc_cache* c, int b, int h, int n) {
   return bh_index(c, b, h) * (size_t)c->capacity + n;
 }
-// V codes: token-major rows of d*bits/8 bytes; channel ch at byte ch*bits/8,
-// bit (ch mod (8/bits))*bits.
-inline size_t v_row_byte(const orc_cache* c, int b, int h, int n) {
-  return (bh_index(c, b, h) * (size_t)c->capacity + n) * (size_t)(c->head_dim * c->v_bits / 8);
+// V codes: channel-major inside each block of kBlock tokens.  A block holds
+// one row per channel; a row packs the block's kBlock codes of that channel in
+// token order, little-endian (token t at bits ((t mod (8/bits)) * bits) of
+// byte t / (8/bits)), and is split into 16-byte chunks.  Chunk i of channel
+// ch is stored at chunk position i ^ chunk_swizzle(ch), so that the rows of 8
+// consecutive channels touch 8 different 16-byte bank groups.
+inline int v_row_bytes(const orc_cache* c) { return kBlock * c->v_bits / 8; }
+inline int v_chunk_swizzle(const orc_cache* c, int ch) {
+  return c->v_bits == 4 ? (ch >> 1) & 3 : (ch >> 2) & 1;
+}
+// byte holding the code of channel ch, token n of (b, h); *shift = its bit offset
+inline size_t v_code_byte(const orc_cache* c, int b, int h, int ch, int n, int* shift) {
+  const int per_byte = 8 / c->v_bits;
+  const int tokens_per_chunk = 16 * per_byte;
+  const int t = n % kBlock;
+  const int chunk = (t / tokens_per_chunk) ^ v_chunk_swizzle(c, ch);
+  const size_t blk = bh_index(c, b, h) * n_blocks(c) + n / kBlock;
+  *shift = (t % per_byte) * c->v_bits;
+  return (blk * c->head_dim + ch) * (size_t)v_row_bytes(c) + (size_t)chunk * 16 + (t % tokens_per_chunk) / per_byte;
 }
 inline size_t v_scale_index(const orc_cache* c, int b, int h, int n, int g) {
   return (bh_index(c, b, h) * (size_t)c->capacity + n) * (c->head_dim / kGroup) + g;
@@ -249,7 +264,7 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
         for (int i = 0; i < kGranule; ++i) word |= (uint32_t)codes[pg * kGranule + i] << (i * c->k_bits);
         store_k_word(c, b, h, pg, n, word);
       }
-      // ---- values: no rotation, quantize, pack token-major ----
+      // ---- values: no rotation, quantize, pack into the channel rows of the block ----
       for (int i = 0; i < d; ++i) xr[i] = v_new[row + i];
       row_ex = 0;
       for (int g = 0; g < ngroups; ++g) {
@@ -269,11 +284,13 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
         }
       }
       if (v_row_exempt) v_row_exempt[(size_t)bh * n_new + t] = (uint8_t)row_ex;
-      const size_t vb = v_row_byte(c, b, h, n);
-      const int per_byte = 8 / c->v_bits;
-      for (int i = 0; i < d * c->v_bits / 8; ++i) c->v_codes[vb + i] = 0;
-      for (int ch = 0; ch < d; ++ch)
-        c->v_codes[vb + ch / per_byte] |= (uint8_t)(codes[ch] << ((ch % per_byte) * c->v_bits));
+      const uint32_t vmask = (1u << c->v_bits) - 1;
+      for (int ch = 0; ch < d; ++ch) {
+        int sh;
+        const size_t i = v_code_byte(c, b, h, ch, n, &sh);
+        // only this token's bits change; the byte's other tokens keep theirs
+        c->v_codes[i] = (uint8_t)((c->v_codes[i] & ~(vmask << sh)) | ((uint32_t)codes[ch] << sh));
+      }
     }
 #pragma omp critical
     {
@@ -299,11 +316,12 @@ void orc_unpack_codes(const orc_cache* c, int32_t b, int32_t h, int32_t n, int32
       for (int i = 0; i < kGranule; ++i) codes[pg * kGranule + i] = (uint8_t)((w >> (i * c->k_bits)) & mask);
     }
   } else {
-    const size_t vb = v_row_byte(c, b, h, n);
-    const int per_byte = 8 / c->v_bits;
     const uint32_t mask = (1u << c->v_bits) - 1;
-    for (int ch = 0; ch < d; ++ch)
-      codes[ch] = (uint8_t)((c->v_codes[vb + ch / per_byte] >> ((ch % per_byte) * c->v_bits)) & mask);
+    for (int ch = 0; ch < d; ++ch) {
+      int sh;
+      const size_t i = v_code_byte(c, b, h, ch, n, &sh);
+      codes[ch] = (uint8_t)((c->v_codes[i] >> sh) & mask);
+    }
   }
 }
 

@@ -43,7 +43,8 @@ typedef struct {
   uint8_t* k_codes;   /* [B][Hkv][ceil(cap/128)][d/4][128] x (4*k_bits/8) bytes     */
   uint16_t* k_scales; /* [B][Hkv][ceil(cap/128)][d/32][128] x {fp16 scale, fp16 zero} */
   uint16_t* k_ch0;    /* [B][Hkv][cap] bf16, or NULL                        */
-  uint8_t* v_codes;   /* [B][Hkv][cap][d*v_bits/8]                          */
+  uint8_t* v_codes;   /* [B][Hkv][ceil(cap/128)][d][128*v_bits/8]: per block of 128 tokens one
+                         row per channel, 16-byte chunks swizzled by channel        */
   uint16_t* v_scales; /* [B][Hkv][cap][d/32] x {fp16 scale, fp16 zero}      */
 } orc_cache;
 

@@ -121,11 +121,11 @@ class Cache:
     def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0):
         self.B, self.Hkv, self.d, self.capacity = B, Hkv, d, capacity
         self.k_bits, self.v_bits, self.rotate_k, self.keep_ch0 = k_bits, v_bits, rotate_k, keep_ch0
-        blocked = -(-capacity // 128) * 128  # keys are stored in blocks of 128 tokens
+        blocked = -(-capacity // 128) * 128  # codes are stored in blocks of 128 tokens
         self.k_codes = np.zeros(B * Hkv * (d // 4) * blocked * (4 * k_bits // 8), np.uint8)
         self.k_scales = np.zeros(B * Hkv * (d // 32) * blocked * 2, np.uint16)
         self.k_ch0 = np.zeros(B * Hkv * capacity, np.uint16) if keep_ch0 else None
-        self.v_codes = np.zeros(B * Hkv * capacity * (d * v_bits // 8), np.uint8)
+        self.v_codes = np.zeros(B * Hkv * d * blocked * v_bits // 8, np.uint8)  # channel rows per block
         self.v_scales = np.zeros(B * Hkv * capacity * (d // 32) * 2, np.uint16)
         self.struct = OrcCache(B, Hkv, d, capacity, k_bits, v_bits, rotate_k, keep_ch0, _p(self.k_codes),
                                _p(self.k_scales), _p(self.k_ch0), _p(self.v_codes), _p(self.v_scales))

@@ -1,6 +1,6 @@
-// C ABI of libkvq: argument checks, split planning, workspace carving and
-// kernel launches.  Every check happens on the host before anything is
-// enqueued; no exception leaves this file.
+// C ABI of libkvq: argument checks, workspace carving and kernel launches.
+// Every check happens on the host before anything is enqueued; no exception
+// leaves this file.
 #include <cmath>
 #include <cstdint>
 
@@ -9,8 +9,6 @@
 namespace kvq {
 namespace {
 
-constexpr int kSMs = 148;            // B200
-constexpr long kTargetCtas = 8L * kSMs;  // split CTAs aimed at for a full-length batch
 constexpr size_t kAlign = 256;
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -45,8 +43,6 @@ kvq_status check_heads(const kvq_cache* c, int32_t q_heads) {
   return KVQ_OK;
 }
 
-bool decode_g_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
-
 CacheView view(const kvq_cache* c) {
   CacheView v;
   v.B = c->batch;
@@ -66,42 +62,18 @@ CacheView view(const kvq_cache* c) {
 
 double inv_sqrt_d() { return 1.0 / std::sqrt((double)kHeadDim); }
 
-// Tokens per split: a multiple of the 128-token tile chosen so that a batch
-// of full-length sequences yields about kTargetCtas split CTAs.
-int32_t plan_split_tokens(int B, int H, int max_len) {
-  if (max_len <= kDecodeTile) return kDecodeTile;
-  const long units = (long)B * H;
-  const long splits = (kTargetCtas + units - 1) / units;
-  long s = (max_len + splits - 1) / splits;
-  s = (long)round_up((size_t)s, kDecodeTile);
-  if (s < 2 * kDecodeTile) s = 2 * kDecodeTile;
-  return (int32_t)s;
-}
-
-// Decode kernels: the persistent warp-specialized tensor-core kernel for GQA
-// groups of 4 or 8 query heads, the per-split tensor-core kernel for 16, the
-// CUDA-core kernel for 1 or 2.
-enum DecodePath { kPathSimt = 0, kPathTc = 1, kPathWs = 2 };
-
+// Workspace of the decode: one partial row (128-channel accumulator, running
+// max and sum) per (slot, query head of the GQA group), decode_slots slots.
 struct DecodePlan {
-  int path;
-  int32_t split_tokens, max_splits;
   size_t acc_bytes, ml_offset, bytes;
 };
 
-DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
+DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   DecodePlan p;
-  const int g = q_heads / c->kv_heads;
-  p.path = decode_ws_supported(g) ? kPathWs : (decode_tc_supported(g) ? kPathTc : kPathSimt);
-  p.split_tokens = plan_split_tokens(c->batch, c->kv_heads, max_len);
-  p.max_splits = (max_len + p.split_tokens - 1) / p.split_tokens;
-  // partial rows: per (sequence, query head, split), or per (slot, query head of the group)
-  const size_t units = p.path == kPathWs ? (size_t)decode_ws_slots(c->batch, c->kv_heads) * g
-                                         : (size_t)c->batch * q_heads * (size_t)p.max_splits;
-  p.acc_bytes = units * kHeadDim * sizeof(float);
+  const size_t rows = (size_t)decode_slots(c->batch, c->kv_heads) * (q_heads / c->kv_heads);
+  p.acc_bytes = rows * kHeadDim * sizeof(float);
   p.ml_offset = round_up(p.acc_bytes, kAlign);
-  p.bytes = p.ml_offset + round_up(units * sizeof(float2), kAlign);
-  if (p.bytes == 0) p.bytes = kAlign;
+  p.bytes = p.ml_offset + round_up(rows * sizeof(float2), kAlign);
   return p;
 }
 
@@ -124,19 +96,14 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.mask = mask;
   a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);  // log2(e)
   a.inv_sqrt_d = inv_sqrt_d();
-  a.split_tokens = plan.split_tokens;
-  a.max_splits = plan.max_splits;
   a.part_acc = static_cast<float*>(workspace);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
-  if ((parts & kRunSplit) && plan.max_splits > 0) {
-    cudaError_t e = plan.path == kPathWs   ? launch_decode_split_ws(a, s)
-                    : plan.path == kPathTc ? launch_decode_split_tc(a, s)
-                                           : launch_decode_split(a, s);
-    kvq_status st = cuda_status(e);
+  if ((parts & kRunSplit) && max_len > 0) {
+    kvq_status st = cuda_status(launch_decode(a, s));
     if (st != KVQ_OK) return st;
   }
-  if (parts & kRunCombine) return cuda_status(plan.path == kPathWs ? launch_combine_ws(a, s) : launch_combine(a, s));
+  if (parts & kRunCombine) return cuda_status(launch_combine(a, s));
   return KVQ_OK;
 }
 
@@ -153,7 +120,7 @@ kvq_status check_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, int3
   if (max_len < 0) return KVQ_ERR_INVALID_ARG;
   if (max_len > c->capacity) return KVQ_ERR_CAPACITY;
   if (!decode_g_supported(q_heads / c->kv_heads)) return KVQ_ERR_UNSUPPORTED;
-  if (workspace_bytes < plan_decode(c, q_heads, max_len).bytes) return KVQ_ERR_WORKSPACE;
+  if (workspace_bytes < plan_decode(c, q_heads).bytes) return KVQ_ERR_WORKSPACE;
   return KVQ_OK;
 }
 
@@ -166,7 +133,7 @@ kvq_status decode_into(const kvq_cache* c, const void* q, kvq_dtype dtype, int32
                                workspace_bytes, true);
   if (st != KVQ_OK) return st;
   return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, out, workspace,
-                        plan_decode(c, q_heads, max_len), s);
+                        plan_decode(c, q_heads), s);
 }
 
 }  // namespace kvq
@@ -228,16 +195,10 @@ KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dt
   return cuda_status(launch_select(a, static_cast<cudaStream_t>(stream)));
 }
 
-KVQ_API int32_t kvq_decode_split_tokens(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
-  if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK) return 0;
-  if (max_len < 0 || max_len > c->capacity) return 0;
-  return plan_split_tokens(c->batch, c->kv_heads, max_len);
-}
-
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
   if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK) return 0;
   if (max_len < 0 || max_len > c->capacity) return 0;
-  return plan_decode(c, q_heads, max_len).bytes;
+  return plan_decode(c, q_heads).bytes;
 }
 
 KVQ_API kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
@@ -248,7 +209,7 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_d
                                workspace_bytes, true);
   if (st != KVQ_OK) return st;
   return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, out, workspace,
-                        plan_decode(c, q_heads, max_len), static_cast<cudaStream_t>(stream));
+                        plan_decode(c, q_heads), static_cast<cudaStream_t>(stream));
 }
 
 KVQ_API kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
@@ -258,7 +219,7 @@ KVQ_API kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dt
                                workspace_bytes, true);
   if (st != KVQ_OK) return st;
   return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, nullptr, workspace,
-                        plan_decode(c, q_heads, max_len), static_cast<cudaStream_t>(stream), kRunSplit);
+                        plan_decode(c, q_heads), static_cast<cudaStream_t>(stream), kRunSplit);
 }
 
 KVQ_API kvq_status kvq_decode_combine(const kvq_cache* c, int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
@@ -267,7 +228,7 @@ KVQ_API kvq_status kvq_decode_combine(const kvq_cache* c, int32_t q_heads, const
                                workspace_bytes, false);
   if (st != KVQ_OK) return st;
   return enqueue_decode(c, nullptr, KVQ_F32, q_heads, seq_lens, max_len, nullptr, 1.0f, out,
-                        const_cast<void*>(workspace), plan_decode(c, q_heads, max_len),
+                        const_cast<void*>(workspace), plan_decode(c, q_heads),
                         static_cast<cudaStream_t>(stream), kRunCombine);
 }
 
@@ -278,7 +239,7 @@ KVQ_API size_t kvq_decode_step_workspace_bytes(const kvq_cache* c, kvq_dtype dty
   const size_t qb = (size_t)c->batch * q_heads * kHeadDim * dtype_size(dtype);
   const size_t mb = (size_t)c->batch * c->kv_heads * sizeof(uint32_t);
   const size_t ob = (size_t)c->batch * q_heads * kHeadDim * sizeof(float);
-  return round_up(qb, kAlign) + round_up(mb, kAlign) + round_up(ob, kAlign) + plan_decode(c, q_heads, max_len).bytes;
+  return round_up(qb, kAlign) + round_up(mb, kAlign) + round_up(ob, kAlign) + plan_decode(c, q_heads).bytes;
 }
 
 KVQ_API kvq_status kvq_decode_step_host(const kvq_cache* c, const void* q_host, kvq_dtype dtype, int32_t q_heads,
@@ -311,7 +272,7 @@ KVQ_API kvq_status kvq_decode_step_host(const kvq_cache* c, const void* q_host, 
     if (st != KVQ_OK) return st;
     mask = mask_dev;
   }
-  const DecodePlan plan = plan_decode(c, q_heads, max_len);
+  const DecodePlan plan = plan_decode(c, q_heads);
   st = enqueue_decode(c, q_dev, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, out_dev, dec_ws, plan, s);
   if (st != KVQ_OK) return st;
   return cuda_status(cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, s));

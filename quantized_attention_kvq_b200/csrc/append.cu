@@ -1,21 +1,24 @@
 // Fused rotate + quantize + pack + append kernel.
 //
-// One CTA handles a tile of 64 new tokens of one (sequence, kv head); each of
-// its 8 warps takes every 8th token, one 128-channel row at a time with lane
-// l owning channels 4l..4l+3 (= pruning group l).  Keys: fp64 Walsh-Hadamard
-// butterflies (Dual-QK summary Sec. 1; gist.science KQV scheme), optional
-// bf16 channel 0 (Dual-QK Sec. 3.3, App. C.3), per-32-channel asymmetric
-// quantization (Dual-QK Sec. 3.3).  Values: the same quantizer without
-// rotation (Dual-QK App. B.2).  Key code words are staged in shared memory and
-// written channel-major so every row store is coalesced; value rows and their
-// scales go straight out token-major.  Only tokens [offset, offset+n_new) are
-// touched (tq-kv incremental cache).
+// One CTA handles the new tokens of one (sequence, kv head) that fall in one
+// 64-token-aligned window of the cache; each of its 8 warps takes every 8th
+// token, one 128-channel row at a time with lane l owning channels 4l..4l+3
+// (= pruning group l).  Keys: fp64 Walsh-Hadamard butterflies (Dual-QK
+// summary Sec. 1; gist.science KQV scheme), optional bf16 channel 0 (Dual-QK
+// Sec. 3.3, App. C.3), per-32-channel asymmetric quantization (Dual-QK
+// Sec. 3.3).  Values: the same quantizer without rotation (Dual-QK App. B.2).
+// Both code kinds are staged in shared memory and leave channel-major: key
+// words one coalesced row per pruning group, value codes packed into each
+// channel's row of the 128-token block.  Only tokens [offset, offset+n_new)
+// change (tq-kv incremental cache); value-code words that also hold tokens
+// outside that range are read, patched and written back by the one CTA whose
+// window contains them.
 #include "common.cuh"
 
 namespace kvq {
 namespace {
 
-constexpr int kAppendTile = 64;
+constexpr int kAppendTile = 64;  // tokens per CTA window, aligned to absolute token positions
 constexpr int kAppendWarps = 8;
 
 // Quantize the 4 channels this lane holds; the 8 lanes of a group agree on
@@ -59,35 +62,45 @@ __device__ __forceinline__ uint32_t quantize_lane(const float x[4], bool skip0, 
 
 template <int KB, int VB, bool ROT, bool CH0, typename In>
 __global__ void __launch_bounds__(kAppendWarps * 32) k_quantize_append(AppendArgs a) {
+  constexpr int TPW = 32 / VB;                  // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
+  constexpr int WPR = kAppendTile / TPW;        // value words per channel in the window: 8 or 4
   __shared__ uint16_t kw[kPruneGroups][kAppendTile + 2];
   __shared__ __half2 ksz[kGroups][kAppendTile];
   __shared__ __nv_bfloat16 k0s[kAppendTile];
+  __shared__ __align__(16) uint8_t vcode[kAppendTile][kHeadDim];  // [token][channel] value codes
+  __shared__ uint32_t vword[kHeadDim][WPR + 1];                   // packed value words, padded rows
 
   const CacheView& c = a.c;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int t0 = blockIdx.x * kAppendTile;
-  const int ntok = min(kAppendTile, a.n_new - t0);
+  const int w0 = (a.offset / kAppendTile + blockIdx.x) * kAppendTile;  // absolute first token of the window
+  const int lo = max(a.offset - w0, 0);                                // window tokens [lo, hi) are new
+  const int hi = min(a.offset + a.n_new - w0, kAppendTile);
   const size_t bh = (size_t)b * c.H + h;
-  const In* kin = static_cast<const In*>(a.k_new) + (bh * a.n_new + t0) * kHeadDim;
-  const In* vin = static_cast<const In*>(a.v_new) + (bh * a.n_new + t0) * kHeadDim;
+  // input row of window token tt: (bh * n_new + w0 + tt - offset), never negative for tt >= lo
+  const size_t row0 = bh * a.n_new + (w0 + lo - a.offset);
+  const In* kin = static_cast<const In*>(a.k_new) + (row0 - lo) * kHeadDim;
+  const In* vin = static_cast<const In*>(a.v_new) + (row0 - lo) * kHeadDim;
 
   // one-deep prefetch of the next row pair
   float kx[4], vx[4], kn[4], vn[4];
-  int tt = warp;
-  if (tt < ntok) {
+  int tt = lo + warp;
+  if (tt < hi) {
     load4(kin + (size_t)tt * kHeadDim + 4 * lane, kn);
     load4(vin + (size_t)tt * kHeadDim + 4 * lane, vn);
   }
-  for (; tt < ntok; tt += kAppendWarps) {
+  for (; tt < hi; tt += kAppendWarps) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) { kx[i] = kn[i]; vx[i] = vn[i]; }
+    for (int i = 0; i < 4; ++i) {
+      kx[i] = kn[i];
+      vx[i] = vn[i];
+    }
     const int nx = tt + kAppendWarps;
-    if (nx < ntok) {
+    if (nx < hi) {
       load4(kin + (size_t)nx * kHeadDim + 4 * lane, kn);
       load4(vin + (size_t)nx * kHeadDim + 4 * lane, vn);
     }
-    const size_t n = (size_t)a.offset + t0 + tt;
+    const size_t n = (size_t)w0 + tt;
 
     // ---- key row
     if (ROT) rotate_row_warp(kx, a.inv_sqrt_d, lane);
@@ -97,38 +110,72 @@ __global__ void __launch_bounds__(kAppendWarps * 32) k_quantize_append(AppendArg
     kw[lane][tt] = (uint16_t)kword;
     if ((lane & 7) == 0) ksz[lane >> 3][tt] = sz;
 
-    // ---- value row: token-major, written directly (coalesced 32/64 bytes)
-    const uint32_t vword = quantize_lane<VB>(vx, false, sz);
-    uint8_t* vrow = c.vc + (bh * c.cap + n) * (kHeadDim * VB / 8);
-    if (VB == 4)
-      reinterpret_cast<uint16_t*>(vrow)[lane] = (uint16_t)vword;
-    else
-      vrow[lane] = (uint8_t)vword;
+    // ---- value row: codes of channels 4l..4l+3 as bytes; scales token-major, written directly
+    const uint32_t vw = quantize_lane<VB>(vx, false, sz);
+    constexpr uint32_t L = (1u << VB) - 1;
+    *reinterpret_cast<uint32_t*>(&vcode[tt][4 * lane]) =
+        (vw & L) | (((vw >> VB) & L) << 8) | (((vw >> (2 * VB)) & L) << 16) | (((vw >> (3 * VB)) & L) << 24);
     if ((lane & 7) == 0) c.vs[(bh * c.cap + n) * kGroups + (lane >> 3)] = sz;
   }
   __syncthreads();
 
   // ---- key rows out: channel-major, one coalesced run per pruning group
-  const size_t n0 = (size_t)a.offset + t0;
+  const int ntok = hi - lo;
   for (int i = threadIdx.x; i < kPruneGroups * ntok; i += blockDim.x) {
-    const int pg = i / ntok, t = i - pg * ntok;
-    const size_t idx = key_word_index(bh, c.cap, pg, (int)n0 + t);
+    const int pg = i / ntok, t = lo + i % ntok;
+    const size_t idx = key_word_index(bh, c.cap, pg, w0 + t);
     if (KB == 4)
       reinterpret_cast<uint16_t*>(c.kc)[idx] = kw[pg][t];
     else
       c.kc[idx] = (uint8_t)kw[pg][t];
   }
   for (int i = threadIdx.x; i < kGroups * ntok; i += blockDim.x) {
-    const int g = i / ntok, t = i - g * ntok;
-    c.ks[key_scale_index(bh, c.cap, g, (int)n0 + t)] = ksz[g][t];
+    const int g = i / ntok, t = lo + i % ntok;
+    c.ks[key_scale_index(bh, c.cap, g, w0 + t)] = ksz[g][t];
   }
   if (CH0)
-    for (int t = threadIdx.x; t < ntok; t += blockDim.x) c.k0[bh * c.cap + n0 + t] = k0s[t];
+    for (int t = lo + threadIdx.x; t < hi; t += blockDim.x) c.k0[bh * c.cap + w0 + t] = k0s[t];
+
+  // ---- value codes: pack each channel's window into words (token order, low bits first)
+  for (int i = threadIdx.x; i < kHeadDim * WPR; i += blockDim.x) {
+    const int ch = i % kHeadDim, w = i / kHeadDim;  // a warp: 32 channels of one word position
+    uint32_t word = 0;
+#pragma unroll
+    for (int k = 0; k < TPW; ++k) {
+      const int t = w * TPW + k;
+      const uint32_t code = (t >= lo && t < hi) ? vcode[t][ch] : 0u;
+      word |= code << (VB * k);
+    }
+    vword[ch][w] = word;
+  }
+  __syncthreads();
+  // ...and store them into the channel rows of the 128-token block
+  const int blk = w0 / kKeyBlock;
+  const int tb0 = w0 % kKeyBlock;               // window start inside the block: 0 or 64
+  constexpr int TPC = 16 * 8 / VB;              // tokens per 16-byte chunk: 32 or 64
+  for (int i = threadIdx.x; i < kHeadDim * WPR; i += blockDim.x) {
+    const int ch = i / WPR, w = i % WPR;        // a warp: 32 / WPR channels, all their words
+    const int t0 = w * TPW;                     // first window token of the word
+    const int tb = tb0 + t0;                    // ... inside the block
+    const int chunk = (tb / TPC) ^ v_chunk_swizzle(VB, ch);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(c.vc + v_row_offset(bh, c.cap, blk, ch, VB) + chunk * 16 +
+                                                (tb % TPC) / (8 / VB));
+    const int a0 = max(lo - t0, 0), a1 = min(hi - t0, TPW);  // new tokens of this word: [a0, a1)
+    if (a0 >= a1) continue;
+    uint32_t word = vword[ch][w];
+    if (a0 > 0 || a1 < TPW) {
+      const uint32_t keep_lo = a0 * VB >= 32 ? ~0u : ((1u << (a0 * VB)) - 1u);
+      const uint32_t keep_hi = a1 * VB >= 32 ? 0u : ~((1u << (a1 * VB)) - 1u);
+      word |= *dst & (keep_lo | keep_hi);  // the other tokens' codes stay as they were
+    }
+    *dst = word;
+  }
 }
 
 template <int KB, int VB, bool ROT, bool CH0>
 cudaError_t launch_typed(const AppendArgs& a, cudaStream_t s) {
-  dim3 grid((a.n_new + kAppendTile - 1) / kAppendTile, a.c.H, a.c.B);
+  const int first = a.offset / kAppendTile, last = (a.offset + a.n_new - 1) / kAppendTile;
+  dim3 grid(last - first + 1, a.c.H, a.c.B);
   dim3 block(kAppendWarps * 32);
   switch (a.dtype) {
     case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, float><<<grid, block, 0, s>>>(a); break;

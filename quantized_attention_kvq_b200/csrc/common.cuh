@@ -15,7 +15,6 @@ constexpr int kGroup = 32;         // channels per quantization group
 constexpr int kGroups = kHeadDim / kGroup;      // 4
 constexpr int kGranule = 4;        // channels per pruning group
 constexpr int kPruneGroups = kHeadDim / kGranule;  // 32
-constexpr int kDecodeTile = 128;   // tokens per decode tile; split lengths are multiples of it
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---------------------------------------------------------------- loads
@@ -88,10 +87,11 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// ---------------------------------------------------------------- key layout
+// ---------------------------------------------------------------- cache layout
 // Keys are stored in blocks of kKeyBlock tokens; inside a block, one row of
 // kKeyBlock code words per channel group of 4, then (separately) one row of
-// kKeyBlock (scale, zero) pairs per 32-channel group.
+// kKeyBlock (scale, zero) pairs per 32-channel group.  Value codes use the
+// same blocks with one row per channel (see v_code_byte).
 constexpr int kKeyBlock = 128;
 // index of the code word of (unit bh, channel group pg, token n)
 __host__ __device__ __forceinline__ size_t key_word_index(size_t bh, int cap, int pg, int n) {
@@ -100,6 +100,19 @@ __host__ __device__ __forceinline__ size_t key_word_index(size_t bh, int cap, in
 // index of the (scale, zero) pair of (unit bh, 32-channel group g, token n)
 __host__ __device__ __forceinline__ size_t key_scale_index(size_t bh, int cap, int g, int n) {
   return (((bh * (size_t)(cap / kKeyBlock) + n / kKeyBlock) * kGroups + g) * kKeyBlock) + n % kKeyBlock;
+}
+
+// Value codes: per block of kKeyBlock tokens, one row per channel holding the
+// block's codes in token order (little-endian inside a byte), cut into
+// 16-byte chunks; chunk i of channel ch sits at chunk position
+// i ^ v_chunk_swizzle(ch), so 8 consecutive channels' rows start in 8
+// different shared-memory bank groups.
+__host__ __device__ __forceinline__ int v_chunk_swizzle(int v_bits, int ch) {
+  return v_bits == 4 ? (ch >> 1) & 3 : (ch >> 2) & 1;
+}
+// byte offset of the row of (unit bh, block blk, channel ch)
+__host__ __device__ __forceinline__ size_t v_row_offset(size_t bh, int cap, int blk, int ch, int v_bits) {
+  return ((bh * (size_t)(cap / kKeyBlock) + blk) * kHeadDim + ch) * (size_t)(kKeyBlock * v_bits / 8);
 }
 
 // ---------------------------------------------------------------- launch plumbing
@@ -136,25 +149,19 @@ struct DecodeArgs {
   const uint32_t* mask;
   float scale_log2;  // softmax_scale * log2(e): scores live in the exp2 domain
   double inv_sqrt_d;
-  int split_tokens, max_splits;
-  float* part_acc;  // [B][Hq][max_splits][128]
-  float2* part_ml;  // [B][Hq][max_splits] (running max, running sum)
+  float* part_acc;  // [decode_slots][G][128] unnormalized accumulators
+  float2* part_ml;  // [decode_slots][G] (running max, running sum)
   float* out;       // [B][Hq][128]
 };
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
-cudaError_t launch_decode_split(const DecodeArgs& a, cudaStream_t s);
+// persistent tensor-core split decode (GQA groups of 1, 2, 4, 8 or 16 query
+// heads) and its combine; partial slots: one per (unit + CTA), decode_slots of them
+bool decode_g_supported(int g);
+int decode_slots(int B, int H);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
-// tensor-core split decode: GQA groups of 4, 8 or 16 query heads
-bool decode_tc_supported(int g);
-cudaError_t launch_decode_split_tc(const DecodeArgs& a, cudaStream_t s);
-// persistent warp-specialized tensor-core decode (GQA groups of 4 or 8) and
-// its combine; partial slots: one per (unit + CTA), decode_ws_slots of them
-bool decode_ws_supported(int g);
-int decode_ws_slots(int B, int H);
-cudaError_t launch_decode_split_ws(const DecodeArgs& a, cudaStream_t s);
-cudaError_t launch_combine_ws(const DecodeArgs& a, cudaStream_t s);
 
 // Checked split decode + combine into a caller-chosen scratch buffer of
 // `workspace_bytes` bytes (the body of kvq_decode_attention).

@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a features the tensor-core decode
 // uses: mbarriers, 1-D bulk async copies (TMA), tcgen05 tensor-memory
-// allocation, UMMA issue/commit and tensor-memory loads.  Each wrapper is one
+// allocation, UMMA issue/commit and tensor-memory loads and stores.  Each wrapper is one
 // PTX instruction (or a bounded loop around one).
 #pragma once
 
@@ -26,6 +26,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Non-blocking: whether phase `parity` of the barrier has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -111,6 +123,33 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
+// D[tmem] (+)= A[tmem] * B[smem]^T, issued by one thread.  A sits in tensor
+// memory: row m of A in lane m, its K elements packed two per 32-bit column.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+// Instruction descriptor for kind::i8: unsigned 8-bit A, signed 8-bit B, s32 accumulation, both K-major.
+__host__ __device__ constexpr uint32_t idesc_u8s8_s32(int M, int N) {
+  return (2u << 4)                        // D format: s32
+         | (0u << 7) | (1u << 10)         // A: unsigned 8-bit, B: signed 8-bit
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T on 8-bit integers (K = 32 per instruction), issued by one thread.
+__device__ __forceinline__ void umma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
 // Arrive once on `bar` when every UMMA this thread issued so far has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -137,7 +176,216 @@ __device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, uint32_t (&r)[8]) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                : "r"(taddr));
 }
+template <>
+__device__ __forceinline__ void tmem_ld<1>(uint32_t taddr, uint32_t (&r)[1]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Loads that complete inside the same asm statement: the destination
+// registers of tcgen05.ld are only defined after tcgen05.wait::ld, so the
+// wait is issued before the compiler may touch them.
+// N consecutive columns at taddr.
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[N]);
+template <>
+__device__ __forceinline__ void tmem_ld_wait<1>(uint32_t taddr, uint32_t (&r)[1]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0])
+      : "r"(taddr)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_wait<2>(uint32_t taddr, uint32_t (&r)[2]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1])
+      : "r"(taddr)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_wait<4>(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+      : "r"(taddr)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_wait<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+// Four runs of N columns at taddr + k * stride (k = 0..3), one wait for all.
+template <int N>
+__device__ __forceinline__ void tmem_ld4_wait(uint32_t taddr, uint32_t stride, uint32_t (&r)[4][N]);
+template <>
+__device__ __forceinline__ void tmem_ld4_wait<1>(uint32_t taddr, uint32_t stride, uint32_t (&r)[4][1]) {
+  asm volatile(
+      "{\n\t.reg .b32 a;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%4];\n\t"
+      "add.u32 a, %4, %5;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%1}, [a];\n\t"
+      "add.u32 a, a, %5;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%2}, [a];\n\t"
+      "add.u32 a, a, %5;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%3}, [a];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0][0]), "=r"(r[1][0]), "=r"(r[2][0]), "=r"(r[3][0])
+      : "r"(taddr), "r"(stride)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld4_wait<2>(uint32_t taddr, uint32_t stride, uint32_t (&r)[4][2]) {
+  asm volatile(
+      "{\n\t.reg .b32 a;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%8];\n\t"
+      "add.u32 a, %8, %9;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%2, %3}, [a];\n\t"
+      "add.u32 a, a, %9;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%4, %5}, [a];\n\t"
+      "add.u32 a, a, %9;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%6, %7}, [a];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[3][0]),
+        "=r"(r[3][1])
+      : "r"(taddr), "r"(stride)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld4_wait<4>(uint32_t taddr, uint32_t stride, uint32_t (&r)[4][4]) {
+  asm volatile(
+      "{\n\t.reg .b32 a;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%16];\n\t"
+      "add.u32 a, %16, %17;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [a];\n\t"
+      "add.u32 a, a, %17;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [a];\n\t"
+      "add.u32 a, a, %17;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%12, %13, %14, %15}, [a];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]),
+        "=r"(r[1][3]), "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[2][2]), "=r"(r[2][3]), "=r"(r[3][0]), "=r"(r[3][1]),
+        "=r"(r[3][2]), "=r"(r[3][3])
+      : "r"(taddr), "r"(stride)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld4_wait<8>(uint32_t taddr, uint32_t stride, uint32_t (&r)[4][8]) {
+  asm volatile(
+      "{\n\t.reg .b32 a;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%32];\n\t"
+      "add.u32 a, %32, %33;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [a];\n\t"
+      "add.u32 a, a, %33;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16, %17, %18, %19, %20, %21, %22, %23}, [a];\n\t"
+      "add.u32 a, a, %33;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%24, %25, %26, %27, %28, %29, %30, %31}, [a];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[0][4]), "=r"(r[0][5]), "=r"(r[0][6]),
+        "=r"(r[0][7]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]), "=r"(r[1][3]), "=r"(r[1][4]), "=r"(r[1][5]),
+        "=r"(r[1][6]), "=r"(r[1][7]), "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[2][2]), "=r"(r[2][3]), "=r"(r[2][4]),
+        "=r"(r[2][5]), "=r"(r[2][6]), "=r"(r[2][7]), "=r"(r[3][0]), "=r"(r[3][1]), "=r"(r[3][2]), "=r"(r[3][3]),
+        "=r"(r[3][4]), "=r"(r[3][5]), "=r"(r[3][6]), "=r"(r[3][7])
+      : "r"(taddr), "r"(stride)
+      : "memory");
+}
+
+// Two sets of four runs of N columns (at taddr + k * stride and taddr + off2 +
+// k * stride, k = 0..3), one wait for all eight loads.
+template <int N>
+__device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, uint32_t stride, uint32_t off2, uint32_t (&r)[4][N],
+                                              uint32_t (&q)[4][N]);
+template <>
+__device__ __forceinline__ void tmem_ld8_wait<2>(uint32_t taddr, uint32_t stride, uint32_t off2, uint32_t (&r)[4][2],
+                                                 uint32_t (&q)[4][2]) {
+  asm volatile(
+      "{\n\t.reg .b32 a, b;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%16];\n\t"
+      "add.u32 b, %16, %18;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%8, %9}, [b];\n\t"
+      "add.u32 a, %16, %17;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%2, %3}, [a];\n\t"
+      "add.u32 b, a, %18;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%10, %11}, [b];\n\t"
+      "add.u32 a, a, %17;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%4, %5}, [a];\n\t"
+      "add.u32 b, a, %18;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%12, %13}, [b];\n\t"
+      "add.u32 a, a, %17;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%6, %7}, [a];\n\t"
+      "add.u32 b, a, %18;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%14, %15}, [b];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[3][0]),
+        "=r"(r[3][1]), "=r"(q[0][0]), "=r"(q[0][1]), "=r"(q[1][0]), "=r"(q[1][1]), "=r"(q[2][0]), "=r"(q[2][1]),
+        "=r"(q[3][0]), "=r"(q[3][1])
+      : "r"(taddr), "r"(stride), "r"(off2)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld8_wait<4>(uint32_t taddr, uint32_t stride, uint32_t off2, uint32_t (&r)[4][4],
+                                                 uint32_t (&q)[4][4]) {
+  asm volatile(
+      "{\n\t.reg .b32 a, b;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%32];\n\t"
+      "add.u32 b, %32, %34;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%16, %17, %18, %19}, [b];\n\t"
+      "add.u32 a, %32, %33;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [a];\n\t"
+      "add.u32 b, a, %34;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%20, %21, %22, %23}, [b];\n\t"
+      "add.u32 a, a, %33;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [a];\n\t"
+      "add.u32 b, a, %34;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%24, %25, %26, %27}, [b];\n\t"
+      "add.u32 a, a, %33;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%12, %13, %14, %15}, [a];\n\t"
+      "add.u32 b, a, %34;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%28, %29, %30, %31}, [b];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]),
+        "=r"(r[1][3]), "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[2][2]), "=r"(r[2][3]), "=r"(r[3][0]), "=r"(r[3][1]),
+        "=r"(r[3][2]), "=r"(r[3][3]), "=r"(q[0][0]), "=r"(q[0][1]), "=r"(q[0][2]), "=r"(q[0][3]), "=r"(q[1][0]),
+        "=r"(q[1][1]), "=r"(q[1][2]), "=r"(q[1][3]), "=r"(q[2][0]), "=r"(q[2][1]), "=r"(q[2][2]), "=r"(q[2][3]),
+        "=r"(q[3][0]), "=r"(q[3][1]), "=r"(q[3][2]), "=r"(q[3][3])
+      : "r"(taddr), "r"(stride), "r"(off2)
+      : "memory");
+}
+
+// Each thread of the warp writes N consecutive 32-bit columns of its own lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+// The calling thread's earlier tcgen05.st have completed.
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- code -> f16
 // Eight 4-bit codes n0..n7 (n_i in bits 4i..4i+3 of x) -> exact f16 integers,

@@ -18,8 +18,7 @@ KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORK
 KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 
 # every exported symbol the header declares
-SYMBOLS = ("kvq_cache_sizes", "kvq_quantize_append", "kvq_select_channels", "kvq_decode_split_tokens",
-           "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
+SYMBOLS = ("kvq_cache_sizes", "kvq_quantize_append", "kvq_select_channels", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
            "kvq_decode_step_workspace_bytes",
            "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_status_string")
 
@@ -56,8 +55,6 @@ def lib():
         L.kvq_quantize_append.restype = ctypes.c_int
         L.kvq_select_channels.argtypes = [C, _P, ctypes.c_int, _I32, _I32, _P, _P]
         L.kvq_select_channels.restype = ctypes.c_int
-        L.kvq_decode_split_tokens.argtypes = [C, _I32, _I32]
-        L.kvq_decode_split_tokens.restype = _I32
         L.kvq_decode_workspace_bytes.argtypes = [C, _I32, _I32]
         L.kvq_decode_workspace_bytes.restype = ctypes.c_size_t
         L.kvq_decode_attention.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _P, ctypes.c_float, _P, _P,
@@ -181,8 +178,6 @@ class KVQCache:
     def workspace_bytes(self, q_heads: int, max_len: int) -> int:
         return lib().kvq_decode_workspace_bytes(ctypes.byref(self.desc), q_heads, max_len)
 
-    def split_tokens(self, q_heads: int, max_len: int) -> int:
-        return lib().kvq_decode_split_tokens(ctypes.byref(self.desc), q_heads, max_len)
 
     def decode(self, q: torch.Tensor, seq_lens: torch.Tensor, max_len: int, mask: torch.Tensor | None = None,
                softmax_scale: float | None = None, out: torch.Tensor | None = None,

@@ -132,17 +132,17 @@ def test_decode_step_host_argument_checks(L):
     assert rc == native.KVQ_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("B,H,max_len", [(8, 8, 32768), (4, 8, 131072), (64, 8, 16384), (1, 1, 1024),
-                                         (16, 8, 12288), (2, 2, 100), (1, 1, 0), (3, 7, 4096)])
-def test_split_plan_covers_sequence(L, B, H, max_len):
+@pytest.mark.parametrize("B,H,G,max_len", [(8, 8, 4, 32768), (4, 8, 4, 131072), (64, 8, 8, 16384), (1, 1, 1, 1024),
+                                           (16, 8, 2, 12288), (2, 2, 16, 100), (1, 1, 1, 0), (3, 7, 8, 4096)])
+def test_decode_workspace_holds_one_partial_per_slot_and_head(L, B, H, G, max_len):
+    # the decode spreads all tiles over 148 persistent CTAs; a (sequence, kv head)
+    # unit leaves at most one partial per CTA its tiles touch, and consecutive
+    # units share at most one CTA, so B*H + 148 slots of G partial rows suffice
     d = native.describe(B, H, max(128, (max_len + 127) // 128 * 128), 4, 4)
-    S = L.kvq_decode_split_tokens(ctypes.byref(d), H, max_len)
-    assert S > 0 and S % 128 == 0
-    splits = (max_len + S - 1) // S
-    ws = L.kvq_decode_workspace_bytes(ctypes.byref(d), H * 2, max_len)
-    assert ws >= B * H * 2 * splits * (128 * 4 + 8)
-    if max_len >= 4096 and B * H <= 1184:
-        assert B * H * splits >= 148  # enough split CTAs to cover every SM
+    ws = L.kvq_decode_workspace_bytes(ctypes.byref(d), H * G, max_len)
+    rows = (B * H + 148) * G
+    assert ws >= rows * (128 * 4 + 8)
+    assert ws <= rows * (128 * 4 + 8) + 512  # two 256-byte aligned regions
 
 
 def test_status_strings(L):

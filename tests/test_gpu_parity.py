@@ -134,7 +134,9 @@ def test_decode_matches_oracle(case):
         ref_mask, _ = orc.select(host_f32(q, fmt), H, rot, keep)
         np.testing.assert_array_equal(mask_u32(mask_d), ref_mask)
     out = gc.decode(qd, lens_d, T, mask_d, softmax_scale())
+    again = gc.decode(qd, lens_d, T, mask_d, softmax_scale())
     torch.cuda.synchronize()
+    assert torch.equal(out, again), "two identical decode calls differ"
     o_ref = oc.attention(host_f32(q, fmt), lens_np, ref_mask, softmax_scale())
     o_gpu = out.cpu().numpy().reshape(-1, 128)
     for b in range(B):

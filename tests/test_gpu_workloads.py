@@ -12,6 +12,7 @@ import pytest
 import torch
 
 from kvq_testlib import ATOL_REL, TIE_BUDGET, host_f32, mask_u32
+from kvq_testlib import _token_of as token_of
 from oracle import oracle as orc
 from quantized_attention_kvq_b200 import native, synth, workloads
 
@@ -58,24 +59,17 @@ def check_slice_bytes(got: dict, c: orc.Cache, st: dict, wl):
         diff = np.nonzero(got[name] != r)[0]
         if diff.size:
             # every differing byte must sit in a token the oracle flagged as a near-tie
-            cap = wl.capacity
-            if name == "k_codes":  # [block of 128 tokens][32 channel groups][128]
-                w = diff // (2 if wl.k_bits == 4 else 1)
-                tok = (w // (32 * 128)) * 128 + w % 128
-            elif name == "k_scales":  # [block][4 groups][128]
-                i = diff // 4
-                tok = (i // (4 * 128)) * 128 + i % 128
-            elif name == "k_ch0":
-                tok = (diff // 2) % cap
-            elif name == "v_codes":
-                tok = diff // (16 * wl.v_bits)
-            else:
-                tok = diff // 16
-            t = tok - wl.offset
-            assert ((t >= 0) & (t < wl.T)).all(), f"{name}: bytes outside the appended range differ"
+            # (a value-code byte holds several tokens: any of them may carry the tie)
+            _, tok = token_of(name, diff, wl.capacity, wl.k_bits, wl.v_bits)
+            span = 8 // wl.v_bits if name == "v_codes" else 1
             flags = st["k_row_exempt" if name.startswith("k_") else "v_row_exempt"][0, 0]
-            assert flags[t].all(), f"{name}: {diff.size} differing bytes outside near-tie tokens"
-            bad_rows += np.unique(t).size
+            ok = np.zeros(diff.size, bool)
+            for i in range(span):
+                t = tok + i - wl.offset
+                inside = (t >= 0) & (t < wl.T)
+                ok |= inside & flags[np.clip(t, 0, wl.T - 1)].astype(bool)
+            assert ok.all(), f"{name}: {int((~ok).sum())} differing bytes outside near-tie tokens"
+            bad_rows += np.unique(tok).size
     assert bad_rows <= TIE_BUDGET * (st["k_elems"] + st["v_elems"]) + 1
 
 
@@ -127,7 +121,6 @@ def test_decode_workload(wid):
     gc.decode_combine(wl.Hq, lens_d, max_len, out, ws)
     out2 = gc.decode(qd, lens_d, max_len, mask_d, scale)
     torch.cuda.synchronize()
-    assert torch.equal(out, out2)
     o_gpu = out.cpu().numpy()
     assert np.isfinite(o_gpu).all()
     G = wl.G
@@ -140,6 +133,9 @@ def test_decode_workload(wid):
         got = o_gpu[b, h * G:(h + 1) * G].astype(np.float64)
         err = np.abs(got - o_ref).max()
         assert err <= ATOL_REL * np.abs(o_ref).max(), (wl.name, b, h, err, np.abs(o_ref).max())
+    diff = (out - out2).abs().reshape(wl.B, wl.Hq, 128).amax(dim=2)
+    rows = torch.nonzero(diff).tolist()
+    assert not rows, f"identical decode calls differ in {len(rows)} rows, e.g. {rows[:8]}, max {diff.max().item():.3e}"
 
 
 def test_append_workload():

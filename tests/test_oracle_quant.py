@@ -147,15 +147,47 @@ def test_key_layout_is_channel_major_words():
     assert not sc.any()
 
 
-def test_value_layout_is_token_major_nibbles():
+def test_value_layout_is_channel_major_rows_with_swizzled_chunks():
+    # INT2, rotation off, one token at position 129 = block 1, token 1 of the
+    # block; value of channel ch is ch % 4, which is also its code (min 0, max 3)
     d = 128
     v = np.zeros((1, 1, 1, d), np.float32)
-    v[0, 0, 0, :] = np.tile(np.array([0, 1, 2, 3], np.float32), 32)  # INT2: codes = values
-    k = np.zeros_like(v)
-    c, _ = _cache_with(k, v, 2, 2, 0, 0, capacity=2, offset=1)
-    row = c.v_codes.reshape(2, 32)[1]
-    assert np.all(row == (0 | 1 << 2 | 2 << 4 | 3 << 6))
-    assert not c.v_codes.reshape(2, 32)[0].any()
+    v[0, 0, 0, :] = np.tile(np.array([0, 1, 2, 3], np.float32), 32)
+    c, _ = _cache_with(np.zeros_like(v), v, 2, 2, 0, 0, capacity=256, offset=129)
+    rows = c.v_codes.reshape(2, 128, 32)  # [block][channel][128 tokens x 2 bits]
+    # hand-placed: token 1 is the second crumb (bits 2-3) of byte 0 of chunk 0;
+    # chunk 0 of channels 4-7, 12-15, ... sits in the second 16-byte half of the row
+    assert rows[1, 1, 0] == 1 << 2
+    assert rows[1, 2, 0] == 2 << 2
+    assert rows[1, 3, 0] == 3 << 2
+    assert rows[1, 5, 16] == 1 << 2
+    assert rows[1, 6, 16] == 2 << 2
+    assert rows[1, 127, 16] == 3 << 2
+    assert rows[1, 9, 0] == 1 << 2
+    rows[1, :, 0] = 0
+    rows[1, :, 16] = 0
+    assert not rows.any()
+
+
+def test_value_rows_share_bytes_between_tokens_without_clobbering():
+    # INT4: tokens 32 and 33 of a block share byte 0 of chunk 1 (low, high nibble)
+    d = 128
+    v = np.zeros((1, 1, 2, d), np.float32)
+    v[0, 0, 0, :] = np.tile(np.array([0, 15], np.float32), 64)  # codes 0, 15, 0, 15, ...
+    v[0, 0, 1, :] = np.tile(np.array([15, 0], np.float32), 64)  # codes 15, 0, 15, 0, ...
+    c = orc.Cache(1, 1, d, 128, 4, 4, 0, 0)
+    c.append(np.zeros((1, 1, 1, d), np.float32), v[:, :, :1], 32)
+    c.append(np.zeros((1, 1, 1, d), np.float32), v[:, :, 1:], 33)
+    rows = c.v_codes.reshape(128, 64)  # [channel][128 tokens x 4 bits]
+    # chunk 1 of channel ch lands at chunk position 1 ^ ((ch >> 1) & 3)
+    assert rows[0, 16] == 0xF0   # ch 0: token 32 code 0, token 33 code 15
+    assert rows[1, 16] == 0x0F   # ch 1: token 32 code 15, token 33 code 0
+    assert rows[2, 0] == 0xF0    # ch 2: chunk position 0
+    assert rows[5, 48] == 0x0F   # ch 5: chunk position 3
+    assert rows[7, 32] == 0x0F   # ch 7: chunk position 2
+    assert np.count_nonzero(rows) == 128
+    assert list(c.unpack(0, 0, 32, 1)) == [0, 15] * 64
+    assert list(c.unpack(0, 0, 33, 1)) == [15, 0] * 64
 
 
 def test_channel0_outlier_is_excluded_from_range():
