@@ -18,7 +18,8 @@
 //           so the per-token group scale applies exactly afterwards;
 //   PV:     8 MMAs of kind::f16 (K = 16 tokens each): value codes as exact
 //           f16 integers in tensor memory x P' = p * value scale, spread over
-//           independent partial accumulators.
+//           independent partial accumulators that stay in tensor memory for a
+//           whole segment (one accumulator set per segment parity).
 //
 // Roles inside a CTA, pipelined over tiles with mbarriers:
 //   producer warp   : 1-D bulk async copies of a tile's kept key-code rows
@@ -35,10 +36,11 @@
 //   epilogue warps  : thread = (token, heads): score = delta * sum_g s_g S_g +
 //                     sum_g z_g sum(q_g) (+ q_0 k_0), online softmax with a
 //                     lazily raised max, P' into shared memory, the value
-//                     zero-point terms sum_t p_t z_t in registers; later,
-//                     thread = (channel, heads): O from tensor memory into a
-//                     rescaled register accumulator; at a segment end, the
-//                     partial.
+//                     zero-point terms sum_t p_t z_t in registers; when the max
+//                     rises inside a segment, thread = (channel, heads) rescales
+//                     the segment's PV accumulator in tensor memory; two tiles
+//                     after a segment ends, the accumulator is read out into
+//                     the segment's partial.
 // Scores come straight from the codes; no dequantized key is ever formed
 // (tq-kv abstract; Dual-QK summary Sec. 3.2, 3.3).  Every mbarrier wait is
 // bounded; after a give-up all waits fall through and the CTA writes NaN
@@ -60,7 +62,7 @@ constexpr float kQSteps = 16000.0f;  // |q| / delta <= 16000: pieces q1 in [-125
 
 template <int G, int KB, int VB, bool CH0>
 struct Shape {
-  static constexpr int TPT = G > 1 ? 2 : 1;  // epilogue threads per token (head parts)
+  static constexpr int TPT = G > 4 ? 2 : 1;  // epilogue threads per token (head parts)
   static constexpr int HH = G / TPT;         // heads per epilogue thread: 1, 2, 4 or 8
   static constexpr int EPI_WARPS = 4 * TPT;
   static constexpr int EPI_THREADS = 32 * EPI_WARPS;
@@ -70,13 +72,13 @@ struct Shape {
   static constexpr int NS = 2 * G < 16 ? 16 : 2 * G;  // score columns per group: q1 rows, then q2 rows
   static constexpr int NO = 4 * G < 16 ? 16 : 4 * G;  // PV columns: (value group, head)
   static constexpr int STG = G > 8 ? 1 : 2;           // operand stages in tensor memory (keys and values)
-  static constexpr int OB = G > 8 ? 2 : 3;            // PV accumulator sets in flight
+  static constexpr int OB = 2;                        // PV accumulator sets: one per segment parity
   static constexpr int PP = G > 8 ? 1 : (G > 4 ? 2 : 4);  // partial accumulators per PV (independent chains)
   // tensor-memory columns; every accumulator starts at a multiple of its width
   static constexpr int TM_AK = 0;                   // STG key stages x 32 columns (128 u8 codes)
   static constexpr int TM_AV = 32 * STG;            // STG value stages x 64 columns (128 f16 codes)
   static constexpr int TM_S = STG == 2 ? 192 : 128; // 2 score buffers x 4 groups x NS
-  static constexpr int TM_O = TM_S + 2 * 4 * NS;    // OB PV sets x PP partials x NO
+  static constexpr int TM_O = TM_S + 2 * 4 * NS;    // 2 PV sets x PP partials x NO
   static constexpr int TMEM_COLS = 512;
   static_assert(TM_AK + 32 * STG <= TM_AV && TM_AV + 64 * STG <= TM_S, "operand columns");
   static_assert(TM_O + OB * PP * NO <= TMEM_COLS, "tensor memory");
@@ -103,10 +105,9 @@ struct Shape {
   static constexpr int F_QD = F_Q0 + 2 * QV;         // [2][G] f32: delta of the query pieces
   static constexpr int F_RED = F_QD + 2 * QV;        // [2 tiles][TPT][4 warps][16] f32
   static constexpr int F_RED2 = F_RED + 2 * TPT * 4 * 16 * 4;    // [TPT][4 warps][16] f32
-  static constexpr int F_PEND = F_RED2 + TPT * 4 * 16 * 4;       // [2 parities][TPT][6 HH] f32
-  static constexpr int F_ALPHA = F_PEND + 2 * TPT * 6 * HH * 4;  // [OB][TPT][HH] f32: rescale per tile
-  static constexpr int F_BAR = (F_ALPHA + OB * TPT * HH * 4 + 15) / 16 * 16;
-  static constexpr int NBAR_FIXED = 15;  // kready[2] vready[2] pready[2] sdone[2] pvdone[3] qready[2] qfree[2]
+  static constexpr int F_PEND = F_RED2 + TPT * 4 * 16 * 4;       // [2 segment parities][TPT][6 HH] f32
+  static constexpr int F_BAR = (F_PEND + 2 * TPT * 6 * HH * 4 + 15) / 16 * 16;
+  static constexpr int NBAR_FIXED = 14;  // kready[2] vready[2] pready[2] sdone[2] pvdone[2] qready[2] qfree[2]
   static constexpr int F_REST_NO_RING = F_BAR + NBAR_FIXED * 8 + 16;  // + tmem slot, error flag
   static constexpr int STAGES_FIT = (kSmemLimit - F_REST_NO_RING - 2 * kMaxStages * 8) / STAGE;
   static constexpr int STAGES = STAGES_FIT < kMaxStages ? STAGES_FIT : kMaxStages;
@@ -201,17 +202,32 @@ struct TileIter {
   __device__ size_t bh(const DecodeArgs& a) const { return (size_t)b * a.c.H + h; }
 };
 
-// Bounded wait.  A non-blocking test first (a completed phase costs little);
-// then each poll may keep the thread suspended (not issuing) for up to 0.5 us
-// while the phase is incomplete and resumes it as soon as the phase completes;
-// the wait gives up after 2^21 polls (about a second), or at once after any
-// earlier give-up in the CTA.
+// Bounded waits.  Both test the phase without blocking first (a completed
+// phase costs a few instructions).  ws_wait then keeps polling with
+// try_wait, for the epilogue, whose waits are on the critical path; ws_wait_nap
+// sleeps between polls (32 ns doubling to `cap_ns`), for the warps that run
+// ahead of the epilogue and would otherwise take issue slots from it while they
+// wait.  Both give up after about a second, or at once after any earlier
+// give-up in the CTA, and report false.
 __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile int* err) {
   if (mbar_test_wait(bar, parity)) return true;
 #pragma unroll 1
   for (uint32_t it = 0; it < (1u << 21); ++it) {
     if (mbar_try_wait_sleep(bar, parity, 500u)) return true;
     if (*err) return false;
+  }
+  *err = 1;
+  return false;
+}
+__device__ __forceinline__ bool ws_wait_nap(uint32_t bar, uint32_t parity, volatile int* err, uint32_t cap_ns) {
+  if (mbar_test_wait(bar, parity)) return true;
+  uint32_t ns = 32;
+#pragma unroll 1
+  for (uint32_t it = 0; it < (1u << 22); ++it) {
+    __nanosleep(ns);
+    if (mbar_test_wait(bar, parity)) return true;
+    if (*err) return false;
+    if (ns < cap_ns) ns <<= 1;
   }
   *err = 1;
   return false;
@@ -246,9 +262,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   auto VREADY = [&](int k) { return bar0 + 8 * (2 + k); };
   auto PREADY = [&](int k) { return bar0 + 8 * (4 + k); };
   auto SDONE = [&](int k) { return bar0 + 8 * (6 + k); };
-  auto PVDONE = [&](int k) { return bar0 + 8 * (8 + k); };  // k < OB
-  auto QREADY = [&](int k) { return bar0 + 8 * (11 + k); };  // a segment's query data is in buffer k
-  auto QFREE = [&](int k) { return bar0 + 8 * (13 + k); };   // the epilogue is done with buffer k
+  auto PVDONE = [&](int k) { return bar0 + 8 * (8 + k); };   // PV UMMAs of tiles of parity k
+  auto QREADY = [&](int k) { return bar0 + 8 * (10 + k); };  // a segment's query data is in buffer k
+  auto QFREE = [&](int k) { return bar0 + 8 * (12 + k); };   // the epilogue is done with buffer k
   auto FULL = [&](int s) { return bar0 + 8 * (S::NBAR_FIXED + s); };
   auto EMPTY = [&](int s) { return bar0 + 8 * (S::NBAR_FIXED + ST + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fix + S::F_SLOT);
@@ -265,7 +281,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       mbar_init(PREADY(k), S::EPI_THREADS);
       mbar_init(SDONE(k), 1);
     }
-    for (int k = 0; k < OB; ++k) mbar_init(PVDONE(k), 1);
+    for (int k = 0; k < 2; ++k) mbar_init(PVDONE(k), 1);
     for (int k = 0; k < 2; ++k) {
       mbar_init(QREADY(k), 128);
       mbar_init(QFREE(k), S::EPI_THREADS);
@@ -294,7 +310,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     const int nblk = c.cap / kTile;
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int s = t % ST;
-      if (t >= ST) ws_wait(EMPTY(s), ((t / ST) - 1) & 1, err);
+      if (t >= ST) ws_wait_nap(EMPTY(s), ((t / ST) - 1) & 1, err, 512);
       const size_t bh = it.bh(a);
       const uint32_t msk = it.msk;
       const int n0 = it.i * kTile;
@@ -323,11 +339,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     const uint32_t idesc_o = idesc_f16_f32(kTile, S::NO, 0, 1);
     const uint32_t bp = smem_addr(fix + S::F_BP);
     int sseg = -1;  // segment of the tile being scored
+    uint32_t firstbits = 0, setbits = 0;  // bit (t & 3): tile t opens a segment / its PV set
     auto score = [&](int t) {
       if (it.first) ++sseg;
+      firstbits = (firstbits & ~(1u << (t & 3))) | ((it.first ? 1u : 0u) << (t & 3));
+      setbits = (setbits & ~(1u << (t & 3))) | ((uint32_t)(sseg & 1) << (t & 3));
       const uint32_t bq = smem_addr(fix + S::F_BQ + (sseg & 1) * S::BQ_BYTES);
       it.next(a);
-      ws_wait(KREADY(t & 1), (t >> 1) & 1, err);
+      ws_wait_nap(KREADY(t & 1), (t >> 1) & 1, err, 64);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t a0 = tmem + S::TM_AK + (S::STG == 2 ? (t & 1) * 32 : 0);
@@ -343,20 +362,21 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     score(0);
     for (int t = 0; t < ntiles; ++t) {
       if (t + 1 < ntiles) score(t + 1);
-      ws_wait(PREADY(t & 1), (t >> 1) & 1, err);
-      ws_wait(VREADY(t & 1), (t >> 1) & 1, err);
+      ws_wait_nap(PREADY(t & 1), (t >> 1) & 1, err, 64);
+      ws_wait_nap(VREADY(t & 1), (t >> 1) & 1, err, 64);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t a0 = tmem + S::TM_AV + (S::STG == 2 ? (t & 1) * 64 : 0);
         const uint32_t b0 = bp + (t & 1) * S::BP_BYTES;
-        const uint32_t d0 = tmem + S::TM_O + (t % OB) * PP * S::NO;
+        const uint32_t d0 = tmem + S::TM_O + ((setbits >> (t & 3)) & 1u) * PP * S::NO;
+        const bool fresh = (firstbits >> (t & 3)) & 1u;  // the segment's first tile starts its sums
         // 16 tokens per MMA; K step s accumulates into partial s % PP, so
         // consecutive MMAs of one accumulator are PP issues apart
 #pragma unroll
         for (int s = 0; s < kTile / 16; ++s)
           umma_f16_tmem_a(d0 + (s % PP) * S::NO, a0 + s * 8, smem_desc(b0 + s * 256, 128, 2048), idesc_o,
-                          s >= PP ? 1u : 0u);
-        umma_commit(PVDONE(t % OB));
+                          (fresh && s < PP) ? 0u : 1u);
+        umma_commit(PVDONE(t & 1));
       }
       __syncwarp();
     }
@@ -368,9 +388,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int s = t % ST;
       const uint8_t* raw = smem + s * S::STAGE + S::R_KC;
-      ws_wait(FULL(s), (t / ST) & 1, err);
+      ws_wait_nap(FULL(s), (t / ST) & 1, err, 256);
       // this key stage was read by the score UMMAs of tile t - STG
-      if (t >= S::STG) ws_wait(SDONE((t - S::STG) & 1), ((t - S::STG) >> 1) & 1, err);
+      if (t >= S::STG) ws_wait_nap(SDONE((t - S::STG) & 1), ((t - S::STG) >> 1) & 1, err, 256);
       tc_fence_after();
       if (it.first) {
         // query data of segment kseg into buffer kseg & 1: per head, delta =
@@ -381,7 +401,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         // buffer's two barriers see one phase per use, in order, so no parity wait
         // can pass on a later or an earlier phase.
         const int qb = kseg & 1;
-        if (kseg >= 2) ws_wait(QFREE(qb), ((kseg - 2) >> 1) & 1, err);
+        if (kseg >= 2) ws_wait_nap(QFREE(qb), ((kseg - 2) >> 1) & 1, err, 256);
         uint8_t* BQ = fix + S::F_BQ + qb * S::BQ_BYTES;
         float* qsum = reinterpret_cast<float*>(fix + S::F_QS + qb * G * 16);
         float* q0s = reinterpret_cast<float*>(fix + S::F_Q0 + qb * S::QV);
@@ -464,9 +484,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % ST;
       const uint8_t* row = smem + s * S::STAGE + S::R_VC + ch * S::VROW;
-      ws_wait(FULL(s), (t / ST) & 1, err);
+      ws_wait_nap(FULL(s), (t / ST) & 1, err, 256);
       // this value stage was read by the PV UMMAs of tile t - STG
-      if (t >= S::STG) ws_wait(PVDONE((t - S::STG) % OB), ((t - S::STG) / OB) & 1, err);
+      if (t >= S::STG) ws_wait_nap(PVDONE((t - S::STG) & 1), ((t - S::STG) >> 1) & 1, err, 256);
       tc_fence_after();
       const uint32_t col = tl + S::TM_AV + (S::STG == 2 ? (t & 1) * 64 : 0);
       constexpr int CHUNKS = S::VROW / 16;  // 4 (INT4: 32 tokens each) or 2 (INT2: 64 tokens each)
@@ -517,30 +537,30 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     float* red = reinterpret_cast<float*>(fix + S::F_RED);      // [2][TPT][4][16]
     float* red2 = reinterpret_cast<float*>(fix + S::F_RED2);    // [TPT][4][16]
     float* pend = reinterpret_cast<float*>(fix + S::F_PEND);    // [2][TPT][6 HH]
-    float* alphas = reinterpret_cast<float*>(fix + S::F_ALPHA) + part * HH;  // [OB][TPT][HH]
     const float NEG_INF = -__int_as_float(0x7f800000);
 
-    float m_run[HH], l_acc[HH], zacc[kGroups][HH], o[HH];
+    float m_run[HH], l_acc[HH], zacc[kGroups][HH];
     int nseg = 0;  // segments begun so far
-    int qb = 0;    // query buffer of the current segment
-    bool first1 = false, last1 = false, first2 = false, last2 = false;
-    int slot_even = 0, slot_odd = 0;  // partial slot of a segment ending at an even / odd tile
+    int qb = 0;    // query buffer and PV accumulator set of the current segment (its parity)
+    // tiles t-1 and t-2: whether they ended a segment, its set and partial slot
+    bool last1 = false, last2 = false;
+    int set1 = 0, set2 = 0, slot1 = 0, slot2 = 0;
     bool ok = true;
 #pragma unroll
     for (int i = 0; i < HH; ++i) {
       m_run[i] = NEG_INF;
-      l_acc[i] = o[i] = 0.0f;
+      l_acc[i] = 0.0f;
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) zacc[g][i] = 0.0f;
     }
 
-    // PV of tile tp into o (thread = channel j), rescaled by the tile's factor;
-    // at a segment end, the partial (plus the group's value zero-point term)
-    auto readback = [&](int tp, bool first, bool last) {
-      ok &= ws_wait(PVDONE(tp % OB), (tp / OB) & 1, err);
-      tc_fence_after();
-      const uint32_t base = tmem + lane_base + S::TM_O + (tp % OB) * PP * S::NO + wq * G + part * HH;
-      float d[HH];
+    // this thread's PV accumulator columns (channel j, its HH heads) of partial 0 of set os
+    auto obase = [&](int os) {
+      return tmem + lane_base + S::TM_O + os * PP * S::NO + wq * G + part * HH;
+    };
+    // sum of the PP partials of set os (after the last PV into it completed)
+    auto load_out = [&](int os, float (&d)[HH]) {
+      const uint32_t base = obase(os);
       if constexpr (PP == 4) {
         uint32_t r[4][HH];
         tmem_ld4_wait<HH>(base, S::NO, r);
@@ -560,21 +580,23 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 #pragma unroll
         for (int i = 0; i < HH; ++i) d[i] = __uint_as_float(r0[i]);
       }
-      const float* al = alphas + (tp % OB) * S::TPT * HH;
-#pragma unroll
-      for (int i = 0; i < HH; ++i) o[i] = first ? d[i] : fmaf(o[i], al[i], d[i]);
+    };
+    // a segment that ended at tile tp: its PV output (plus the group's value
+    // zero-point term) and its running max and sum into partial slot `slot`
+    auto readout = [&](int tp, int os, int slot) {
+      ok &= ws_wait(PVDONE(tp & 1), (tp >> 1) & 1, err);
+      tc_fence_after();
+      float d[HH];
+      load_out(os, d);
       tc_fence_before();
-      if (last) {
-        const float nan = __int_as_float(0x7fc00000);
-        const bool good = ok && !*err;
-        const float* pd = pend + ((tp & 1) * S::TPT + part) * 6 * HH;
-        const int slot = (tp & 1) ? slot_odd : slot_even;
+      const float nan = __int_as_float(0x7fc00000);
+      const bool good = ok && !*err;
+      const float* pd = pend + (os * S::TPT + part) * 6 * HH;
 #pragma unroll
-        for (int i = 0; i < HH; ++i) {
-          const size_t row = (size_t)slot * G + part * HH + i;
-          a.part_acc[row * kHeadDim + j] = good ? o[i] + pd[(2 + wq) * HH + i] : nan;
-          if (j == 0) a.part_ml[row] = good ? make_float2(pd[i], pd[HH + i]) : make_float2(nan, nan);
-        }
+      for (int i = 0; i < HH; ++i) {
+        const size_t row = (size_t)slot * G + part * HH + i;
+        a.part_acc[row * kHeadDim + j] = good ? d[i] + pd[(2 + wq) * HH + i] : nan;
+        if (j == 0) a.part_ml[row] = good ? make_float2(pd[i], pd[HH + i]) : make_float2(nan, nan);
       }
     };
 
@@ -590,9 +612,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           for (int g = 0; g < kGroups; ++g) zacc[g][i] = 0.0f;
         }
       }
-      // PV of tile t-2 (its accumulator set is reused by tile t+1, or by tile t with two
-      // sets; its P' buffer is rewritten below)
-      if (t >= 2) readback(t - 2, first2, last2);
+      // the segment that ended two tiles ago: its accumulator set is reused by the
+      // segment after next, whose first PV comes after this tile's
+      if (last2) readout(t - 2, set2, slot2);
       // per-token scales, zeros and channel 0 from the ring (zero past the sequence end)
       const int s = t % ST;
       ok &= ws_wait(FULL(s), (t / ST) & 1, err);
@@ -667,8 +689,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       if (lane == 0) rt[wq * 16 + 8] = any ? 1.0f : 0.0f;
       named_sync(bar_id, 128);
       const bool raise = (rt[8] + rt[24] + rt[40] + rt[56]) > 0.0f;
-      float m_new[HH];
+      float alpha[HH];
       if (raise) {  // uniform across the part
+        float m_new[HH];
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           const float mx = warp_max(sc[i]);
@@ -676,26 +699,43 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         }
         named_sync(bar_id, 128);
 #pragma unroll
-        for (int i = 0; i < HH; ++i)
+        for (int i = 0; i < HH; ++i) {
           m_new[i] = fmaxf(m_run[i], fmaxf(fmaxf(rt[i], rt[16 + i]), fmaxf(rt[32 + i], rt[48 + i])));
+          alpha[i] = exp2f(m_run[i] - m_new[i]);
+          m_run[i] = m_new[i];
+        }
+        if (!it.first) {
+          // rescale the segment's PV sums so far (this thread: channel j, its heads)
+          // once the PV of tile t-1 has landed; tile t's PV adds after PREADY below
+          ok &= ws_wait(PVDONE((t - 1) & 1), ((t - 1) >> 1) & 1, err);
+          tc_fence_after();
+          const uint32_t base = obase(qb);
+#pragma unroll
+          for (int pp = 0; pp < PP; ++pp) {
+            uint32_t r[HH];
+            tmem_ld_wait<HH>(base + pp * S::NO, r);
+#pragma unroll
+            for (int i = 0; i < HH; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha[i]);
+            tmem_st_n<HH>(base + pp * S::NO, r);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+        }
       } else {
 #pragma unroll
-        for (int i = 0; i < HH; ++i) m_new[i] = m_run[i];
+        for (int i = 0; i < HH; ++i) alpha[i] = 1.0f;
       }
       float p[HH];
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        const float alpha = exp2f(m_run[i] - m_new[i]);  // uniform across the part
-        if (j == 0) alphas[(t % OB) * S::TPT * HH + i] = alpha;
-        m_run[i] = m_new[i];
-        p[i] = valid ? exp2f(sc[i] - m_new[i]) : 0.0f;
-        l_acc[i] = fmaf(l_acc[i], alpha, p[i]);
+        p[i] = valid ? exp2f(sc[i] - m_run[i]) : 0.0f;
+        l_acc[i] = fmaf(l_acc[i], alpha[i], p[i]);
 #pragma unroll
-        for (int g = 0; g < kGroups; ++g) zacc[g][i] = fmaf(zacc[g][i], alpha, p[i] * vsz[g].y);
+        for (int g = 0; g < kGroups; ++g) zacc[g][i] = fmaf(zacc[g][i], alpha[i], p[i] * vsz[g].y);
       }
       // P' = p * value scale into the MN-major operand: column (group g, head),
-      // K position pos.  This buffer was last read by the PV UMMAs of tile t-2,
-      // complete since the readback above.
+      // K position pos.  This buffer was last read by the PV UMMAs of tile t-2.
+      if (t >= 2) ok &= ws_wait(PVDONE(k), ((t - 2) >> 1) & 1, err);
       uint8_t* BP = fix + S::F_BP + k * S::BP_BYTES;
       if constexpr (G == 1) {
         // one head: columns 0..3 = groups 0..3, one 8-byte store
@@ -703,11 +743,20 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         const __half2 a23 = __floats2half2_rn(p[0] * vsz[2].x, p[0] * vsz[3].x);
         *reinterpret_cast<uint2*>(BP + mnmajor(0, pos)) =
             make_uint2(*reinterpret_cast<const uint32_t*>(&a01), *reinterpret_cast<const uint32_t*>(&a23));
-      } else if constexpr (HH == 1) {
-        // G = 2: this part's head of group g is column 2g + part
+      } else if constexpr (S::TPT == 1) {
+        // columns g*G + i, 0 .. 4G-1, contiguous: 8 per 16-byte store
+        uint32_t pk[2 * G];
 #pragma unroll
         for (int g = 0; g < kGroups; ++g)
-          *reinterpret_cast<__half*>(BP + mnmajor(2 * g + part, pos)) = __float2half_rn(p[0] * vsz[g].x);
+#pragma unroll
+          for (int i = 0; i < HH; i += 2) {
+            const __half2 h2 = __floats2half2_rn(p[i] * vsz[g].x, p[i + 1] * vsz[g].x);
+            pk[(g * HH + i) / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+#pragma unroll
+        for (int n = 0; n < 4 * G; n += 8)
+          *reinterpret_cast<uint4*>(BP + mnmajor(n, pos)) =
+              make_uint4(pk[n / 2], pk[n / 2 + 1], pk[n / 2 + 2], pk[n / 2 + 3]);
       } else {
         // HH consecutive columns g*G + part*HH .. per group
 #pragma unroll
@@ -719,7 +768,6 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             pk[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
           }
           uint8_t* dst = BP + mnmajor(g * G + part * HH, pos);
-          if constexpr (HH == 2) *reinterpret_cast<uint32_t*>(dst) = pk[0];
           if constexpr (HH == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
           if constexpr (HH == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
@@ -727,16 +775,12 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       fence_proxy_async();
       mbar_arrive(PREADY(k));
 
-      first2 = first1;
-      last2 = last1;
-      first1 = it.first;
-      last1 = it.last;
-
+      int slot_t = 0;
       if (it.last) {
         // segment totals over this part's 128 tokens (max, sum, value zero-point terms),
-        // parked in shared memory until the segment's last PV is read back
+        // parked in shared memory until the segment's output is read out
         float* r2 = red2 + part * 64;
-        float* pd = pend + (k * S::TPT + part) * 6 * HH;
+        float* pd = pend + (qb * S::TPT + part) * 6 * HH;
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           const float sm = warp_sum(l_acc[i]);
@@ -765,16 +809,18 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           }
         }
         named_sync(bar_id, 128);
-        if (k)
-          slot_odd = (int)it.bh(a) + blockIdx.x;
-        else
-          slot_even = (int)it.bh(a) + blockIdx.x;
+        slot_t = (int)it.bh(a) + blockIdx.x;
       }
+      last2 = last1;
+      set2 = set1;
+      slot2 = slot1;
+      last1 = it.last;
+      set1 = qb;
+      slot1 = slot_t;
     }
-    if (ntiles >= 2) readback(ntiles - 2, first2, last2);
-    readback(ntiles - 1, first1, last1);
+    if (ntiles >= 2 && last2) readout(ntiles - 2, set2, slot2);
+    readout(ntiles - 1, set1, slot1);  // the last tile always ends a segment
   }
-
   tc_fence_before();
   __syncthreads();
   if (warp == S::MMA_WARP) {
