@@ -9,6 +9,9 @@ the split decode kernel against the measured copy bandwidth.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl kvq|reference] [--workload ID]
 
+Workload 3 (quantize-append) measures the append kernel instead: appended
+tokens/s and its HBM GB/s.
+
 With N > 1 it runs under torchrun, one rank per GPU, each rank decoding its
 own batch (independent sequences, no collective on the data path); the
 timed region is bracketed by barriers and the step time is the max over ranks.
@@ -408,6 +411,130 @@ def run_kvq(args):
         dist.destroy_process_group()
 
 
+def append_algorithmic_bytes(wl: workloads.Workload) -> int:
+    """Bytes one append of the workload must move: the new K and V rows read,
+    and their codes, scale/zero pairs (and channel 0) written."""
+    esize = 4 if wl.fmt == "f32" else 2
+    per = 2 * 128 * esize  # K and V rows in
+    per += 128 * wl.k_bits // 8 + 16 + (2 if wl.keep_ch0 else 0)  # key codes, scales, channel 0
+    per += 128 * wl.v_bits // 8 + 16  # value codes, scales
+    return wl.B * wl.Hkv * wl.T * per
+
+
+def run_append(args):
+    """Quantize-append throughput: one step appends T new tokens to every
+    (sequence, kv head) of the workload at its offset, from K/V rows resident
+    in HBM.  Metric: appended tokens/s (sequence positions) and achieved HBM
+    GB/s of the append kernel against its algorithmic bytes."""
+    import torch
+
+    from quantized_attention_kvq_b200 import native
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = workloads.by_id(args.workload)
+    s = synth.Synth(workloads.BASE_SEED + wl.id + 1000 * rank, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt,
+                    wl.len_range)
+
+    def up(a):
+        if wl.fmt == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    kd, vd = up(s.k_full()), up(s.v_full())
+    cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        cache.append(kd, vd, wl.offset)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        torch.cuda._sleep(50_000_000)
+        for a_, b_ in evs:
+            flush.zero_()
+            a_.record(stream)
+            cache.append(kd, vd, wl.offset)
+            b_.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = sum(a_.elapsed_time(b_) for a_, b_ in evs) / len(evs)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end: K/V rows from pinned host memory, then the append, then one
+    # code word read back (the host sees the cache updated)
+    k_pin, v_pin = kd.cpu().pin_memory(), vd.cpu().pin_memory()
+    probe = torch.empty(16, dtype=torch.uint8).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a_, b_ in e2e_ev:
+        flush.zero_()
+        a_.record(stream)
+        kd.copy_(k_pin, non_blocking=True)
+        vd.copy_(v_pin, non_blocking=True)
+        cache.append(kd, vd, wl.offset)
+        probe.copy_(cache.k_codes[:16], non_blocking=True)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a_.elapsed_time(b_) for a_, b_ in e2e_ev) / len(e2e_ev)
+
+    peak, peak_src = measured_hbm_peak()
+    abytes = append_algorithmic_bytes(wl)
+    achieved = abytes / (ms * 1e-3) / 1e9
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import oracle as orc
+
+        c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0)
+        k1 = orc.as_f32(np.stack([s.k_slice(0, h) for h in range(wl.Hkv)])[None])
+        v1 = orc.as_f32(np.stack([s.v_slice(0, h) for h in range(wl.Hkv)])[None])
+        t0 = time.perf_counter()
+        done = 0
+        while time.perf_counter() - t0 < args.cpu_seconds:
+            c.append(k1, v1, wl.offset)
+            done += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": done * wl.T / dt, "unit": "appended tokens/s", "cores": host_cores(), "kind": "oracle",
+               "sample": f"{done} appends of sequence 0 ({wl.Hkv} kv heads x {wl.T} tokens), {dt:.1f} s"}
+    if rank == 0:
+        line = {
+            "metric": "quantize-append tokens/sec & achieved HBM GB/s (fraction of B200 peak) at 1 GPU",
+            "value": world * wl.B * wl.T / (ms * 1e-3), "unit": "appended tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": f"{wl.fmt} in, u{wl.k_bits}k/u{wl.v_bits}v codes out",
+            "data": "synthetic (seeded SplitMix64 + Box-Muller, workload recipe distributions)",
+            "config": workload_config(wl),
+            "e2e": {"value": world * wl.B * wl.T / (e2e_ms * 1e-3), "unit": "appended tokens/s",
+                    "h2d_bytes_per_step": int(2 * kd.numel() * kd.element_size()), "d2h_bytes_per_step": 16},
+            "gpu_launches": args.steps,
+            "roofline": {"bound": "hbm", "kernel": "quantize-append (kvq_quantize_append)", "achieved": achieved,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "algorithmic_bytes_per_launch": abytes, "peak_source": peak_src, "kernel_ms": ms},
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -420,6 +547,8 @@ def main():
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == 3:
+        run_append(args)
     else:
         run_kvq(args)
 

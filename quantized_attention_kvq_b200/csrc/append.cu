@@ -1,9 +1,9 @@
 // Fused rotate + quantize + pack + append kernel.
 //
 // One CTA handles the new tokens of one (sequence, kv head) that fall in one
-// 64-token-aligned window of the cache; each of its 8 warps takes every 8th
-// token, one 128-channel row at a time with lane l owning channels 4l..4l+3
-// (= pruning group l).  Keys: fp64 Walsh-Hadamard butterflies (Dual-QK
+// 64-token-aligned window of the cache; each of its 8 warps takes 8 tokens,
+// four lanes per token, lane g of a token owning the 32 channels of
+// quantization group g.  Keys: fp64 Walsh-Hadamard butterflies (Dual-QK
 // summary Sec. 1; gist.science KQV scheme), optional bf16 channel 0 (Dual-QK
 // Sec. 3.3, App. C.3), per-32-channel asymmetric quantization (Dual-QK
 // Sec. 3.3).  Values: the same quantizer without rotation (Dual-QK App. B.2).
@@ -21,54 +21,170 @@ namespace {
 constexpr int kAppendTile = 64;  // tokens per CTA window, aligned to absolute token positions
 constexpr int kAppendWarps = 8;
 
-// Quantize the 4 channels this lane holds; the 8 lanes of a group agree on
-// (scale, zero).  skip0: channel 0 of this lane is kept out of the range and
-// gets code 0.  Returns the lane's packed word (4 codes of BITS bits).
+// 3-input fp32 max / min (sm_100)
+template <bool MAX>
+__device__ __forceinline__ float mm3(float a, float b, float c) {
+  float r;
+  if (MAX)
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  else
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// max / min of v0, v[1..31] as a depth-4 tree
+template <bool MAX>
+__device__ __forceinline__ float reduce32(float v0, const float (&v)[32]) {
+  float a[11];
+  a[0] = mm3<MAX>(v0, v[1], v[2]);
+#pragma unroll
+  for (int i = 1; i < 10; ++i) a[i] = mm3<MAX>(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  a[10] = mm3<MAX>(v[30], v[31], v[31]);
+  const float b0 = mm3<MAX>(a[0], a[1], a[2]), b1 = mm3<MAX>(a[3], a[4], a[5]);
+  const float b2 = mm3<MAX>(a[6], a[7], a[8]), b3 = mm3<MAX>(a[9], a[10], a[10]);
+  return mm3<MAX>(mm3<MAX>(b0, b1, b2), b3, b3);
+}
+
+// 1.5 * 2^23: for 0 <= q <= 2^22, q + kRoundMagic rounds q to the nearest
+// integer (ties to even) and leaves it in the low significand bits
+constexpr float kRoundMagic = 12582912.0f;
+constexpr float kNear = 0.5f - 1e-5f;  // |q - round(q)| beyond this: next to a rounding boundary
+
+// low bytes of four words -> one word, a in byte 0
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+// four codes (bytes 0..3 of x, each < 2^BITS) -> one BITS*4-bit word, byte 0 lowest
 template <int BITS>
-__device__ __forceinline__ uint32_t quantize_lane(const float x[4], bool skip0, __half2& sz) {
-  float mn = __int_as_float(0x7f800000), mx = -__int_as_float(0x7f800000);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    if (!(skip0 && i == 0)) {
-      mn = fminf(mn, x[i]);
-      mx = fmaxf(mx, x[i]);
-    }
-#pragma unroll
-  for (int m = 1; m < 8; m <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(kFull, mn, m));
-    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+__device__ __forceinline__ uint32_t compress_codes(uint32_t x) {
+  if (BITS == 4) {
+    x |= x >> 4;  // byte 0: c0 | c1 << 4, byte 2: c2 | c3 << 4
+    return __byte_perm(x, 0, 0x0020) & 0xFFFFu;
+  } else {
+    x |= x >> 6;  // byte 0: c0 | c1 << 2, byte 2: c2 | c3 << 2
+    return (x | (x >> 12)) & 0xFFu;
   }
+}
+
+// Quantize one 32-channel group held by this lane (v[0..31]); skip0: element 0
+// is kept out of the range and gets code 0.  Returns the fp16 (scale, zero)
+// pair; byte j of packed[p] is the code of element 4p + j.
+//
+// The code is round_half_even((x - zero) / scale) clamped to [0, L], the
+// quotient as IEEE fp32 division gives it.  It is formed as
+// q = (x - zero) * rcp(scale) with a correctly rounded reciprocal and clamped
+// to [0, L] (the bounds are integers, so clamp and round commute); q is then
+// within 2^-22 * q < 4e-6 of the clamped IEEE quotient.  When an element's q
+// lies within 1e-5 of a rounding boundary (k + 1/2) the group is coded again
+// with the IEEE division for such elements, so every code is the division's.
+template <int BITS>
+__device__ __forceinline__ __half2 quantize_group32(const float (&v)[32], bool skip0, uint32_t (&packed)[8]) {
+  const float v0 = skip0 ? v[1] : v[0];
   // -0 and +0 are the same extreme; take it as +0 so the stored bits are unique
-  mn = __fadd_rn(mn, 0.0f);
-  mx = __fadd_rn(mx, 0.0f);
+  const float mn = __fadd_rn(reduce32<false>(v0, v), 0.0f);
+  const float mx = __fadd_rn(reduce32<true>(v0, v), 0.0f);
   constexpr int L = (1 << BITS) - 1;
-  float s32 = fminf(__fdiv_rn(__fsub_rn(mx, mn), (float)L), 65504.0f);
-  float zc = fminf(fmaxf(mn, -65504.0f), 65504.0f);
+  const float s32 = fminf(__fdiv_rn(__fsub_rn(mx, mn), (float)L), 65504.0f);
+  const float zc = fminf(fmaxf(mn, -65504.0f), 65504.0f);
   const __half s16 = __float2half_rn(s32), z16 = __float2half_rn(zc);
-  sz = __halves2half2(s16, z16);
   const float sf = __half2float(s16), zf = __half2float(z16);
-  uint32_t word = 0;
+  const float rs = sf != 0.0f ? __frcp_rn(sf) : 0.0f;  // sf == 0: every code is 0
+  float near[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int code = 0;
-    if (!(skip0 && i == 0) && sf != 0.0f) {
-      code = __float2int_rn(__fdiv_rn(__fsub_rn(x[i], zf), sf));  // IEEE fp32, ties to even
-      code = min(max(code, 0), L);
+  for (int p = 0; p < 8; ++p) {
+    uint32_t m[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float q = fminf(fmaxf(__fmul_rn(__fsub_rn(v[4 * p + j], zf), rs), 0.0f), (float)L);
+      const float mq = __fadd_rn(q, kRoundMagic);
+      const float d = fabsf(__fsub_rn(q, __fsub_rn(mq, kRoundMagic)));  // exact: |q - round(q)|
+      near[j] = fmaxf(near[j], (p == 0 && j == 0 && skip0) ? 0.0f : d);
+      m[j] = __float_as_uint(mq);
     }
-    word |= (uint32_t)code << (BITS * i);
+    packed[p] = pack_low_bytes(m[0], m[1], m[2], m[3]);
   }
-  return word;
+  if (mm3<true>(mm3<true>(near[0], near[1], near[2]), near[3], near[3]) > kNear) {
+    // rare: code the group again, with the IEEE division next to a boundary
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      uint32_t m[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float d = __fsub_rn(v[4 * p + j], zf);
+        float q = fminf(fmaxf(__fmul_rn(d, rs), 0.0f), (float)L);
+        if (fabsf(__fsub_rn(q, rintf(q))) > kNear) q = fminf(fmaxf(rintf(__fdiv_rn(d, sf)), 0.0f), (float)L);
+        m[j] = __float_as_uint(__fadd_rn(q, kRoundMagic));
+      }
+      packed[p] = pack_low_bytes(m[0], m[1], m[2], m[3]);
+    }
+  }
+  if (skip0) packed[0] &= 0xFFFFFF00u;
+  return __halves2half2(s16, z16);
+}
+
+// 32 consecutive input elements held raw: 64 bytes (16-bit types) or 128 (fp32)
+template <typename In>
+struct Raw32 {
+  uint4 w[sizeof(In) * 2];
+};
+template <typename In>
+__device__ __forceinline__ void load_raw(const In* p, Raw32<In>& r) {
+#pragma unroll
+  for (int j = 0; j < (int)sizeof(In) * 2; ++j) r.w[j] = reinterpret_cast<const uint4*>(p)[j];
+}
+__device__ __forceinline__ void widen2(uint32_t u, const __nv_bfloat16*, float& a, float& b) {
+  a = __uint_as_float(u << 16);
+  b = __uint_as_float(u & 0xFFFF0000u);
+}
+__device__ __forceinline__ void widen2(uint32_t u, const __half*, float& a, float& b) {
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
+  a = f.x;
+  b = f.y;
+}
+// exact widening to fp32
+template <typename In>
+__device__ __forceinline__ void widen(const Raw32<In>& r, float (&f)[32]) {
+  if constexpr (sizeof(In) == 4) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      f[4 * j] = __uint_as_float(r.w[j].x);
+      f[4 * j + 1] = __uint_as_float(r.w[j].y);
+      f[4 * j + 2] = __uint_as_float(r.w[j].z);
+      f[4 * j + 3] = __uint_as_float(r.w[j].w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      widen2(r.w[j].x, (const In*)nullptr, f[8 * j], f[8 * j + 1]);
+      widen2(r.w[j].y, (const In*)nullptr, f[8 * j + 2], f[8 * j + 3]);
+      widen2(r.w[j].z, (const In*)nullptr, f[8 * j + 4], f[8 * j + 5]);
+      widen2(r.w[j].w, (const In*)nullptr, f[8 * j + 6], f[8 * j + 7]);
+    }
+  }
+}
+
+// 4x4 byte transpose: out[j] byte k = byte j of in[k]
+__device__ __forceinline__ void transpose_bytes4(const uint32_t (&in)[4], uint32_t (&out)[4]) {
+  const uint32_t t0 = __byte_perm(in[0], in[1], 0x5140), t1 = __byte_perm(in[0], in[1], 0x7362);
+  const uint32_t t2 = __byte_perm(in[2], in[3], 0x5140), t3 = __byte_perm(in[2], in[3], 0x7362);
+  out[0] = __byte_perm(t0, t2, 0x5410);
+  out[1] = __byte_perm(t0, t2, 0x7632);
+  out[2] = __byte_perm(t1, t3, 0x5410);
+  out[3] = __byte_perm(t1, t3, 0x7632);
 }
 
 template <int KB, int VB, bool ROT, bool CH0, typename In>
-__global__ void __launch_bounds__(kAppendWarps * 32) k_quantize_append(AppendArgs a) {
-  constexpr int TPW = 32 / VB;                  // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
-  constexpr int WPR = kAppendTile / TPW;        // value words per channel in the window: 8 or 4
-  __shared__ uint16_t kw[kPruneGroups][kAppendTile + 2];
-  __shared__ __half2 ksz[kGroups][kAppendTile];
-  __shared__ __nv_bfloat16 k0s[kAppendTile];
-  __shared__ __align__(16) uint8_t vcode[kAppendTile][kHeadDim];  // [token][channel] value codes
-  __shared__ uint32_t vword[kHeadDim][WPR + 1];                   // packed value words, padded rows
+__global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(AppendArgs a) {
+  constexpr int TPW = 32 / VB;            // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
+  constexpr int WPR = kAppendTile / TPW;  // value words per channel in the window: 8 or 4
+  // key words [pruning group][token], 16 bits a token (its KB * 4 low bits used)
+  __shared__ __align__(16) uint16_t kw[kPruneGroups][kAppendTile + 2];
+  // value codes [token][channel], one byte each; rows padded to 144 bytes so
+  // that the 16-byte stores of the 8 tokens a quarter-warp holds fall on
+  // distinct banks
+  __shared__ __align__(16) uint8_t vcode[kAppendTile][kHeadDim + 16];
+  // packed value words [word][channel]; rows padded by TPW words so that the
+  // TPW-channel x WPR-word block a warp reads falls on distinct banks
+  __shared__ __align__(16) uint32_t vword[WPR][kHeadDim + TPW];
 
   const CacheView& c = a.c;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -77,92 +193,142 @@ __global__ void __launch_bounds__(kAppendWarps * 32) k_quantize_append(AppendArg
   const int lo = max(a.offset - w0, 0);                                // window tokens [lo, hi) are new
   const int hi = min(a.offset + a.n_new - w0, kAppendTile);
   const size_t bh = (size_t)b * c.H + h;
-  // input row of window token tt: (bh * n_new + w0 + tt - offset), never negative for tt >= lo
-  const size_t row0 = bh * a.n_new + (w0 + lo - a.offset);
-  const In* kin = static_cast<const In*>(a.k_new) + (row0 - lo) * kHeadDim;
-  const In* vin = static_cast<const In*>(a.v_new) + (row0 - lo) * kHeadDim;
+  const int tb0 = w0 % kKeyBlock;                                      // window start inside its block: 0 or 64
+  const size_t unit_blk = bh * (size_t)(c.cap / kKeyBlock) + w0 / kKeyBlock;  // (unit, block) index
+  // four lanes per token, lane group g = lane & 3 holding channels 32g .. 32g+31
+  const int g = lane & 3;
+  const int tt = warp * 8 + (lane >> 2);  // window token of this lane
+  const bool active = tt >= lo && tt < hi;
+  // input row of window token tt: (bh * n_new + w0 + tt - offset), never negative when active
+  const size_t row = bh * a.n_new + (size_t)(w0 + (active ? tt : lo) - a.offset);
+  const In* kin = static_cast<const In*>(a.k_new) + row * kHeadDim + 32 * g;
+  const In* vin = static_cast<const In*>(a.v_new) + row * kHeadDim + 32 * g;
 
-  // one-deep prefetch of the next row pair
-  float kx[4], vx[4], kn[4], vn[4];
-  int tt = lo + warp;
-  if (tt < hi) {
-    load4(kin + (size_t)tt * kHeadDim + 4 * lane, kn);
-    load4(vin + (size_t)tt * kHeadDim + 4 * lane, vn);
-  }
-  for (; tt < hi; tt += kAppendWarps) {
+  Raw32<In> kraw, vraw;  // value loads issued together with the key loads
+  if (active) {
+    load_raw(kin, kraw);
+    load_raw(vin, vraw);
+  } else {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      kx[i] = kn[i];
-      vx[i] = vn[i];
-    }
-    const int nx = tt + kAppendWarps;
-    if (nx < hi) {
-      load4(kin + (size_t)nx * kHeadDim + 4 * lane, kn);
-      load4(vin + (size_t)nx * kHeadDim + 4 * lane, vn);
-    }
-    const size_t n = (size_t)w0 + tt;
+    for (int j = 0; j < (int)sizeof(In) * 2; ++j) kraw.w[j] = vraw.w[j] = make_uint4(0, 0, 0, 0);
+  }
+  float kx[32];
+  widen(kraw, kx);
 
-    // ---- key row
-    if (ROT) rotate_row_warp(kx, a.inv_sqrt_d, lane);
-    if (CH0 && lane == 0) k0s[tt] = __float2bfloat16_rn(kx[0]);
-    __half2 sz;
-    const uint32_t kword = quantize_lane<KB>(kx, CH0 && lane == 0, sz);
-    kw[lane][tt] = (uint16_t)kword;
-    if ((lane & 7) == 0) ksz[lane >> 3][tt] = sz;
-
-    // ---- value row: codes of channels 4l..4l+3 as bytes; scales token-major, written directly
-    const uint32_t vw = quantize_lane<VB>(vx, false, sz);
-    constexpr uint32_t L = (1u << VB) - 1;
-    *reinterpret_cast<uint32_t*>(&vcode[tt][4 * lane]) =
-        (vw & L) | (((vw >> VB) & L) << 8) | (((vw >> (2 * VB)) & L) << 16) | (((vw >> (3 * VB)) & L) << 24);
-    if ((lane & 7) == 0) c.vs[(bh * c.cap + n) * kGroups + (lane >> 3)] = sz;
+  // ---- key row: Walsh-Hadamard butterflies in fp64, natural Sylvester order
+  // (stage h pairs channels i and i + h, i & h == 0, -> (a + b, a - b)); the
+  // stages below 32 stay inside the lane, 32 and 64 pair lanes g ^ 1, g ^ 2
+  if (ROT) {
+    double x[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = kx[i];
+#pragma unroll
+    for (int hs = 1; hs < 32; hs <<= 1)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if ((i & hs) == 0) {
+          const double u = x[i], w = x[i + hs];
+          x[i] = __dadd_rn(u, w);
+          x[i + hs] = __dsub_rn(u, w);
+        }
+#pragma unroll
+    for (int m = 1; m <= 2; m <<= 1) {
+      const bool upper = (g & m) != 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        // lower lane: x + o; upper lane: o - x = o + (-x), the same IEEE sum
+        const double o = __shfl_xor_sync(kFull, x[i], m);
+        x[i] = __dadd_rn(upper ? -x[i] : x[i], o);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) kx[i] = __double2float_rn(__dmul_rn(x[i], a.inv_sqrt_d));
+  }
+  uint32_t code[8];
+  {
+    const bool skip0 = CH0 && g == 0;
+    const __half2 sz = quantize_group32<KB>(kx, skip0, code);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) kw[8 * g + p][tt] = (uint16_t)compress_codes<KB>(code[p]);
+    if (active) {
+      c.ks[(unit_blk * kGroups + g) * kKeyBlock + tb0 + tt] = sz;
+      if (skip0) c.k0[bh * c.cap + w0 + tt] = __float2bfloat16_rn(kx[0]);
+    }
+  }
+  // ---- value row: the same quantizer, no rotation; codes as bytes, scales token-major
+  {
+    float vx[32];
+    widen(vraw, vx);
+    const __half2 sz = quantize_group32<VB>(vx, false, code);
+    if (!active) {
+#pragma unroll
+      for (int p = 0; p < 8; ++p) code[p] = 0;  // tokens outside the append contribute zero bits
+    } else {
+      c.vs[(bh * c.cap + w0 + tt) * kGroups + g] = sz;
+    }
+    *reinterpret_cast<uint4*>(&vcode[tt][32 * g]) = make_uint4(code[0], code[1], code[2], code[3]);
+    *reinterpret_cast<uint4*>(&vcode[tt][32 * g + 16]) = make_uint4(code[4], code[5], code[6], code[7]);
   }
   __syncthreads();
 
-  // ---- key rows out: channel-major, one coalesced run per pruning group
-  const int ntok = hi - lo;
-  for (int i = threadIdx.x; i < kPruneGroups * ntok; i += blockDim.x) {
-    const int pg = i / ntok, t = lo + i % ntok;
-    const size_t idx = key_word_index(bh, c.cap, pg, w0 + t);
-    if (KB == 4)
-      reinterpret_cast<uint16_t*>(c.kc)[idx] = kw[pg][t];
-    else
-      c.kc[idx] = (uint8_t)kw[pg][t];
-  }
-  for (int i = threadIdx.x; i < kGroups * ntok; i += blockDim.x) {
-    const int g = i / ntok, t = lo + i % ntok;
-    c.ks[key_scale_index(bh, c.cap, g, w0 + t)] = ksz[g][t];
-  }
-  if (CH0)
-    for (int t = lo + threadIdx.x; t < hi; t += blockDim.x) c.k0[bh * c.cap + w0 + t] = k0s[t];
-
-  // ---- value codes: pack each channel's window into words (token order, low bits first)
-  for (int i = threadIdx.x; i < kHeadDim * WPR; i += blockDim.x) {
-    const int ch = i % kHeadDim, w = i / kHeadDim;  // a warp: 32 channels of one word position
-    uint32_t word = 0;
-#pragma unroll
-    for (int k = 0; k < TPW; ++k) {
-      const int t = w * TPW + k;
-      const uint32_t code = (t >= lo && t < hi) ? vcode[t][ch] : 0u;
-      word |= code << (VB * k);
+  // ---- key rows out: one pruning group's run per warp, two tokens a lane
+  {
+    const int t = 2 * lane;  // window tokens t, t + 1
+    const bool a0 = t >= lo && t < hi, a1 = t + 1 >= lo && t + 1 < hi;
+    for (int pg = warp; pg < kPruneGroups; pg += kAppendWarps) {
+      const size_t idx = (unit_blk * kPruneGroups + pg) * kKeyBlock + tb0 + t;
+      const uint32_t w2 = *reinterpret_cast<const uint32_t*>(&kw[pg][t]);  // token t in the low half
+      if (KB == 4) {
+        uint16_t* dst = reinterpret_cast<uint16_t*>(c.kc) + idx;
+        if (a0 && a1)
+          *reinterpret_cast<uint32_t*>(dst) = w2;
+        else if (a0)
+          dst[0] = (uint16_t)w2;
+        else if (a1)
+          dst[1] = (uint16_t)(w2 >> 16);
+      } else {
+        uint8_t* dst = c.kc + idx;
+        const uint32_t b2 = (w2 & 0xFFu) | ((w2 >> 8) & 0xFF00u);
+        if (a0 && a1)
+          *reinterpret_cast<uint16_t*>(dst) = (uint16_t)b2;
+        else if (a0)
+          dst[0] = (uint8_t)b2;
+        else if (a1)
+          dst[1] = (uint8_t)(b2 >> 8);
+      }
     }
-    vword[ch][w] = word;
+  }
+
+  // ---- value codes: each thread packs 4 channels x TPW tokens into 4 words
+  // (token order, low bits first) with byte transposes
+  if (threadIdx.x < 32 * WPR) {
+    const int c4 = threadIdx.x & 31, w = threadIdx.x >> 5;  // channels 4 c4 .. 4 c4 + 3, word w
+    uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int k = 0; k < TPW / 4; ++k) {
+      uint32_t in[4], col[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) in[r] = *reinterpret_cast<const uint32_t*>(&vcode[w * TPW + 4 * k + r][4 * c4]);
+      transpose_bytes4(in, col);  // col[j]: channel 4 c4 + j, tokens 4k .. 4k + 3
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] |= compress_codes<VB>(col[j]) << (4 * VB * k);
+    }
+    *reinterpret_cast<uint4*>(&vword[w][4 * c4]) = make_uint4(out[0], out[1], out[2], out[3]);
   }
   __syncthreads();
   // ...and store them into the channel rows of the 128-token block
-  const int blk = w0 / kKeyBlock;
-  const int tb0 = w0 % kKeyBlock;               // window start inside the block: 0 or 64
-  constexpr int TPC = 16 * 8 / VB;              // tokens per 16-byte chunk: 32 or 64
+  constexpr int TPC = 16 * 8 / VB;  // tokens per 16-byte chunk: 32 or 64
+  uint8_t* vblk = c.vc + unit_blk * (size_t)(kHeadDim * (kKeyBlock * VB / 8));
   for (int i = threadIdx.x; i < kHeadDim * WPR; i += blockDim.x) {
-    const int ch = i / WPR, w = i % WPR;        // a warp: 32 / WPR channels, all their words
-    const int t0 = w * TPW;                     // first window token of the word
-    const int tb = tb0 + t0;                    // ... inside the block
-    const int chunk = (tb / TPC) ^ v_chunk_swizzle(VB, ch);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(c.vc + v_row_offset(bh, c.cap, blk, ch, VB) + chunk * 16 +
-                                                (tb % TPC) / (8 / VB));
+    const int ch = i / WPR, w = i % WPR;  // a warp: 32 / WPR channels, all their words
+    const int t0 = w * TPW;               // first window token of the word
     const int a0 = max(lo - t0, 0), a1 = min(hi - t0, TPW);  // new tokens of this word: [a0, a1)
     if (a0 >= a1) continue;
-    uint32_t word = vword[ch][w];
+    const int tb = tb0 + t0;  // ... inside the block
+    const int chunk = (tb / TPC) ^ v_chunk_swizzle(VB, ch);
+    uint32_t* dst =
+        reinterpret_cast<uint32_t*>(vblk + ch * (kKeyBlock * VB / 8) + chunk * 16 + (tb % TPC) / (8 / VB));
+    uint32_t word = vword[w][ch];
     if (a0 > 0 || a1 < TPW) {
       const uint32_t keep_lo = a0 * VB >= 32 ? ~0u : ((1u << (a0 * VB)) - 1u);
       const uint32_t keep_hi = a1 * VB >= 32 ? 0u : ~((1u << (a1 * VB)) - 1u);
