@@ -38,6 +38,7 @@ from quantized_attention_kvq_b200 import synth, workloads  # noqa: E402
 DEFAULT_WORKLOAD = 1  # GQA INT4 decode, batch 8, 32/8 heads, 32768 cached tokens
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("decode.cu", "common.cuh", "sm100.cuh")
+APPEND_SOURCES = ("append.cu", "common.cuh")
 
 
 # ------------------------------------------------------------------ helpers
@@ -73,18 +74,19 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def decode_source_sha() -> str:
+def source_sha(names=DECODE_SOURCES) -> str:
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in names:
         with open(os.path.join(ROOT, "quantized_attention_kvq_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name: str):
-    """DRAM bytes per launch of the split kernel from the committed ncu summary,
-    or None when the summary is missing or the kernel source changed since."""
-    p = os.path.join(ROOT, "profiles", "decode_split_traffic.md")
+def recorded_traffic(workload_name: str, summary: str = "decode_split_traffic.md", sources=DECODE_SOURCES):
+    """DRAM bytes per launch of a kernel from its committed ncu summary, or None
+    when the summary is missing, covers another workload, or the kernel source
+    changed since."""
+    p = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(p):
         return None
     fields = {}
@@ -92,7 +94,7 @@ def recorded_traffic(workload_name: str):
         if ":" in line and line.startswith("- "):
             k, v = line[2:].split(":", 1)
             fields[k.strip()] = v.strip()
-    if fields.get("source_sha") != decode_source_sha() or fields.get("workload") != workload_name:
+    if fields.get("source_sha") != source_sha(sources) or fields.get("workload") != workload_name:
         return None
     try:
         return float(fields["traffic_bytes_per_launch"])
@@ -525,7 +527,8 @@ def run_append(args):
                     "h2d_bytes_per_step": int(2 * kd.numel() * kd.element_size()), "d2h_bytes_per_step": 16},
             "gpu_launches": args.steps,
             "roofline": {"bound": "hbm", "kernel": "quantize-append (kvq_quantize_append)", "achieved": achieved,
-                         "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": recorded_traffic(wl.name, "append_traffic.md", APPEND_SOURCES),
                          "algorithmic_bytes_per_launch": abytes, "peak_source": peak_src, "kernel_ms": ms},
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

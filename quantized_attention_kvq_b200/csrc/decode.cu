@@ -71,16 +71,21 @@ struct Shape {
   static constexpr int THREADS = 32 * (PROD_WARP + 1);
   static constexpr int NS = 2 * G < 16 ? 16 : 2 * G;  // score columns per group: q1 rows, then q2 rows
   static constexpr int NO = 4 * G < 16 ? 16 : 4 * G;  // PV columns: (value group, head)
-  static constexpr int STG = G > 8 ? 1 : 2;           // operand stages in tensor memory (keys and values)
+  static constexpr int KST = G > 8 ? 1 : 2;  // key operand stages in tensor memory
+  static constexpr int VST = G > 8 ? 1 : 2;  // value operand stages in tensor memory
+  static constexpr int SB = 2;               // score accumulator buffers
+  static constexpr int LA = SB - 1;          // score MMAs are issued LA tiles ahead of the PV MMAs
+  static constexpr int NKR = KST > 1 ? KST : 2;  // key-ready barriers
   static constexpr int OB = 2;                        // PV accumulator sets: one per segment parity
   static constexpr int PP = G > 8 ? 1 : (G > 4 ? 2 : 4);  // partial accumulators per PV (independent chains)
   // tensor-memory columns; every accumulator starts at a multiple of its width
-  static constexpr int TM_AK = 0;                   // STG key stages x 32 columns (128 u8 codes)
-  static constexpr int TM_AV = 32 * STG;            // STG value stages x 64 columns (128 f16 codes)
-  static constexpr int TM_S = STG == 2 ? 192 : 128; // 2 score buffers x 4 groups x NS
-  static constexpr int TM_O = TM_S + 2 * 4 * NS;    // 2 PV sets x PP partials x NO
+  static constexpr int TM_AK = 0;                                  // KST key stages x 32 columns (128 u8 codes)
+  static constexpr int TM_AV = 32 * KST;                           // VST value stages x 64 columns (128 f16 codes)
+  static constexpr int TM_S = (TM_AV + 64 * VST + 63) / 64 * 64;   // SB score buffers x 4 groups x NS
+  static constexpr int TM_O = TM_S + SB * 4 * NS;                  // 2 PV sets x PP partials x NO
   static constexpr int TMEM_COLS = 512;
-  static_assert(TM_AK + 32 * STG <= TM_AV && TM_AV + 64 * STG <= TM_S, "operand columns");
+  static_assert(TM_AK + 32 * KST <= TM_AV && TM_AV + 64 * VST <= TM_S, "operand columns");
+  static_assert(SB >= LA + 1 && KST >= 1 && VST <= 2, "stage counts");
   static_assert(TM_O + OB * PP * NO <= TMEM_COLS, "tensor memory");
   static_assert(TM_S % NS == 0 && TM_O % NO == 0, "accumulator alignment");
   // one ring stage: key-code rows, value-code rows, key (scale, zero) rows,
@@ -107,7 +112,8 @@ struct Shape {
   static constexpr int F_RED2 = F_RED + 2 * TPT * 4 * 16 * 4;    // [TPT][4 warps][16] f32
   static constexpr int F_PEND = F_RED2 + TPT * 4 * 16 * 4;       // [2 segment parities][TPT][6 HH] f32
   static constexpr int F_BAR = (F_PEND + 2 * TPT * 6 * HH * 4 + 15) / 16 * 16;
-  static constexpr int NBAR_FIXED = 14;  // kready[2] vready[2] pready[2] sdone[2] pvdone[2] qready[2] qfree[2]
+  // kready[3] vready[2] pready[2] sdone[3] pvdone[2] qready[2] qfree[2]
+  static constexpr int NBAR_FIXED = 16;
   static constexpr int F_REST_NO_RING = F_BAR + NBAR_FIXED * 8 + 16;  // + tmem slot, error flag
   static constexpr int STAGES_FIT = (kSmemLimit - F_REST_NO_RING - 2 * kMaxStages * 8) / STAGE;
   static constexpr int STAGES = STAGES_FIT < kMaxStages ? STAGES_FIT : kMaxStages;
@@ -258,13 +264,15 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
   uint8_t* fix = smem + ST * S::STAGE;
   const uint32_t bar0 = smem_addr(fix + S::F_BAR);
+  // Tile t's barriers: key-ready t % NKR, score-done t % SB, the others t % 2;
+  // a wait for tile t takes the parity of t's use of its barrier.
   auto KREADY = [&](int k) { return bar0 + 8 * k; };
-  auto VREADY = [&](int k) { return bar0 + 8 * (2 + k); };
-  auto PREADY = [&](int k) { return bar0 + 8 * (4 + k); };
-  auto SDONE = [&](int k) { return bar0 + 8 * (6 + k); };
-  auto PVDONE = [&](int k) { return bar0 + 8 * (8 + k); };   // PV UMMAs of tiles of parity k
-  auto QREADY = [&](int k) { return bar0 + 8 * (10 + k); };  // a segment's query data is in buffer k
-  auto QFREE = [&](int k) { return bar0 + 8 * (12 + k); };   // the epilogue is done with buffer k
+  auto VREADY = [&](int k) { return bar0 + 8 * (3 + k); };
+  auto PREADY = [&](int k) { return bar0 + 8 * (5 + k); };
+  auto SDONE = [&](int k) { return bar0 + 8 * (7 + k); };
+  auto PVDONE = [&](int k) { return bar0 + 8 * (10 + k); };  // PV UMMAs of tiles of parity k
+  auto QREADY = [&](int k) { return bar0 + 8 * (12 + k); };  // a segment's query data is in buffer k
+  auto QFREE = [&](int k) { return bar0 + 8 * (14 + k); };   // the epilogue is done with buffer k
   auto FULL = [&](int s) { return bar0 + 8 * (S::NBAR_FIXED + s); };
   auto EMPTY = [&](int s) { return bar0 + 8 * (S::NBAR_FIXED + ST + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fix + S::F_SLOT);
@@ -275,11 +283,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       mbar_init(FULL(s), 1);
       mbar_init(EMPTY(s), 256 + S::EPI_THREADS);
     }
+    for (int k = 0; k < S::NKR; ++k) mbar_init(KREADY(k), 128);
+    for (int k = 0; k < S::SB; ++k) mbar_init(SDONE(k), 1);
     for (int k = 0; k < 2; ++k) {
-      mbar_init(KREADY(k), 128);
       mbar_init(VREADY(k), 128);
       mbar_init(PREADY(k), S::EPI_THREADS);
-      mbar_init(SDONE(k), 1);
     }
     for (int k = 0; k < 2; ++k) mbar_init(PVDONE(k), 1);
     for (int k = 0; k < 2; ++k) {
@@ -346,27 +354,31 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       setbits = (setbits & ~(1u << (t & 3))) | ((uint32_t)(sseg & 1) << (t & 3));
       const uint32_t bq = smem_addr(fix + S::F_BQ + (sseg & 1) * S::BQ_BYTES);
       it.next(a);
-      ws_wait_nap(KREADY(t & 1), (t >> 1) & 1, err, 64);
+      ws_wait_nap(KREADY(t % S::NKR), (t / S::NKR) & 1, err, 64);
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a0 = tmem + S::TM_AK + (S::STG == 2 ? (t & 1) * 32 : 0);
-        const uint32_t d0 = tmem + S::TM_S + (t & 1) * 4 * S::NS;
+        const uint32_t a0 = tmem + S::TM_AK + (t % S::KST) * 32;
+        const uint32_t d0 = tmem + S::TM_S + (t % S::SB) * 4 * S::NS;
         // one MMA per 32-channel group (8 columns of u8 codes, 32 query bytes), all independent
 #pragma unroll
         for (int g = 0; g < kGroups; ++g)
           umma_i8_tmem_a(d0 + g * S::NS, a0 + g * 8, smem_desc(bq + g * 256, 128, 1024), idesc_s, 0u);
-        umma_commit(SDONE(t & 1));
+        umma_commit(SDONE(t % S::SB));
       }
       __syncwarp();
     };
-    score(0);
+    // The score MMAs of tile t + LA go ahead of the PV MMAs of tile t, so the
+    // epilogue finds tile t + 1's scores done while it works on tile t.  Score
+    // buffer (t + LA) % SB was last read by the epilogue of tile t + LA - SB
+    // <= t - 1, whose P' (PREADY) was waited for in the previous iteration.
+    for (int u = 0; u < S::LA && u < ntiles; ++u) score(u);
     for (int t = 0; t < ntiles; ++t) {
-      if (t + 1 < ntiles) score(t + 1);
+      if (t + S::LA < ntiles) score(t + S::LA);
       ws_wait_nap(PREADY(t & 1), (t >> 1) & 1, err, 64);
       ws_wait_nap(VREADY(t & 1), (t >> 1) & 1, err, 64);
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a0 = tmem + S::TM_AV + (S::STG == 2 ? (t & 1) * 64 : 0);
+        const uint32_t a0 = tmem + S::TM_AV + (t % S::VST) * 64;
         const uint32_t b0 = bp + (t & 1) * S::BP_BYTES;
         const uint32_t d0 = tmem + S::TM_O + ((setbits >> (t & 3)) & 1u) * PP * S::NO;
         const bool fresh = (firstbits >> (t & 3)) & 1u;  // the segment's first tile starts its sums
@@ -389,8 +401,8 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       const int s = t % ST;
       const uint8_t* raw = smem + s * S::STAGE + S::R_KC;
       ws_wait_nap(FULL(s), (t / ST) & 1, err, 256);
-      // this key stage was read by the score UMMAs of tile t - STG
-      if (t >= S::STG) ws_wait_nap(SDONE((t - S::STG) & 1), ((t - S::STG) >> 1) & 1, err, 256);
+      // this key stage was read by the score UMMAs of tile t - KST
+      if (t >= S::KST) ws_wait_nap(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err, 256);
       tc_fence_after();
       if (it.first) {
         // query data of segment kseg into buffer kseg & 1: per head, delta =
@@ -465,13 +477,13 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           for (int k = 0; k < 4; ++k) r[4 * q + k] = (x >> (2 * k)) & 0x03030303u;
         }
       }
-      const uint32_t col = tl + S::TM_AK + (S::STG == 2 ? (t & 1) * 32 : 0);
+      const uint32_t col = tl + S::TM_AK + (t % S::KST) * 32;
       tmem_st16(col, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
       tmem_st16(col + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
       tmem_wait_st();
       fence_proxy_async();  // query operand (generic writes) -> tensor core
       tc_fence_before();
-      mbar_arrive(KREADY(t & 1));
+      mbar_arrive(KREADY(t % S::NKR));
       mbar_arrive(EMPTY(s));
     }
   } else if (warp < 8) {
@@ -485,10 +497,10 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       const int s = t % ST;
       const uint8_t* row = smem + s * S::STAGE + S::R_VC + ch * S::VROW;
       ws_wait_nap(FULL(s), (t / ST) & 1, err, 256);
-      // this value stage was read by the PV UMMAs of tile t - STG
-      if (t >= S::STG) ws_wait_nap(PVDONE((t - S::STG) & 1), ((t - S::STG) >> 1) & 1, err, 256);
+      // this value stage was read by the PV UMMAs of tile t - VST
+      if (t >= S::VST) ws_wait_nap(PVDONE((t - S::VST) & 1), ((t - S::VST) >> 1) & 1, err, 256);
       tc_fence_after();
-      const uint32_t col = tl + S::TM_AV + (S::STG == 2 ? (t & 1) * 64 : 0);
+      const uint32_t col = tl + S::TM_AV + (t % S::VST) * 64;
       constexpr int CHUNKS = S::VROW / 16;  // 4 (INT4: 32 tokens each) or 2 (INT2: 64 tokens each)
 #pragma unroll
       for (int k = 0; k < CHUNKS; ++k) {
@@ -647,13 +659,13 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       const float* qsum = reinterpret_cast<const float*>(fix + S::F_QS + qb * G * 16);
       const float* q0s = reinterpret_cast<const float*>(fix + S::F_Q0 + qb * S::QV);
       const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * S::QV);
-      ok &= ws_wait(SDONE(k), (t >> 1) & 1, err);
+      ok &= ws_wait(SDONE(t % S::SB), (t / S::SB) & 1, err);
       tc_fence_after();
       float sc[HH];
       {
         // S_g = sum_c u8 code * (128 q1 + q2): q1 in column h, q2 in column G + h of group g
         uint32_t d1[kGroups][HH], d2[kGroups][HH];
-        const uint32_t sbase = tmem + lane_base + S::TM_S + k * 4 * S::NS + part * HH;
+        const uint32_t sbase = tmem + lane_base + S::TM_S + (t % S::SB) * 4 * S::NS + part * HH;
         if constexpr (HH == 2 || HH == 4) {
           tmem_ld8_wait<HH>(sbase, S::NS, G, d1, d2);
         } else {
@@ -768,6 +780,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             pk[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
           }
           uint8_t* dst = BP + mnmajor(g * G + part * HH, pos);
+          if constexpr (HH == 2) *reinterpret_cast<uint32_t*>(dst) = pk[0];
           if constexpr (HH == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
           if constexpr (HH == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
