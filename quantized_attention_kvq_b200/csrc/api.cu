@@ -70,7 +70,8 @@ struct DecodePlan {
 
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   DecodePlan p;
-  const size_t rows = (size_t)decode_slots(c->batch, c->kv_heads) * (q_heads / c->kv_heads);
+  const int G = q_heads / c->kv_heads;
+  const size_t rows = (size_t)decode_slots(c->batch, c->kv_heads, G) * G;
   p.acc_bytes = rows * kHeadDim * sizeof(float);
   p.ml_offset = round_up(p.acc_bytes, kAlign);
   p.bytes = p.ml_offset + round_up(rows * sizeof(float2), kAlign);

@@ -157,9 +157,11 @@ struct DecodeArgs {
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t s);
 // persistent tensor-core split decode (GQA groups of 1, 2, 4, 8 or 16 query
-// heads) and its combine; partial slots: one per (unit + CTA), decode_slots of them
+// heads) and its combine; partial slots: decode_groups(G) per (unit + CTA),
+// decode_slots of them
 bool decode_g_supported(int g);
-int decode_slots(int B, int H);
+int decode_groups(int G);
+int decode_slots(int B, int H, int G);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 

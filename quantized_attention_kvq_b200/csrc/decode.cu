@@ -64,7 +64,8 @@ template <int G, int KB, int VB, bool CH0>
 struct Shape {
   static constexpr int TPT = G > 4 ? 2 : 1;  // epilogue threads per token (head parts)
   static constexpr int HH = G / TPT;         // heads per epilogue thread: 1, 2, 4 or 8
-  static constexpr int EPI_WARPS = 4 * TPT;
+  static constexpr int NGRP = 1;  // epilogue groups, group g taking tiles t with t % NGRP == g (2 measured no faster)
+  static constexpr int EPI_WARPS = 4 * TPT * NGRP;
   static constexpr int EPI_THREADS = 32 * EPI_WARPS;
   static constexpr int MMA_WARP = 8 + EPI_WARPS;
   static constexpr int PROD_WARP = MMA_WARP + 1;
@@ -77,16 +78,16 @@ struct Shape {
   static constexpr int LA = SB - 1;          // score MMAs are issued LA tiles ahead of the PV MMAs
   static constexpr int NKR = KST > 1 ? KST : 2;  // key-ready barriers
   static constexpr int OB = 2;                        // PV accumulator sets: one per segment parity
-  static constexpr int PP = G > 8 ? 1 : (G > 4 ? 2 : 4);  // partial accumulators per PV (independent chains)
+  static constexpr int PP = G > 8 ? 1 : 2;  // partial accumulators per PV (independent chains)
   // tensor-memory columns; every accumulator starts at a multiple of its width
   static constexpr int TM_AK = 0;                                  // KST key stages x 32 columns (128 u8 codes)
   static constexpr int TM_AV = 32 * KST;                           // VST value stages x 64 columns (128 f16 codes)
   static constexpr int TM_S = (TM_AV + 64 * VST + 63) / 64 * 64;   // SB score buffers x 4 groups x NS
-  static constexpr int TM_O = TM_S + SB * 4 * NS;                  // 2 PV sets x PP partials x NO
+  static constexpr int TM_O = TM_S + SB * 4 * NS;                  // NGRP x 2 PV sets x PP partials x NO
   static constexpr int TMEM_COLS = 512;
   static_assert(TM_AK + 32 * KST <= TM_AV && TM_AV + 64 * VST <= TM_S, "operand columns");
   static_assert(SB >= LA + 1 && KST >= 1 && VST <= 2, "stage counts");
-  static_assert(TM_O + OB * PP * NO <= TMEM_COLS, "tensor memory");
+  static_assert(TM_O + NGRP * OB * PP * NO <= TMEM_COLS, "tensor memory");
   static_assert(TM_S % NS == 0 && TM_O % NO == 0, "accumulator alignment");
   // one ring stage: key-code rows, value-code rows, key (scale, zero) rows,
   // value (scale, zero) per token, channel 0
@@ -109,9 +110,9 @@ struct Shape {
   static constexpr int F_Q0 = F_QS + 2 * G * 16;     // [2][G] f32: q_0 (channel 0 kept in bf16)
   static constexpr int F_QD = F_Q0 + 2 * QV;         // [2][G] f32: delta of the query pieces
   static constexpr int F_RED = F_QD + 2 * QV;        // [2 tiles][TPT][4 warps][16] f32
-  static constexpr int F_RED2 = F_RED + 2 * TPT * 4 * 16 * 4;    // [TPT][4 warps][16] f32
-  static constexpr int F_PEND = F_RED2 + TPT * 4 * 16 * 4;       // [2 segment parities][TPT][6 HH] f32
-  static constexpr int F_BAR = (F_PEND + 2 * TPT * 6 * HH * 4 + 15) / 16 * 16;
+  static constexpr int F_RED2 = F_RED + 2 * TPT * 4 * 16 * 4;         // [NGRP][TPT][4 warps][16] f32
+  static constexpr int F_PEND = F_RED2 + NGRP * TPT * 4 * 16 * 4;     // [NGRP][2 segment parities][TPT][6 HH] f32
+  static constexpr int F_BAR = (F_PEND + NGRP * 2 * TPT * 6 * HH * 4 + 15) / 16 * 16;
   // kready[3] vready[2] pready[2] sdone[3] pvdone[2] qready[2] qfree[2]
   static constexpr int NBAR_FIXED = 16;
   static constexpr int F_REST_NO_RING = F_BAR + NBAR_FIXED * 8 + 16;  // + tmem slot, error flag
@@ -208,32 +209,17 @@ struct TileIter {
   __device__ size_t bh(const DecodeArgs& a) const { return (size_t)b * a.c.H + h; }
 };
 
-// Bounded waits.  Both test the phase without blocking first (a completed
-// phase costs a few instructions).  ws_wait then keeps polling with
-// try_wait, for the epilogue, whose waits are on the critical path; ws_wait_nap
-// sleeps between polls (32 ns doubling to `cap_ns`), for the warps that run
-// ahead of the epilogue and would otherwise take issue slots from it while they
-// wait.  Both give up after about a second, or at once after any earlier
-// give-up in the CTA, and report false.
+// Bounded wait: tests the phase without blocking first (a completed phase
+// costs a few instructions), then waits with try_wait, which suspends the
+// thread until the phase completes (or a time hint passes) without taking issue
+// slots.  Gives up after about a second, or at once after any earlier give-up
+// in the CTA, and reports false.
 __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile int* err) {
   if (mbar_test_wait(bar, parity)) return true;
 #pragma unroll 1
   for (uint32_t it = 0; it < (1u << 21); ++it) {
     if (mbar_try_wait_sleep(bar, parity, 500u)) return true;
     if (*err) return false;
-  }
-  *err = 1;
-  return false;
-}
-__device__ __forceinline__ bool ws_wait_nap(uint32_t bar, uint32_t parity, volatile int* err, uint32_t cap_ns) {
-  if (mbar_test_wait(bar, parity)) return true;
-  uint32_t ns = 32;
-#pragma unroll 1
-  for (uint32_t it = 0; it < (1u << 22); ++it) {
-    __nanosleep(ns);
-    if (mbar_test_wait(bar, parity)) return true;
-    if (*err) return false;
-    if (ns < cap_ns) ns <<= 1;
   }
   *err = 1;
   return false;
@@ -281,13 +267,13 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(FULL(s), 1);
-      mbar_init(EMPTY(s), 256 + S::EPI_THREADS);
+      mbar_init(EMPTY(s), 256 + S::EPI_THREADS / S::NGRP);  // key, value and the tile's epilogue group
     }
     for (int k = 0; k < S::NKR; ++k) mbar_init(KREADY(k), 128);
     for (int k = 0; k < S::SB; ++k) mbar_init(SDONE(k), 1);
     for (int k = 0; k < 2; ++k) {
       mbar_init(VREADY(k), 128);
-      mbar_init(PREADY(k), S::EPI_THREADS);
+      mbar_init(PREADY(k), S::EPI_THREADS / S::NGRP);
     }
     for (int k = 0; k < 2; ++k) mbar_init(PVDONE(k), 1);
     for (int k = 0; k < 2; ++k) {
@@ -318,7 +304,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     const int nblk = c.cap / kTile;
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int s = t % ST;
-      if (t >= ST) ws_wait_nap(EMPTY(s), ((t / ST) - 1) & 1, err, 512);
+      if (t >= ST) ws_wait(EMPTY(s), ((t / ST) - 1) & 1, err);
       const size_t bh = it.bh(a);
       const uint32_t msk = it.msk;
       const int n0 = it.i * kTile;
@@ -346,15 +332,20 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     const uint32_t idesc_s = idesc_u8s8_s32(kTile, S::NS);
     const uint32_t idesc_o = idesc_f16_f32(kTile, S::NO, 0, 1);
     const uint32_t bp = smem_addr(fix + S::F_BP);
-    int sseg = -1;  // segment of the tile being scored
-    uint32_t firstbits = 0, setbits = 0;  // bit (t & 3): tile t opens a segment / its PV set
+    int sseg = -1;    // segment of the tile being scored
+    int sstart = 0;   // its first tile
+    // bit (t & 3): tile t is its epilogue group's first of the segment / the segment's parity
+    uint32_t firstbits = 0, setbits = 0;
     auto score = [&](int t) {
-      if (it.first) ++sseg;
-      firstbits = (firstbits & ~(1u << (t & 3))) | ((it.first ? 1u : 0u) << (t & 3));
+      if (it.first) {
+        ++sseg;
+        sstart = t;
+      }
+      firstbits = (firstbits & ~(1u << (t & 3))) | ((t - sstart < S::NGRP ? 1u : 0u) << (t & 3));
       setbits = (setbits & ~(1u << (t & 3))) | ((uint32_t)(sseg & 1) << (t & 3));
       const uint32_t bq = smem_addr(fix + S::F_BQ + (sseg & 1) * S::BQ_BYTES);
       it.next(a);
-      ws_wait_nap(KREADY(t % S::NKR), (t / S::NKR) & 1, err, 64);
+      ws_wait(KREADY(t % S::NKR), (t / S::NKR) & 1, err);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t a0 = tmem + S::TM_AK + (t % S::KST) * 32;
@@ -374,14 +365,16 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     for (int u = 0; u < S::LA && u < ntiles; ++u) score(u);
     for (int t = 0; t < ntiles; ++t) {
       if (t + S::LA < ntiles) score(t + S::LA);
-      ws_wait_nap(PREADY(t & 1), (t >> 1) & 1, err, 64);
-      ws_wait_nap(VREADY(t & 1), (t >> 1) & 1, err, 64);
+      ws_wait(PREADY(t & 1), (t >> 1) & 1, err);
+      ws_wait(VREADY(t & 1), (t >> 1) & 1, err);
       tc_fence_after();
       if (lane == 0) {
         const uint32_t a0 = tmem + S::TM_AV + (t % S::VST) * 64;
         const uint32_t b0 = bp + (t & 1) * S::BP_BYTES;
-        const uint32_t d0 = tmem + S::TM_O + ((setbits >> (t & 3)) & 1u) * PP * S::NO;
-        const bool fresh = (firstbits >> (t & 3)) & 1u;  // the segment's first tile starts its sums
+        // accumulator set: (epilogue group of tile t, segment parity)
+        const uint32_t set = (S::NGRP == 2 ? (uint32_t)(t & 1) * OB : 0u) + ((setbits >> (t & 3)) & 1u);
+        const uint32_t d0 = tmem + S::TM_O + set * PP * S::NO;
+        const bool fresh = (firstbits >> (t & 3)) & 1u;  // the group's first tile of the segment starts its sums
         // 16 tokens per MMA; K step s accumulates into partial s % PP, so
         // consecutive MMAs of one accumulator are PP issues apart
 #pragma unroll
@@ -400,9 +393,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int s = t % ST;
       const uint8_t* raw = smem + s * S::STAGE + S::R_KC;
-      ws_wait_nap(FULL(s), (t / ST) & 1, err, 256);
+      ws_wait(FULL(s), (t / ST) & 1, err);
       // this key stage was read by the score UMMAs of tile t - KST
-      if (t >= S::KST) ws_wait_nap(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err, 256);
+      if (t >= S::KST) ws_wait(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err);
       tc_fence_after();
       if (it.first) {
         // query data of segment kseg into buffer kseg & 1: per head, delta =
@@ -413,7 +406,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         // buffer's two barriers see one phase per use, in order, so no parity wait
         // can pass on a later or an earlier phase.
         const int qb = kseg & 1;
-        if (kseg >= 2) ws_wait_nap(QFREE(qb), ((kseg - 2) >> 1) & 1, err, 256);
+        if (kseg >= 2) ws_wait(QFREE(qb), ((kseg - 2) >> 1) & 1, err);
         uint8_t* BQ = fix + S::F_BQ + qb * S::BQ_BYTES;
         float* qsum = reinterpret_cast<float*>(fix + S::F_QS + qb * G * 16);
         float* q0s = reinterpret_cast<float*>(fix + S::F_Q0 + qb * S::QV);
@@ -496,9 +489,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     for (int t = 0; t < ntiles; ++t) {
       const int s = t % ST;
       const uint8_t* row = smem + s * S::STAGE + S::R_VC + ch * S::VROW;
-      ws_wait_nap(FULL(s), (t / ST) & 1, err, 256);
+      ws_wait(FULL(s), (t / ST) & 1, err);
       // this value stage was read by the PV UMMAs of tile t - VST
-      if (t >= S::VST) ws_wait_nap(PVDONE((t - S::VST) & 1), ((t - S::VST) >> 1) & 1, err, 256);
+      if (t >= S::VST) ws_wait(PVDONE((t - S::VST) & 1), ((t - S::VST) >> 1) & 1, err);
       tc_fence_after();
       const uint32_t col = tl + S::TM_AV + (t % S::VST) * 64;
       constexpr int CHUNKS = S::VROW / 16;  // 4 (INT4: 32 tokens each) or 2 (INT2: 64 tokens each)
@@ -538,25 +531,37 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     }
   } else if (warp < 8 + S::EPI_WARPS) {
     // ================================================================ epilogue
-    const int e = tid - 256;    // 0 .. EPI_THREADS-1
-    const int j = e & 127;      // token (score phase) == tensor-memory lane == channel (PV phase)
-    const int part = e >> 7;    // head part: heads part*HH .. part*HH + HH - 1
-    const int wq = warp & 3;    // lane quarter == value group in the PV phase
-    const int bar_id = 1 + part;
+    // With NGRP epilogue groups, group g takes the tiles t with t % NGRP == g,
+    // so one tile's chain of waits and latencies can overlap another's; each
+    // group keeps its own online softmax and PV accumulator sets per segment and
+    // leaves its own partial, which the combine merges like any other split.
+    // (Two groups measured no faster than one at G = 4, so NGRP is 1.)
+    const int e = tid - 256;                  // 0 .. EPI_THREADS-1
+    const int grp = e / (128 * S::TPT);       // epilogue group
+    const int j = e & 127;                    // token (score phase) == tensor-memory lane == channel (PV phase)
+    const int part = (e >> 7) % S::TPT;       // head part: heads part*HH .. part*HH + HH - 1
+    const int wq = warp & 3;                  // lane quarter == value group in the PV phase
+    const int bar_id = 1 + grp * S::TPT + part;
     const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
     // K position of token j in the P' operand (the value conversion's pairing)
     const int pos = VB == 4 ? (j & ~7) + vpos_of<4>(j & 7) : (j & ~15) + vpos_of<2>(j & 15);
     float* red = reinterpret_cast<float*>(fix + S::F_RED);      // [2][TPT][4][16]
-    float* red2 = reinterpret_cast<float*>(fix + S::F_RED2);    // [TPT][4][16]
-    float* pend = reinterpret_cast<float*>(fix + S::F_PEND);    // [2][TPT][6 HH]
+    float* red2 = reinterpret_cast<float*>(fix + S::F_RED2) + grp * S::TPT * 64;         // [TPT][4][16]
+    float* pend = reinterpret_cast<float*>(fix + S::F_PEND) + grp * 2 * S::TPT * 6 * HH;  // [2][TPT][6 HH]
     const float NEG_INF = -__int_as_float(0x7f800000);
 
     float m_run[HH], l_acc[HH], zacc[kGroups][HH];
-    int nseg = 0;  // segments begun so far
-    int qb = 0;    // query buffer and PV accumulator set of the current segment (its parity)
-    // tiles t-1 and t-2: whether they ended a segment, its set and partial slot
-    bool last1 = false, last2 = false;
-    int set1 = 0, set2 = 0, slot1 = 0, slot2 = 0;
+    // this segment's query data for the thread's heads (per-group sums of the
+    // kept q, q_0, the step of the query pieces), held in registers when one
+    // thread takes a token's heads, else read from shared memory per tile
+    constexpr bool QREG = S::TPT == 1;
+    float qsg[QREG ? HH : 1][kGroups], q0r[QREG ? HH : 1], qdr[QREG ? HH : 1];
+    int nseg = 0;       // segments begun so far
+    int qb = 0;         // query buffer and PV accumulator set of the current segment (its parity)
+    int seg_tiles = 0;  // tiles of the current segment this group has taken
+    int last_own = 0;   // the last tile this group took
+    // segments waiting for their read-out: last tile into the set, set, partial slot
+    int pn = 0, p0_tile = 0, p0_set = 0, p0_slot = 0, p1_tile = 0, p1_set = 0, p1_slot = 0;
     bool ok = true;
 #pragma unroll
     for (int i = 0; i < HH; ++i) {
@@ -568,7 +573,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
     // this thread's PV accumulator columns (channel j, its HH heads) of partial 0 of set os
     auto obase = [&](int os) {
-      return tmem + lane_base + S::TM_O + os * PP * S::NO + wq * G + part * HH;
+      return tmem + lane_base + S::TM_O + (grp * OB + os) * PP * S::NO + wq * G + part * HH;
     };
     // sum of the PP partials of set os (after the last PV into it completed)
     auto load_out = [&](int os, float (&d)[HH]) {
@@ -612,9 +617,22 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       }
     };
 
+    // Read out the pending segments whose last PV tile is at least two tiles
+    // before tile u.  A set is next written by the group's first tile of the
+    // segment after next, at or after u, whose PV follows this tile's P'.
+    auto drain = [&](int u) {
+      while (pn > 0 && u >= p0_tile + 2) {
+        readout(p0_tile, p0_set, p0_slot);
+        p0_tile = p1_tile;
+        p0_set = p1_set;
+        p0_slot = p1_slot;
+        --pn;
+      }
+    };
+
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int k = t & 1;
-      const bool valid = it.i * kTile + j < it.len;
+      const bool own = S::NGRP == 1 || k == grp;
       if (it.first) {
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
@@ -623,10 +641,28 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) zacc[g][i] = 0.0f;
         }
+        seg_tiles = 0;
+        qb = nseg & 1;  // this segment's query data
+        ok &= ws_wait(QREADY(qb), (nseg >> 1) & 1, err);
+        ++nseg;
+        const float* qsum = reinterpret_cast<const float*>(fix + S::F_QS + qb * G * 16);
+        const float* q0s = reinterpret_cast<const float*>(fix + S::F_Q0 + qb * S::QV);
+        const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * S::QV);
+#pragma unroll
+        for (int i = 0; i < (QREG ? HH : 0); ++i) {
+          const int hh = part * HH + i;
+          const float4 qs = reinterpret_cast<const float4*>(qsum)[hh];
+          qsg[i][0] = qs.x;
+          qsg[i][1] = qs.y;
+          qsg[i][2] = qs.z;
+          qsg[i][3] = qs.w;
+          q0r[i] = CH0 ? q0s[hh] : 0.0f;
+          qdr[i] = qds[hh];
+        }
       }
-      // the segment that ended two tiles ago: its accumulator set is reused by the
-      // segment after next, whose first PV comes after this tile's
-      if (last2) readout(t - 2, set2, slot2);
+      if (own) {
+      drain(t);
+      const bool valid = it.i * kTile + j < it.len;
       // per-token scales, zeros and channel 0 from the ring (zero past the sequence end)
       const int s = t % ST;
       ok &= ws_wait(FULL(s), (t / ST) & 1, err);
@@ -651,14 +687,6 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         k0v = 0.0f;
       }
 
-      if (it.first) {  // this segment's query data
-        qb = nseg & 1;
-        ok &= ws_wait(QREADY(qb), (nseg >> 1) & 1, err);
-        ++nseg;
-      }
-      const float* qsum = reinterpret_cast<const float*>(fix + S::F_QS + qb * G * 16);
-      const float* q0s = reinterpret_cast<const float*>(fix + S::F_Q0 + qb * S::QV);
-      const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * S::QV);
       ok &= ws_wait(SDONE(t % S::SB), (t / S::SB) & 1, err);
       tc_fence_after();
       float sc[HH];
@@ -672,19 +700,35 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           tmem_ld4_wait<HH>(sbase, S::NS, d1);
           tmem_ld4_wait<HH>(sbase + G, S::NS, d2);
         }
+        const float* qsum = reinterpret_cast<const float*>(fix + S::F_QS + qb * G * 16);
+        const float* q0s = reinterpret_cast<const float*>(fix + S::F_Q0 + qb * S::QV);
+        const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * S::QV);
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           const int hh = part * HH + i;
-          const float4 qs = reinterpret_cast<const float4*>(qsum)[hh];
-          const float qsg[kGroups] = {qs.x, qs.y, qs.z, qs.w};
-          float dot = 0.0f, zt = CH0 ? q0s[hh] * k0v : 0.0f;
+          float qg[kGroups], q0, qd;
+          if constexpr (QREG) {
+#pragma unroll
+            for (int g = 0; g < kGroups; ++g) qg[g] = qsg[i][g];
+            q0 = q0r[i];
+            qd = qdr[i];
+          } else {
+            const float4 qs = reinterpret_cast<const float4*>(qsum)[hh];
+            qg[0] = qs.x;
+            qg[1] = qs.y;
+            qg[2] = qs.z;
+            qg[3] = qs.w;
+            q0 = CH0 ? q0s[hh] : 0.0f;
+            qd = qds[hh];
+          }
+          float dot = 0.0f, zt = CH0 ? q0 * k0v : 0.0f;
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) {
             const int dg = (int)d1[g][i] * 128 + (int)d2[g][i];  // exact: |dg| < 2^23
             dot = fmaf(ksz[g].x, (float)dg, dot);
-            zt = fmaf(ksz[g].y, qsg[g], zt);
+            zt = fmaf(ksz[g].y, qg[g], zt);
           }
-          sc[i] = fmaf(dot, qds[hh], zt);
+          sc[i] = fmaf(dot, qd, zt);
         }
       }
       tc_fence_before();
@@ -716,10 +760,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           alpha[i] = exp2f(m_run[i] - m_new[i]);
           m_run[i] = m_new[i];
         }
-        if (!it.first) {
-          // rescale the segment's PV sums so far (this thread: channel j, its heads)
-          // once the PV of tile t-1 has landed; tile t's PV adds after PREADY below
-          ok &= ws_wait(PVDONE((t - 1) & 1), ((t - 1) >> 1) & 1, err);
+        if (seg_tiles > 0) {
+          // rescale the group's PV sums of the segment so far (this thread: channel
+          // j, its heads) once the PV of its previous tile has landed; tile t's PV
+          // adds after PREADY below
+          ok &= ws_wait(PVDONE(last_own & 1), (last_own >> 1) & 1, err);
           tc_fence_after();
           const uint32_t base = obase(qb);
 #pragma unroll
@@ -787,9 +832,19 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       }
       fence_proxy_async();
       mbar_arrive(PREADY(k));
+      ++seg_tiles;
+      last_own = t;
+      } else if (it.last) {
+        mbar_arrive(QFREE(qb));  // done with this segment's query data
+      }
 
-      int slot_t = 0;
-      if (it.last) {
+      if (it.last && seg_tiles == 0) {
+        // no tile of this segment fell to this group: an empty partial (the combine skips it)
+        const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
+        if (j == 0)
+#pragma unroll
+          for (int i = 0; i < HH; ++i) a.part_ml[(size_t)slot * G + part * HH + i] = make_float2(NEG_INF, 0.0f);
+      } else if (it.last) {
         // segment totals over this part's 128 tokens (max, sum, value zero-point terms),
         // parked in shared memory until the segment's output is read out
         float* r2 = red2 + part * 64;
@@ -822,17 +877,20 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           }
         }
         named_sync(bar_id, 128);
-        slot_t = (int)it.bh(a) + blockIdx.x;
+        const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
+        if (pn == 0) {
+          p0_tile = last_own;
+          p0_set = qb;
+          p0_slot = slot;
+        } else {
+          p1_tile = last_own;
+          p1_set = qb;
+          p1_slot = slot;
+        }
+        ++pn;
       }
-      last2 = last1;
-      set2 = set1;
-      slot2 = slot1;
-      last1 = it.last;
-      set1 = qb;
-      slot1 = slot_t;
     }
-    if (ntiles >= 2 && last2) readout(ntiles - 2, set2, slot2);
-    readout(ntiles - 1, set1, slot1);  // the last tile always ends a segment
+    drain(ntiles + 2);
   }
   tc_fence_before();
   __syncthreads();
@@ -844,7 +902,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
 // Merges a unit's partials (one per CTA its tiles were spread over) into one
 // softmax over the whole sequence: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
-__global__ void __launch_bounds__(kHeadDim) k_combine(DecodeArgs a, int G) {
+__global__ void __launch_bounds__(kHeadDim) k_combine(DecodeArgs a, int G, int ngrp) {
   const int row = blockIdx.x;  // b * Hq + query head
   const int b = row / a.Hq, hq = row - b * a.Hq;
   const int h = hq / G, hl = hq - h * G;
@@ -861,12 +919,15 @@ __global__ void __launch_bounds__(kHeadDim) k_combine(DecodeArgs a, int G) {
     const int u = b * a.c.H + h;
     const int tu = tb + h * nt;
     const int c0 = tu / per, c1 = (tu + nt - 1) / per;
-    float M = -__int_as_float(0x7f800000);
-    for (int cc = c0; cc <= c1; ++cc) M = fmaxf(M, a.part_ml[(size_t)(u + cc) * G + hl].x);
+    // slots (u + CTA) * ngrp + epilogue group; an empty one has max -inf and is skipped
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    float M = NEG_INF;
+    for (int sl = (u + c0) * ngrp; sl < (u + c1 + 1) * ngrp; ++sl) M = fmaxf(M, a.part_ml[(size_t)sl * G + hl].x);
     float l = 0.0f, o = 0.0f;
-    for (int cc = c0; cc <= c1; ++cc) {
-      const size_t r = (size_t)(u + cc) * G + hl;
+    for (int sl = (u + c0) * ngrp; sl < (u + c1 + 1) * ngrp; ++sl) {
+      const size_t r = (size_t)sl * G + hl;
       const float2 v = a.part_ml[r];
+      if (v.x == NEG_INF) continue;
       const float w = exp2f(v.x - M);
       l = fmaf(w, v.y, l);
       o = fmaf(w, a.part_acc[r * kHeadDim + chn], o);
@@ -915,7 +976,8 @@ cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool decode_g_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
-int decode_slots(int B, int H) { return B * H + kCtas; }
+int decode_groups(int) { return 1; }
+int decode_slots(int B, int H, int G) { return (B * H + kCtas) * decode_groups(G); }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.c.k_bits == 4 && a.c.v_bits == 4) return launch_bits<4, 4>(a, s);
@@ -925,7 +987,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
-  k_combine<<<a.c.B * a.Hq, kHeadDim, 0, s>>>(a, a.Hq / a.c.H);
+  k_combine<<<a.c.B * a.Hq, kHeadDim, 0, s>>>(a, a.Hq / a.c.H, decode_groups(a.Hq / a.c.H));
   return cudaGetLastError();
 }
 
