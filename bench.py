@@ -211,6 +211,55 @@ def oracle_rate(leg: OracleLeg, budget_s: float, warmup: int = 1):
     return done / dt, done, dt
 
 
+# ------------------------------------------------------------------ replicas
+class Replicas:
+    """One process per GPU, launched by torchrun, each rank working on its own
+    batch: the units are independent, so the data path has no collective.  This
+    is the host-side glue: rank and world from the environment, a process group
+    for the barriers around the timed region, distinct seeds per rank, the step
+    time as the max over ranks, and the whole-job throughput."""
+
+    def __init__(self, backend: str = "nccl", timeout_s: float = 120.0):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.dist = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+            self.dist = dist
+
+    def seed(self, wl: workloads.Workload) -> int:
+        """Seed of this rank's synthetic batch (rank 0 draws the single-GPU inputs)."""
+        return workloads.BASE_SEED + wl.id + 1000 * self.rank
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float, device) -> float:
+        """The max of x over ranks (a device-timed duration: the slowest rank sets the step)."""
+        if self.dist is None:
+            return x
+        import torch
+
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def whole_job(self, units_per_rank: float, ms: float) -> float:
+        """Units all ranks processed per second, given the max-over-ranks step time."""
+        return self.world * units_per_rank / (ms * 1e-3)
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
 # ------------------------------------------------------------------ main arms
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
@@ -253,22 +302,15 @@ def workload_config(wl):
 
 def run_kvq(args):
     import torch
-    import torch.distributed as dist
 
     from quantized_attention_kvq_b200 import native
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    rep = Replicas()
+    world, rank, local = rep.world, rep.rank, rep.local
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = workloads.by_id(args.workload)
-    s = synth.Synth(workloads.BASE_SEED + wl.id + 1000 * rank, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt,
-                    wl.len_range)
+    s = synth.Synth(rep.seed(wl), wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt, wl.len_range)
 
     def up(a):
         if wl.fmt == "bf16":
@@ -319,25 +361,19 @@ def run_kvq(args):
     abytes = algorithmic_bytes(wl, masks_np, lens_np)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
+    rep.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         torch.cuda._sleep(50_000_000)  # let the host queue the steps ahead of the device
         for i in range(args.steps):
             step(evs[i])
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    rep.barrier()
     step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     split_ms = [e[1].elapsed_time(e[2]) for e in evs]
     select_ms = [e[0].elapsed_time(e[1]) for e in evs]
     combine_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    ms_step = sum(step_ms) / len(step_ms)
-    if world > 1:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = rep.max(sum(step_ms) / len(step_ms), dev)
 
     # -- end to end through the host-buffer entry point: q H2D, select, decode, out D2H
     q_pin = qd.cpu().pin_memory()
@@ -347,8 +383,7 @@ def run_kvq(args):
         flush.zero_()
         cache.decode_step_host(q_pin, lens, max_len, keep, scale, out_pin, ws2)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
+    rep.barrier()
     torch.cuda.synchronize()
     torch.cuda._sleep(50_000_000)
     for a, b in e2e_ev:
@@ -357,13 +392,8 @@ def run_kvq(args):
         cache.decode_step_host(q_pin, lens, max_len, keep, scale, out_pin, ws2)
         b.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    rep.barrier()
+    e2e_ms = rep.max(sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev), dev)
 
     peak, peak_src = measured_hbm_peak()
     split_avg = sum(split_ms) / len(split_ms)
@@ -381,7 +411,7 @@ def run_kvq(args):
     if rank == 0:
         line = {
             "metric": METRIC,
-            "value": world * wl.B / (ms_step * 1e-3),
+            "value": rep.whole_job(wl.B, ms_step),
             "unit": "tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -393,7 +423,7 @@ def run_kvq(args):
             "dtype": f"u{wl.k_bits}k/u{wl.v_bits}v codes, f32 accumulate",
             "data": "synthetic (seeded SplitMix64 + Box-Muller, workload recipe distributions)",
             "config": workload_config(wl),
-            "e2e": {"value": world * wl.B / (e2e_ms * 1e-3), "unit": "tokens/s",
+            "e2e": {"value": rep.whole_job(wl.B, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(q_pin.numel() * q_pin.element_size()),
                     "d2h_bytes_per_step": int(out_pin.numel() * 4)},
             "gpu_launches": args.steps * (2 + (1 if keep < 32 else 0)),
@@ -409,8 +439,7 @@ def run_kvq(args):
                                  "(CPU, AVX2); Dual-QK estimated 8.3x KV-read reduction at 128K"},
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    rep.close()
 
 
 def append_algorithmic_bytes(wl: workloads.Workload) -> int:
@@ -432,20 +461,12 @@ def run_append(args):
 
     from quantized_attention_kvq_b200 import native
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    rep = Replicas()
+    world, rank, local = rep.world, rep.rank, rep.local
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = workloads.by_id(args.workload)
-    s = synth.Synth(workloads.BASE_SEED + wl.id + 1000 * rank, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt,
-                    wl.len_range)
+    s = synth.Synth(rep.seed(wl), wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt, wl.len_range)
 
     def up(a):
         if wl.fmt == "bf16":
@@ -462,8 +483,7 @@ def run_append(args):
         cache.append(kd, vd, wl.offset)
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
+    rep.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         torch.cuda._sleep(50_000_000)
@@ -473,19 +493,16 @@ def run_append(args):
             cache.append(kd, vd, wl.offset)
             b_.record(stream)
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    ms = sum(a_.elapsed_time(b_) for a_, b_ in evs) / len(evs)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    rep.barrier()
+    ms = rep.max(sum(a_.elapsed_time(b_) for a_, b_ in evs) / len(evs), dev)
 
     # end to end: K/V rows from pinned host memory, then the append, then one
     # code word read back (the host sees the cache updated)
     k_pin, v_pin = kd.cpu().pin_memory(), vd.cpu().pin_memory()
     probe = torch.empty(16, dtype=torch.uint8).pin_memory()
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    rep.barrier()
+    torch.cuda.synchronize()
     for a_, b_ in e2e_ev:
         flush.zero_()
         a_.record(stream)
@@ -495,7 +512,8 @@ def run_append(args):
         probe.copy_(cache.k_codes[:16], non_blocking=True)
         b_.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a_.elapsed_time(b_) for a_, b_ in e2e_ev) / len(e2e_ev)
+    rep.barrier()
+    e2e_ms = rep.max(sum(a_.elapsed_time(b_) for a_, b_ in e2e_ev) / len(e2e_ev), dev)
 
     peak, peak_src = measured_hbm_peak()
     abytes = append_algorithmic_bytes(wl)
@@ -518,12 +536,12 @@ def run_append(args):
     if rank == 0:
         line = {
             "metric": "quantize-append tokens/sec & achieved HBM GB/s (fraction of B200 peak) at 1 GPU",
-            "value": world * wl.B * wl.T / (ms * 1e-3), "unit": "appended tokens/s", "n_gpus": world,
+            "value": rep.whole_job(wl.B * wl.T, ms), "unit": "appended tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": f"{wl.fmt} in, u{wl.k_bits}k/u{wl.v_bits}v codes out",
             "data": "synthetic (seeded SplitMix64 + Box-Muller, workload recipe distributions)",
             "config": workload_config(wl),
-            "e2e": {"value": world * wl.B * wl.T / (e2e_ms * 1e-3), "unit": "appended tokens/s",
+            "e2e": {"value": rep.whole_job(wl.B * wl.T, e2e_ms), "unit": "appended tokens/s",
                     "h2d_bytes_per_step": int(2 * kd.numel() * kd.element_size()), "d2h_bytes_per_step": 16},
             "gpu_launches": args.steps,
             "roofline": {"bound": "hbm", "kernel": "quantize-append (kvq_quantize_append)", "achieved": achieved,
@@ -534,8 +552,7 @@ def run_append(args):
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        torch.distributed.destroy_process_group()
+    rep.close()
 
 
 def main():
