@@ -171,6 +171,11 @@ double orc_bf16_value(uint16_t h) { return decode_format(h, 7, -126, 127, 8); }
 
 int32_t orc_quantize_group(const float* x, const uint8_t* include, int32_t n, int32_t bits, uint16_t* s16,
                            uint16_t* z16, uint8_t* codes, uint8_t* exempt, int64_t* clamped) {
+  return orc_quantize_group_clip(x, include, n, bits, 1.0f, s16, z16, codes, exempt, clamped);
+}
+
+int32_t orc_quantize_group_clip(const float* x, const uint8_t* include, int32_t n, int32_t bits, float clip,
+                                uint16_t* s16, uint16_t* z16, uint8_t* codes, uint8_t* exempt, int64_t* clamped) {
   const int L = (1 << bits) - 1;
   float mn = std::numeric_limits<float>::infinity(), mx = -std::numeric_limits<float>::infinity();
   for (int i = 0; i < n; ++i)
@@ -182,6 +187,10 @@ int32_t orc_quantize_group(const float* x, const uint8_t* include, int32_t n, in
   // scale and zero do not depend on which of the two came first.
   mn = mn + 0.0f;
   mx = mx + 0.0f;
+  // clipping ratio: both ends of the range move toward zero by the same factor
+  // (exact for clip = 1)
+  mn = clip * mn;
+  mx = clip * mx;
   // scale = (max - min) / L and zero = min, both computed in fp32 and stored
   // as fp16; values beyond the fp16 range saturate at +-65504.
   float range = mx - mn;
@@ -264,13 +273,17 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
         for (int i = 0; i < kGranule; ++i) word |= (uint32_t)codes[pg * kGranule + i] << (i * c->k_bits);
         store_k_word(c, b, h, pg, n, word);
       }
-      // ---- values: no rotation, quantize, pack into the channel rows of the block ----
-      for (int i = 0; i < d; ++i) xr[i] = v_new[row + i];
+      // ---- values: optional rotation, quantize with the clipping ratio, pack
+      // into the channel rows of the block ----
+      if (c->rotate_v)
+        orc_rotate(v_new + row, d, xr.data());
+      else
+        for (int i = 0; i < d; ++i) xr[i] = v_new[row + i];
       row_ex = 0;
       for (int g = 0; g < ngroups; ++g) {
         uint16_t s16, z16;
-        int gex = orc_quantize_group(&xr[g * kGroup], nullptr, kGroup, c->v_bits, &s16, &z16, &codes[g * kGroup],
-                                     &ex[g * kGroup], &st.v_clamped);
+        int gex = orc_quantize_group_clip(&xr[g * kGroup], nullptr, kGroup, c->v_bits, c->v_clip, &s16, &z16,
+                                          &codes[g * kGroup], &ex[g * kGroup], &st.v_clamped);
         size_t si = v_scale_index(c, b, h, n, g);
         c->v_scales[2 * si] = s16;
         c->v_scales[2 * si + 1] = z16;
@@ -429,6 +442,12 @@ void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t
       for (int ch = 0; ch < d; ++ch) o[ch] += s[j] * vhat[ch];
     }
     for (int ch = 0; ch < d; ++ch) o[ch] /= l;
+    if (c->rotate_v) {
+      // back from the rotated value basis: the orthonormal transform is its own inverse
+      orc_fwht(o, d);
+      const double inv = 1.0 / std::sqrt((double)d);
+      for (int ch = 0; ch < d; ++ch) o[ch] *= inv;
+    }
   }
 }
 

@@ -22,6 +22,11 @@
  *    n-bit scalar quantization of keys.
  *  - "CASK-Q" (decentralizedcompute.company), Method: scalar codes + FP16
  *    scales as the stored format.
+ *  - Dual-QK App. B.2 and Sec. 3.3: values rotated (the Hadamard part of the
+ *    rotation the pages take from OSCAR) and quantized with a 0.92 clipping
+ *    ratio; the ratio scales the group's minimum and maximum before the scale
+ *    and zero are formed (keys are not clipped).  The attention output then
+ *    leaves the rotated basis through the same orthonormal transform.
  *
  * Precision: FWHT in fp64 (natural Sylvester order), rotated values rounded
  * to fp32; quantization in fp32 with IEEE round-half-to-even; dequantization,
@@ -40,6 +45,8 @@ typedef struct {
   int32_t batch, kv_heads, head_dim, capacity;
   int32_t k_bits, v_bits; /* 2 or 4 */
   int32_t rotate_k, keep_ch0;
+  int32_t rotate_v; /* 1: values pass through the orthonormal Walsh-Hadamard transform before quantization */
+  float v_clip;     /* value clipping ratio in (0, 1]; 1 = no clipping                              */
   uint8_t* k_codes;   /* [B][Hkv][ceil(cap/128)][d/4][128] x (4*k_bits/8) bytes     */
   uint16_t* k_scales; /* [B][Hkv][ceil(cap/128)][d/32][128] x {fp16 scale, fp16 zero} */
   uint16_t* k_ch0;    /* [B][Hkv][cap] bf16, or NULL                        */
@@ -74,6 +81,10 @@ double orc_bf16_value(uint16_t h);
  */
 int32_t orc_quantize_group(const float* x, const uint8_t* include, int32_t n, int32_t bits, uint16_t* s16,
                            uint16_t* z16, uint8_t* codes, uint8_t* exempt, int64_t* clamped);
+/* the same with a clipping ratio: min and max are multiplied by clip (fp32)
+   before the scale and zero are formed; codes outside [0, L] clamp */
+int32_t orc_quantize_group_clip(const float* x, const uint8_t* include, int32_t n, int32_t bits, float clip,
+                                uint16_t* s16, uint16_t* z16, uint8_t* codes, uint8_t* exempt, int64_t* clamped);
 
 /*
  * Quantize k_new/v_new ([B][Hkv][n_new][d] fp32 values) and write them at
@@ -102,6 +113,9 @@ void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, i
 
 /*
  * Decode attention over the oracle cache for rows r = b*Hq + hq listed in
+ * `rows` (all B*Hq rows when rows == NULL); with rotate_v the output is the
+ * orthonormal Walsh-Hadamard transform (its own inverse) of the attention
+ * over the rotated values.  Remaining arguments:
  * `rows` (all B*Hq rows when rows == NULL).  q as in orc_select; lens[b]
  * tokens of sequence b; mask NULL = all channels.  out[r][d] fp64 (row-major
  * in the order of `rows`).

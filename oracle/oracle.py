@@ -20,6 +20,7 @@ _I32 = ctypes.c_int32
 class OrcCache(ctypes.Structure):
     _fields_ = [("batch", _I32), ("kv_heads", _I32), ("head_dim", _I32), ("capacity", _I32),
                 ("k_bits", _I32), ("v_bits", _I32), ("rotate_k", _I32), ("keep_ch0", _I32),
+                ("rotate_v", _I32), ("v_clip", ctypes.c_float),
                 ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P)]
 
 
@@ -45,6 +46,8 @@ def lib():
         L.orc_bf16_value.restype = ctypes.c_double
         L.orc_quantize_group.argtypes = [_P, _P, _I32, _I32, _P, _P, _P, _P, _P]
         L.orc_quantize_group.restype = _I32
+        L.orc_quantize_group_clip.argtypes = [_P, _P, _I32, _I32, ctypes.c_float, _P, _P, _P, _P, _P]
+        L.orc_quantize_group_clip.restype = _I32
         L.orc_quantize_append.argtypes = [ctypes.POINTER(OrcCache), _P, _P, _I32, _I32, ctypes.POINTER(OrcStats),
                                           _P, _P]
         L.orc_quantize_append.restype = _I32
@@ -100,7 +103,7 @@ def bf16_value(h: int) -> float:
     return lib().orc_bf16_value(int(h))
 
 
-def quantize_group(x, bits: int, include=None):
+def quantize_group(x, bits: int, include=None, clip: float = 1.0):
     """-> (s16 bits, z16 bits, codes, exempt flags, group_exempt, clamped count)"""
     xi = np.ascontiguousarray(x, dtype=np.float32)
     n = xi.size
@@ -110,24 +113,26 @@ def quantize_group(x, bits: int, include=None):
     codes = np.zeros(n, np.uint8)
     ex = np.zeros(n, np.uint8)
     clamped = ctypes.c_int64(0)
-    gex = lib().orc_quantize_group(_p(xi), _p(inc), n, bits, ctypes.byref(s), ctypes.byref(z), _p(codes), _p(ex),
-                                   ctypes.byref(clamped))
+    gex = lib().orc_quantize_group_clip(_p(xi), _p(inc), n, bits, float(clip), ctypes.byref(s), ctypes.byref(z),
+                                        _p(codes), _p(ex), ctypes.byref(clamped))
     return s.value, z.value, codes, ex, gex, clamped.value
 
 
 class Cache:
     """Host copy of the packed cache, written by the oracle."""
 
-    def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0):
+    def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, rotate_v=0, v_clip=1.0):
         self.B, self.Hkv, self.d, self.capacity = B, Hkv, d, capacity
         self.k_bits, self.v_bits, self.rotate_k, self.keep_ch0 = k_bits, v_bits, rotate_k, keep_ch0
+        self.rotate_v, self.v_clip = rotate_v, v_clip
         blocked = -(-capacity // 128) * 128  # codes are stored in blocks of 128 tokens
         self.k_codes = np.zeros(B * Hkv * (d // 4) * blocked * (4 * k_bits // 8), np.uint8)
         self.k_scales = np.zeros(B * Hkv * (d // 32) * blocked * 2, np.uint16)
         self.k_ch0 = np.zeros(B * Hkv * capacity, np.uint16) if keep_ch0 else None
         self.v_codes = np.zeros(B * Hkv * d * blocked * v_bits // 8, np.uint8)  # channel rows per block
         self.v_scales = np.zeros(B * Hkv * capacity * (d // 32) * 2, np.uint16)
-        self.struct = OrcCache(B, Hkv, d, capacity, k_bits, v_bits, rotate_k, keep_ch0, _p(self.k_codes),
+        self.struct = OrcCache(B, Hkv, d, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v, v_clip,
+                               _p(self.k_codes),
                                _p(self.k_scales), _p(self.k_ch0), _p(self.v_codes), _p(self.v_scales))
 
     def append(self, k_new: np.ndarray, v_new: np.ndarray, offset: int, want_exempt: bool = False):
