@@ -181,7 +181,8 @@ class OracleLeg:
         self.caches = []
         self.q = orc.as_f32(q)
         for b in range(n_seqs):
-            c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0)
+            c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
+                          wl.v_clip)
             k = np.stack([s.k_slice(b, h) for h in range(wl.Hkv)])[None]
             v = np.stack([s.v_slice(b, h) for h in range(wl.Hkv)])[None]
             c.append(orc.as_f32(k), orc.as_f32(v), wl.offset)
@@ -296,7 +297,8 @@ def workload_config(wl):
     return {"workload": wl.name, "batch": wl.B, "q_heads": wl.Hq, "kv_heads": wl.Hkv, "head_dim": wl.d,
             "seq_len": wl.T if wl.len_range is None else f"U[{wl.len_range[0]},{wl.len_range[1]}]",
             "k_bits": wl.k_bits, "v_bits": wl.v_bits, "group": 32, "rotate_k": wl.rotate_k,
-            "keep_ch0": wl.keep_ch0, "keep_groups": wl.keep_groups, "input_dtype": wl.fmt,
+            "keep_ch0": wl.keep_ch0, "keep_groups": wl.keep_groups, "rotate_v": wl.rotate_v, "v_clip": wl.v_clip,
+            "input_dtype": wl.fmt,
             "l2": "flushed between steps (memset of 2x L2)", "parallelism": "replicas (one batch per GPU)"}
 
 
@@ -319,7 +321,8 @@ def run_kvq(args):
 
     # -- resident cache (built by the append kernel, not timed here)
     q_np = s.q()
-    cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev)
+    cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev,
+                            rotate_v=wl.rotate_v, v_clip=wl.v_clip)
     for b in range(wl.B):  # one sequence at a time keeps host memory small
         kd = up(np.stack([s.k_slice(b, h) for h in range(wl.Hkv)]))
         vd = up(np.stack([s.v_slice(b, h) for h in range(wl.Hkv)]))
@@ -474,7 +477,8 @@ def run_append(args):
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
     kd, vd = up(s.k_full()), up(s.v_full())
-    cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev)
+    cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev,
+                            rotate_v=wl.rotate_v, v_clip=wl.v_clip)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -522,7 +526,8 @@ def run_append(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import oracle as orc
 
-        c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0)
+        c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
+                      wl.v_clip)
         k1 = orc.as_f32(np.stack([s.k_slice(0, h) for h in range(wl.Hkv)])[None])
         v1 = orc.as_f32(np.stack([s.v_slice(0, h) for h in range(wl.Hkv)])[None])
         t0 = time.perf_counter()
@@ -567,7 +572,7 @@ def main():
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
-    elif args.workload == 3:
+    elif workloads.by_id(args.workload).kind == "append":
         run_append(args)
     else:
         run_kvq(args)

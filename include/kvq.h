@@ -83,6 +83,10 @@ typedef struct {
   int32_t k_bits, v_bits, group_size, prune_granule;
   int32_t rotate_k; /* 1: keys (and queries) pass through the orthonormal Walsh-Hadamard transform */
   int32_t keep_ch0; /* 1: rotated channel 0 of each key is kept in bf16, unquantized               */
+  int32_t rotate_v; /* 1: values pass through the orthonormal Walsh-Hadamard transform before they
+                       are quantized, and decode outputs are rotated back [DQK App. B.2]           */
+  float v_clip;     /* value clipping ratio in (0, 1]: each value group's min and max are scaled
+                       by it before scale and zero are formed, values beyond saturate; 1 = none  */
   void* k_codes;
   void* k_scales;
   void* k_ch0;
@@ -110,8 +114,10 @@ KVQ_API kvq_status kvq_cache_sizes(const kvq_cache* cache, size_t bytes_out[5]);
  * bf16 when keep_ch0; then per token and per 32-channel group
  * scale = fp16((max - min) / L), zero = fp16(min), L = 2^bits - 1,
  * code = clamp(round_half_even((x - zero) / scale), 0, L) with IEEE fp32
- * subtract and divide [DQK Sec. 3.3].  Values: same quantizer, no rotation
- * [DQK App. B.2].  n_new == 0 is a no-op.
+ * subtract and divide [DQK Sec. 3.3].  Values: the same quantizer [DQK App.
+ * B.2], after the same rotation when rotate_v, with min and max multiplied by
+ * v_clip (fp32) before scale and zero are formed (keys are not clipped).
+ * n_new == 0 is a no-op.
  */
 KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new, const void* v_new,
                                        kvq_dtype dtype, int32_t n_new, int32_t offset, void* stream);

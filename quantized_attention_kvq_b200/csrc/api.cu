@@ -21,6 +21,7 @@ kvq_status check_shape(const kvq_cache* c) {
   if (!c) return KVQ_ERR_INVALID_ARG;
   if (c->batch < 1 || c->kv_heads < 1 || c->capacity < 1 || c->head_dim < 1) return KVQ_ERR_INVALID_ARG;
   if ((c->rotate_k != 0 && c->rotate_k != 1) || (c->keep_ch0 != 0 && c->keep_ch0 != 1)) return KVQ_ERR_INVALID_ARG;
+  if ((c->rotate_v != 0 && c->rotate_v != 1) || !(c->v_clip > 0.0f && c->v_clip <= 1.0f)) return KVQ_ERR_INVALID_ARG;
   if (c->head_dim != kHeadDim || c->group_size != kGroup || c->prune_granule != kGranule) return KVQ_ERR_UNSUPPORTED;
   if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return KVQ_ERR_UNSUPPORTED;
   if (c->capacity % kKeyBlock != 0) return KVQ_ERR_UNSUPPORTED;
@@ -52,6 +53,8 @@ CacheView view(const kvq_cache* c) {
   v.v_bits = c->v_bits;
   v.rotate = c->rotate_k;
   v.keep_ch0 = c->keep_ch0;
+  v.rotate_v = c->rotate_v;
+  v.v_clip = c->v_clip;
   v.kc = static_cast<uint8_t*>(c->k_codes);
   v.ks = static_cast<__half2*>(c->k_scales);
   v.k0 = static_cast<__nv_bfloat16*>(c->k_ch0);

@@ -6,7 +6,8 @@
 // quantization group g.  Keys: fp64 Walsh-Hadamard butterflies (Dual-QK
 // summary Sec. 1; gist.science KQV scheme), optional bf16 channel 0 (Dual-QK
 // Sec. 3.3, App. C.3), per-32-channel asymmetric quantization (Dual-QK
-// Sec. 3.3).  Values: the same quantizer without rotation (Dual-QK App. B.2).
+// Sec. 3.3).  Values: the same quantizer, optionally after the same rotation
+// and with a clipping ratio on each group's range (Dual-QK App. B.2).
 // Both code kinds are staged in shared memory and leave channel-major: key
 // words one coalesced row per pruning group, value codes packed into each
 // channel's row of the 128-token block.  Only tokens [offset, offset+n_new)
@@ -66,8 +67,9 @@ __device__ __forceinline__ uint32_t compress_codes(uint32_t x) {
 }
 
 // Quantize one 32-channel group held by this lane (v[0..31]); skip0: element 0
-// is kept out of the range and gets code 0.  Returns the fp16 (scale, zero)
-// pair; byte j of packed[p] is the code of element 4p + j.
+// is kept out of the range and gets code 0; clip: the clipping ratio applied to
+// the group's minimum and maximum.  Returns the fp16 (scale, zero) pair; byte j
+// of packed[p] is the code of element 4p + j.
 //
 // The code is round_half_even((x - zero) / scale) clamped to [0, L], the
 // quotient as IEEE fp32 division gives it.  It is formed as
@@ -77,11 +79,13 @@ __device__ __forceinline__ uint32_t compress_codes(uint32_t x) {
 // lies within 1e-5 of a rounding boundary (k + 1/2) the group is coded again
 // with the IEEE division for such elements, so every code is the division's.
 template <int BITS>
-__device__ __forceinline__ __half2 quantize_group32(const float (&v)[32], bool skip0, uint32_t (&packed)[8]) {
+__device__ __forceinline__ __half2 quantize_group32(const float (&v)[32], bool skip0, float clip,
+                                                   uint32_t (&packed)[8]) {
   const float v0 = skip0 ? v[1] : v[0];
-  // -0 and +0 are the same extreme; take it as +0 so the stored bits are unique
-  const float mn = __fadd_rn(reduce32<false>(v0, v), 0.0f);
-  const float mx = __fadd_rn(reduce32<true>(v0, v), 0.0f);
+  // -0 and +0 are the same extreme; take it as +0 so the stored bits are unique;
+  // then the clipping ratio scales both ends (exact for clip = 1)
+  const float mn = __fmul_rn(clip, __fadd_rn(reduce32<false>(v0, v), 0.0f));
+  const float mx = __fmul_rn(clip, __fadd_rn(reduce32<true>(v0, v), 0.0f));
   constexpr int L = (1 << BITS) - 1;
   const float s32 = fminf(__fdiv_rn(__fsub_rn(mx, mn), (float)L), 65504.0f);
   const float zc = fminf(fmaxf(mn, -65504.0f), 65504.0f);
@@ -172,6 +176,39 @@ __device__ __forceinline__ void transpose_bytes4(const uint32_t (&in)[4], uint32
   out[3] = __byte_perm(t1, t3, 0x7632);
 }
 
+// Orthonormal Walsh-Hadamard transform of one 128-channel row held by four
+// lanes, lane g holding channels 32g .. 32g+31: butterflies in fp64, natural
+// Sylvester order (stage h pairs channels i and i + h, i & h == 0, -> (a + b,
+// a - b)); the stages below 32 stay inside the lane, 32 and 64 pair lanes g ^ 1
+// and g ^ 2; then one fp64 multiply by 1/sqrt(128) and a round to fp32.  All
+// 32 lanes of the warp take part.
+__device__ __forceinline__ void rotate_row_4lanes(float (&v)[32], int g, double inv_sqrt_d) {
+  double x[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) x[i] = v[i];
+#pragma unroll
+  for (int hs = 1; hs < 32; hs <<= 1)
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if ((i & hs) == 0) {
+        const double u = x[i], w = x[i + hs];
+        x[i] = __dadd_rn(u, w);
+        x[i + hs] = __dsub_rn(u, w);
+      }
+#pragma unroll
+  for (int m = 1; m <= 2; m <<= 1) {
+    const bool upper = (g & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      // lower lane: x + o; upper lane: o - x = o + (-x), the same IEEE sum
+      const double o = __shfl_xor_sync(kFull, x[i], m);
+      x[i] = __dadd_rn(upper ? -x[i] : x[i], o);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __double2float_rn(__dmul_rn(x[i], inv_sqrt_d));
+}
+
 template <int KB, int VB, bool ROT, bool CH0, typename In>
 __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(AppendArgs a) {
   constexpr int TPW = 32 / VB;            // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
@@ -215,39 +252,12 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
   float kx[32];
   widen(kraw, kx);
 
-  // ---- key row: Walsh-Hadamard butterflies in fp64, natural Sylvester order
-  // (stage h pairs channels i and i + h, i & h == 0, -> (a + b, a - b)); the
-  // stages below 32 stay inside the lane, 32 and 64 pair lanes g ^ 1, g ^ 2
-  if (ROT) {
-    double x[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[i] = kx[i];
-#pragma unroll
-    for (int hs = 1; hs < 32; hs <<= 1)
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if ((i & hs) == 0) {
-          const double u = x[i], w = x[i + hs];
-          x[i] = __dadd_rn(u, w);
-          x[i + hs] = __dsub_rn(u, w);
-        }
-#pragma unroll
-    for (int m = 1; m <= 2; m <<= 1) {
-      const bool upper = (g & m) != 0;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        // lower lane: x + o; upper lane: o - x = o + (-x), the same IEEE sum
-        const double o = __shfl_xor_sync(kFull, x[i], m);
-        x[i] = __dadd_rn(upper ? -x[i] : x[i], o);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) kx[i] = __double2float_rn(__dmul_rn(x[i], a.inv_sqrt_d));
-  }
+  // ---- key row: rotated, then quantized (keys are not clipped)
+  if (ROT) rotate_row_4lanes(kx, g, a.inv_sqrt_d);
   uint32_t code[8];
   {
     const bool skip0 = CH0 && g == 0;
-    const __half2 sz = quantize_group32<KB>(kx, skip0, code);
+    const __half2 sz = quantize_group32<KB>(kx, skip0, 1.0f, code);
 #pragma unroll
     for (int p = 0; p < 8; ++p) kw[8 * g + p][tt] = (uint16_t)compress_codes<KB>(code[p]);
     if (active) {
@@ -255,11 +265,13 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
       if (skip0) c.k0[bh * c.cap + w0 + tt] = __float2bfloat16_rn(kx[0]);
     }
   }
-  // ---- value row: the same quantizer, no rotation; codes as bytes, scales token-major
+  // ---- value row: optionally rotated, the same quantizer with the clipping
+  // ratio; codes as bytes, scales token-major
   {
     float vx[32];
     widen(vraw, vx);
-    const __half2 sz = quantize_group32<VB>(vx, false, code);
+    if (c.rotate_v) rotate_row_4lanes(vx, g, a.inv_sqrt_d);  // uniform across the CTA
+    const __half2 sz = quantize_group32<VB>(vx, false, c.v_clip, code);
     if (!active) {
 #pragma unroll
       for (int p = 0; p < 8; ++p) code[p] = 0;  // tokens outside the append contribute zero bits

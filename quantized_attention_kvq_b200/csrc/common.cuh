@@ -117,7 +117,8 @@ __host__ __device__ __forceinline__ size_t v_row_offset(size_t bh, int cap, int 
 
 // ---------------------------------------------------------------- launch plumbing
 struct CacheView {
-  int B, H, cap, k_bits, v_bits, rotate, keep_ch0;
+  int B, H, cap, k_bits, v_bits, rotate, keep_ch0, rotate_v;
+  float v_clip;
   uint8_t* kc;
   __half2* ks;
   __nv_bfloat16* k0;

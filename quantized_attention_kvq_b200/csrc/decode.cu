@@ -686,6 +686,10 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         for (int g = 0; g < kGroups; ++g) ksz[g] = vsz[g] = make_float2(0.0f, 0.0f);
         k0v = 0.0f;
       }
+      // the value operand holds c - L/2, so the zero point carries the L/2 steps
+      constexpr float kHalfL = ((1 << VB) - 1) * 0.5f;
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) vsz[g].y = fmaf(kHalfL, vsz[g].x, vsz[g].y);
 
       ok &= ws_wait(SDONE(t % S::SB), (t / S::SB) & 1, err);
       tc_fence_after();
@@ -901,7 +905,8 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 }
 
 // Merges a unit's partials (one per CTA its tiles were spread over) into one
-// softmax over the whole sequence: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// softmax over the whole sequence: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,
+// rotated back into the value basis when the values were stored rotated.
 __global__ void __launch_bounds__(kHeadDim) k_combine(DecodeArgs a, int G, int ngrp) {
   const int row = blockIdx.x;  // b * Hq + query head
   const int b = row / a.Hq, hq = row - b * a.Hq;
@@ -933,6 +938,20 @@ __global__ void __launch_bounds__(kHeadDim) k_combine(DecodeArgs a, int G, int n
       o = fmaf(w, a.part_acc[r * kHeadDim + chn], o);
     }
     out = o / l;
+  }
+  if (a.c.rotate_v) {
+    // back from the rotated value basis: the orthonormal Walsh-Hadamard
+    // transform is its own inverse (fp32 butterflies over the 128 channels)
+    __shared__ float x[kHeadDim];
+    x[chn] = out;
+    for (int hs = 1; hs < kHeadDim; hs <<= 1) {
+      __syncthreads();
+      const float mine = x[chn], other = x[chn ^ hs];
+      __syncthreads();
+      x[chn] = (chn & hs) ? other - mine : mine + other;
+    }
+    __syncthreads();
+    out = x[chn] * (float)a.inv_sqrt_d;
   }
   a.out[(size_t)row * kHeadDim + chn] = out;
 }

@@ -407,41 +407,48 @@ __device__ __forceinline__ void tmem_st_n<8>(uint32_t taddr, const uint32_t (&r)
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- code -> f16
-// Eight 4-bit codes n0..n7 (n_i in bits 4i..4i+3 of x) -> exact f16 integers,
-// returned as half2 pairs (n0,n4) (n1,n5) (n2,n6) (n3,n7).  Each nibble is
-// OR-ed into the mantissa of 1024.0 (0x6400), then 1024 (or 16*1024 for the
-// high nibble of a byte, rescaled by 1/16) is subtracted; all exact in f16.
+// Value codes enter the PV MMA centred, as c - L/2 (exact f16 values): the
+// products then average out instead of all being positive, which keeps the
+// fp32 accumulator near the size of the result (the zero point takes the L/2).
+//
+// Eight 4-bit codes n0..n7 (n_i in bits 4i..4i+3 of x) -> f16 (n_i - 7.5) as
+// half2 pairs (n0,n4) (n1,n5) (n2,n6) (n3,n7).  Each nibble is moved to bits
+// 4..7 of its half and OR-ed into the mantissa of 1024.0 (0x6400), giving
+// 1024 + 16 n; one fma (x 1/16, - 71.5) leaves n - 7.5; all exact in f16.
 __device__ __forceinline__ void codes4_to_f16(uint32_t x, uint32_t (&r)[4]) {
   const uint32_t magic = 0x64006400u;
+  const uint32_t sel = 0x00F000F0u;
   uint32_t a, b, c, d;
-  const uint32_t x2 = x >> 8;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(a) : "r"(x), "r"(0x000F000Fu), "r"(magic));
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(b) : "r"(x), "r"(0x00F000F0u), "r"(magic));
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(c) : "r"(x2), "r"(0x000F000Fu), "r"(magic));
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(x2), "r"(0x00F000F0u), "r"(magic));
-  const uint32_t sub = 0x64006400u;    // (1024, 1024)
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(a) : "r"(x << 4), "r"(sel), "r"(magic));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(b) : "r"(x), "r"(sel), "r"(magic));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(c) : "r"(x >> 4), "r"(sel), "r"(magic));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(x >> 8), "r"(sel), "r"(magic));
   const uint32_t mul16 = 0x2C002C00u;  // (1/16, 1/16)
-  const uint32_t add64 = 0xD400D400u;  // (-64, -64)
-  asm("sub.f16x2 %0, %1, %2;" : "=r"(r[0]) : "r"(a), "r"(sub));
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[1]) : "r"(b), "r"(mul16), "r"(add64));
-  asm("sub.f16x2 %0, %1, %2;" : "=r"(r[2]) : "r"(c), "r"(sub));
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[3]) : "r"(d), "r"(mul16), "r"(add64));
+  const uint32_t add = 0xD478D478u;    // (-71.5, -71.5)
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[0]) : "r"(a), "r"(mul16), "r"(add));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[1]) : "r"(b), "r"(mul16), "r"(add));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[2]) : "r"(c), "r"(mul16), "r"(add));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[3]) : "r"(d), "r"(mul16), "r"(add));
 }
 
-// Sixteen 2-bit codes f0..f15 (f_i in bits 2i..2i+1) -> exact f16 integers as
-// half2 pairs (f0,f8) (f1,f9) ... (f7,f15).
+// Sixteen 2-bit codes f0..f15 (f_i in bits 2i..2i+1) -> f16 (f_i - 1.5) as
+// half2 pairs (f0,f8) (f1,f9) ... (f7,f15).  Field k (k = 1..3) of each half,
+// OR-ed in place into 1024.0, is 1024 + 4^k f; one fma (x 4^-k, -1024 4^-k -
+// 1.5) leaves f - 1.5.  Field 0 is first moved to field 1's bits (-1025.5 is
+// not an f16 value).  All exact in f16.
 __device__ __forceinline__ void codes2_to_f16(uint32_t x, uint32_t (&r)[8]) {
   const uint32_t magic = 0x64006400u;
-  // field k of the low byte pair sits at bit 2k of each half: value 1024 + 4^k f
-  const uint32_t mul[4] = {0x3C003C00u, 0x34003400u, 0x2C002C00u, 0x24002400u};  // 1, 1/4, 1/16, 1/64
-  const uint32_t add[4] = {0xE400E400u, 0xDC00DC00u, 0xD400D400u, 0xCC00CC00u};  // -1024, -256, -64, -16
+  const uint32_t mul[4] = {0x34003400u, 0x34003400u, 0x2C002C00u, 0x24002400u};  // 1/4, 1/4, 1/16, 1/64
+  const uint32_t add[4] = {0xDC06DC06u, 0xDC06DC06u, 0xD418D418u, 0xCC60CC60u};  // -257.5, -257.5, -65.5, -17.5
   const uint32_t xs[2] = {x, x >> 8};
 #pragma unroll
   for (int half = 0; half < 2; ++half)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint32_t t;
-      asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(t) : "r"(xs[half]), "r"(0x00030003u << (2 * k)), "r"(magic));
+      const uint32_t src = k == 0 ? xs[half] << 2 : xs[half];
+      const uint32_t m = 0x00030003u << (2 * (k == 0 ? 1 : k));
+      asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(t) : "r"(src), "r"(m), "r"(magic));
       asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r[half * 4 + k]) : "r"(t), "r"(mul[k]), "r"(add[k]));
     }
 }

@@ -29,7 +29,7 @@ _I32 = ctypes.c_int32
 class KvqCacheStruct(ctypes.Structure):
     _fields_ = [("batch", _I32), ("kv_heads", _I32), ("head_dim", _I32), ("capacity", _I32),
                 ("k_bits", _I32), ("v_bits", _I32), ("group_size", _I32), ("prune_granule", _I32),
-                ("rotate_k", _I32), ("keep_ch0", _I32),
+                ("rotate_k", _I32), ("keep_ch0", _I32), ("rotate_v", _I32), ("v_clip", ctypes.c_float),
                 ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P)]
 
 
@@ -107,8 +107,8 @@ def _stream(stream) -> int | None:
     return stream.cuda_stream
 
 
-def describe(B, H, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, d=128) -> KvqCacheStruct:
-    return KvqCacheStruct(B, H, d, capacity, k_bits, v_bits, 32, 4, rotate_k, keep_ch0)
+def describe(B, H, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, d=128, rotate_v=0, v_clip=1.0) -> KvqCacheStruct:
+    return KvqCacheStruct(B, H, d, capacity, k_bits, v_bits, 32, 4, rotate_k, keep_ch0, rotate_v, v_clip)
 
 
 def cache_sizes(desc: KvqCacheStruct) -> list[int]:
@@ -121,8 +121,8 @@ class KVQCache:
     """Packed quantized KV cache in device memory (torch-allocated, library-laid-out)."""
 
     def __init__(self, B: int, H: int, capacity: int, k_bits: int, v_bits: int, rotate_k: int = 1,
-                 keep_ch0: int = 0, device="cuda", zero: bool = True):
-        self.desc = describe(B, H, capacity, k_bits, v_bits, rotate_k, keep_ch0)
+                 keep_ch0: int = 0, device="cuda", zero: bool = True, rotate_v: int = 0, v_clip: float = 1.0):
+        self.desc = describe(B, H, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v=rotate_v, v_clip=v_clip)
         sizes = cache_sizes(self.desc)
         alloc = torch.zeros if zero else torch.empty
         self.k_codes = alloc(sizes[0], dtype=torch.uint8, device=device)
@@ -142,7 +142,7 @@ class KVQCache:
         with the sequence outermost, so this is a pointer offset per array."""
         per = [x // self.B for x in cache_sizes(self.desc)]
         d = describe(1, self.H, self.capacity, self.desc.k_bits, self.desc.v_bits, self.desc.rotate_k,
-                     self.desc.keep_ch0)
+                     self.desc.keep_ch0, rotate_v=self.desc.rotate_v, v_clip=self.desc.v_clip)
         d.k_codes = self.desc.k_codes + b * per[0]
         d.k_scales = self.desc.k_scales + b * per[1]
         d.k_ch0 = self.desc.k_ch0 + b * per[2] if self.desc.keep_ch0 else None

@@ -1,4 +1,4 @@
-"""The five synthetic workloads of the quantized-KV decode path.
+"""The synthetic workloads of the quantized-KV decode path.
 
 Each names its shapes, code widths and flags; inputs are drawn by
 ``synth.Synth`` with seed ``base_seed + id``.
@@ -26,6 +26,9 @@ class Workload:
     keep_ch0: int
     keep_groups: int    # channel groups of 4 kept by the query-channel pruning (32 = none)
     len_range: tuple | None = None  # per-sequence lengths U[lo, hi] (ragged), else all T
+    rotate_v: int = 0   # values rotated before quantization (decode output rotated back)
+    v_clip: float = 1.0  # value clipping ratio on each group's min and max
+    kind: str = "decode"  # what bench.py times: "decode" or "append"
 
     @property
     def G(self) -> int:
@@ -36,9 +39,15 @@ WORKLOADS = [
     Workload(0, "tiny_int4", 1, 1, 1, 128, 1024, 1024, 0, "f32", 4, 4, 1, 0, 32),
     Workload(1, "gqa_int4_b8_h32x8_n32k", 8, 32, 8, 128, 32768, 32768, 0, "bf16", 4, 4, 1, 0, 32),
     Workload(2, "dualqk_int2_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16", 2, 2, 1, 1, 19),
-    Workload(3, "append_b16_h8_t4096_at8192", 16, 8, 8, 128, 4096, 12288, 8192, "bf16", 4, 2, 1, 0, 32),
+    Workload(3, "append_b16_h8_t4096_at8192", 16, 8, 8, 128, 4096, 12288, 8192, "bf16", 4, 2, 1, 0, 32,
+             kind="append"),
     Workload(4, "ragged_b64_h64x8_n1k16k_keep24", 64, 64, 8, 128, 16384, 16384, 0, "bf16", 4, 2, 1, 1, 24,
              (1024, 16384)),
+    # values rotated and clipped at 0.92 before INT2 quantization (Dual-QK App. B.2)
+    Workload(5, "dualqk_int2_vrot_clip092_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16", 2, 2,
+             1, 1, 19, rotate_v=1, v_clip=0.92),
+    Workload(6, "append_vrot_clip092_b16_h8_t4096_at8192", 16, 8, 8, 128, 4096, 12288, 8192, "bf16", 4, 2, 1, 0,
+             32, rotate_v=1, v_clip=0.92, kind="append"),
 ]
 
 BASE_SEED = 0

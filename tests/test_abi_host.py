@@ -63,13 +63,24 @@ def test_cache_sizes_follow_layout(L):
     ("group_size", 64, native.KVQ_ERR_UNSUPPORTED), ("prune_granule", 8, native.KVQ_ERR_UNSUPPORTED),
     ("batch", 0, native.KVQ_ERR_INVALID_ARG), ("rotate_k", 2, native.KVQ_ERR_INVALID_ARG),
     ("k_codes", 0, native.KVQ_ERR_INVALID_ARG), ("k_ch0", 0, native.KVQ_ERR_INVALID_ARG),
-    ("v_scales", FAKE + 4, native.KVQ_ERR_INVALID_ARG),
+    ("v_scales", FAKE + 4, native.KVQ_ERR_INVALID_ARG), ("rotate_v", 2, native.KVQ_ERR_INVALID_ARG),
+    ("v_clip", 0.0, native.KVQ_ERR_INVALID_ARG), ("v_clip", 1.5, native.KVQ_ERR_INVALID_ARG),
+    ("v_clip", float("nan"), native.KVQ_ERR_INVALID_ARG), ("v_clip", -0.5, native.KVQ_ERR_INVALID_ARG),
 ])
 def test_bad_cache_rejected(L, field, value, status):
     d = desc()
     setattr(d, field, value)
     rc = L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 0, None)
     assert rc == status
+
+
+def test_rotated_clipped_values_are_accepted(L):
+    # the flags leave the layout alone: same sizes, and the host checks pass
+    # (the enqueue itself is left to the GPU tests)
+    d = desc(rotate_v=1, v_clip=0.92)
+    assert native.cache_sizes(d) == native.cache_sizes(desc())
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 250, None) == \
+        native.KVQ_ERR_CAPACITY
 
 
 def test_append_argument_checks(L):

@@ -25,11 +25,11 @@ def draw(seed, B, Hq, H, T, fmt):
     return q, k, v
 
 
-def build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset=0, chunks=None):
+def build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset=0, chunks=None, rotate_v=0, v_clip=1.0):
     """Append the same inputs through the C ABI and through the oracle.
     Returns (gpu cache, oracle cache, near-tie row flags, comparison geometry)."""
-    gc = native.KVQCache(B, H, cap, kb, vb, rot, ch0)
-    oc = orc.Cache(B, H, 128, cap, kb, vb, rot, ch0)
+    gc = native.KVQCache(B, H, cap, kb, vb, rot, ch0, rotate_v=rotate_v, v_clip=v_clip)
+    oc = orc.Cache(B, H, 128, cap, kb, vb, rot, ch0, rotate_v=rotate_v, v_clip=v_clip)
     T = k.shape[2]
     chunks = chunks or [T]
     flags = {"k": np.zeros((B, H, cap), np.uint8), "v": np.zeros((B, H, cap), np.uint8)}
@@ -60,6 +60,21 @@ def test_append_bitexact(kb, vb, rot, ch0, fmt, T, offset, cap):
     B, H = 2, 3
     _, k, v = draw(100 + T, B, H, H, T, fmt)
     gc, oc, flags, geom = build_both(B, H, cap, kb, vb, rot, ch0, k, v, fmt, offset)
+    compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), flags, geom)
+
+
+@pytest.mark.parametrize("kb,vb,ch0,fmt,T,offset,cap,clip", [
+    (4, 2, 1, "bf16", 200, 0, 256, 0.92),
+    (2, 2, 0, "f32", 129, 7, 256, 0.92),
+    (4, 4, 0, "f16", 64, 64, 128, 1.0),
+    (2, 4, 1, "bf16", 33, 95, 128, 0.5),
+])
+def test_append_bitexact_rotated_clipped_values(kb, vb, ch0, fmt, T, offset, cap, clip):
+    # values rotated like the keys and quantized with a clipping ratio on each
+    # group's range (Dual-QK App. B.2)
+    B, H = 2, 3
+    _, k, v = draw(700 + T, B, H, H, T, fmt)
+    gc, oc, flags, geom = build_both(B, H, cap, kb, vb, 1, ch0, k, v, fmt, offset, rotate_v=1, v_clip=clip)
     compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), flags, geom)
 
 
@@ -145,6 +160,31 @@ def test_decode_matches_oracle(case):
             assert not o_gpu[rows].any()
         else:
             assert_close_output(o_gpu[rows], o_ref[rows], f"sequence {b}")
+
+
+@pytest.mark.parametrize("B,G,H,kb,vb,ch0,keep,clip,lens", [
+    (2, 4, 2, 2, 2, 1, 19, 0.92, [1000, 129]),
+    (2, 8, 1, 4, 2, 1, 24, 0.92, [2048, 1]),
+    (1, 1, 2, 4, 4, 0, 32, 1.0, [777]),
+])
+def test_decode_with_rotated_values_matches_oracle(B, G, H, kb, vb, ch0, keep, clip, lens):
+    # the decode works in the rotated value basis; the combine rotates back
+    T = 2048
+    q, k, v = draw(900 + G + kb, B, G * H, H, T, "bf16")
+    gc, oc, flags, geom = build_both(B, H, T, kb, vb, 1, ch0, k, v, "bf16", rotate_v=1, v_clip=clip)
+    compare_cache_bytes(gpu_arrays(gc), oracle_arrays(oc), flags, geom)
+    qd = to_device(q, "bf16")
+    lens_np = np.array(lens, np.int32)
+    lens_d = torch.from_numpy(lens_np).cuda()
+    mask_d = gc.select(qd, keep) if keep < 32 else None
+    ref_mask = orc.select(host_f32(q, "bf16"), H, 1, keep)[0] if keep < 32 else None
+    out = gc.decode(qd, lens_d, T, mask_d, softmax_scale())
+    torch.cuda.synchronize()
+    o_ref = oc.attention(host_f32(q, "bf16"), lens_np, ref_mask, softmax_scale())
+    o_gpu = out.cpu().numpy().reshape(-1, 128)
+    for b in range(B):
+        rows = slice(b * G * H, (b + 1) * G * H)
+        assert_close_output(o_gpu[rows], o_ref[rows], f"sequence {b}")
 
 
 def test_full_mask_is_bit_identical_to_no_mask_and_split_plan_is_exact():
