@@ -198,7 +198,24 @@ class OracleLeg:
         return self.caches[b].attention(qb, self.lens[b:b + 1], mask, 1.0 / math.sqrt(128))
 
 
-def oracle_rate(leg: OracleLeg, budget_s: float, warmup: int = 1):
+class OracleAppendLeg:
+    """The CPU oracle's quantize-append: per step it appends the workload's
+    new tokens of sequence 0 (every kv head) into an oracle cache."""
+
+    def __init__(self, wl: workloads.Workload, s: synth.Synth):
+        from oracle import oracle as orc
+
+        self.wl = wl
+        self.c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
+                           wl.v_clip)
+        self.k = orc.as_f32(np.stack([s.k_slice(0, h) for h in range(wl.Hkv)])[None])
+        self.v = orc.as_f32(np.stack([s.v_slice(0, h) for h in range(wl.Hkv)])[None])
+
+    def step(self, i: int):
+        self.c.append(self.k, self.v, self.wl.offset)
+
+
+def oracle_rate(leg, budget_s: float, warmup: int = 1):
     for i in range(warmup):
         leg.step(i)
     t0 = time.perf_counter()
@@ -268,29 +285,34 @@ def run_reference(args):
         return  # the oracle leg runs on rank 0 only
     wl = workloads.by_id(args.workload)
     s = synth.Synth(workloads.BASE_SEED + wl.id, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt, wl.len_range)
-    leg = OracleLeg(wl, s, s.q(), n_seqs=1)
+    if wl.kind == "append":
+        leg, per_step, unit, metric = OracleAppendLeg(wl, s), wl.T, "appended tokens/s", APPEND_METRIC
+        sample = f"the {wl.T} new tokens of sequence 0 ({wl.Hkv} kv heads) appended per step"
+    else:
+        leg, per_step, unit, metric = OracleLeg(wl, s, s.q(), n_seqs=1), 1, "tokens/s", METRIC
+        sample = f"all {wl.Hq} query heads of sequence 0 over its {int(s.lens[0])} cached tokens per step"
     for i in range(args.warmup):
         leg.step(i)
     t0 = time.perf_counter()
     for i in range(args.steps):
         leg.step(i)
     dt = time.perf_counter() - t0
-    value = args.steps / dt
-    sample = f"all {wl.Hq} query heads of sequence 0 over its {int(s.lens[0])} cached tokens per step"
+    value = per_step * args.steps / dt
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 oracle",
         "data": "synthetic (seeded SplitMix64 + Box-Muller, workload recipe distributions)",
         "config": workload_config(wl),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": unit, "cores": host_cores(), "kind": "oracle",
                          "sample": sample},
-        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 METRIC = "decode tokens/sec & achieved HBM GB/s (fraction of B200 peak) at 1 GPU"
+APPEND_METRIC = "quantize-append tokens/sec & achieved HBM GB/s (fraction of B200 peak) at 1 GPU"
 
 
 def workload_config(wl):
@@ -524,23 +546,12 @@ def run_append(args):
     achieved = abytes / (ms * 1e-3) / 1e9
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from oracle import oracle as orc
-
-        c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
-                      wl.v_clip)
-        k1 = orc.as_f32(np.stack([s.k_slice(0, h) for h in range(wl.Hkv)])[None])
-        v1 = orc.as_f32(np.stack([s.v_slice(0, h) for h in range(wl.Hkv)])[None])
-        t0 = time.perf_counter()
-        done = 0
-        while time.perf_counter() - t0 < args.cpu_seconds:
-            c.append(k1, v1, wl.offset)
-            done += 1
-        dt = time.perf_counter() - t0
-        cpu = {"value": done * wl.T / dt, "unit": "appended tokens/s", "cores": host_cores(), "kind": "oracle",
+        rate, done, dt = oracle_rate(OracleAppendLeg(wl, s), args.cpu_seconds, warmup=0)
+        cpu = {"value": rate * wl.T, "unit": "appended tokens/s", "cores": host_cores(), "kind": "oracle",
                "sample": f"{done} appends of sequence 0 ({wl.Hkv} kv heads x {wl.T} tokens), {dt:.1f} s"}
     if rank == 0:
         line = {
-            "metric": "quantize-append tokens/sec & achieved HBM GB/s (fraction of B200 peak) at 1 GPU",
+            "metric": APPEND_METRIC,
             "value": rep.whole_job(wl.B * wl.T, ms), "unit": "appended tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": f"{wl.fmt} in, u{wl.k_bits}k/u{wl.v_bits}v codes out",
