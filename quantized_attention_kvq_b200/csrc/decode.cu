@@ -228,6 +228,19 @@ __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile 
 __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// named barrier that also ORs a predicate over the participating threads
+__device__ __forceinline__ bool named_sync_or(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -745,12 +758,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         exceed |= sc[i] > m_run[i] + kLazyMax;
       }
       float* rt = red + (k * S::TPT + part) * 64;
-      const unsigned any = __any_sync(kFull, exceed);
-      if (lane == 0) rt[wq * 16 + 8] = any ? 1.0f : 0.0f;
-      named_sync(bar_id, 128);
-      const bool raise = (rt[8] + rt[24] + rt[40] + rt[56]) > 0.0f;
-      float alpha[HH];
+      const bool raise = named_sync_or(bar_id, 128, exceed);
       if (raise) {  // uniform across the part
+        float alpha[HH];
         float m_new[HH];
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
@@ -763,6 +773,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           m_new[i] = fmaxf(m_run[i], fmaxf(fmaxf(rt[i], rt[16 + i]), fmaxf(rt[32 + i], rt[48 + i])));
           alpha[i] = exp2f(m_run[i] - m_new[i]);
           m_run[i] = m_new[i];
+          l_acc[i] *= alpha[i];
+#pragma unroll
+          for (int g = 0; g < kGroups; ++g) zacc[g][i] *= alpha[i];
         }
         if (seg_tiles > 0) {
           // rescale the group's PV sums of the segment so far (this thread: channel
@@ -782,17 +795,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           tmem_wait_st();
           tc_fence_before();
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < HH; ++i) alpha[i] = 1.0f;
       }
       float p[HH];
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
         p[i] = valid ? exp2f(sc[i] - m_run[i]) : 0.0f;
-        l_acc[i] = fmaf(l_acc[i], alpha[i], p[i]);
+        l_acc[i] += p[i];
 #pragma unroll
-        for (int g = 0; g < kGroups; ++g) zacc[g][i] = fmaf(zacc[g][i], alpha[i], p[i] * vsz[g].y);
+        for (int g = 0; g < kGroups; ++g) zacc[g][i] = fmaf(p[i], vsz[g].y, zacc[g][i]);
       }
       // P' = p * value scale into the MN-major operand: column (group g, head),
       // K position pos.  This buffer was last read by the PV UMMAs of tile t-2.
