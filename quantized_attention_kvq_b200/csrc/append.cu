@@ -209,7 +209,7 @@ __device__ __forceinline__ void rotate_row_4lanes(float (&v)[32], int g, double 
   for (int i = 0; i < 32; ++i) v[i] = __double2float_rn(__dmul_rn(x[i], inv_sqrt_d));
 }
 
-template <int KB, int VB, bool ROT, bool CH0, typename In>
+template <int KB, int VB, bool ROT, bool CH0, bool ROTV, typename In>
 __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(AppendArgs a) {
   constexpr int TPW = 32 / VB;            // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
   constexpr int WPR = kAppendTile / TPW;  // value words per channel in the window: 8 or 4
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
   {
     float vx[32];
     widen(vraw, vx);
-    if (c.rotate_v) rotate_row_4lanes(vx, g, a.inv_sqrt_d);  // uniform across the CTA
+    if (ROTV) rotate_row_4lanes(vx, g, a.inv_sqrt_d);
     const __half2 sz = quantize_group32<VB>(vx, false, c.v_clip, code);
     if (!active) {
 #pragma unroll
@@ -350,26 +350,32 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
   }
 }
 
-template <int KB, int VB, bool ROT, bool CH0>
+template <int KB, int VB, bool ROT, bool CH0, bool ROTV>
 cudaError_t launch_typed(const AppendArgs& a, cudaStream_t s) {
   const int first = a.offset / kAppendTile, last = (a.offset + a.n_new - 1) / kAppendTile;
   dim3 grid(last - first + 1, a.c.H, a.c.B);
   dim3 block(kAppendWarps * 32);
   switch (a.dtype) {
-    case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, float><<<grid, block, 0, s>>>(a); break;
-    case KVQ_BF16: k_quantize_append<KB, VB, ROT, CH0, __nv_bfloat16><<<grid, block, 0, s>>>(a); break;
-    default: k_quantize_append<KB, VB, ROT, CH0, __half><<<grid, block, 0, s>>>(a); break;
+    case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, ROTV, float><<<grid, block, 0, s>>>(a); break;
+    case KVQ_BF16: k_quantize_append<KB, VB, ROT, CH0, ROTV, __nv_bfloat16><<<grid, block, 0, s>>>(a); break;
+    default: k_quantize_append<KB, VB, ROT, CH0, ROTV, __half><<<grid, block, 0, s>>>(a); break;
   }
   return cudaGetLastError();
 }
 
+// value rotation is a template flag, so kernels without it stay as small as before
+template <int KB, int VB, bool ROTV>
+cudaError_t launch_flags(const AppendArgs& a, cudaStream_t s) {
+  const bool rot = a.c.rotate != 0, ch0 = a.c.keep_ch0 != 0;
+  if (rot && ch0) return launch_typed<KB, VB, true, true, ROTV>(a, s);
+  if (rot) return launch_typed<KB, VB, true, false, ROTV>(a, s);
+  if (ch0) return launch_typed<KB, VB, false, true, ROTV>(a, s);
+  return launch_typed<KB, VB, false, false, ROTV>(a, s);
+}
+
 template <int KB, int VB>
 cudaError_t launch_bits(const AppendArgs& a, cudaStream_t s) {
-  const bool rot = a.c.rotate != 0, ch0 = a.c.keep_ch0 != 0;
-  if (rot && ch0) return launch_typed<KB, VB, true, true>(a, s);
-  if (rot) return launch_typed<KB, VB, true, false>(a, s);
-  if (ch0) return launch_typed<KB, VB, false, true>(a, s);
-  return launch_typed<KB, VB, false, false>(a, s);
+  return a.c.rotate_v ? launch_flags<KB, VB, true>(a, s) : launch_flags<KB, VB, false>(a, s);
 }
 
 }  // namespace
