@@ -142,7 +142,9 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_head
  * Fused decode attention over the packed cache [DQK Sec. 3.2-3.4; TQ].
  * For each sequence b and query head j (kv head h = j / G):
  *  s_n = softmax_scale * sum over kept channels c of q_rot[c] * k_hat_n[c],
- *  o = sum_n softmax(s)_n * v_hat_n over n < seq_lens[b],
+ *  o = sum_n softmax(s)_n * v_hat_n over n < seq_lens[b]
+ *  (with rotate_v, v_hat_n is the rotated value and o is rotated back by the
+ *  same orthonormal transform before it is written),
  * scored directly from the key codes (no dequantized key is written):
  * per group, scale * (q . codes) + zero * sum(q), plus q_rot[0] * k_ch0 when
  * channel 0 is kept.  Sequences are cut into 128-token tiles and the tiles
