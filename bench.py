@@ -23,6 +23,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -74,11 +75,21 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_tokens(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace collapsed, so
+    that only code changes change the hash below."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_sha(names=DECODE_SOURCES) -> str:
+    """First 16 hex digits of the SHA-256 of the kernel sources' code (comments
+    and whitespace removed): the key a recorded ncu traffic figure is valid for."""
     h = hashlib.sha256()
     for name in names:
-        with open(os.path.join(ROOT, "quantized_attention_kvq_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "quantized_attention_kvq_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_tokens(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -16,10 +16,11 @@
 //           codes as u8 in tensor memory x the rotated query as two exact s8
 //           pieces (q = delta * (128 q1 + q2)), one s32 accumulator per group,
 //           so the per-token group scale applies exactly afterwards;
-//   PV:     8 MMAs of kind::f16 (K = 16 tokens each): value codes as exact
-//           f16 integers in tensor memory x P' = p * value scale, spread over
-//           independent partial accumulators that stay in tensor memory for a
-//           whole segment (one accumulator set per segment parity).
+//   PV:     8 MMAs of kind::f16 (K = 16 tokens each): value codes centred as
+//           c - L/2 (exact f16) in tensor memory x P' = p * value scale, spread
+//           over independent partial accumulators that stay in tensor memory
+//           for a whole segment (one accumulator set per segment parity); the
+//           zero point, with the L/2 steps folded in, is summed in registers.
 //
 // Roles inside a CTA, pipelined over tiles with mbarriers:
 //   producer warp   : 1-D bulk async copies of a tile's kept key-code rows
