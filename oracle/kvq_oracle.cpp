@@ -6,6 +6,7 @@
 
 #include <cfenv>
 #include <cmath>
+#include <algorithm>
 #include <cstring>
 #include <limits>
 #include <vector>
@@ -135,6 +136,22 @@ uint32_t load_k_word(const orc_cache* c, int b, int h, int pg, int n) {
   return c->k_codes[i];
 }
 
+// bf16 window of a cache: sink + recent slots per (b, h)
+inline long wsize(const orc_cache* c) { return (long)c->sink + c->recent; }
+// slot written for token n by an append, or -1
+inline long window_slot(const orc_cache* c, long n) {
+  if (n < c->sink) return n;
+  if (c->recent > 0) return c->sink + (n - c->sink) % c->recent;
+  return -1;
+}
+// window row of token j when a decode of a length-len sequence reads it from
+// the window (j < sink, or j among the last `recent` tokens), else NULL
+inline const uint16_t* window_row(const orc_cache* c, const uint16_t* win, int b, int h, long j, long len) {
+  const bool in = j < c->sink || (c->recent > 0 && j >= std::max((long)c->sink, len - c->recent));
+  if (!in || !win) return nullptr;
+  return win + (((size_t)b * c->kv_heads + h) * wsize(c) + window_slot(c, j)) * c->head_dim;
+}
+
 }  // namespace
 
 extern "C" {
@@ -244,6 +261,9 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
         orc_rotate(k_new + row, d, xr.data());
       else
         for (int i = 0; i < d; ++i) xr[i] = k_new[row + i];
+      const long ws = window_slot(c, n);
+      if (ws >= 0)
+        for (int i = 0; i < d; ++i) c->k_win[(((size_t)b * c->kv_heads + h) * wsize(c) + ws) * d + i] = orc_bf16_rn(xr[i]);
       for (int i = 0; i < d; ++i) incl[i] = 1;
       if (c->keep_ch0) {
         c->k_ch0[ch0_index(c, b, h, n)] = orc_bf16_rn(xr[0]);
@@ -279,6 +299,8 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
         orc_rotate(v_new + row, d, xr.data());
       else
         for (int i = 0; i < d; ++i) xr[i] = v_new[row + i];
+      if (ws >= 0)
+        for (int i = 0; i < d; ++i) c->v_win[(((size_t)b * c->kv_heads + h) * wsize(c) + ws) * d + i] = orc_bf16_rn(xr[i]);
       row_ex = 0;
       for (int g = 0; g < ngroups; ++g) {
         uint16_t s16, z16;
@@ -424,10 +446,15 @@ void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t
     std::vector<double> s(len), khat(d), vhat(d);
     double smax = -std::numeric_limits<double>::infinity();
     for (int j = 0; j < len; ++j) {
-      orc_dequantize(c, b, hk, j, 1, khat.data(), nullptr);
+      const uint16_t* kw = window_row(c, c->k_win, b, hk, j, len);
       double acc = 0.0;
-      for (int ch = 0; ch < d; ++ch)
-        if ((m >> (ch / kGranule)) & 1u) acc += (double)qr[ch] * khat[ch];
+      if (kw) {  // bf16 window token: every channel
+        for (int ch = 0; ch < d; ++ch) acc += (double)qr[ch] * orc_bf16_value(kw[ch]);
+      } else {
+        orc_dequantize(c, b, hk, j, 1, khat.data(), nullptr);
+        for (int ch = 0; ch < d; ++ch)
+          if ((m >> (ch / kGranule)) & 1u) acc += (double)qr[ch] * khat[ch];
+      }
       s[j] = scale * acc;
       if (s[j] > smax) smax = s[j];
     }
@@ -438,7 +465,11 @@ void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t
       l += s[j];
     }
     for (int j = 0; j < len; ++j) {
-      orc_dequantize(c, b, hk, j, 1, nullptr, vhat.data());
+      const uint16_t* vw = window_row(c, c->v_win, b, hk, j, len);
+      if (vw)
+        for (int ch = 0; ch < d; ++ch) vhat[ch] = orc_bf16_value(vw[ch]);
+      else
+        orc_dequantize(c, b, hk, j, 1, nullptr, vhat.data());
       for (int ch = 0; ch < d; ++ch) o[ch] += s[j] * vhat[ch];
     }
     for (int ch = 0; ch < d; ++ch) o[ch] /= l;

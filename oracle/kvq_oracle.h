@@ -27,6 +27,10 @@
  *    ratio; the ratio scales the group's minimum and maximum before the scale
  *    and zero are formed (keys are not clipped).  The attention output then
  *    leaves the rotated basis through the same orthonormal transform.
+ *  - Dual-QK Sec. 3.3 (the first 64 and the most recent 256 tokens remain
+ *    BF16) and tq-kv's sink-token preservation: window tokens are kept as bf16
+ *    copies of the rotated key and of the (rotated) value and scored in full
+ *    (all channels), under the same softmax as the quantized tokens.
  *
  * Precision: FWHT in fp64 (natural Sylvester order), rotated values rounded
  * to fp32; quantization in fp32 with IEEE round-half-to-even; dequantization,
@@ -53,6 +57,12 @@ typedef struct {
   uint8_t* v_codes;   /* [B][Hkv][ceil(cap/128)][d][128*v_bits/8]: per block of 128 tokens one
                          row per channel, 16-byte chunks swizzled by channel        */
   uint16_t* v_scales; /* [B][Hkv][cap][d/32] x {fp16 scale, fp16 zero}      */
+  /* bf16 windows: token n < sink at slot n, token n >= sink at ring slot
+     sink + (n - sink) % recent; at decode, tokens n < sink and
+     n >= max(sink, len - recent) are taken from the window */
+  int32_t sink, recent;
+  uint16_t* k_win; /* [B][Hkv][sink + recent][d] bf16 rotated key, or NULL   */
+  uint16_t* v_win; /* [B][Hkv][sink + recent][d] bf16 (rotated) value, or NULL */
 } orc_cache;
 
 typedef struct {

@@ -21,7 +21,8 @@ class OrcCache(ctypes.Structure):
     _fields_ = [("batch", _I32), ("kv_heads", _I32), ("head_dim", _I32), ("capacity", _I32),
                 ("k_bits", _I32), ("v_bits", _I32), ("rotate_k", _I32), ("keep_ch0", _I32),
                 ("rotate_v", _I32), ("v_clip", ctypes.c_float),
-                ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P)]
+                ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P),
+                ("sink", _I32), ("recent", _I32), ("k_win", _P), ("v_win", _P)]
 
 
 class OrcStats(ctypes.Structure):
@@ -121,10 +122,14 @@ def quantize_group(x, bits: int, include=None, clip: float = 1.0):
 class Cache:
     """Host copy of the packed cache, written by the oracle."""
 
-    def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, rotate_v=0, v_clip=1.0):
+    def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, rotate_v=0, v_clip=1.0,
+                 sink=0, recent=0):
         self.B, self.Hkv, self.d, self.capacity = B, Hkv, d, capacity
         self.k_bits, self.v_bits, self.rotate_k, self.keep_ch0 = k_bits, v_bits, rotate_k, keep_ch0
-        self.rotate_v, self.v_clip = rotate_v, v_clip
+        self.rotate_v, self.v_clip, self.sink, self.recent = rotate_v, v_clip, sink, recent
+        w = B * Hkv * (sink + recent) * d
+        self.k_win = np.zeros(w, np.uint16) if w else None  # bf16 windows
+        self.v_win = np.zeros(w, np.uint16) if w else None
         blocked = -(-capacity // 128) * 128  # codes are stored in blocks of 128 tokens
         self.k_codes = np.zeros(B * Hkv * (d // 4) * blocked * (4 * k_bits // 8), np.uint8)
         self.k_scales = np.zeros(B * Hkv * (d // 32) * blocked * 2, np.uint16)
@@ -132,8 +137,8 @@ class Cache:
         self.v_codes = np.zeros(B * Hkv * d * blocked * v_bits // 8, np.uint8)  # channel rows per block
         self.v_scales = np.zeros(B * Hkv * capacity * (d // 32) * 2, np.uint16)
         self.struct = OrcCache(B, Hkv, d, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v, v_clip,
-                               _p(self.k_codes),
-                               _p(self.k_scales), _p(self.k_ch0), _p(self.v_codes), _p(self.v_scales))
+                               _p(self.k_codes), _p(self.k_scales), _p(self.k_ch0), _p(self.v_codes),
+                               _p(self.v_scales), sink, recent, _p(self.k_win), _p(self.v_win))
 
     def append(self, k_new: np.ndarray, v_new: np.ndarray, offset: int, want_exempt: bool = False):
         """k_new, v_new: [B][Hkv][n][d] (bf16 as uint16, or fp32)."""
