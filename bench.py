@@ -52,18 +52,22 @@ def algorithmic_bytes(wl: workloads.Workload, masks: np.ndarray, lens: np.ndarra
     scale/zero of touched key groups, channel 0 when its group is kept, every
     value code and value scale/zero of the sequence, plus q in and out."""
     kword = 2 if wl.k_bits == 4 else 1
-    split = 0
+    split = window = 0
     for b in range(wl.B):
         n = int(lens[b])
+        # tokens read from the bf16 windows (the first `sink` and the last `recent`)
+        nw = min(wl.sink, n) + (max(0, n - max(wl.sink, n - wl.recent)) if wl.recent else 0)
         for h in range(wl.Hkv):
             m = int(masks[b, h]) & 0xFFFFFFFF
             kept = popcount32(m)
             touched = sum(1 for g in range(4) if (m >> (8 * g)) & 0xFF)
-            split += n * (kept * kword + touched * 4 + (2 if wl.keep_ch0 and (m & 1) else 0))
-            split += n * (128 * wl.v_bits // 8 + 16)
+            split += (n - nw) * (kept * kword + touched * 4 + (2 if wl.keep_ch0 and (m & 1) else 0))
+            split += (n - nw) * (128 * wl.v_bits // 8 + 16)
+            window += nw * 2 * 128 * 2  # bf16 key and value rows
     esize = 4 if wl.fmt == "f32" else 2
     q_bytes = wl.B * wl.Hq * 128 * esize
-    return {"split_kernel": split + q_bytes, "step": split + q_bytes + wl.B * wl.Hq * 128 * 4}
+    return {"split_kernel": split + q_bytes, "window": window,
+            "step": split + window + q_bytes + wl.B * wl.Hq * 128 * 4}
 
 
 def measured_hbm_peak():
@@ -193,7 +197,7 @@ class OracleLeg:
         self.q = orc.as_f32(q)
         for b in range(n_seqs):
             c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
-                          wl.v_clip)
+                          wl.v_clip, wl.sink, wl.recent)
             k = np.stack([s.k_slice(b, h) for h in range(wl.Hkv)])[None]
             v = np.stack([s.v_slice(b, h) for h in range(wl.Hkv)])[None]
             c.append(orc.as_f32(k), orc.as_f32(v), wl.offset)
@@ -218,7 +222,7 @@ class OracleAppendLeg:
 
         self.wl = wl
         self.c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
-                           wl.v_clip)
+                           wl.v_clip, wl.sink, wl.recent)
         self.k = orc.as_f32(np.stack([s.k_slice(0, h) for h in range(wl.Hkv)])[None])
         self.v = orc.as_f32(np.stack([s.v_slice(0, h) for h in range(wl.Hkv)])[None])
 
@@ -331,6 +335,7 @@ def workload_config(wl):
             "seq_len": wl.T if wl.len_range is None else f"U[{wl.len_range[0]},{wl.len_range[1]}]",
             "k_bits": wl.k_bits, "v_bits": wl.v_bits, "group": 32, "rotate_k": wl.rotate_k,
             "keep_ch0": wl.keep_ch0, "keep_groups": wl.keep_groups, "rotate_v": wl.rotate_v, "v_clip": wl.v_clip,
+            "bf16_sink": wl.sink, "bf16_recent": wl.recent,
             "input_dtype": wl.fmt,
             "l2": "flushed between steps (memset of 2x L2)", "parallelism": "replicas (one batch per GPU)"}
 
@@ -355,7 +360,7 @@ def run_kvq(args):
     # -- resident cache (built by the append kernel, not timed here)
     q_np = s.q()
     cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev,
-                            rotate_v=wl.rotate_v, v_clip=wl.v_clip)
+                            rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent)
     for b in range(wl.B):  # one sequence at a time keeps host memory small
         kd = up(np.stack([s.k_slice(b, h) for h in range(wl.Hkv)]))
         vd = up(np.stack([s.v_slice(b, h) for h in range(wl.Hkv)]))
@@ -462,7 +467,7 @@ def run_kvq(args):
             "e2e": {"value": rep.whole_job(wl.B, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(q_pin.numel() * q_pin.element_size()),
                     "d2h_bytes_per_step": int(out_pin.numel() * 4)},
-            "gpu_launches": args.steps * (2 + (1 if keep < 32 else 0)),
+            "gpu_launches": args.steps * (2 + (1 if keep < 32 else 0) + (1 if wl.sink + wl.recent else 0)),
             "roofline": {"bound": "hbm", "kernel": "decode split (kvq_decode_partials)", "achieved": achieved,
                          "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": abytes["split_kernel"], "peak_source": peak_src,
@@ -511,7 +516,7 @@ def run_append(args):
 
     kd, vd = up(s.k_full()), up(s.v_full())
     cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev,
-                            rotate_v=wl.rotate_v, v_clip=wl.v_clip)
+                            rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()

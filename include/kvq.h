@@ -92,6 +92,23 @@ typedef struct {
   void* k_ch0;
   void* v_codes;
   void* v_scales;
+  /* bf16 token windows [DQK Sec. 3.3: the first 64 and the most recent 256
+     tokens stay BF16; TQ: sink tokens preserved]; 0 and NULL = none.
+     k_window, v_window: [B][H][sink_tokens + recent_tokens][d] bf16, sizes
+     from kvq_window_bytes: the rotated key and the value (rotated when
+     rotate_v) of token n, at slot n when n < sink_tokens, else at ring slot
+     sink_tokens + (n - sink_tokens) % recent_tokens: an append writes its
+     tokens n < sink_tokens and its last recent_tokens tokens (the end state of
+     writing every token in order).
+     A decode over seq_lens[b] = len takes tokens n < sink_tokens and
+     n >= max(sink_tokens, len - recent_tokens) from the windows, scored over
+     every channel (the channel mask applies to the coded tokens only), so the
+     ring must hold the last recent_tokens appended: decode len equal to the
+     tokens appended so far.  sink_tokens + recent_tokens <= min(capacity,
+     2048) (larger: KVQ_ERR_UNSUPPORTED). */
+  int32_t sink_tokens, recent_tokens;
+  void* k_window;
+  void* v_window;
 } kvq_cache;
 
 /*
@@ -99,6 +116,9 @@ typedef struct {
  * k_ch0 (0 unless keep_ch0), v_codes, v_scales.  Pointer fields are ignored.
  */
 KVQ_API kvq_status kvq_cache_sizes(const kvq_cache* cache, size_t bytes_out[5]);
+
+/* Bytes of each of k_window and v_window (0 without windows or on bad arguments). */
+KVQ_API size_t kvq_window_bytes(const kvq_cache* cache);
 
 /*
  * Quantize and append n_new tokens per (sequence, kv head) at token positions

@@ -22,6 +22,9 @@ kvq_status check_shape(const kvq_cache* c) {
   if (c->batch < 1 || c->kv_heads < 1 || c->capacity < 1 || c->head_dim < 1) return KVQ_ERR_INVALID_ARG;
   if ((c->rotate_k != 0 && c->rotate_k != 1) || (c->keep_ch0 != 0 && c->keep_ch0 != 1)) return KVQ_ERR_INVALID_ARG;
   if ((c->rotate_v != 0 && c->rotate_v != 1) || !(c->v_clip > 0.0f && c->v_clip <= 1.0f)) return KVQ_ERR_INVALID_ARG;
+  if (c->sink_tokens < 0 || c->recent_tokens < 0 || (int64_t)c->sink_tokens + c->recent_tokens > c->capacity)
+    return KVQ_ERR_INVALID_ARG;
+  if (c->sink_tokens + c->recent_tokens > 2048) return KVQ_ERR_UNSUPPORTED;  // the window kernel's shared memory
   if (c->head_dim != kHeadDim || c->group_size != kGroup || c->prune_granule != kGranule) return KVQ_ERR_UNSUPPORTED;
   if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return KVQ_ERR_UNSUPPORTED;
   if (c->capacity % kKeyBlock != 0) return KVQ_ERR_UNSUPPORTED;
@@ -35,6 +38,9 @@ kvq_status check_cache(const kvq_cache* c) {
     return KVQ_ERR_INVALID_ARG;
   if (!aligned16(c->k_codes) || !aligned16(c->k_scales) || !aligned16(c->v_codes) || !aligned16(c->v_scales) ||
       (c->keep_ch0 && !aligned16(c->k_ch0)))
+    return KVQ_ERR_INVALID_ARG;
+  if (c->sink_tokens + c->recent_tokens > 0 &&
+      (!c->k_window || !c->v_window || !aligned16(c->k_window) || !aligned16(c->v_window)))
     return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
@@ -55,6 +61,10 @@ CacheView view(const kvq_cache* c) {
   v.keep_ch0 = c->keep_ch0;
   v.rotate_v = c->rotate_v;
   v.v_clip = c->v_clip;
+  v.sink = c->sink_tokens;
+  v.recent = c->recent_tokens;
+  v.kwin = static_cast<__nv_bfloat16*>(c->k_window);
+  v.vwin = static_cast<__nv_bfloat16*>(c->v_window);
   v.kc = static_cast<uint8_t*>(c->k_codes);
   v.ks = static_cast<__half2*>(c->k_scales);
   v.k0 = static_cast<__nv_bfloat16*>(c->k_ch0);
@@ -74,7 +84,8 @@ struct DecodePlan {
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   DecodePlan p;
   const int G = q_heads / c->kv_heads;
-  const size_t rows = (size_t)decode_slots(c->batch, c->kv_heads, G) * G;
+  const bool win = c->sink_tokens + c->recent_tokens > 0;  // one more partial per unit for the windows
+  const size_t rows = ((size_t)decode_slots(c->batch, c->kv_heads, G) + (win ? c->batch * c->kv_heads : 0)) * G;
   p.acc_bytes = rows * kHeadDim * sizeof(float);
   p.ml_offset = round_up(p.acc_bytes, kAlign);
   p.bytes = p.ml_offset + round_up(rows * sizeof(float2), kAlign);
@@ -100,11 +111,16 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.mask = mask;
   a.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);  // log2(e)
   a.inv_sqrt_d = inv_sqrt_d();
+  a.win_base = decode_slots(c->batch, c->kv_heads, q_heads / c->kv_heads);
   a.part_acc = static_cast<float*>(workspace);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
   if ((parts & kRunSplit) && max_len > 0) {
     kvq_status st = cuda_status(launch_decode(a, s));
+    if (st != KVQ_OK) return st;
+  }
+  if ((parts & kRunSplit) && c->sink_tokens + c->recent_tokens > 0) {
+    kvq_status st = cuda_status(launch_window(a, s));
     if (st != KVQ_OK) return st;
   }
   if (parts & kRunCombine) return cuda_status(launch_combine(a, s));
@@ -157,6 +173,11 @@ KVQ_API kvq_status kvq_cache_sizes(const kvq_cache* c, size_t bytes_out[5]) {
   bytes_out[3] = rows * (kHeadDim * c->v_bits / 8);
   bytes_out[4] = rows * kGroups * 4;
   return KVQ_OK;
+}
+
+KVQ_API size_t kvq_window_bytes(const kvq_cache* c) {
+  if (check_shape(c) != KVQ_OK) return 0;
+  return (size_t)c->batch * c->kv_heads * (size_t)(c->sink_tokens + c->recent_tokens) * kHeadDim * 2;
 }
 
 KVQ_API kvq_status kvq_quantize_append(const kvq_cache* c, const void* k_new, const void* v_new, kvq_dtype dtype,

@@ -209,6 +209,19 @@ __device__ __forceinline__ void rotate_row_4lanes(float (&v)[32], int g, double 
   for (int i = 0; i < 32; ++i) v[i] = __double2float_rn(__dmul_rn(x[i], inv_sqrt_d));
 }
 
+// bf16 (round to nearest even) copy of this lane's 32 channels into a window row
+__device__ __forceinline__ void store_bf16_32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
 template <int KB, int VB, bool ROT, bool CH0, bool ROTV, typename In>
 __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(AppendArgs a) {
   constexpr int TPW = 32 / VB;            // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
@@ -254,6 +267,14 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
 
   // ---- key row: rotated, then quantized (keys are not clipped)
   if (ROT) rotate_row_4lanes(kx, g, a.inv_sqrt_d);
+  // bf16 window copies (rotated key, then the value below) for tokens with a
+  // window slot: every sink token, and of the later tokens only this append's
+  // last `recent`, the ones that still own their ring slot when it ends (an
+  // earlier token of the same append would race with them for the slot)
+  const int wn = w0 + tt;
+  const int wslot = active && (wn < c.sink || wn >= a.offset + a.n_new - c.recent)
+                        ? window_slot(c.sink, c.recent, wn) : -1;
+  if (wslot >= 0) store_bf16_32(c.kwin + (bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, kx);
   uint32_t code[8];
   {
     const bool skip0 = CH0 && g == 0;
@@ -271,6 +292,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
     float vx[32];
     widen(vraw, vx);
     if (ROTV) rotate_row_4lanes(vx, g, a.inv_sqrt_d);
+    if (wslot >= 0) store_bf16_32(c.vwin + (bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, vx);
     const __half2 sz = quantize_group32<VB>(vx, false, c.v_clip, code);
     if (!active) {
 #pragma unroll

@@ -107,6 +107,17 @@ __host__ __device__ __forceinline__ size_t key_scale_index(size_t bh, int cap, i
 // 16-byte chunks; chunk i of channel ch sits at chunk position
 // i ^ v_chunk_swizzle(ch), so 8 consecutive channels' rows start in 8
 // different shared-memory bank groups.
+// bf16 window slot of token n (written by appends), or -1: slot n below the
+// sink, else a ring of `recent` slots
+__host__ __device__ __forceinline__ int window_slot(int sink, int recent, int n) {
+  if (n < sink) return n;
+  return recent > 0 ? sink + (n - sink) % recent : -1;
+}
+// whether a decode over a length-len sequence takes token n from the windows
+__host__ __device__ __forceinline__ bool in_window(int sink, int recent, int n, int len) {
+  return n < sink || (recent > 0 && n >= (sink > len - recent ? sink : len - recent));
+}
+
 __host__ __device__ __forceinline__ int v_chunk_swizzle(int v_bits, int ch) {
   return v_bits == 4 ? (ch >> 1) & 3 : (ch >> 2) & 1;
 }
@@ -119,6 +130,9 @@ __host__ __device__ __forceinline__ size_t v_row_offset(size_t bh, int cap, int 
 struct CacheView {
   int B, H, cap, k_bits, v_bits, rotate, keep_ch0, rotate_v;
   float v_clip;
+  int sink, recent;                    // bf16 token windows (0, 0: none)
+  __nv_bfloat16* kwin;                 // [B][H][sink + recent][128]
+  __nv_bfloat16* vwin;
   uint8_t* kc;
   __half2* ks;
   __nv_bfloat16* k0;
@@ -150,6 +164,7 @@ struct DecodeArgs {
   const uint32_t* mask;
   float scale_log2;  // softmax_scale * log2(e): scores live in the exp2 domain
   double inv_sqrt_d;
+  int win_base;     // first partial slot of the bf16 windows: one slot per unit after decode_slots
   float* part_acc;  // [decode_slots][G][128] unnormalized accumulators
   float2* part_ml;  // [decode_slots][G] (running max, running sum)
   float* out;       // [B][Hq][128]
@@ -164,6 +179,8 @@ bool decode_g_supported(int g);
 int decode_groups(int G);
 int decode_slots(int B, int H, int G);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+// attention over the bf16 window tokens of every unit: one partial per unit at win_base + unit
+cudaError_t launch_window(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s);
 
 // Checked split decode + combine into a caller-chosen scratch buffer of

@@ -18,7 +18,7 @@ KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORK
 KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 
 # every exported symbol the header declares
-SYMBOLS = ("kvq_cache_sizes", "kvq_quantize_append", "kvq_select_channels", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
+SYMBOLS = ("kvq_cache_sizes", "kvq_window_bytes", "kvq_quantize_append", "kvq_select_channels", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
            "kvq_decode_step_workspace_bytes",
            "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_status_string")
 
@@ -30,7 +30,8 @@ class KvqCacheStruct(ctypes.Structure):
     _fields_ = [("batch", _I32), ("kv_heads", _I32), ("head_dim", _I32), ("capacity", _I32),
                 ("k_bits", _I32), ("v_bits", _I32), ("group_size", _I32), ("prune_granule", _I32),
                 ("rotate_k", _I32), ("keep_ch0", _I32), ("rotate_v", _I32), ("v_clip", ctypes.c_float),
-                ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P)]
+                ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P),
+                ("sink_tokens", _I32), ("recent_tokens", _I32), ("k_window", _P), ("v_window", _P)]
 
 
 class KvqError(RuntimeError):
@@ -51,6 +52,8 @@ def lib():
         C = ctypes.POINTER(KvqCacheStruct)
         L.kvq_cache_sizes.argtypes = [C, ctypes.POINTER(ctypes.c_size_t)]
         L.kvq_cache_sizes.restype = ctypes.c_int
+        L.kvq_window_bytes.argtypes = [C]
+        L.kvq_window_bytes.restype = ctypes.c_size_t
         L.kvq_quantize_append.argtypes = [C, _P, _P, ctypes.c_int, _I32, _I32, _P]
         L.kvq_quantize_append.restype = ctypes.c_int
         L.kvq_select_channels.argtypes = [C, _P, ctypes.c_int, _I32, _I32, _P, _P]
@@ -107,8 +110,11 @@ def _stream(stream) -> int | None:
     return stream.cuda_stream
 
 
-def describe(B, H, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, d=128, rotate_v=0, v_clip=1.0) -> KvqCacheStruct:
-    return KvqCacheStruct(B, H, d, capacity, k_bits, v_bits, 32, 4, rotate_k, keep_ch0, rotate_v, v_clip)
+def describe(B, H, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, d=128, rotate_v=0, v_clip=1.0, sink=0,
+             recent=0) -> KvqCacheStruct:
+    d_ = KvqCacheStruct(B, H, d, capacity, k_bits, v_bits, 32, 4, rotate_k, keep_ch0, rotate_v, v_clip)
+    d_.sink_tokens, d_.recent_tokens = sink, recent
+    return d_
 
 
 def cache_sizes(desc: KvqCacheStruct) -> list[int]:
@@ -121,8 +127,10 @@ class KVQCache:
     """Packed quantized KV cache in device memory (torch-allocated, library-laid-out)."""
 
     def __init__(self, B: int, H: int, capacity: int, k_bits: int, v_bits: int, rotate_k: int = 1,
-                 keep_ch0: int = 0, device="cuda", zero: bool = True, rotate_v: int = 0, v_clip: float = 1.0):
-        self.desc = describe(B, H, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v=rotate_v, v_clip=v_clip)
+                 keep_ch0: int = 0, device="cuda", zero: bool = True, rotate_v: int = 0, v_clip: float = 1.0,
+                 sink: int = 0, recent: int = 0):
+        self.desc = describe(B, H, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v=rotate_v, v_clip=v_clip,
+                             sink=sink, recent=recent)
         sizes = cache_sizes(self.desc)
         alloc = torch.zeros if zero else torch.empty
         self.k_codes = alloc(sizes[0], dtype=torch.uint8, device=device)
@@ -135,6 +143,11 @@ class KVQCache:
         self.desc.k_ch0 = _dev_ptr(self.k_ch0)
         self.desc.v_codes = _dev_ptr(self.v_codes)
         self.desc.v_scales = _dev_ptr(self.v_scales)
+        wb = lib().kvq_window_bytes(ctypes.byref(self.desc)) if sink + recent else 0
+        self.k_window = alloc(wb, dtype=torch.uint8, device=device) if wb else None  # bf16 token windows
+        self.v_window = alloc(wb, dtype=torch.uint8, device=device) if wb else None
+        self.desc.k_window = _dev_ptr(self.k_window)
+        self.desc.v_window = _dev_ptr(self.v_window)
         self.B, self.H, self.capacity = B, H, capacity
 
     def sequence_desc(self, b: int) -> KvqCacheStruct:
@@ -142,12 +155,17 @@ class KVQCache:
         with the sequence outermost, so this is a pointer offset per array."""
         per = [x // self.B for x in cache_sizes(self.desc)]
         d = describe(1, self.H, self.capacity, self.desc.k_bits, self.desc.v_bits, self.desc.rotate_k,
-                     self.desc.keep_ch0, rotate_v=self.desc.rotate_v, v_clip=self.desc.v_clip)
+                     self.desc.keep_ch0, rotate_v=self.desc.rotate_v, v_clip=self.desc.v_clip,
+                     sink=self.desc.sink_tokens, recent=self.desc.recent_tokens)
         d.k_codes = self.desc.k_codes + b * per[0]
         d.k_scales = self.desc.k_scales + b * per[1]
         d.k_ch0 = self.desc.k_ch0 + b * per[2] if self.desc.keep_ch0 else None
         d.v_codes = self.desc.v_codes + b * per[3]
         d.v_scales = self.desc.v_scales + b * per[4]
+        if self.k_window is not None:
+            wper = self.k_window.numel() // self.B
+            d.k_window = self.desc.k_window + b * wper
+            d.v_window = self.desc.v_window + b * wper
         return d
 
     def append_sequence(self, b: int, k_new: torch.Tensor, v_new: torch.Tensor, offset: int, stream=None):

@@ -29,6 +29,8 @@ class Workload:
     rotate_v: int = 0   # values rotated before quantization (decode output rotated back)
     v_clip: float = 1.0  # value clipping ratio on each group's min and max
     kind: str = "decode"  # what bench.py times: "decode" or "append"
+    sink: int = 0       # bf16 window: the first tokens of each sequence
+    recent: int = 0     # bf16 window: the most recent tokens of each sequence
 
     @property
     def G(self) -> int:
@@ -48,6 +50,9 @@ WORKLOADS = [
              1, 1, 19, rotate_v=1, v_clip=0.92),
     Workload(6, "append_vrot_clip092_b16_h8_t4096_at8192", 16, 8, 8, 128, 4096, 12288, 8192, "bf16", 4, 2, 1, 0,
              32, rotate_v=1, v_clip=0.92, kind="append"),
+    # and the first 64 and most recent 256 tokens kept in bf16 (Dual-QK Sec. 3.3)
+    Workload(7, "dualqk_int2_vrot_win64x256_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16", 2,
+             2, 1, 1, 19, rotate_v=1, v_clip=0.92, sink=64, recent=256),
 ]
 
 BASE_SEED = 0

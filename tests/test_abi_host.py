@@ -83,6 +83,30 @@ def test_rotated_clipped_values_are_accepted(L):
         native.KVQ_ERR_CAPACITY
 
 
+@pytest.mark.parametrize("sink,recent,kw,vw,status", [
+    (-1, 0, None, None, native.KVQ_ERR_INVALID_ARG), (0, -3, None, None, native.KVQ_ERR_INVALID_ARG),
+    (200, 100, FAKE, FAKE, native.KVQ_ERR_INVALID_ARG),          # more than the capacity
+    (64, 0, 0, FAKE, native.KVQ_ERR_INVALID_ARG), (0, 8, FAKE, FAKE + 8, native.KVQ_ERR_INVALID_ARG),
+])
+def test_bad_windows_rejected(L, sink, recent, kw, vw, status):
+    d = desc(sink_tokens=sink, recent_tokens=recent)
+    if kw is not None:
+        d.k_window, d.v_window = kw, vw
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == status
+
+
+def test_window_sizes(L):
+    d = native.describe(3, 2, 4096, 2, 2, 1, 1, sink=64, recent=256)
+    assert L.kvq_window_bytes(ctypes.byref(d)) == 3 * 2 * 320 * 128 * 2
+    assert L.kvq_window_bytes(ctypes.byref(native.describe(3, 2, 4096, 2, 2))) == 0
+    big = native.describe(1, 1, 8192, 4, 4, sink=1024, recent=1025)
+    big.k_window = big.v_window = FAKE
+    for f in ("k_codes", "k_scales", "v_codes", "v_scales"):
+        setattr(big, f, FAKE)
+    assert L.kvq_quantize_append(ctypes.byref(big), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
+        native.KVQ_ERR_UNSUPPORTED
+
+
 def test_append_argument_checks(L):
     d = desc()
     assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 200, 100, None) == \

@@ -53,3 +53,15 @@ def test_traffic_key_ignores_comments_and_layout():
 
 def test_recorded_traffic_only_for_its_workload():
     assert bench.recorded_traffic("no_such_workload") is None
+
+
+def test_decode_bytes_with_bf16_windows():
+    wl = workloads.by_id(7)
+    masks = np.full((wl.B, wl.Hkv), (1 << 19) - 1, np.uint32)
+    lens = np.array([wl.T, 300, 64, 10], np.int32)  # long, inside both windows, the sink alone, shorter than it
+    got = bench.algorithmic_bytes(wl, masks, lens)
+    per_code = 19 * 4 * 2 // 8 + 3 * 4 + 2 + 128 * 2 // 8 + 4 * 4
+    windowed = [64 + 256, 300, 64, 10]  # tokens read as bf16 rows
+    split = sum((int(n) - w) * per_code for n, w in zip(lens, windowed)) * wl.Hkv
+    assert got["split_kernel"] == split + wl.B * wl.Hq * 128 * 2
+    assert got["window"] == sum(windowed) * wl.Hkv * 2 * 128 * 2

@@ -187,6 +187,40 @@ def test_decode_with_rotated_values_matches_oracle(B, G, H, kb, vb, ch0, keep, c
         assert_close_output(o_gpu[rows], o_ref[rows], f"sequence {b}")
 
 
+@pytest.mark.parametrize("G,H,kb,vb,ch0,keep,rotv,sink,recent,L", [
+    (4, 2, 2, 2, 1, 19, 1, 64, 256, 1000),   # the Dual-QK recipe: INT2, pruned keys, bf16 windows
+    (1, 2, 4, 4, 0, 32, 0, 4, 8, 10),        # the whole sequence inside the windows
+    (8, 1, 4, 2, 1, 24, 0, 16, 0, 300),      # sink only
+    (2, 2, 4, 4, 0, 9, 0, 0, 100, 129),      # recent only
+    (16, 1, 4, 4, 1, 32, 1, 3, 5, 2),        # shorter than the sink
+])
+def test_decode_with_bf16_windows_matches_oracle(G, H, kb, vb, ch0, keep, rotv, sink, recent, L):
+    # window tokens come from bf16 copies of the rotated key and value, scored over
+    # every channel; the others from the codes (Dual-QK Sec. 3.3); decode length =
+    # tokens appended, as the ring holds the last `recent` of them
+    T = 1024
+    clip = 0.92 if rotv else 1.0
+    q, k, v = draw(1100 + G + L, 1, G * H, H, T, "bf16")
+    k, v = k[:, :, :L], v[:, :, :L]
+    gc = native.KVQCache(1, H, T, kb, vb, 1, ch0, rotate_v=rotv, v_clip=clip, sink=sink, recent=recent)
+    oc = orc.Cache(1, H, 128, T, kb, vb, 1, ch0, rotv, clip, sink, recent)
+    gc.append(to_device(k, "bf16"), to_device(v, "bf16"), 0)
+    oc.append(host_f32(k, "bf16"), host_f32(v, "bf16"), 0)
+    torch.cuda.synchronize()
+    # the bf16 windows are bit-exact (bf16 of the same fp32 rows)
+    assert np.array_equal(gc.k_window.cpu().numpy(), oc.k_win.view(np.uint8))
+    assert np.array_equal(gc.v_window.cpu().numpy(), oc.v_win.view(np.uint8))
+    qd = to_device(q, "bf16")
+    lens_np = np.array([L], np.int32)
+    lens_d = torch.from_numpy(lens_np).cuda()
+    mask_d = gc.select(qd, keep) if keep < 32 else None
+    ref_mask = orc.select(host_f32(q, "bf16"), H, 1, keep)[0] if keep < 32 else None
+    out = gc.decode(qd, lens_d, T, mask_d, softmax_scale())
+    torch.cuda.synchronize()
+    o_ref = oc.attention(host_f32(q, "bf16"), lens_np, ref_mask, softmax_scale())
+    assert_close_output(out.cpu().numpy().reshape(-1, 128), o_ref, "bf16 windows")
+
+
 def test_full_mask_is_bit_identical_to_no_mask_and_split_plan_is_exact():
     B, G, H, T = 2, 4, 2, 1024
     q, k, v = draw(9, B, G * H, H, T, "bf16")

@@ -42,7 +42,8 @@ def slice_bytes(gc: native.KVQCache, b: int, h: int):
 
 
 def oracle_slice(wl, s, b, h):
-    c = orc.Cache(1, 1, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v, wl.v_clip)
+    c = orc.Cache(1, 1, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v, wl.v_clip,
+                  wl.sink, wl.recent)
     k = s.k_slice(b, h)[None, None]
     v = s.v_slice(b, h)[None, None]
     st = c.append(host_f32(k, wl.fmt), host_f32(v, wl.fmt), wl.offset, want_exempt=True)
@@ -75,7 +76,7 @@ def check_slice_bytes(got: dict, c: orc.Cache, st: dict, wl):
 
 def build_cache(wl, s):
     gc = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0,
-                         rotate_v=wl.rotate_v, v_clip=wl.v_clip)
+                         rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent)
     for b in range(wl.B):
         kd = up(np.stack([s.k_slice(b, h) for h in range(wl.Hkv)]), wl.fmt)
         vd = up(np.stack([s.v_slice(b, h) for h in range(wl.Hkv)]), wl.fmt)
@@ -97,7 +98,7 @@ def sampled_pairs(wl, n=2, seed=0):
     return sorted(pairs)
 
 
-@pytest.mark.parametrize("wid", [0, 1, 2, 4, 5])
+@pytest.mark.parametrize("wid", [0, 1, 2, 4, 5, 7])
 def test_decode_workload(wid):
     wl = workloads.by_id(wid)
     s = synth.Synth(workloads.BASE_SEED + wl.id, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt, wl.len_range)
@@ -144,7 +145,7 @@ def test_append_workload(wid):
     wl = workloads.by_id(wid)
     s = synth.Synth(workloads.BASE_SEED + wl.id, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt, wl.len_range)
     gc = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0,
-                         rotate_v=wl.rotate_v, v_clip=wl.v_clip)
+                         rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent)
     # one launch over the whole batch, as timed for the append workload
     kd = up(s.k_full(), wl.fmt)
     vd = up(s.v_full(), wl.fmt)
