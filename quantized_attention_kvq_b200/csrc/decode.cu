@@ -925,7 +925,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 // weights, thread = channel for the value sums.
 template <int G, typename In>
 __global__ void __launch_bounds__(kHeadDim) k_window(DecodeArgs a) {
-  extern __shared__ float wsm[];  // q [G][128], weights [G][sink + recent], reductions [G][4]
+  extern __shared__ float wsm[];  // q [G][128], weights [G][sink + recent], reductions [G][4], slots [sink + recent]
   const CacheView& c = a.c;
   const int u = blockIdx.x, b = u / c.H, h = u - b * c.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -937,8 +937,10 @@ __global__ void __launch_bounds__(kHeadDim) k_window(DecodeArgs a) {
   float* qs = wsm;
   float* pw = wsm + G * kHeadDim;
   float* red = pw + G * WS;
+  int* slot = reinterpret_cast<int*>(red + G * 4);  // window slot of window token w
   const size_t row0 = (size_t)u * WS;
-  auto token = [&](int w) { return w < n_sink ? w : r0 + (w - n_sink); };
+  for (int w = tid; w < W; w += kHeadDim)
+    slot[w] = window_slot(c.sink, c.recent, w < n_sink ? w : r0 + (w - n_sink));
   // the query rows, rotated as the keys are, one warp per head
   for (int g = warp; g < G; g += kHeadDim / 32) {
     float x[4];
@@ -953,19 +955,24 @@ __global__ void __launch_bounds__(kHeadDim) k_window(DecodeArgs a) {
 #pragma unroll
   for (int g = 0; g < G; ++g) mloc[g] = -__int_as_float(0x7f800000);
   for (int w = tid; w < W; w += kHeadDim) {
-    const __nv_bfloat16* kr = c.kwin + (row0 + window_slot(c.sink, c.recent, token(w))) * kHeadDim;
+    // the whole bf16 key row in flight at once (16 independent 16-byte loads)
+    const uint4* kr = reinterpret_cast<const uint4*>(c.kwin + (row0 + slot[w]) * kHeadDim);
+    uint4 raw[kHeadDim / 8];
+#pragma unroll
+    for (int i = 0; i < kHeadDim / 8; ++i) raw[i] = kr[i];
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = 0.0f;
-    for (int cc = 0; cc < kHeadDim; cc += 8) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(kr + cc);
-      const uint32_t pr[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i8 = 0; i8 < kHeadDim / 8; ++i8) {
+      const uint32_t pr[4] = {raw[i8].x, raw[i8].y, raw[i8].z, raw[i8].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
+        const int cc = 8 * i8 + 2 * i;
         const float k0 = __uint_as_float(pr[i] << 16), k1 = __uint_as_float(pr[i] & 0xFFFF0000u);
 #pragma unroll
         for (int g = 0; g < G; ++g)
-          acc[g] = fmaf(qs[g * kHeadDim + cc + 2 * i + 1], k1, fmaf(qs[g * kHeadDim + cc + 2 * i], k0, acc[g]));
+          acc[g] = fmaf(qs[g * kHeadDim + cc + 1], k1, fmaf(qs[g * kHeadDim + cc], k0, acc[g]));
       }
     }
 #pragma unroll
@@ -1007,8 +1014,21 @@ __global__ void __launch_bounds__(kHeadDim) k_window(DecodeArgs a) {
   float o[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) o[g] = 0.0f;
-  for (int w = 0; w < W; ++w) {
-    const float v = __bfloat162float(c.vwin[(row0 + window_slot(c.sink, c.recent, token(w))) * kHeadDim + ch]);
+  // sixteen tokens' loads in flight before their multiply-adds
+  constexpr int kBatch = 16;
+  const __nv_bfloat16* vb = c.vwin + row0 * kHeadDim + ch;
+  int w = 0;
+  for (; w + kBatch <= W; w += kBatch) {
+    float v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) v[i] = __bfloat162float(vb[(size_t)slot[w + i] * kHeadDim]);
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i)
+#pragma unroll
+      for (int g = 0; g < G; ++g) o[g] = fmaf(pw[g * WS + w + i], v[i], o[g]);
+  }
+  for (; w < W; ++w) {
+    const float v = __bfloat162float(vb[(size_t)slot[w] * kHeadDim]);
 #pragma unroll
     for (int g = 0; g < G; ++g) o[g] = fmaf(pw[g * WS + w], v, o[g]);
   }
@@ -1130,7 +1150,7 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
 template <int G>
 cudaError_t launch_window_g(const DecodeArgs& a, cudaStream_t s) {
   const int ws = a.c.sink + a.c.recent;
-  const size_t smem = (size_t)(G * kHeadDim + G * ws + G * 4) * sizeof(float);
+  const size_t smem = (size_t)(G * kHeadDim + G * ws + G * 4 + ws) * sizeof(float);
   auto kern = a.dtype == KVQ_F32 ? k_window<G, float> : (a.dtype == KVQ_BF16 ? k_window<G, __nv_bfloat16> : k_window<G, __half>);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
