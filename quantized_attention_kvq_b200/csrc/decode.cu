@@ -917,131 +917,6 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   }
 }
 
-// Attention over the bf16 window tokens of one unit (sequence b, kv head h):
-// tokens n < sink and the last `recent` tokens, scored over every channel from
-// the bf16 rotated keys (Dual-QK Sec. 3.3; tq-kv sink tokens), one partial
-// (max and sum in base-2 units, unnormalized values) per query head at slot
-// win_base + unit for the combine.  Thread = window token for the scores and
-// weights, thread = channel for the value sums.
-template <int G, typename In>
-__global__ void __launch_bounds__(kHeadDim) k_window(DecodeArgs a) {
-  extern __shared__ float wsm[];  // q [G][128], weights [G][sink + recent], reductions [G][4], slots [sink + recent]
-  const CacheView& c = a.c;
-  const int u = blockIdx.x, b = u / c.H, h = u - b * c.H;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int WS = c.sink + c.recent;
-  const int len = min(max(a.seq_lens[b], 0), a.max_len);
-  const int n_sink = min(c.sink, len);
-  const int r0 = c.recent > 0 ? max(c.sink, len - c.recent) : len;  // first recent token
-  const int W = n_sink + max(len - r0, 0);                            // window tokens
-  float* qs = wsm;
-  float* pw = wsm + G * kHeadDim;
-  float* red = pw + G * WS;
-  int* slot = reinterpret_cast<int*>(red + G * 4);  // window slot of window token w
-  const size_t row0 = (size_t)u * WS;
-  for (int w = tid; w < W; w += kHeadDim)
-    slot[w] = window_slot(c.sink, c.recent, w < n_sink ? w : r0 + (w - n_sink));
-  // the query rows, rotated as the keys are, one warp per head
-  for (int g = warp; g < G; g += kHeadDim / 32) {
-    float x[4];
-    load_row_warp(static_cast<const In*>(a.q) + ((size_t)b * a.Hq + (size_t)h * G + g) * kHeadDim, c.rotate != 0,
-                  a.inv_sqrt_d, lane, x);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) qs[g * kHeadDim + 4 * lane + i] = x[i];
-  }
-  __syncthreads();
-  // scores (base-2 units) of every window token, all channels
-  float mloc[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) mloc[g] = -__int_as_float(0x7f800000);
-  for (int w = tid; w < W; w += kHeadDim) {
-    // the whole bf16 key row in flight at once (16 independent 16-byte loads)
-    const uint4* kr = reinterpret_cast<const uint4*>(c.kwin + (row0 + slot[w]) * kHeadDim);
-    uint4 raw[kHeadDim / 8];
-#pragma unroll
-    for (int i = 0; i < kHeadDim / 8; ++i) raw[i] = kr[i];
-    float acc[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = 0.0f;
-#pragma unroll
-    for (int i8 = 0; i8 < kHeadDim / 8; ++i8) {
-      const uint32_t pr[4] = {raw[i8].x, raw[i8].y, raw[i8].z, raw[i8].w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int cc = 8 * i8 + 2 * i;
-        const float k0 = __uint_as_float(pr[i] << 16), k1 = __uint_as_float(pr[i] & 0xFFFF0000u);
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-          acc[g] = fmaf(qs[g * kHeadDim + cc + 1], k1, fmaf(qs[g * kHeadDim + cc], k0, acc[g]));
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float sc = acc[g] * a.scale_log2;
-      pw[g * WS + w] = sc;
-      mloc[g] = fmaxf(mloc[g], sc);
-    }
-  }
-  // per head: the max, then weights 2^(s - max) and their sum
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float mx = warp_max(mloc[g]);
-    if (lane == 0) red[g * 4 + warp] = mx;
-  }
-  __syncthreads();
-  float m[G], lsum[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = fmaxf(fmaxf(red[g * 4], red[g * 4 + 1]), fmaxf(red[g * 4 + 2], red[g * 4 + 3]));
-    lsum[g] = 0.0f;
-  }
-  __syncthreads();
-  for (int w = tid; w < W; w += kHeadDim)
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float p = exp2f(pw[g * WS + w] - m[g]);
-      pw[g * WS + w] = p;
-      lsum[g] += p;
-    }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float sm = warp_sum(lsum[g]);
-    if (lane == 0) red[g * 4 + warp] = sm;
-  }
-  __syncthreads();
-  // value sums, thread = channel
-  const int ch = tid;
-  float o[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) o[g] = 0.0f;
-  // sixteen tokens' loads in flight before their multiply-adds
-  constexpr int kBatch = 16;
-  const __nv_bfloat16* vb = c.vwin + row0 * kHeadDim + ch;
-  int w = 0;
-  for (; w + kBatch <= W; w += kBatch) {
-    float v[kBatch];
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) v[i] = __bfloat162float(vb[(size_t)slot[w + i] * kHeadDim]);
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i)
-#pragma unroll
-      for (int g = 0; g < G; ++g) o[g] = fmaf(pw[g * WS + w + i], v[i], o[g]);
-  }
-  for (; w < W; ++w) {
-    const float v = __bfloat162float(vb[(size_t)slot[w] * kHeadDim]);
-#pragma unroll
-    for (int g = 0; g < G; ++g) o[g] = fmaf(pw[g * WS + w], v, o[g]);
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const size_t r = (size_t)(a.win_base + u) * G + g;
-    a.part_acc[r * kHeadDim + ch] = o[g];
-    if (ch == 0)
-      a.part_ml[r] = W > 0 ? make_float2(m[g], red[g * 4] + red[g * 4 + 1] + red[g * 4 + 2] + red[g * 4 + 3])
-                           : make_float2(-__int_as_float(0x7f800000), 0.0f);
-  }
-}
-
 // Merges a unit's partials (one per CTA its tiles were spread over) into one
 // softmax over the whole sequence: o = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s,
 // rotated back into the value basis when the values were stored rotated.
@@ -1145,30 +1020,6 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.c.k_bits == 4) return launch_bits<4, 2>(a, s);
   if (a.c.v_bits == 4) return launch_bits<2, 4>(a, s);
   return launch_bits<2, 2>(a, s);
-}
-
-template <int G>
-cudaError_t launch_window_g(const DecodeArgs& a, cudaStream_t s) {
-  const int ws = a.c.sink + a.c.recent;
-  const size_t smem = (size_t)(G * kHeadDim + G * ws + G * 4 + ws) * sizeof(float);
-  auto kern = a.dtype == KVQ_F32 ? k_window<G, float> : (a.dtype == KVQ_BF16 ? k_window<G, __nv_bfloat16> : k_window<G, __half>);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  kern<<<a.c.B * a.c.H, kHeadDim, smem, s>>>(a);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_window(const DecodeArgs& a, cudaStream_t s) {
-  switch (a.Hq / a.c.H) {
-    case 1: return launch_window_g<1>(a, s);
-    case 2: return launch_window_g<2>(a, s);
-    case 4: return launch_window_g<4>(a, s);
-    case 8: return launch_window_g<8>(a, s);
-    case 16: return launch_window_g<16>(a, s);
-    default: return cudaErrorInvalidValue;
-  }
 }
 
 cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
