@@ -167,6 +167,14 @@ void orc_fwht(double* x, int32_t d) {
       }
 }
 
+void orc_transform(const float* A, const float* x, int32_t d, float* out) {
+  for (int i = 0; i < d; ++i) {
+    double acc = 0.0;
+    for (int j = 0; j < d; ++j) acc += (double)A[(size_t)i * d + j] * (double)x[j];
+    out[i] = (float)acc;
+  }
+}
+
 void orc_rotate(const float* x, int32_t d, float* out) {
   std::vector<double> t(d);
   for (int i = 0; i < d; ++i) t[i] = (double)x[i];
@@ -243,6 +251,7 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
                             int32_t offset, orc_stats* stats, uint8_t* k_row_exempt, uint8_t* v_row_exempt) {
   const int d = c->head_dim;
   if (d % kGroup != 0 || n_new < 0 || offset < 0 || offset + n_new > c->capacity) return -1;
+  if (c->rotate_k == 2 && !c->t_k) return -1;
   if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return -1;
   const int ngroups = d / kGroup, npg = d / kGranule;
   orc_stats total = {0, 0, 0, 0, 0, 0, 0};
@@ -257,7 +266,9 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
       const int n = offset + t;
       const size_t row = ((size_t)bh * n_new + t) * d;
       // ---- keys: rotate, optional channel 0 in bf16, quantize, pack ----
-      if (c->rotate_k)
+      if (c->rotate_k == 2)
+        orc_transform(c->t_k + (size_t)h * d * d, k_new + row, d, xr.data());
+      else if (c->rotate_k)
         orc_rotate(k_new + row, d, xr.data());
       else
         for (int i = 0; i < d; ++i) xr[i] = k_new[row + i];
@@ -388,8 +399,8 @@ void orc_dequantize(const orc_cache* c, int32_t b, int32_t h, int32_t n0, int32_
   }
 }
 
-void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t rotate, int32_t keep,
-                uint32_t* mask, double* energy) {
+void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t rotate, const float* t_q,
+                int32_t keep, uint32_t* mask, double* energy) {
   const int G = Hq / Hkv, npg = d / kGranule;
   std::vector<float> qr((size_t)G * d);
   std::vector<double> E(npg);
@@ -397,7 +408,9 @@ void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, i
     for (int hk = 0; hk < Hkv; ++hk) {
       for (int g = 0; g < G; ++g) {
         const float* qi = q + ((size_t)b * Hq + (size_t)hk * G + g) * d;
-        if (rotate)
+        if (rotate == 2)
+          orc_transform(t_q + (size_t)hk * d * d, qi, d, &qr[(size_t)g * d]);
+        else if (rotate)
           orc_rotate(qi, d, &qr[(size_t)g * d]);
         else
           for (int i = 0; i < d; ++i) qr[(size_t)g * d + i] = qi[i];
@@ -438,7 +451,9 @@ void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t
     const int len = lens[b];
     if (len <= 0) continue;
     std::vector<float> qr(d);
-    if (c->rotate_k)
+    if (c->rotate_k == 2)
+      orc_transform(c->t_q + (size_t)hk * d * d, q + (size_t)row * d, d, qr.data());
+    else if (c->rotate_k)
       orc_rotate(q + (size_t)row * d, d, qr.data());
     else
       for (int i = 0; i < d; ++i) qr[i] = q[(size_t)row * d + i];

@@ -31,6 +31,13 @@
  *    BF16) and tq-kv's sink-token preservation: window tokens are kept as bf16
  *    copies of the rotated key and of the (rotated) value and scored in full
  *    (all channels), under the same softmax as the quantized tokens.
+ *  - Dual-QK Sec. 1 and Sec. 3.1: a general dual transform pair, fixed per
+ *    KV head.  Queries take an invertible d x d matrix T and keys its inverse
+ *    transpose, so that (T q).(T^{-T} k) = q.k before quantization and
+ *    pruning; both matrices are supplied by the caller (calibrating them is
+ *    outside the decode path).  Each output is the fp64 sum over j = 0..d-1,
+ *    in that order, of A[i][j] x[j] (product and sum each rounded once),
+ *    rounded to fp32.
  *
  * Precision: FWHT in fp64 (natural Sylvester order), rotated values rounded
  * to fp32; quantization in fp32 with IEEE round-half-to-even; dequantization,
@@ -48,7 +55,8 @@ extern "C" {
 typedef struct {
   int32_t batch, kv_heads, head_dim, capacity;
   int32_t k_bits, v_bits; /* 2 or 4 */
-  int32_t rotate_k, keep_ch0;
+  int32_t rotate_k; /* 0: none; 1: orthonormal Walsh-Hadamard on keys and queries; 2: the caller's pair */
+  int32_t keep_ch0;
   int32_t rotate_v; /* 1: values pass through the orthonormal Walsh-Hadamard transform before quantization */
   float v_clip;     /* value clipping ratio in (0, 1]; 1 = no clipping                              */
   uint8_t* k_codes;   /* [B][Hkv][ceil(cap/128)][d/4][128] x (4*k_bits/8) bytes     */
@@ -63,6 +71,10 @@ typedef struct {
   int32_t sink, recent;
   uint16_t* k_win; /* [B][Hkv][sink + recent][d] bf16 rotated key, or NULL   */
   uint16_t* v_win; /* [B][Hkv][sink + recent][d] bf16 (rotated) value, or NULL */
+  /* rotate_k == 2: per kv head, row-major d x d fp32 matrices, T for queries
+     and T^{-T} for keys; NULL otherwise */
+  const float* t_q; /* [Hkv][d][d] */
+  const float* t_k; /* [Hkv][d][d] */
 } orc_cache;
 
 typedef struct {
@@ -76,6 +88,9 @@ typedef struct {
 void orc_fwht(double* x, int32_t d);
 /* out = fp32(FWHT(x) * (1/sqrt(d))) */
 void orc_rotate(const float* x, int32_t d, float* out);
+
+/* out[i] = fp32(sum_j A[i][j] * x[j]), fp64 products and sums in order j = 0..d-1 */
+void orc_transform(const float* A, const float* x, int32_t d, float* out);
 
 /* IEEE binary16 / bfloat16 round-to-nearest-even from fp32, and widening */
 uint16_t orc_half_rn(float x);
@@ -114,12 +129,13 @@ void orc_dequantize(const orc_cache* c, int32_t b, int32_t h, int32_t n0, int32_
 /*
  * Channel selection: per (b, kv head) keep the `keep` channel groups of 4
  * with the largest query energy summed over the GQA group.  q is
- * [B][Hq][d] fp32 values (un-rotated; rotated here when rotate != 0).
+ * [B][Hq][d] fp32 values (un-rotated; rotated here when rotate == 1, taken
+ * through t_q[h] ([Hkv][d][d], the pair's query matrix) when rotate == 2).
  * mask[b*Hkv + h] bit p set = group p kept.  energy (may be NULL) receives
  * [B][Hkv][d/4] fp64 energies.
  */
-void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t rotate, int32_t keep,
-                uint32_t* mask, double* energy);
+void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, int32_t rotate, const float* t_q,
+                int32_t keep, uint32_t* mask, double* energy);
 
 /*
  * Decode attention over the oracle cache for rows r = b*Hq + hq listed in

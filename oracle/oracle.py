@@ -22,7 +22,7 @@ class OrcCache(ctypes.Structure):
                 ("k_bits", _I32), ("v_bits", _I32), ("rotate_k", _I32), ("keep_ch0", _I32),
                 ("rotate_v", _I32), ("v_clip", ctypes.c_float),
                 ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P),
-                ("sink", _I32), ("recent", _I32), ("k_win", _P), ("v_win", _P)]
+                ("sink", _I32), ("recent", _I32), ("k_win", _P), ("v_win", _P), ("t_q", _P), ("t_k", _P)]
 
 
 class OrcStats(ctypes.Structure):
@@ -37,6 +37,7 @@ def lib():
         L = ctypes.CDLL(so)
         L.orc_fwht.argtypes = [_P, _I32]
         L.orc_rotate.argtypes = [_P, _I32, _P]
+        L.orc_transform.argtypes = [_P, _P, _I32, _P]
         L.orc_half_rn.argtypes = [ctypes.c_float]
         L.orc_half_rn.restype = ctypes.c_uint16
         L.orc_half_value.argtypes = [ctypes.c_uint16]
@@ -54,7 +55,7 @@ def lib():
         L.orc_quantize_append.restype = _I32
         L.orc_unpack_codes.argtypes = [ctypes.POINTER(OrcCache), _I32, _I32, _I32, _I32, _P]
         L.orc_dequantize.argtypes = [ctypes.POINTER(OrcCache), _I32, _I32, _I32, _I32, _P, _P]
-        L.orc_select.argtypes = [_P, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P]
+        L.orc_select.argtypes = [_P, _I32, _I32, _I32, _I32, _I32, _P, _I32, _P, _P]
         L.orc_attention.argtypes = [ctypes.POINTER(OrcCache), _P, _I32, _P, _P, ctypes.c_double, _P, _I32, _P]
         L.orc_dual_score.argtypes = [_P, _I32, _P, _P]
         L.orc_dual_score.restype = ctypes.c_double
@@ -85,6 +86,15 @@ def rotate(x: np.ndarray) -> np.ndarray:
     xi = np.ascontiguousarray(x, dtype=np.float32)
     out = np.empty_like(xi)
     lib().orc_rotate(_p(xi), xi.size, _p(out))
+    return out
+
+
+def transform(A: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """fp32 of the fp64 product A x (sum over j in order) of one row."""
+    Ac = np.ascontiguousarray(A, dtype=np.float32)
+    xi = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty_like(xi)
+    lib().orc_transform(_p(Ac), _p(xi), xi.size, _p(out))
     return out
 
 
@@ -123,8 +133,14 @@ class Cache:
     """Host copy of the packed cache, written by the oracle."""
 
     def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, rotate_v=0, v_clip=1.0,
-                 sink=0, recent=0):
+                 sink=0, recent=0, t_q=None, t_k=None):
+        """rotate_k = 2 takes the caller's pair: t_q [Hkv][d][d] on queries and
+        t_k [Hkv][d][d] (its inverse transpose) on keys, fp32 row-major."""
         self.B, self.Hkv, self.d, self.capacity = B, Hkv, d, capacity
+        if rotate_k == 2:
+            t_q = np.ascontiguousarray(t_q, dtype=np.float32).reshape(Hkv, d, d)
+            t_k = np.ascontiguousarray(t_k, dtype=np.float32).reshape(Hkv, d, d)
+        self.t_q, self.t_k = t_q, t_k
         self.k_bits, self.v_bits, self.rotate_k, self.keep_ch0 = k_bits, v_bits, rotate_k, keep_ch0
         self.rotate_v, self.v_clip, self.sink, self.recent = rotate_v, v_clip, sink, recent
         w = B * Hkv * (sink + recent) * d
@@ -138,7 +154,8 @@ class Cache:
         self.v_scales = np.zeros(B * Hkv * capacity * (d // 32) * 2, np.uint16)
         self.struct = OrcCache(B, Hkv, d, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v, v_clip,
                                _p(self.k_codes), _p(self.k_scales), _p(self.k_ch0), _p(self.v_codes),
-                               _p(self.v_scales), sink, recent, _p(self.k_win), _p(self.v_win))
+                               _p(self.v_scales), sink, recent, _p(self.k_win), _p(self.v_win),
+                               _p(self.t_q) if rotate_k == 2 else None, _p(self.t_k) if rotate_k == 2 else None)
 
     def append(self, k_new: np.ndarray, v_new: np.ndarray, offset: int, want_exempt: bool = False):
         """k_new, v_new: [B][Hkv][n][d] (bf16 as uint16, or fp32)."""
@@ -184,13 +201,15 @@ class Cache:
         return out
 
 
-def select(q: np.ndarray, Hkv: int, rotate: int, keep: int):
-    """-> (mask [B][Hkv] uint32, energy [B][Hkv][d/4] fp64)"""
+def select(q: np.ndarray, Hkv: int, rotate: int, keep: int, t_q: np.ndarray | None = None):
+    """-> (mask [B][Hkv] uint32, energy [B][Hkv][d/4] fp64); rotate = 2 takes
+    the pair's query matrices t_q [Hkv][d][d]."""
     qf = as_f32(q)
+    tq = np.ascontiguousarray(t_q, dtype=np.float32) if rotate == 2 else None
     B, Hq, d = qf.shape
     mask = np.zeros((B, Hkv), np.uint32)
     energy = np.zeros((B, Hkv, d // 4), np.float64)
-    lib().orc_select(_p(qf), B, Hq, Hkv, d, rotate, keep, _p(mask), _p(energy))
+    lib().orc_select(_p(qf), B, Hq, Hkv, d, rotate, _p(tq), keep, _p(mask), _p(energy))
     return mask, energy
 
 
