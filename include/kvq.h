@@ -81,7 +81,8 @@ typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1, KVQ_F16 = 2 } kvq_dtype;
 typedef struct {
   int32_t batch, kv_heads, head_dim, capacity;
   int32_t k_bits, v_bits, group_size, prune_granule;
-  int32_t rotate_k; /* 1: keys (and queries) pass through the orthonormal Walsh-Hadamard transform */
+  int32_t rotate_k; /* 1: keys (and queries) pass through the orthonormal Walsh-Hadamard transform;
+                       2: through the caller's dual transform pair t_query / t_key (below)       */
   int32_t keep_ch0; /* 1: rotated channel 0 of each key is kept in bf16, unquantized               */
   int32_t rotate_v; /* 1: values pass through the orthonormal Walsh-Hadamard transform before they
                        are quantized, and decode outputs are rotated back [DQK App. B.2]           */
@@ -109,6 +110,18 @@ typedef struct {
   int32_t sink_tokens, recent_tokens;
   void* k_window;
   void* v_window;
+  /* Dual transform pair [DQK Sec. 1, Sec. 3.1], used when rotate_k == 2 (NULL
+     otherwise): per kv head an invertible d x d matrix T applied to queries
+     and its inverse transpose applied to keys, so that (T q).(T^-T k) = q.k
+     before quantization and pruning.  Both are caller-owned device fp32
+     arrays [H][d][d], row-major, 16-byte aligned, read but never written; the
+     library does not check that t_key is T^-T.  Each transformed channel i is
+     sum_j A[i][j] x[j] over j = 0..d-1 in that order, fp64 products and sums
+     each rounded once, rounded to fp32.  Keys, their bf16 window copies and
+     channel 0 (keep_ch0) are taken after the transform; values are not
+     affected. */
+  const float* t_query;
+  const float* t_key;
 } kvq_cache;
 
 /*
@@ -129,8 +142,9 @@ KVQ_API size_t kvq_window_bytes(const kvq_cache* cache);
  * same sequence whose ranges touch the same 64-token window must not run
  * concurrently (on different streams without ordering).
  *  k_new, v_new: device [B][H][n_new][d] of `dtype`.
- * Keys: x = H_d k / sqrt(d) when rotate_k (fp64 butterflies in natural
- * Sylvester order, rounded to fp32) [DQK Sec. 1; SIQ KQV; TQ]; channel 0 to
+ * Keys: x = H_d k / sqrt(d) when rotate_k == 1 (fp64 butterflies in natural
+ * Sylvester order, rounded to fp32) [DQK Sec. 1; SIQ KQV; TQ], x = t_key[h] k
+ * when rotate_k == 2 (fp64 in-order sums, rounded to fp32); channel 0 to
  * bf16 when keep_ch0; then per token and per 32-channel group
  * scale = fp16((max - min) / L), zero = fp16(min), L = 2^bits - 1,
  * code = clamp(round_half_even((x - zero) / scale), 0, L) with IEEE fp32
@@ -150,7 +164,8 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new
  * the keep_groups largest energies are kept, equal energies keeping the
  * lower p.  mask_out[b*H + h] (device uint32) gets bit p set for a kept group.
  *  q: device [B][q_heads][d] of `dtype`, un-rotated (rotated here when
- *  rotate_k).  Query head j belongs to kv head j / G.  keep_groups in [1, 32].
+ *  rotate_k == 1, q_rot = t_query[h] q when rotate_k == 2).  Query head j
+ *  belongs to kv head j / G.  keep_groups in [1, 32].
  */
 KVQ_API kvq_status kvq_select_channels(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
                                        int32_t keep_groups, uint32_t* mask_out, void* stream);
@@ -173,7 +188,8 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_head
  * max and sum, and a combine pass merges the pieces into one softmax over the
  * whole sequence [DQK Sec. 3.4].  Supported GQA group sizes
  * G = q_heads / kv_heads: 1, 2, 4, 8, 16 (others: KVQ_ERR_UNSUPPORTED).
- *  q:        device [B][q_heads][d] of `dtype`, un-rotated.
+ *  q:        device [B][q_heads][d] of `dtype`, un-rotated (with rotate_k == 2
+ *            the workspace also holds the transformed fp32 query rows).
  *  seq_lens: device int32 [B]; entries are clamped to [0, max_len]; a
  *            sequence of length 0 gets a zero output.
  *  max_len:  host bound on seq_lens, 0 <= max_len <= capacity; sizes the grid.

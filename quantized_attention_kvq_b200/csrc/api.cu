@@ -4,7 +4,7 @@
 #include <cmath>
 #include <cstdint>
 
-#include "common.cuh"
+#include "transform.cuh"
 
 namespace kvq {
 namespace {
@@ -20,7 +20,7 @@ inline bool dtype_ok(int t) { return t == KVQ_F32 || t == KVQ_BF16 || t == KVQ_F
 kvq_status check_shape(const kvq_cache* c) {
   if (!c) return KVQ_ERR_INVALID_ARG;
   if (c->batch < 1 || c->kv_heads < 1 || c->capacity < 1 || c->head_dim < 1) return KVQ_ERR_INVALID_ARG;
-  if ((c->rotate_k != 0 && c->rotate_k != 1) || (c->keep_ch0 != 0 && c->keep_ch0 != 1)) return KVQ_ERR_INVALID_ARG;
+  if (c->rotate_k < 0 || c->rotate_k > 2 || (c->keep_ch0 != 0 && c->keep_ch0 != 1)) return KVQ_ERR_INVALID_ARG;
   if ((c->rotate_v != 0 && c->rotate_v != 1) || !(c->v_clip > 0.0f && c->v_clip <= 1.0f)) return KVQ_ERR_INVALID_ARG;
   if (c->sink_tokens < 0 || c->recent_tokens < 0 || (int64_t)c->sink_tokens + c->recent_tokens > c->capacity)
     return KVQ_ERR_INVALID_ARG;
@@ -31,9 +31,16 @@ kvq_status check_shape(const kvq_cache* c) {
   return KVQ_OK;
 }
 
+// the caller's transform pair, when rotate_k selects it
+bool pair_ok(const kvq_cache* c, bool query, bool key) {
+  if (c->rotate_k != 2) return true;
+  return (!query || (c->t_query && aligned16(c->t_query))) && (!key || (c->t_key && aligned16(c->t_key)));
+}
+
 kvq_status check_cache(const kvq_cache* c) {
   kvq_status st = check_shape(c);
   if (st != KVQ_OK) return st;
+  if (!pair_ok(c, true, true)) return KVQ_ERR_INVALID_ARG;
   if (!c->k_codes || !c->k_scales || !c->v_codes || !c->v_scales || (c->keep_ch0 && !c->k_ch0))
     return KVQ_ERR_INVALID_ARG;
   if (!aligned16(c->k_codes) || !aligned16(c->k_scales) || !aligned16(c->v_codes) || !aligned16(c->v_scales) ||
@@ -76,9 +83,10 @@ CacheView view(const kvq_cache* c) {
 double inv_sqrt_d() { return 1.0 / std::sqrt((double)kHeadDim); }
 
 // Workspace of the decode: one partial row (128-channel accumulator, running
-// max and sum) per (slot, query head of the GQA group), decode_slots slots.
+// max and sum) per (slot, query head of the GQA group), decode_slots slots;
+// with the caller's transform pair, then the transformed fp32 query rows.
 struct DecodePlan {
-  size_t acc_bytes, ml_offset, bytes;
+  size_t acc_bytes, ml_offset, tq_offset, bytes;
 };
 
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
@@ -88,7 +96,9 @@ DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   const size_t rows = ((size_t)decode_slots(c->batch, c->kv_heads, G) + (win ? c->batch * c->kv_heads : 0)) * G;
   p.acc_bytes = rows * kHeadDim * sizeof(float);
   p.ml_offset = round_up(p.acc_bytes, kAlign);
-  p.bytes = p.ml_offset + round_up(rows * sizeof(float2), kAlign);
+  p.tq_offset = p.ml_offset + round_up(rows * sizeof(float2), kAlign);
+  p.bytes = p.tq_offset;
+  if (c->rotate_k == 2) p.bytes += round_up((size_t)c->batch * q_heads * kHeadDim * sizeof(float), kAlign);
   return p;
 }
 
@@ -115,6 +125,15 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.part_acc = static_cast<float*>(workspace);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
+  if ((parts & kRunSplit) && c->rotate_k == 2) {
+    // the kernels below read the transformed rows as untransformed fp32 queries
+    float* qt = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.tq_offset);
+    kvq_status st = cuda_status(launch_transform_q(q, dtype, c->t_query, c->batch, q_heads, c->kv_heads, qt, s));
+    if (st != KVQ_OK) return st;
+    a.q = qt;
+    a.dtype = KVQ_F32;
+    a.c.rotate = 0;
+  }
   if ((parts & kRunSplit) && max_len > 0) {
     kvq_status st = cuda_status(launch_decode(a, s));
     if (st != KVQ_OK) return st;
@@ -196,7 +215,7 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* c, const void* k_new, co
   a.n_new = n_new;
   a.offset = offset;
   a.inv_sqrt_d = inv_sqrt_d();
-  return cuda_status(launch_append(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_append_pair(a, c->t_key, static_cast<cudaStream_t>(stream)));
 }
 
 KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
@@ -204,7 +223,7 @@ KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dt
   kvq_status st = check_shape(c);
   if (st != KVQ_OK) return st;
   if ((st = check_heads(c, q_heads)) != KVQ_OK) return st;
-  if (!dtype_ok(dtype) || !q || !mask_out || !aligned16(q)) return KVQ_ERR_INVALID_ARG;
+  if (!dtype_ok(dtype) || !q || !mask_out || !aligned16(q) || !pair_ok(c, true, false)) return KVQ_ERR_INVALID_ARG;
   if (keep_groups < 1 || keep_groups > kPruneGroups) return KVQ_ERR_INVALID_ARG;
   if (q_heads / c->kv_heads > 64) return KVQ_ERR_UNSUPPORTED;
   SelectArgs a;
@@ -217,7 +236,7 @@ KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dt
   a.keep = keep_groups;
   a.inv_sqrt_d = inv_sqrt_d();
   a.mask = mask_out;
-  return cuda_status(launch_select(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_select_pair(a, c->t_query, static_cast<cudaStream_t>(stream)));
 }
 
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* c, int32_t q_heads, int32_t max_len) {

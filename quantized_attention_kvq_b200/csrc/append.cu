@@ -4,7 +4,8 @@
 // 64-token-aligned window of the cache; each of its 8 warps takes 8 tokens,
 // four lanes per token, lane g of a token owning the 32 channels of
 // quantization group g.  Keys: fp64 Walsh-Hadamard butterflies (Dual-QK
-// summary Sec. 1; gist.science KQV scheme), optional bf16 channel 0 (Dual-QK
+// summary Sec. 1; gist.science KQV scheme) or the kv head's key matrix of the
+// caller's dual transform pair (Dual-QK Sec. 1, Sec. 3.1), optional bf16 channel 0 (Dual-QK
 // Sec. 3.3, App. C.3), per-32-channel asymmetric quantization (Dual-QK
 // Sec. 3.3).  Values: the same quantizer, optionally after the same rotation
 // and with a clipping ratio on each group's range (Dual-QK App. B.2).
@@ -14,7 +15,7 @@
 // change (tq-kv incremental cache); value-code words that also hold tokens
 // outside that range are read, patched and written back by the one CTA whose
 // window contains them.
-#include "common.cuh"
+#include "transform.cuh"
 
 namespace kvq {
 namespace {
@@ -209,6 +210,38 @@ __device__ __forceinline__ void rotate_row_4lanes(float (&v)[32], int g, double 
   for (int i = 0; i < 32; ++i) v[i] = __double2float_rn(__dmul_rn(x[i], inv_sqrt_d));
 }
 
+// Key row through the kv head's matrix A of the caller's transform pair, held
+// by four lanes as above: channel 32g + r is the fp64 sum over j = 0..127, in
+// order, of A[32g + r][j] x_j (product and sum each rounded once), rounded to
+// fp32; x_j comes from lane j / 32 of the quad by shuffles.  All 32 lanes of
+// the warp take part.
+__device__ __forceinline__ void transform_row_4lanes(float (&v)[32], int g, int lane, const float* __restrict__ A) {
+  const int base = lane & ~3;
+  const float4* rows = reinterpret_cast<const float4*>(A) + (size_t)32 * g * (kHeadDim / 4);
+  double acc[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) acc[r] = 0.0;
+#pragma unroll 1
+  for (int src = 0; src < 4; ++src) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      double xs[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) xs[k] = (double)__shfl_sync(kFull, v[4 * e + k], base + src);
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        const float4 m = __ldg(rows + r * (kHeadDim / 4) + src * 8 + e);  // A[32g + r][32 src + 4e .. + 3]
+        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.x, xs[0]));
+        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.y, xs[1]));
+        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.z, xs[2]));
+        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.w, xs[3]));
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < 32; ++r) v[r] = __double2float_rn(acc[r]);
+}
+
 // bf16 (round to nearest even) copy of this lane's 32 channels into a window row
 __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* dst, const float (&v)[32]) {
   uint32_t w[16];
@@ -222,8 +255,11 @@ __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* dst, const float (&
   for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
-template <int KB, int VB, bool ROT, bool CH0, bool ROTV, typename In>
-__global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(AppendArgs a) {
+// ROT: 0 keys as given, 1 Walsh-Hadamard rotation, 2 the pair's key matrix
+// tk[h] (its fp64 accumulators need the registers of fewer resident blocks)
+template <int KB, int VB, int ROT, bool CH0, bool ROTV, typename In>
+__global__ void __launch_bounds__(kAppendWarps * 32, ROT == 2 ? 1 : 3)
+    k_quantize_append(AppendArgs a, const float* __restrict__ tk) {
   constexpr int TPW = 32 / VB;            // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
   constexpr int WPR = kAppendTile / TPW;  // value words per channel in the window: 8 or 4
   // key words [pruning group][token], 16 bits a token (its KB * 4 low bits used)
@@ -266,7 +302,8 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
   widen(kraw, kx);
 
   // ---- key row: rotated, then quantized (keys are not clipped)
-  if (ROT) rotate_row_4lanes(kx, g, a.inv_sqrt_d);
+  if (ROT == 1) rotate_row_4lanes(kx, g, a.inv_sqrt_d);
+  if (ROT == 2) transform_row_4lanes(kx, g, lane, tk + (size_t)h * kPairElems);
   // bf16 window copies (rotated key, then the value below) for tokens with a
   // window slot: every sink token, and of the later tokens only this append's
   // last `recent`, the ones that still own their ring slot when it ends (an
@@ -372,41 +409,44 @@ __global__ void __launch_bounds__(kAppendWarps * 32, 3) k_quantize_append(Append
   }
 }
 
-template <int KB, int VB, bool ROT, bool CH0, bool ROTV>
-cudaError_t launch_typed(const AppendArgs& a, cudaStream_t s) {
+template <int KB, int VB, int ROT, bool CH0, bool ROTV>
+cudaError_t launch_typed(const AppendArgs& a, const float* tk, cudaStream_t s) {
   const int first = a.offset / kAppendTile, last = (a.offset + a.n_new - 1) / kAppendTile;
   dim3 grid(last - first + 1, a.c.H, a.c.B);
   dim3 block(kAppendWarps * 32);
   switch (a.dtype) {
-    case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, ROTV, float><<<grid, block, 0, s>>>(a); break;
-    case KVQ_BF16: k_quantize_append<KB, VB, ROT, CH0, ROTV, __nv_bfloat16><<<grid, block, 0, s>>>(a); break;
-    default: k_quantize_append<KB, VB, ROT, CH0, ROTV, __half><<<grid, block, 0, s>>>(a); break;
+    case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, ROTV, float><<<grid, block, 0, s>>>(a, tk); break;
+    case KVQ_BF16: k_quantize_append<KB, VB, ROT, CH0, ROTV, __nv_bfloat16><<<grid, block, 0, s>>>(a, tk); break;
+    default: k_quantize_append<KB, VB, ROT, CH0, ROTV, __half><<<grid, block, 0, s>>>(a, tk); break;
   }
   return cudaGetLastError();
 }
 
 // value rotation is a template flag, so kernels without it stay as small as before
 template <int KB, int VB, bool ROTV>
-cudaError_t launch_flags(const AppendArgs& a, cudaStream_t s) {
-  const bool rot = a.c.rotate != 0, ch0 = a.c.keep_ch0 != 0;
-  if (rot && ch0) return launch_typed<KB, VB, true, true, ROTV>(a, s);
-  if (rot) return launch_typed<KB, VB, true, false, ROTV>(a, s);
-  if (ch0) return launch_typed<KB, VB, false, true, ROTV>(a, s);
-  return launch_typed<KB, VB, false, false, ROTV>(a, s);
+cudaError_t launch_flags(const AppendArgs& a, const float* tk, cudaStream_t s) {
+  const bool ch0 = a.c.keep_ch0 != 0;
+  if (a.c.rotate == 2)
+    return ch0 ? launch_typed<KB, VB, 2, true, ROTV>(a, tk, s) : launch_typed<KB, VB, 2, false, ROTV>(a, tk, s);
+  if (a.c.rotate == 1)
+    return ch0 ? launch_typed<KB, VB, 1, true, ROTV>(a, tk, s) : launch_typed<KB, VB, 1, false, ROTV>(a, tk, s);
+  return ch0 ? launch_typed<KB, VB, 0, true, ROTV>(a, tk, s) : launch_typed<KB, VB, 0, false, ROTV>(a, tk, s);
 }
 
 template <int KB, int VB>
-cudaError_t launch_bits(const AppendArgs& a, cudaStream_t s) {
-  return a.c.rotate_v ? launch_flags<KB, VB, true>(a, s) : launch_flags<KB, VB, false>(a, s);
+cudaError_t launch_bits(const AppendArgs& a, const float* tk, cudaStream_t s) {
+  return a.c.rotate_v ? launch_flags<KB, VB, true>(a, tk, s) : launch_flags<KB, VB, false>(a, tk, s);
 }
 
 }  // namespace
 
-cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
-  if (a.c.k_bits == 4 && a.c.v_bits == 4) return launch_bits<4, 4>(a, s);
-  if (a.c.k_bits == 4) return launch_bits<4, 2>(a, s);
-  if (a.c.v_bits == 4) return launch_bits<2, 4>(a, s);
-  return launch_bits<2, 2>(a, s);
+cudaError_t launch_append_pair(const AppendArgs& a, const float* tk, cudaStream_t s) {
+  if (a.c.k_bits == 4 && a.c.v_bits == 4) return launch_bits<4, 4>(a, tk, s);
+  if (a.c.k_bits == 4) return launch_bits<4, 2>(a, tk, s);
+  if (a.c.v_bits == 4) return launch_bits<2, 4>(a, tk, s);
+  return launch_bits<2, 2>(a, tk, s);
 }
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) { return launch_append_pair(a, nullptr, s); }
 
 }  // namespace kvq

@@ -1,9 +1,10 @@
 // Query-channel selection (Dual-QK summary Sec. 3.2, App. C.2): one CTA per
-// (sequence, kv head).  Its warps rotate the GQA group's query rows; warp 0
+// (sequence, kv head).  Its warps rotate the GQA group's query rows (or take
+// them through the kv head's matrix of the caller's transform pair); warp 0
 // then gives lane p the fp64 energy of channel group p (heads outer, channels
 // inner, the order the mask is defined in), ranks the 32 energies across the
 // warp (ties keep the lower group) and writes the kept-group bitmask.
-#include "common.cuh"
+#include "transform.cuh"
 
 namespace kvq {
 namespace {
@@ -12,7 +13,7 @@ constexpr int kSelectThreads = 128;
 constexpr int kMaxG = 64;
 
 template <typename In>
-__global__ void __launch_bounds__(kSelectThreads) k_select(SelectArgs a) {
+__global__ void __launch_bounds__(kSelectThreads) k_select(SelectArgs a, const float* __restrict__ tq) {
   __shared__ float4 qr[kMaxG][kPruneGroups];  // rotated query rows, 4 channels per entry
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
@@ -20,7 +21,8 @@ __global__ void __launch_bounds__(kSelectThreads) k_select(SelectArgs a) {
   const In* q = static_cast<const In*>(a.q) + ((size_t)b * a.Hq + (size_t)h * G) * kHeadDim;
   for (int j = warp; j < G; j += kSelectThreads / 32) {
     float x[4];
-    load_row_warp(q + (size_t)j * kHeadDim, a.rotate != 0, a.inv_sqrt_d, lane, x);
+    load_row_warp(q + (size_t)j * kHeadDim, a.rotate == 1, a.inv_sqrt_d, lane, x);
+    if (a.rotate == 2) transform_row_warp(x, tq + (size_t)h * kPairElems, lane);
     qr[j][lane] = make_float4(x[0], x[1], x[2], x[3]);
   }
   __syncthreads();
@@ -45,14 +47,16 @@ __global__ void __launch_bounds__(kSelectThreads) k_select(SelectArgs a) {
 
 }  // namespace
 
-cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) {
+cudaError_t launch_select_pair(const SelectArgs& a, const float* tq, cudaStream_t s) {
   dim3 grid(a.H, a.B), block(kSelectThreads);
   switch (a.dtype) {
-    case KVQ_F32: k_select<float><<<grid, block, 0, s>>>(a); break;
-    case KVQ_BF16: k_select<__nv_bfloat16><<<grid, block, 0, s>>>(a); break;
-    default: k_select<__half><<<grid, block, 0, s>>>(a); break;
+    case KVQ_F32: k_select<float><<<grid, block, 0, s>>>(a, tq); break;
+    case KVQ_BF16: k_select<__nv_bfloat16><<<grid, block, 0, s>>>(a, tq); break;
+    default: k_select<__half><<<grid, block, 0, s>>>(a, tq); break;
   }
   return cudaGetLastError();
 }
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t s) { return launch_select_pair(a, nullptr, s); }
 
 }  // namespace kvq

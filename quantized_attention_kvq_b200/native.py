@@ -31,7 +31,8 @@ class KvqCacheStruct(ctypes.Structure):
                 ("k_bits", _I32), ("v_bits", _I32), ("group_size", _I32), ("prune_granule", _I32),
                 ("rotate_k", _I32), ("keep_ch0", _I32), ("rotate_v", _I32), ("v_clip", ctypes.c_float),
                 ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P),
-                ("sink_tokens", _I32), ("recent_tokens", _I32), ("k_window", _P), ("v_window", _P)]
+                ("sink_tokens", _I32), ("recent_tokens", _I32), ("k_window", _P), ("v_window", _P),
+                ("t_query", _P), ("t_key", _P)]
 
 
 class KvqError(RuntimeError):
@@ -128,7 +129,15 @@ class KVQCache:
 
     def __init__(self, B: int, H: int, capacity: int, k_bits: int, v_bits: int, rotate_k: int = 1,
                  keep_ch0: int = 0, device="cuda", zero: bool = True, rotate_v: int = 0, v_clip: float = 1.0,
-                 sink: int = 0, recent: int = 0):
+                 sink: int = 0, recent: int = 0, t_query: torch.Tensor | None = None,
+                 t_key: torch.Tensor | None = None):
+        """rotate_k = 2 takes the caller's dual transform pair: t_query (T) and
+        t_key (T^-T), fp32 device tensors [H][128][128], kept referenced here."""
+        if rotate_k == 2 and (t_query is None or t_key is None):
+            raise ValueError("rotate_k = 2 needs t_query and t_key")
+        if rotate_k == 2 and (t_query.dtype != torch.float32 or t_key.dtype != torch.float32 or
+                              tuple(t_query.shape) != (H, 128, 128) or tuple(t_key.shape) != (H, 128, 128)):
+            raise ValueError("t_query and t_key are fp32 [H][128][128]")
         self.desc = describe(B, H, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v=rotate_v, v_clip=v_clip,
                              sink=sink, recent=recent)
         sizes = cache_sizes(self.desc)
@@ -148,6 +157,10 @@ class KVQCache:
         self.v_window = alloc(wb, dtype=torch.uint8, device=device) if wb else None
         self.desc.k_window = _dev_ptr(self.k_window)
         self.desc.v_window = _dev_ptr(self.v_window)
+        self.t_query = t_query.contiguous() if rotate_k == 2 else None
+        self.t_key = t_key.contiguous() if rotate_k == 2 else None
+        self.desc.t_query = _dev_ptr(self.t_query)
+        self.desc.t_key = _dev_ptr(self.t_key)
         self.B, self.H, self.capacity = B, H, capacity
 
     def sequence_desc(self, b: int) -> KvqCacheStruct:
@@ -166,6 +179,7 @@ class KVQCache:
             wper = self.k_window.numel() // self.B
             d.k_window = self.desc.k_window + b * wper
             d.v_window = self.desc.v_window + b * wper
+        d.t_query, d.t_key = self.desc.t_query, self.desc.t_key  # per kv head, shared by every sequence
         return d
 
     def append_sequence(self, b: int, k_new: torch.Tensor, v_new: torch.Tensor, offset: int, stream=None):

@@ -61,7 +61,8 @@ def test_cache_sizes_follow_layout(L):
     ("head_dim", 64, native.KVQ_ERR_UNSUPPORTED), ("k_bits", 3, native.KVQ_ERR_UNSUPPORTED),
     ("v_bits", 8, native.KVQ_ERR_UNSUPPORTED), ("capacity", 100, native.KVQ_ERR_UNSUPPORTED),
     ("group_size", 64, native.KVQ_ERR_UNSUPPORTED), ("prune_granule", 8, native.KVQ_ERR_UNSUPPORTED),
-    ("batch", 0, native.KVQ_ERR_INVALID_ARG), ("rotate_k", 2, native.KVQ_ERR_INVALID_ARG),
+    ("batch", 0, native.KVQ_ERR_INVALID_ARG), ("rotate_k", 3, native.KVQ_ERR_INVALID_ARG),
+    ("rotate_k", -1, native.KVQ_ERR_INVALID_ARG), ("rotate_k", 2, native.KVQ_ERR_INVALID_ARG),
     ("k_codes", 0, native.KVQ_ERR_INVALID_ARG), ("k_ch0", 0, native.KVQ_ERR_INVALID_ARG),
     ("v_scales", FAKE + 4, native.KVQ_ERR_INVALID_ARG), ("rotate_v", 2, native.KVQ_ERR_INVALID_ARG),
     ("v_clip", 0.0, native.KVQ_ERR_INVALID_ARG), ("v_clip", 1.5, native.KVQ_ERR_INVALID_ARG),
@@ -105,6 +106,36 @@ def test_window_sizes(L):
         setattr(big, f, FAKE)
     assert L.kvq_quantize_append(ctypes.byref(big), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
         native.KVQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("tq,tk", [(None, FAKE), (FAKE, None), (FAKE + 4, FAKE), (FAKE, FAKE + 8)])
+def test_transform_pair_pointers_checked(L, tq, tk):
+    d = desc(rotate_k=2)
+    d.t_query, d.t_key = tq, tk
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    ws = L.kvq_decode_workspace_bytes(ctypes.byref(d), 8, 256)
+    assert L.kvq_decode_attention(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, FAKE, 256, None, 0.088, FAKE, FAKE,
+                                  ws, None) == native.KVQ_ERR_INVALID_ARG
+    # the channel selection reads only the query matrices (called only where
+    # they are bad, so nothing is enqueued)
+    if tq != FAKE:
+        rc = L.kvq_select_channels(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, 4, FAKE, None)
+        assert rc == native.KVQ_ERR_INVALID_ARG
+
+
+def test_transform_pair_workspace_holds_the_transformed_queries(L):
+    d = desc()
+    p = desc(rotate_k=2)
+    p.t_query = p.t_key = FAKE
+    for q_heads in (8, 16):
+        plain = L.kvq_decode_workspace_bytes(ctypes.byref(d), q_heads, 256)
+        pair = L.kvq_decode_workspace_bytes(ctypes.byref(p), q_heads, 256)
+        assert pair - plain == -(-d.batch * q_heads * 128 * 4 // 256) * 256
+    # and the step entry point's workspace grows with it
+    assert L.kvq_decode_step_workspace_bytes(ctypes.byref(p), native.KVQ_BF16, 8, 256) - \
+        L.kvq_decode_step_workspace_bytes(ctypes.byref(d), native.KVQ_BF16, 8, 256) == \
+        L.kvq_decode_workspace_bytes(ctypes.byref(p), 8, 256) - L.kvq_decode_workspace_bytes(ctypes.byref(d), 8, 256)
 
 
 def test_append_argument_checks(L):
