@@ -155,6 +155,69 @@ inline const uint16_t* window_row(const orc_cache* c, const uint16_t* win, int b
 }  // namespace
 
 extern "C" {
+void orc_rope(const float* x, int32_t d, const float* inv_freq, int64_t pos, float* out);
+void orc_transform(const float* A, const float* x, int32_t d, float* out);
+void orc_rotate(const float* x, int32_t d, float* out);
+}
+
+namespace {
+
+// A key (query = false) or query row as the cache scores it: rotary-embedded
+// at `rel` when the cache uses bucket-relative RoPE, then taken through the
+// key or query side of the cache's transform.
+void prepare_row(const orc_cache* c, int h, const float* x, bool query, long rel, float* out) {
+  const int d = c->head_dim;
+  std::vector<float> e(x, x + d);
+  if (c->bucket_w > 0) orc_rope(x, d, c->rope_inv_freq, rel, e.data());
+  if (c->rotate_k == 2)
+    orc_transform((query ? c->t_q : c->t_k) + (size_t)h * d * d, e.data(), d, out);
+  else if (c->rotate_k)
+    orc_rotate(e.data(), d, out);
+  else
+    for (int i = 0; i < d; ++i) out[i] = e[i];
+}
+
+inline int n_buckets(const orc_cache* c) { return c->bucket_w > 0 ? (c->capacity + c->bucket_w - 1) / c->bucket_w : 1; }
+
+// keep the `keep` largest energies of the GQA group's rows qr [G][d]; equal
+// energies rank the lower index first
+uint32_t select_mask(const float* qr, int G, int d, int keep, double* energy) {
+  const int npg = d / kGranule;
+  std::vector<double> E(npg);
+  for (int p = 0; p < npg; ++p) {
+    double e = 0.0;
+    for (int g = 0; g < G; ++g)
+      for (int i = p * kGranule; i < (p + 1) * kGranule; ++i) {
+        double v = (double)qr[(size_t)g * d + i];
+        e += v * v;
+      }
+    E[p] = e;
+    if (energy) energy[p] = e;
+  }
+  uint32_t m = 0;
+  for (int p = 0; p < npg; ++p) {
+    int rank = 0;
+    for (int o = 0; o < npg; ++o)
+      if (E[o] > E[p] || (E[o] == E[p] && o < p)) ++rank;
+    if (rank < keep) m |= 1u << p;
+  }
+  return m;
+}
+
+}  // namespace
+
+extern "C" {
+
+void orc_rope(const float* x, int32_t d, const float* inv_freq, int64_t pos, float* out) {
+  const int hd = d / 2;
+  for (int i = 0; i < hd; ++i) {
+    const double th = (double)pos * (double)inv_freq[i];
+    const double cs = std::cos(th), sn = std::sin(th);
+    const double a = x[i], b = x[i + hd];
+    out[i] = (float)(a * cs - b * sn);
+    out[i + hd] = (float)(b * cs + a * sn);
+  }
+}
 
 void orc_fwht(double* x, int32_t d) {
   // Sylvester order: H[i][j] = (-1)^popcount(i & j); stage h pairs (i, i+h)
@@ -252,6 +315,7 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
   const int d = c->head_dim;
   if (d % kGroup != 0 || n_new < 0 || offset < 0 || offset + n_new > c->capacity) return -1;
   if (c->rotate_k == 2 && !c->t_k) return -1;
+  if (c->bucket_w < 0 || (c->bucket_w > 0 && !c->rope_inv_freq)) return -1;
   if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return -1;
   const int ngroups = d / kGroup, npg = d / kGranule;
   orc_stats total = {0, 0, 0, 0, 0, 0, 0};
@@ -266,12 +330,7 @@ int32_t orc_quantize_append(const orc_cache* c, const float* k_new, const float*
       const int n = offset + t;
       const size_t row = ((size_t)bh * n_new + t) * d;
       // ---- keys: rotate, optional channel 0 in bf16, quantize, pack ----
-      if (c->rotate_k == 2)
-        orc_transform(c->t_k + (size_t)h * d * d, k_new + row, d, xr.data());
-      else if (c->rotate_k)
-        orc_rotate(k_new + row, d, xr.data());
-      else
-        for (int i = 0; i < d; ++i) xr[i] = k_new[row + i];
+      prepare_row(c, h, k_new + row, false, c->bucket_w > 0 ? n % c->bucket_w : 0, xr.data());
       const long ws = window_slot(c, n);
       if (ws >= 0)
         for (int i = 0; i < d; ++i) c->k_win[(((size_t)b * c->kv_heads + h) * wsize(c) + ws) * d + i] = orc_bf16_rn(xr[i]);
@@ -403,7 +462,6 @@ void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, i
                 int32_t keep, uint32_t* mask, double* energy) {
   const int G = Hq / Hkv, npg = d / kGranule;
   std::vector<float> qr((size_t)G * d);
-  std::vector<double> E(npg);
   for (int b = 0; b < B; ++b)
     for (int hk = 0; hk < Hkv; ++hk) {
       for (int g = 0; g < G; ++g) {
@@ -416,26 +474,24 @@ void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, i
           for (int i = 0; i < d; ++i) qr[(size_t)g * d + i] = qi[i];
       }
       // energy of channel group p summed over the GQA group's query heads
-      for (int p = 0; p < npg; ++p) {
-        double e = 0.0;
-        for (int g = 0; g < G; ++g)
-          for (int i = p * kGranule; i < (p + 1) * kGranule; ++i) {
-            double v = (double)qr[(size_t)g * d + i];
-            e += v * v;
-          }
-        E[p] = e;
-        if (energy) energy[((size_t)b * Hkv + hk) * npg + p] = e;
-      }
-      // keep the `keep` largest energies; equal energies rank the lower index first
-      uint32_t m = 0;
-      for (int p = 0; p < npg; ++p) {
-        int rank = 0;
-        for (int o = 0; o < npg; ++o)
-          if (E[o] > E[p] || (E[o] == E[p] && o < p)) ++rank;
-        if (rank < keep) m |= 1u << p;
-      }
-      mask[(size_t)b * Hkv + hk] = m;
+      mask[(size_t)b * Hkv + hk] =
+          select_mask(qr.data(), G, d, keep, energy ? energy + ((size_t)b * Hkv + hk) * npg : nullptr);
     }
+}
+
+void orc_select_buckets(const orc_cache* c, const float* q, int32_t Hq, const int32_t* lens, int32_t keep,
+                        uint32_t* mask, double* energy) {
+  const int d = c->head_dim, Hkv = c->kv_heads, G = Hq / Hkv, npg = d / kGranule, nb = n_buckets(c);
+  std::vector<float> qr((size_t)G * d);
+  for (int b = 0; b < c->batch; ++b)
+    for (int k = 0; k < nb; ++k)
+      for (int hk = 0; hk < Hkv; ++hk) {
+        const long rel = (long)lens[b] - 1 - (long)k * c->bucket_w;  // query offset from bucket k's anchor
+        for (int g = 0; g < G; ++g)
+          prepare_row(c, hk, q + ((size_t)b * Hq + (size_t)hk * G + g) * d, true, rel, &qr[(size_t)g * d]);
+        const size_t u = ((size_t)b * nb + k) * Hkv + hk;
+        mask[u] = select_mask(qr.data(), G, d, keep, energy ? energy + u * npg : nullptr);
+      }
 }
 
 void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t* lens, const uint32_t* mask,
@@ -450,17 +506,17 @@ void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t
     for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
     const int len = lens[b];
     if (len <= 0) continue;
-    std::vector<float> qr(d);
-    if (c->rotate_k == 2)
-      orc_transform(c->t_q + (size_t)hk * d * d, q + (size_t)row * d, d, qr.data());
-    else if (c->rotate_k)
-      orc_rotate(q + (size_t)row * d, d, qr.data());
-    else
-      for (int i = 0; i < d; ++i) qr[i] = q[(size_t)row * d + i];
-    const uint32_t m = mask ? mask[(size_t)b * c->kv_heads + hk] : 0xFFFFFFFFu;
+    // the query as each bucket scores it (one bucket without bucket-relative RoPE)
+    const int nb = n_buckets(c), used = c->bucket_w > 0 ? (len - 1) / c->bucket_w + 1 : 1;
+    std::vector<float> qall((size_t)used * d);
+    for (int k = 0; k < used; ++k)
+      prepare_row(c, hk, q + (size_t)row * d, true, (long)len - 1 - (long)k * c->bucket_w, &qall[(size_t)k * d]);
     std::vector<double> s(len), khat(d), vhat(d);
     double smax = -std::numeric_limits<double>::infinity();
     for (int j = 0; j < len; ++j) {
+      const int k = c->bucket_w > 0 ? j / c->bucket_w : 0;
+      const float* qr = &qall[(size_t)k * d];
+      const uint32_t m = mask ? mask[((size_t)b * nb + k) * c->kv_heads + hk] : 0xFFFFFFFFu;
       const uint16_t* kw = window_row(c, c->k_win, b, hk, j, len);
       double acc = 0.0;
       if (kw) {  // bf16 window token: every channel

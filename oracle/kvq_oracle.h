@@ -38,6 +38,16 @@
  *    outside the decode path).  Each output is the fp64 sum over j = 0..d-1,
  *    in that order, of A[i][j] x[j] (product and sum each rounded once),
  *    rounded to fp32.
+ *  - Dual-QK Sec. 3.4 and App. C.4: bucket-relative RoPE.  Token n belongs to
+ *    bucket n / w (w = 2048 on the pages) with anchor w * (n / w); its key is
+ *    stored rotary-embedded at its offset n mod w from the anchor, then taken
+ *    through the key transform.  The query (at position len - 1, the last
+ *    token appended) is embedded at its offset p - anchor for each bucket,
+ *    which may exceed w, then taken through the query transform; each bucket
+ *    selects its own channel mask from its own query, and one softmax covers
+ *    every bucket.  Rotary embedding pairs channel i with i + d/2 and turns the
+ *    pair by angle pos * inv_freq[i] (fp64 cos and sin), the caller supplying
+ *    the model's inverse frequencies; the embedded row is rounded to fp32.
  *
  * Precision: FWHT in fp64 (natural Sylvester order), rotated values rounded
  * to fp32; quantization in fp32 with IEEE round-half-to-even; dequantization,
@@ -75,6 +85,10 @@ typedef struct {
      and T^{-T} for keys; NULL otherwise */
   const float* t_q; /* [Hkv][d][d] */
   const float* t_k; /* [Hkv][d][d] */
+  /* bucket-relative RoPE: bucket width w (0 = keys and queries used as given,
+     no rotary embedding) and the d/2 inverse frequencies */
+  int32_t bucket_w;
+  const float* rope_inv_freq; /* [d/2] */
 } orc_cache;
 
 typedef struct {
@@ -91,6 +105,10 @@ void orc_rotate(const float* x, int32_t d, float* out);
 
 /* out[i] = fp32(sum_j A[i][j] * x[j]), fp64 products and sums in order j = 0..d-1 */
 void orc_transform(const float* A, const float* x, int32_t d, float* out);
+
+/* rotary embedding of one row at position pos: out[i] = x[i] cos - x[i+d/2] sin,
+   out[i+d/2] = x[i+d/2] cos + x[i] sin, angle pos * inv_freq[i], fp64, rounded to fp32 */
+void orc_rope(const float* x, int32_t d, const float* inv_freq, int64_t pos, float* out);
 
 /* IEEE binary16 / bfloat16 round-to-nearest-even from fp32, and widening */
 uint16_t orc_half_rn(float x);
@@ -138,12 +156,22 @@ void orc_select(const float* q, int32_t B, int32_t Hq, int32_t Hkv, int32_t d, i
                 int32_t keep, uint32_t* mask, double* energy);
 
 /*
+ * Channel selection per bucket of a bucket-relative RoPE cache (bucket_w > 0):
+ * mask[(b * nb + k) * Hkv + h], nb = ceil(capacity / bucket_w), from the query
+ * embedded at offset (lens[b] - 1) - k * bucket_w and transformed like the
+ * keys' partner; energy (may be NULL) [B][nb][Hkv][d/4].
+ */
+void orc_select_buckets(const orc_cache* c, const float* q, int32_t Hq, const int32_t* lens, int32_t keep,
+                        uint32_t* mask, double* energy);
+
+/*
  * Decode attention over the oracle cache for rows r = b*Hq + hq listed in
  * `rows` (all B*Hq rows when rows == NULL); with rotate_v the output is the
  * orthonormal Walsh-Hadamard transform (its own inverse) of the attention
  * over the rotated values.  Remaining arguments:
  * `rows` (all B*Hq rows when rows == NULL).  q as in orc_select; lens[b]
- * tokens of sequence b; mask NULL = all channels.  out[r][d] fp64 (row-major
+ * tokens of sequence b; mask NULL = all channels ([B][nb][Hkv], one per bucket,
+ * with bucket-relative RoPE).  out[r][d] fp64 (row-major
  * in the order of `rows`).
  */
 void orc_attention(const orc_cache* c, const float* q, int32_t Hq, const int32_t* lens, const uint32_t* mask,

@@ -22,7 +22,8 @@ class OrcCache(ctypes.Structure):
                 ("k_bits", _I32), ("v_bits", _I32), ("rotate_k", _I32), ("keep_ch0", _I32),
                 ("rotate_v", _I32), ("v_clip", ctypes.c_float),
                 ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P),
-                ("sink", _I32), ("recent", _I32), ("k_win", _P), ("v_win", _P), ("t_q", _P), ("t_k", _P)]
+                ("sink", _I32), ("recent", _I32), ("k_win", _P), ("v_win", _P), ("t_q", _P), ("t_k", _P),
+                ("bucket_w", _I32), ("rope_inv_freq", _P)]
 
 
 class OrcStats(ctypes.Structure):
@@ -38,6 +39,8 @@ def lib():
         L.orc_fwht.argtypes = [_P, _I32]
         L.orc_rotate.argtypes = [_P, _I32, _P]
         L.orc_transform.argtypes = [_P, _P, _I32, _P]
+        L.orc_rope.argtypes = [_P, _I32, _P, ctypes.c_int64, _P]
+        L.orc_select_buckets.argtypes = [ctypes.POINTER(OrcCache), _P, _I32, _P, _I32, _P, _P]
         L.orc_half_rn.argtypes = [ctypes.c_float]
         L.orc_half_rn.restype = ctypes.c_uint16
         L.orc_half_value.argtypes = [ctypes.c_uint16]
@@ -98,6 +101,15 @@ def transform(A: np.ndarray, x: np.ndarray) -> np.ndarray:
     return out
 
 
+def rope(x: np.ndarray, inv_freq: np.ndarray, pos: int) -> np.ndarray:
+    """Rotary embedding of one row at position pos (channel i paired with i + d/2)."""
+    xi = np.ascontiguousarray(x, dtype=np.float32)
+    fr = np.ascontiguousarray(inv_freq, dtype=np.float32)
+    out = np.empty_like(xi)
+    lib().orc_rope(_p(xi), xi.size, _p(fr), int(pos), _p(out))
+    return out
+
+
 def half_rn(x: float) -> int:
     return lib().orc_half_rn(float(x))
 
@@ -133,14 +145,19 @@ class Cache:
     """Host copy of the packed cache, written by the oracle."""
 
     def __init__(self, B, Hkv, d, capacity, k_bits, v_bits, rotate_k=1, keep_ch0=0, rotate_v=0, v_clip=1.0,
-                 sink=0, recent=0, t_q=None, t_k=None):
+                 sink=0, recent=0, t_q=None, t_k=None, bucket_w=0, inv_freq=None):
         """rotate_k = 2 takes the caller's pair: t_q [Hkv][d][d] on queries and
-        t_k [Hkv][d][d] (its inverse transpose) on keys, fp32 row-major."""
+        t_k [Hkv][d][d] (its inverse transpose) on keys, fp32 row-major.
+        bucket_w > 0: keys and queries arrive before rotary embedding and are
+        embedded relative to their bucket's anchor (inv_freq [d/2] fp32)."""
         self.B, self.Hkv, self.d, self.capacity = B, Hkv, d, capacity
         if rotate_k == 2:
             t_q = np.ascontiguousarray(t_q, dtype=np.float32).reshape(Hkv, d, d)
             t_k = np.ascontiguousarray(t_k, dtype=np.float32).reshape(Hkv, d, d)
         self.t_q, self.t_k = t_q, t_k
+        self.bucket_w = bucket_w
+        self.inv_freq = np.ascontiguousarray(inv_freq, dtype=np.float32) if bucket_w else None
+        self.n_buckets = -(-capacity // bucket_w) if bucket_w else 1
         self.k_bits, self.v_bits, self.rotate_k, self.keep_ch0 = k_bits, v_bits, rotate_k, keep_ch0
         self.rotate_v, self.v_clip, self.sink, self.recent = rotate_v, v_clip, sink, recent
         w = B * Hkv * (sink + recent) * d
@@ -155,7 +172,8 @@ class Cache:
         self.struct = OrcCache(B, Hkv, d, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v, v_clip,
                                _p(self.k_codes), _p(self.k_scales), _p(self.k_ch0), _p(self.v_codes),
                                _p(self.v_scales), sink, recent, _p(self.k_win), _p(self.v_win),
-                               _p(self.t_q) if rotate_k == 2 else None, _p(self.t_k) if rotate_k == 2 else None)
+                               _p(self.t_q) if rotate_k == 2 else None, _p(self.t_k) if rotate_k == 2 else None,
+                               bucket_w, _p(self.inv_freq))
 
     def append(self, k_new: np.ndarray, v_new: np.ndarray, offset: int, want_exempt: bool = False):
         """k_new, v_new: [B][Hkv][n][d] (bf16 as uint16, or fp32)."""
@@ -185,6 +203,16 @@ class Cache:
         vh = np.zeros((n, self.d), np.float64)
         lib().orc_dequantize(ctypes.byref(self.struct), b, h, n0, n, _p(kh), _p(vh))
         return kh, vh
+
+    def select_buckets(self, q: np.ndarray, lens: np.ndarray, keep: int):
+        """-> (mask [B][nb][Hkv] uint32, energy [B][nb][Hkv][d/4]): one mask per bucket."""
+        qf = as_f32(q)
+        Hq = qf.shape[1]
+        ln = np.ascontiguousarray(lens, dtype=np.int32)
+        mask = np.zeros((self.B, self.n_buckets, self.Hkv), np.uint32)
+        energy = np.zeros((self.B, self.n_buckets, self.Hkv, self.d // 4), np.float64)
+        lib().orc_select_buckets(ctypes.byref(self.struct), _p(qf), Hq, _p(ln), keep, _p(mask), _p(energy))
+        return mask, energy
 
     def attention(self, q: np.ndarray, lens: np.ndarray, mask: np.ndarray | None, scale: float,
                   rows: np.ndarray | None = None) -> np.ndarray:
