@@ -122,6 +122,26 @@ typedef struct {
      affected. */
   const float* t_query;
   const float* t_key;
+  /* Bucket-relative RoPE [DQK Sec. 3.4, App. C.4]; 0 and NULL = none (keys
+     and queries are used as given).  With bucket_tokens = w > 0, keys and
+     queries arrive before rotary embedding.  Token n belongs to bucket
+     k = n / w with anchor k * w; its key is embedded at offset n mod w, then
+     transformed (rotate_k) and quantized.  At decode and selection the query
+     of sequence b sits at position L - 1 (L = seq_lens[b]) and is embedded at
+     offset L - 1 - k * w for bucket k (possibly beyond w), then transformed;
+     each bucket has its own channel mask and one softmax covers all buckets.
+     Rotary embedding pairs channel i with i + d/2 at angle
+     offset * rope_inv_freq[i] (fp64 angle, cos and sin; each product and sum
+     rounded once), the row then rounded to fp32.
+     Layout: bucket-major -- every array is laid out as the cache of batch
+     B * (capacity / w) and capacity w, bucket k of sequence b being its
+     sequence b * (capacity / w) + k (kvq_cache_sizes is unchanged).
+     Requires w a multiple of 128 dividing capacity, and no token windows
+     (otherwise KVQ_ERR_UNSUPPORTED); an append must stay inside one bucket
+     (otherwise KVQ_ERR_INVALID_ARG).  rope_inv_freq: caller-owned device
+     fp32 [d/2], 16-byte aligned. */
+  int32_t bucket_tokens;
+  const float* rope_inv_freq;
 } kvq_cache;
 
 /*
@@ -170,6 +190,19 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* cache, const void* k_new
 KVQ_API kvq_status kvq_select_channels(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
                                        int32_t keep_groups, uint32_t* mask_out, void* stream);
 
+/*
+ * The same selection for queries at known positions: without bucket-relative
+ * RoPE identical to kvq_select_channels (seq_lens unused); with it, one mask
+ * per bucket from the query embedded at that bucket's offset [DQK Sec. 3.4:
+ * masks may differ across buckets], mask_out [B][capacity / w][H].
+ *  seq_lens: device int32 [B], the query of sequence b at position
+ *  seq_lens[b] - 1.  kvq_select_channels on a bucketed cache returns
+ *  KVQ_ERR_INVALID_ARG (it has no positions).
+ */
+KVQ_API kvq_status kvq_select_channels_at(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                          const int32_t* seq_lens, int32_t keep_groups, uint32_t* mask_out,
+                                          void* stream);
+
 /* Device workspace bytes kvq_decode_attention needs for these sizes (0 on bad arguments). */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_heads, int32_t max_len);
 
@@ -194,7 +227,8 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_head
  *            sequence of length 0 gets a zero output.
  *  max_len:  host bound on seq_lens, 0 <= max_len <= capacity; sizes the grid.
  *  mask:     device uint32 [B][H] from kvq_select_channels, or NULL = every
- *            channel group.
+ *            channel group ([B][capacity / w][H] from kvq_select_channels_at
+ *            with bucket-relative RoPE).
  *  out:      device fp32 [B][q_heads][d].
  *  workspace: device scratch of at least kvq_decode_workspace_bytes bytes,
  *            owned by the caller; not read by later calls.

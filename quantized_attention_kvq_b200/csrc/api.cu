@@ -28,6 +28,10 @@ kvq_status check_shape(const kvq_cache* c) {
   if (c->head_dim != kHeadDim || c->group_size != kGroup || c->prune_granule != kGranule) return KVQ_ERR_UNSUPPORTED;
   if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return KVQ_ERR_UNSUPPORTED;
   if (c->capacity % kKeyBlock != 0) return KVQ_ERR_UNSUPPORTED;
+  if (c->bucket_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  if (c->bucket_tokens > 0 && (c->bucket_tokens % kKeyBlock != 0 || c->capacity % c->bucket_tokens != 0 ||
+                               c->sink_tokens + c->recent_tokens > 0))
+    return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
 
@@ -41,6 +45,7 @@ kvq_status check_cache(const kvq_cache* c) {
   kvq_status st = check_shape(c);
   if (st != KVQ_OK) return st;
   if (!pair_ok(c, true, true)) return KVQ_ERR_INVALID_ARG;
+  if (c->bucket_tokens > 0 && (!c->rope_inv_freq || !aligned16(c->rope_inv_freq))) return KVQ_ERR_INVALID_ARG;
   if (!c->k_codes || !c->k_scales || !c->v_codes || !c->v_scales || (c->keep_ch0 && !c->k_ch0))
     return KVQ_ERR_INVALID_ARG;
   if (!aligned16(c->k_codes) || !aligned16(c->k_scales) || !aligned16(c->v_codes) || !aligned16(c->v_scales) ||
@@ -82,23 +87,58 @@ CacheView view(const kvq_cache* c) {
 
 double inv_sqrt_d() { return 1.0 / std::sqrt((double)kHeadDim); }
 
+// Buckets of a bucket-relative RoPE cache (1 without): the arrays are those of
+// a cache of batch B * nb and capacity bucket_tokens.
+inline int n_buckets(const kvq_cache* c) { return c->bucket_tokens > 0 ? c->capacity / c->bucket_tokens : 1; }
+
+// Bytes of the five arrays for `batch` sequences of `cap` tokens.
+void array_bytes(const kvq_cache* c, size_t batch, size_t cap, size_t out[5]) {
+  const size_t rows = batch * c->kv_heads * cap;
+  out[0] = rows * kPruneGroups * (c->k_bits == 4 ? 2 : 1);
+  out[1] = rows * kGroups * 4;
+  out[2] = c->keep_ch0 ? rows * 2 : 0;
+  out[3] = rows * (kHeadDim * c->v_bits / 8);
+  out[4] = rows * kGroups * 4;
+}
+
+// The view of bucket sequence vb alone (batch 1, capacity bucket_tokens).
+CacheView bucket_sequence_view(const kvq_cache* c, size_t vb) {
+  CacheView v = view(c);
+  size_t per[5];
+  array_bytes(c, 1, c->bucket_tokens, per);
+  v.B = 1;
+  v.cap = c->bucket_tokens;
+  v.kc = v.kc + vb * per[0];
+  v.ks = reinterpret_cast<__half2*>(reinterpret_cast<char*>(v.ks) + vb * per[1]);
+  if (v.k0) v.k0 = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(v.k0) + vb * per[2]);
+  v.vc = v.vc + vb * per[3];
+  v.vs = reinterpret_cast<__half2*>(reinterpret_cast<char*>(v.vs) + vb * per[4]);
+  return v;
+}
+
 // Workspace of the decode: one partial row (128-channel accumulator, running
 // max and sum) per (slot, query head of the GQA group), decode_slots slots;
 // with the caller's transform pair, then the transformed fp32 query rows.
 struct DecodePlan {
-  size_t acc_bytes, ml_offset, tq_offset, bytes;
+  size_t acc_bytes, ml_offset, tq_offset, qb_offset, vl_offset, bytes;
 };
 
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   DecodePlan p;
   const int G = q_heads / c->kv_heads;
   const bool win = c->sink_tokens + c->recent_tokens > 0;  // one more partial per unit for the windows
-  const size_t rows = ((size_t)decode_slots(c->batch, c->kv_heads, G) + (win ? c->batch * c->kv_heads : 0)) * G;
+  const int Bv = c->batch * n_buckets(c);  // the split decode runs over every bucket as a sequence
+  const size_t rows = ((size_t)decode_slots(Bv, c->kv_heads, G) + (win ? c->batch * c->kv_heads : 0)) * G;
   p.acc_bytes = rows * kHeadDim * sizeof(float);
   p.ml_offset = round_up(p.acc_bytes, kAlign);
   p.tq_offset = p.ml_offset + round_up(rows * sizeof(float2), kAlign);
   p.bytes = p.tq_offset;
   if (c->rotate_k == 2) p.bytes += round_up((size_t)c->batch * q_heads * kHeadDim * sizeof(float), kAlign);
+  // with buckets: each bucket's query rows and length
+  p.qb_offset = p.bytes;
+  if (c->bucket_tokens > 0) p.bytes += round_up((size_t)Bv * q_heads * kHeadDim * sizeof(float), kAlign);
+  p.vl_offset = p.bytes;
+  if (c->bucket_tokens > 0) p.bytes += round_up((size_t)Bv * sizeof(int32_t), kAlign);
   return p;
 }
 
@@ -111,6 +151,40 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
                           const int32_t* seq_lens, int32_t max_len, const uint32_t* mask, float softmax_scale,
                           float* out, void* workspace, const DecodePlan& plan, cudaStream_t s,
                           int parts = kRunSplit | kRunCombine) {
+  if (c->bucket_tokens > 0) {
+    // every bucket is a sequence of the split decode, with its own query and
+    // length; the merge makes one softmax of them
+    const int nb = n_buckets(c), G = q_heads / c->kv_heads;
+    char* ws = static_cast<char*>(workspace);
+    DecodeArgs v;
+    v.c = view(c);
+    v.c.B = c->batch * nb;
+    v.c.cap = c->bucket_tokens;
+    v.c.rotate = 0;
+    v.q = ws + plan.qb_offset;
+    v.dtype = KVQ_F32;
+    v.Hq = q_heads;
+    v.seq_lens = reinterpret_cast<const int32_t*>(ws + plan.vl_offset);
+    v.max_len = max_len < c->bucket_tokens ? max_len : c->bucket_tokens;
+    v.mask = mask;
+    v.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);  // log2(e)
+    v.inv_sqrt_d = inv_sqrt_d();
+    v.win_base = decode_slots(v.c.B, c->kv_heads, G);
+    v.part_acc = reinterpret_cast<float*>(ws);
+    v.part_ml = reinterpret_cast<float2*>(ws + plan.ml_offset);
+    v.out = nullptr;
+    if (parts & kRunSplit) {
+      kvq_status st = cuda_status(launch_bucket_queries(
+          q, dtype, c->rotate_k, c->t_query, c->rope_inv_freq, seq_lens, max_len, c->batch, q_heads, c->kv_heads,
+          c->bucket_tokens, nb, inv_sqrt_d(), reinterpret_cast<float*>(ws + plan.qb_offset),
+          reinterpret_cast<int32_t*>(ws + plan.vl_offset), s));
+      if (st != KVQ_OK) return st;
+      if (v.max_len > 0 && (st = cuda_status(launch_decode(v, s))) != KVQ_OK) return st;
+    }
+    if (parts & kRunCombine)
+      return cuda_status(launch_bucket_merge(v, nb, decode_slots(0, 0, G) / decode_groups(G), out, s));
+    return KVQ_OK;
+  }
   DecodeArgs a;
   a.c = view(c);
   a.q = q;
@@ -185,12 +259,7 @@ KVQ_API kvq_status kvq_cache_sizes(const kvq_cache* c, size_t bytes_out[5]) {
   kvq_status st = check_shape(c);
   if (st != KVQ_OK) return st;
   if (!bytes_out) return KVQ_ERR_INVALID_ARG;
-  const size_t rows = (size_t)c->batch * c->kv_heads * (size_t)c->capacity;
-  bytes_out[0] = rows * kPruneGroups * (c->k_bits == 4 ? 2 : 1);
-  bytes_out[1] = rows * kGroups * 4;
-  bytes_out[2] = c->keep_ch0 ? rows * 2 : 0;
-  bytes_out[3] = rows * (kHeadDim * c->v_bits / 8);
-  bytes_out[4] = rows * kGroups * 4;
+  array_bytes(c, c->batch, c->capacity, bytes_out);
   return KVQ_OK;
 }
 
@@ -207,6 +276,26 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* c, const void* k_new, co
   if ((int64_t)offset + n_new > c->capacity) return KVQ_ERR_CAPACITY;
   if (n_new == 0) return KVQ_OK;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
+  if (c->bucket_tokens > 0) {
+    // one launch per sequence into its bucket's sequence, keys embedded at
+    // their offset from the bucket's anchor
+    const int w = c->bucket_tokens, k = offset / w;
+    if ((offset + n_new - 1) / w != k) return KVQ_ERR_INVALID_ARG;
+    const size_t in_seq = (size_t)c->kv_heads * n_new * kHeadDim * dtype_size(dtype);
+    for (int b = 0; b < c->batch; ++b) {
+      AppendArgs a;
+      a.c = bucket_sequence_view(c, (size_t)b * n_buckets(c) + k);
+      a.k_new = static_cast<const char*>(k_new) + b * in_seq;
+      a.v_new = static_cast<const char*>(v_new) + b * in_seq;
+      a.dtype = dtype;
+      a.n_new = n_new;
+      a.offset = offset - k * w;
+      a.inv_sqrt_d = inv_sqrt_d();
+      kvq_status st = cuda_status(launch_append_ext(a, c->t_key, c->rope_inv_freq, static_cast<cudaStream_t>(stream)));
+      if (st != KVQ_OK) return st;
+    }
+    return KVQ_OK;
+  }
   AppendArgs a;
   a.c = view(c);
   a.k_new = k_new;
@@ -215,15 +304,18 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* c, const void* k_new, co
   a.n_new = n_new;
   a.offset = offset;
   a.inv_sqrt_d = inv_sqrt_d();
-  return cuda_status(launch_append_pair(a, c->t_key, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_append_ext(a, c->t_key, nullptr, static_cast<cudaStream_t>(stream)));
 }
 
-KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
-                                       int32_t keep_groups, uint32_t* mask_out, void* stream) {
+KVQ_API kvq_status kvq_select_channels_at(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                          const int32_t* seq_lens, int32_t keep_groups, uint32_t* mask_out,
+                                          void* stream) {
   kvq_status st = check_shape(c);
   if (st != KVQ_OK) return st;
   if ((st = check_heads(c, q_heads)) != KVQ_OK) return st;
   if (!dtype_ok(dtype) || !q || !mask_out || !aligned16(q) || !pair_ok(c, true, false)) return KVQ_ERR_INVALID_ARG;
+  if (c->bucket_tokens > 0 && (!seq_lens || !c->rope_inv_freq || !aligned16(c->rope_inv_freq)))
+    return KVQ_ERR_INVALID_ARG;
   if (keep_groups < 1 || keep_groups > kPruneGroups) return KVQ_ERR_INVALID_ARG;
   if (q_heads / c->kv_heads > 64) return KVQ_ERR_UNSUPPORTED;
   SelectArgs a;
@@ -236,7 +328,18 @@ KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dt
   a.keep = keep_groups;
   a.inv_sqrt_d = inv_sqrt_d();
   a.mask = mask_out;
-  return cuda_status(launch_select_pair(a, c->t_query, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (c->bucket_tokens > 0)
+    return cuda_status(
+        launch_select_buckets(a, c->t_query, c->rope_inv_freq, seq_lens, c->bucket_tokens, n_buckets(c), s));
+  return cuda_status(launch_select_pair(a, c->t_query, s));
+}
+
+KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                       int32_t keep_groups, uint32_t* mask_out, void* stream) {
+  // bucket-relative RoPE needs the queries' positions: kvq_select_channels_at
+  if (c && c->bucket_tokens != 0) return KVQ_ERR_INVALID_ARG;
+  return kvq_select_channels_at(c, q, dtype, q_heads, nullptr, keep_groups, mask_out, stream);
 }
 
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
@@ -281,7 +384,7 @@ KVQ_API size_t kvq_decode_step_workspace_bytes(const kvq_cache* c, kvq_dtype dty
   if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK || !dtype_ok(dtype)) return 0;
   if (max_len < 0 || max_len > c->capacity) return 0;
   const size_t qb = (size_t)c->batch * q_heads * kHeadDim * dtype_size(dtype);
-  const size_t mb = (size_t)c->batch * c->kv_heads * sizeof(uint32_t);
+  const size_t mb = (size_t)c->batch * n_buckets(c) * c->kv_heads * sizeof(uint32_t);
   const size_t ob = (size_t)c->batch * q_heads * kHeadDim * sizeof(float);
   return round_up(qb, kAlign) + round_up(mb, kAlign) + round_up(ob, kAlign) + plan_decode(c, q_heads).bytes;
 }
@@ -303,7 +406,7 @@ KVQ_API kvq_status kvq_decode_step_host(const kvq_cache* c, const void* q_host, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
   const size_t qb = (size_t)c->batch * q_heads * kHeadDim * dtype_size(dtype);
-  const size_t mb = (size_t)c->batch * c->kv_heads * sizeof(uint32_t);
+  const size_t mb = (size_t)c->batch * n_buckets(c) * c->kv_heads * sizeof(uint32_t);
   const size_t ob = (size_t)c->batch * q_heads * kHeadDim * sizeof(float);
   void* q_dev = ws;
   uint32_t* mask_dev = reinterpret_cast<uint32_t*>(ws + round_up(qb, kAlign));
@@ -312,7 +415,7 @@ KVQ_API kvq_status kvq_decode_step_host(const kvq_cache* c, const void* q_host, 
   if ((st = cuda_status(cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s))) != KVQ_OK) return st;
   const uint32_t* mask = nullptr;
   if (keep_groups < kPruneGroups) {
-    st = kvq_select_channels(c, q_dev, dtype, q_heads, keep_groups, mask_dev, stream);
+    st = kvq_select_channels_at(c, q_dev, dtype, q_heads, seq_lens, keep_groups, mask_dev, stream);
     if (st != KVQ_OK) return st;
     mask = mask_dev;
   }

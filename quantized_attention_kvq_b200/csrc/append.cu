@@ -242,6 +242,24 @@ __device__ __forceinline__ void transform_row_4lanes(float (&v)[32], int g, int 
   for (int r = 0; r < 32; ++r) v[r] = __double2float_rn(acc[r]);
 }
 
+// Rotary embedding of one key row held by four lanes as above, at position
+// pos (Dual-QK Sec. 3.4, bucket-relative RoPE): channel i < 64 pairs with
+// i + 64, held by lane group g ^ 2; angle pos * inv_freq[i mod 64] in fp64,
+// x_i cos - x_{i+64} sin below, x_{i+64} cos + x_i sin above, each product and
+// sum rounded once, then rounded to fp32.  All 32 lanes of the warp take part.
+__device__ __forceinline__ void rope_row_4lanes(float (&v)[32], int g, int pos, const float* __restrict__ inv_freq) {
+  const bool upper = g >= 2;
+  const int f0 = 32 * (g & 1);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const double other = (double)__shfl_xor_sync(kFull, v[i], 2);
+    double sn, cs;
+    sincos(__dmul_rn((double)pos, (double)__ldg(inv_freq + f0 + i)), &sn, &cs);
+    const double own = __dmul_rn((double)v[i], cs), cross = __dmul_rn(other, sn);
+    v[i] = __double2float_rn(upper ? __dadd_rn(own, cross) : __dsub_rn(own, cross));
+  }
+}
+
 // bf16 (round to nearest even) copy of this lane's 32 channels into a window row
 __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* dst, const float (&v)[32]) {
   uint32_t w[16];
@@ -255,11 +273,13 @@ __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* dst, const float (&
   for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
-// ROT: 0 keys as given, 1 Walsh-Hadamard rotation, 2 the pair's key matrix
-// tk[h] (its fp64 accumulators need the registers of fewer resident blocks)
+// ROT & 3: 0 keys as given, 1 Walsh-Hadamard rotation, 2 the pair's key
+// matrix tk[h] (its fp64 accumulators need the registers of fewer resident
+// blocks); ROT & 4: keys first rotary-embedded at their token index in the
+// view (the offset from their bucket's anchor), frequencies inv_freq
 template <int KB, int VB, int ROT, bool CH0, bool ROTV, typename In>
-__global__ void __launch_bounds__(kAppendWarps * 32, ROT == 2 ? 1 : 3)
-    k_quantize_append(AppendArgs a, const float* __restrict__ tk) {
+__global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
+    k_quantize_append(AppendArgs a, const float* __restrict__ tk, const float* __restrict__ inv_freq) {
   constexpr int TPW = 32 / VB;            // value tokens per 32-bit word: 8 (INT4) or 16 (INT2)
   constexpr int WPR = kAppendTile / TPW;  // value words per channel in the window: 8 or 4
   // key words [pruning group][token], 16 bits a token (its KB * 4 low bits used)
@@ -302,8 +322,9 @@ __global__ void __launch_bounds__(kAppendWarps * 32, ROT == 2 ? 1 : 3)
   widen(kraw, kx);
 
   // ---- key row: rotated, then quantized (keys are not clipped)
-  if (ROT == 1) rotate_row_4lanes(kx, g, a.inv_sqrt_d);
-  if (ROT == 2) transform_row_4lanes(kx, g, lane, tk + (size_t)h * kPairElems);
+  if (ROT & 4) rope_row_4lanes(kx, g, w0 + tt, inv_freq);
+  if ((ROT & 3) == 1) rotate_row_4lanes(kx, g, a.inv_sqrt_d);
+  if ((ROT & 3) == 2) transform_row_4lanes(kx, g, lane, tk + (size_t)h * kPairElems);
   // bf16 window copies (rotated key, then the value below) for tokens with a
   // window slot: every sink token, and of the later tokens only this append's
   // last `recent`, the ones that still own their ring slot when it ends (an
@@ -410,43 +431,51 @@ __global__ void __launch_bounds__(kAppendWarps * 32, ROT == 2 ? 1 : 3)
 }
 
 template <int KB, int VB, int ROT, bool CH0, bool ROTV>
-cudaError_t launch_typed(const AppendArgs& a, const float* tk, cudaStream_t s) {
+cudaError_t launch_typed(const AppendArgs& a, const float* tk, const float* fr, cudaStream_t s) {
   const int first = a.offset / kAppendTile, last = (a.offset + a.n_new - 1) / kAppendTile;
   dim3 grid(last - first + 1, a.c.H, a.c.B);
   dim3 block(kAppendWarps * 32);
   switch (a.dtype) {
-    case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, ROTV, float><<<grid, block, 0, s>>>(a, tk); break;
-    case KVQ_BF16: k_quantize_append<KB, VB, ROT, CH0, ROTV, __nv_bfloat16><<<grid, block, 0, s>>>(a, tk); break;
-    default: k_quantize_append<KB, VB, ROT, CH0, ROTV, __half><<<grid, block, 0, s>>>(a, tk); break;
+    case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, ROTV, float><<<grid, block, 0, s>>>(a, tk, fr); break;
+    case KVQ_BF16: k_quantize_append<KB, VB, ROT, CH0, ROTV, __nv_bfloat16><<<grid, block, 0, s>>>(a, tk, fr); break;
+    default: k_quantize_append<KB, VB, ROT, CH0, ROTV, __half><<<grid, block, 0, s>>>(a, tk, fr); break;
   }
   return cudaGetLastError();
 }
 
-// value rotation is a template flag, so kernels without it stay as small as before
-template <int KB, int VB, bool ROTV>
-cudaError_t launch_flags(const AppendArgs& a, const float* tk, cudaStream_t s) {
-  const bool ch0 = a.c.keep_ch0 != 0;
-  if (a.c.rotate == 2)
-    return ch0 ? launch_typed<KB, VB, 2, true, ROTV>(a, tk, s) : launch_typed<KB, VB, 2, false, ROTV>(a, tk, s);
-  if (a.c.rotate == 1)
-    return ch0 ? launch_typed<KB, VB, 1, true, ROTV>(a, tk, s) : launch_typed<KB, VB, 1, false, ROTV>(a, tk, s);
-  return ch0 ? launch_typed<KB, VB, 0, true, ROTV>(a, tk, s) : launch_typed<KB, VB, 0, false, ROTV>(a, tk, s);
+template <int KB, int VB, int ROT, bool ROTV>
+cudaError_t launch_ch0(const AppendArgs& a, const float* tk, const float* fr, cudaStream_t s) {
+  return a.c.keep_ch0 ? launch_typed<KB, VB, ROT, true, ROTV>(a, tk, fr, s)
+                      : launch_typed<KB, VB, ROT, false, ROTV>(a, tk, fr, s);
 }
 
+template <int KB, int VB, bool ROTV>
+cudaError_t launch_flags(const AppendArgs& a, const float* tk, const float* fr, cudaStream_t s) {
+  switch (a.c.rotate + (fr ? 4 : 0)) {
+    case 0: return launch_ch0<KB, VB, 0, ROTV>(a, tk, fr, s);
+    case 1: return launch_ch0<KB, VB, 1, ROTV>(a, tk, fr, s);
+    case 2: return launch_ch0<KB, VB, 2, ROTV>(a, tk, fr, s);
+    case 4: return launch_ch0<KB, VB, 4, ROTV>(a, tk, fr, s);
+    case 5: return launch_ch0<KB, VB, 5, ROTV>(a, tk, fr, s);
+    default: return launch_ch0<KB, VB, 6, ROTV>(a, tk, fr, s);
+  }
+}
+
+// value rotation is a template flag, so kernels without it stay as small as before
 template <int KB, int VB>
-cudaError_t launch_bits(const AppendArgs& a, const float* tk, cudaStream_t s) {
-  return a.c.rotate_v ? launch_flags<KB, VB, true>(a, tk, s) : launch_flags<KB, VB, false>(a, tk, s);
+cudaError_t launch_bits(const AppendArgs& a, const float* tk, const float* fr, cudaStream_t s) {
+  return a.c.rotate_v ? launch_flags<KB, VB, true>(a, tk, fr, s) : launch_flags<KB, VB, false>(a, tk, fr, s);
 }
 
 }  // namespace
 
-cudaError_t launch_append_pair(const AppendArgs& a, const float* tk, cudaStream_t s) {
-  if (a.c.k_bits == 4 && a.c.v_bits == 4) return launch_bits<4, 4>(a, tk, s);
-  if (a.c.k_bits == 4) return launch_bits<4, 2>(a, tk, s);
-  if (a.c.v_bits == 4) return launch_bits<2, 4>(a, tk, s);
-  return launch_bits<2, 2>(a, tk, s);
+cudaError_t launch_append_ext(const AppendArgs& a, const float* tk, const float* fr, cudaStream_t s) {
+  if (a.c.k_bits == 4 && a.c.v_bits == 4) return launch_bits<4, 4>(a, tk, fr, s);
+  if (a.c.k_bits == 4) return launch_bits<4, 2>(a, tk, fr, s);
+  if (a.c.v_bits == 4) return launch_bits<2, 4>(a, tk, fr, s);
+  return launch_bits<2, 2>(a, tk, fr, s);
 }
 
-cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) { return launch_append_pair(a, nullptr, s); }
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) { return launch_append_ext(a, nullptr, nullptr, s); }
 
 }  // namespace kvq

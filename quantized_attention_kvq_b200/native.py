@@ -18,7 +18,8 @@ KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORK
 KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 
 # every exported symbol the header declares
-SYMBOLS = ("kvq_cache_sizes", "kvq_window_bytes", "kvq_quantize_append", "kvq_select_channels", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
+SYMBOLS = ("kvq_cache_sizes", "kvq_window_bytes", "kvq_quantize_append", "kvq_select_channels",
+           "kvq_select_channels_at", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
            "kvq_decode_step_workspace_bytes",
            "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_status_string")
 
@@ -32,7 +33,7 @@ class KvqCacheStruct(ctypes.Structure):
                 ("rotate_k", _I32), ("keep_ch0", _I32), ("rotate_v", _I32), ("v_clip", ctypes.c_float),
                 ("k_codes", _P), ("k_scales", _P), ("k_ch0", _P), ("v_codes", _P), ("v_scales", _P),
                 ("sink_tokens", _I32), ("recent_tokens", _I32), ("k_window", _P), ("v_window", _P),
-                ("t_query", _P), ("t_key", _P)]
+                ("t_query", _P), ("t_key", _P), ("bucket_tokens", _I32), ("rope_inv_freq", _P)]
 
 
 class KvqError(RuntimeError):
@@ -59,6 +60,8 @@ def lib():
         L.kvq_quantize_append.restype = ctypes.c_int
         L.kvq_select_channels.argtypes = [C, _P, ctypes.c_int, _I32, _I32, _P, _P]
         L.kvq_select_channels.restype = ctypes.c_int
+        L.kvq_select_channels_at.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _P, _P]
+        L.kvq_select_channels_at.restype = ctypes.c_int
         L.kvq_decode_workspace_bytes.argtypes = [C, _I32, _I32]
         L.kvq_decode_workspace_bytes.restype = ctypes.c_size_t
         L.kvq_decode_attention.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _P, ctypes.c_float, _P, _P,
@@ -130,7 +133,8 @@ class KVQCache:
     def __init__(self, B: int, H: int, capacity: int, k_bits: int, v_bits: int, rotate_k: int = 1,
                  keep_ch0: int = 0, device="cuda", zero: bool = True, rotate_v: int = 0, v_clip: float = 1.0,
                  sink: int = 0, recent: int = 0, t_query: torch.Tensor | None = None,
-                 t_key: torch.Tensor | None = None):
+                 t_key: torch.Tensor | None = None, bucket_tokens: int = 0,
+                 rope_inv_freq: torch.Tensor | None = None):
         """rotate_k = 2 takes the caller's dual transform pair: t_query (T) and
         t_key (T^-T), fp32 device tensors [H][128][128], kept referenced here."""
         if rotate_k == 2 and (t_query is None or t_key is None):
@@ -138,6 +142,9 @@ class KVQCache:
         if rotate_k == 2 and (t_query.dtype != torch.float32 or t_key.dtype != torch.float32 or
                               tuple(t_query.shape) != (H, 128, 128) or tuple(t_key.shape) != (H, 128, 128)):
             raise ValueError("t_query and t_key are fp32 [H][128][128]")
+        if bucket_tokens and (rope_inv_freq is None or rope_inv_freq.dtype != torch.float32 or
+                              tuple(rope_inv_freq.shape) != (64,)):
+            raise ValueError("bucket-relative RoPE needs rope_inv_freq, fp32 [64]")
         self.desc = describe(B, H, capacity, k_bits, v_bits, rotate_k, keep_ch0, rotate_v=rotate_v, v_clip=v_clip,
                              sink=sink, recent=recent)
         sizes = cache_sizes(self.desc)
@@ -161,6 +168,10 @@ class KVQCache:
         self.t_key = t_key.contiguous() if rotate_k == 2 else None
         self.desc.t_query = _dev_ptr(self.t_query)
         self.desc.t_key = _dev_ptr(self.t_key)
+        self.rope_inv_freq = rope_inv_freq.contiguous() if bucket_tokens else None
+        self.desc.bucket_tokens = bucket_tokens
+        self.desc.rope_inv_freq = _dev_ptr(self.rope_inv_freq)
+        self.n_buckets = capacity // bucket_tokens if bucket_tokens else 1
         self.B, self.H, self.capacity = B, H, capacity
 
     def sequence_desc(self, b: int) -> KvqCacheStruct:
@@ -180,6 +191,7 @@ class KVQCache:
             d.k_window = self.desc.k_window + b * wper
             d.v_window = self.desc.v_window + b * wper
         d.t_query, d.t_key = self.desc.t_query, self.desc.t_key  # per kv head, shared by every sequence
+        d.bucket_tokens, d.rope_inv_freq = self.desc.bucket_tokens, self.desc.rope_inv_freq
         return d
 
     def append_sequence(self, b: int, k_new: torch.Tensor, v_new: torch.Tensor, offset: int, stream=None):
@@ -205,6 +217,18 @@ class KVQCache:
         _check(lib().kvq_select_channels(ctypes.byref(self.desc), _dev_ptr(q), torch_dtype_code(q.dtype),
                                          q.shape[1], keep_groups, _dev_ptr(mask_out), _stream(stream)),
                "kvq_select_channels")
+        return mask_out
+
+    def select_at(self, q: torch.Tensor, seq_lens: torch.Tensor, keep_groups: int,
+                  mask_out: torch.Tensor | None = None, stream=None):
+        """Selection for queries at positions seq_lens - 1; returns mask [B][nb][H]
+        (nb buckets, 1 without bucket-relative RoPE)."""
+        if mask_out is None:
+            mask_out = torch.empty((self.B, self.n_buckets, self.H), dtype=torch.int32, device=q.device)
+        _check(lib().kvq_select_channels_at(ctypes.byref(self.desc), _dev_ptr(q), torch_dtype_code(q.dtype),
+                                            q.shape[1], _dev_ptr(seq_lens), keep_groups, _dev_ptr(mask_out),
+                                            _stream(stream)),
+               "kvq_select_channels_at")
         return mask_out
 
     def workspace_bytes(self, q_heads: int, max_len: int) -> int:

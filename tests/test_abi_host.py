@@ -138,6 +138,46 @@ def test_transform_pair_workspace_holds_the_transformed_queries(L):
         L.kvq_decode_workspace_bytes(ctypes.byref(p), 8, 256) - L.kvq_decode_workspace_bytes(ctypes.byref(d), 8, 256)
 
 
+@pytest.mark.parametrize("w,sink,status", [(100, 0, native.KVQ_ERR_UNSUPPORTED), (128, 4, native.KVQ_ERR_UNSUPPORTED),
+                                           (-128, 0, native.KVQ_ERR_INVALID_ARG)])
+def test_bad_buckets_rejected(L, w, sink, status):
+    d = desc(cap=512, bucket_tokens=w, sink_tokens=sink)
+    d.rope_inv_freq = FAKE
+    if sink:
+        d.k_window = d.v_window = FAKE
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == status
+
+
+def test_bucket_rope_host_checks(L):
+    d = desc(cap=512, bucket_tokens=256)  # 384 does not divide 512: checked below
+    # no frequencies
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    d.rope_inv_freq = FAKE
+    # an append may not cross a bucket boundary
+    assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 8, 250, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    # the plain selection has no query positions
+    assert L.kvq_select_channels(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, 4, FAKE, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_select_channels_at(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, None, 4, FAKE, None) == \
+        native.KVQ_ERR_INVALID_ARG
+    odd = desc(cap=512, bucket_tokens=384)
+    odd.rope_inv_freq = FAKE
+    assert L.kvq_quantize_append(ctypes.byref(odd), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
+        native.KVQ_ERR_UNSUPPORTED
+    # same array sizes; the decode workspace holds the bucket batch's partials,
+    # query rows and lengths
+    assert native.cache_sizes(d) == native.cache_sizes(desc(cap=512))
+    plain = L.kvq_decode_workspace_bytes(ctypes.byref(desc(cap=512)), 8, 512)
+    ws = L.kvq_decode_workspace_bytes(ctypes.byref(d), 8, 512)
+    B, H, G, nb = 2, 2, 4, 2
+    extra = (B * nb - B) * H * G * (128 * 4 + 8)
+    assert ws >= plain + extra + B * nb * 8 * 128 * 4 + B * nb * 4
+    # a step's mask holds one word per bucket
+    assert L.kvq_decode_step_workspace_bytes(ctypes.byref(d), native.KVQ_BF16, 8, 512) >= ws + B * nb * H * 4
+
+
 def test_append_argument_checks(L):
     d = desc()
     assert L.kvq_quantize_append(ctypes.byref(d), FAKE, FAKE, native.KVQ_BF16, 200, 100, None) == \
