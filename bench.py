@@ -50,22 +50,34 @@ def popcount32(x: int) -> int:
 def algorithmic_bytes(wl: workloads.Workload, masks: np.ndarray, lens: np.ndarray) -> dict:
     """Bytes the method must move for one decode step: kept key-code rows, the
     scale/zero of touched key groups, channel 0 when its group is kept, every
-    value code and value scale/zero of the sequence, plus q in and out."""
+    value code and value scale/zero of the sequence, plus q in and out.  With
+    bucket-relative RoPE, masks is [B][nb][H] and each bucket's tokens count
+    with its own mask; the split decode then reads one fp32 query row per
+    bucket that holds tokens (and one per head with the dual pair alone)."""
     kword = 2 if wl.k_bits == 4 else 1
     split = window = 0
+    q_rows = 0
     for b in range(wl.B):
         n = int(lens[b])
         # tokens read from the bf16 windows (the first `sink` and the last `recent`)
         nw = min(wl.sink, n) + (max(0, n - max(wl.sink, n - wl.recent)) if wl.recent else 0)
-        for h in range(wl.Hkv):
-            m = int(masks[b, h]) & 0xFFFFFFFF
-            kept = popcount32(m)
-            touched = sum(1 for g in range(4) if (m >> (8 * g)) & 0xFF)
-            split += (n - nw) * (kept * kword + touched * 4 + (2 if wl.keep_ch0 and (m & 1) else 0))
-            split += (n - nw) * (128 * wl.v_bits // 8 + 16)
-            window += nw * 2 * 128 * 2  # bf16 key and value rows
-    esize = 4 if wl.fmt == "f32" else 2
-    q_bytes = wl.B * wl.Hq * 128 * esize
+        if wl.bucket:
+            segs = [(min(n - k * wl.bucket, wl.bucket), masks[b, k]) for k in range(-(-n // wl.bucket))]
+        else:
+            segs = [(n - nw, masks[b])]
+        q_rows += max(len(segs), 1) * wl.Hq
+        for nt, mrow in segs:
+            for h in range(wl.Hkv):
+                m = int(mrow[h]) & 0xFFFFFFFF
+                kept = popcount32(m)
+                touched = sum(1 for g in range(4) if (m >> (8 * g)) & 0xFF)
+                split += nt * (kept * kword + touched * 4 + (2 if wl.keep_ch0 and (m & 1) else 0))
+                split += nt * (128 * wl.v_bits // 8 + 16)
+        window += nw * wl.Hkv * 2 * 128 * 2  # bf16 key and value rows
+    if wl.bucket or wl.rotate_k == 2:
+        q_bytes = q_rows * 128 * 4  # transformed fp32 query rows
+    else:
+        q_bytes = wl.B * wl.Hq * 128 * (4 if wl.fmt == "f32" else 2)
     return {"split_kernel": split + q_bytes, "window": window,
             "step": split + window + q_bytes + wl.B * wl.Hq * 128 * 4}
 
@@ -189,15 +201,16 @@ class OracleLeg:
     """The CPU oracle on this host's cores: per step it selects channels and
     decodes every query head of one sequence over the oracle's own cache."""
 
-    def __init__(self, wl: workloads.Workload, s: synth.Synth, q: np.ndarray, n_seqs: int):
+    def __init__(self, wl: workloads.Workload, s: synth.Synth, q: np.ndarray, n_seqs: int, tq=None, tk=None,
+                 fr=None):
         from oracle import oracle as orc
 
-        self.orc, self.wl, self.n = orc, wl, n_seqs
+        self.orc, self.wl, self.n, self.tq = orc, wl, n_seqs, tq
         self.caches = []
         self.q = orc.as_f32(q)
         for b in range(n_seqs):
             c = orc.Cache(1, wl.Hkv, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
-                          wl.v_clip, wl.sink, wl.recent)
+                          wl.v_clip, wl.sink, wl.recent, tq, tk, bucket_w=wl.bucket, inv_freq=fr)
             k = np.stack([s.k_slice(b, h) for h in range(wl.Hkv)])[None]
             v = np.stack([s.v_slice(b, h) for h in range(wl.Hkv)])[None]
             c.append(orc.as_f32(k), orc.as_f32(v), wl.offset)
@@ -208,8 +221,10 @@ class OracleLeg:
         b = i % self.n
         qb = self.q[b:b + 1]
         mask = None
-        if self.wl.keep_groups < 32:
-            mask, _ = self.orc.select(qb, self.wl.Hkv, self.wl.rotate_k, self.wl.keep_groups)
+        if self.wl.keep_groups < 32 and self.wl.bucket:
+            mask, _ = self.caches[b].select_buckets(qb, self.lens[b:b + 1], self.wl.keep_groups)
+        elif self.wl.keep_groups < 32:
+            mask, _ = self.orc.select(qb, self.wl.Hkv, self.wl.rotate_k, self.wl.keep_groups, self.tq)
         return self.caches[b].attention(qb, self.lens[b:b + 1], mask, 1.0 / math.sqrt(128))
 
 
@@ -336,6 +351,7 @@ def workload_config(wl):
             "k_bits": wl.k_bits, "v_bits": wl.v_bits, "group": 32, "rotate_k": wl.rotate_k,
             "keep_ch0": wl.keep_ch0, "keep_groups": wl.keep_groups, "rotate_v": wl.rotate_v, "v_clip": wl.v_clip,
             "bf16_sink": wl.sink, "bf16_recent": wl.recent,
+            "dual_pair": wl.rotate_k == 2, "rope_bucket": wl.bucket,
             "input_dtype": wl.fmt,
             "l2": "flushed between steps (memset of 2x L2)", "parallelism": "replicas (one batch per GPU)"}
 
@@ -359,12 +375,23 @@ def run_kvq(args):
 
     # -- resident cache (built by the append kernel, not timed here)
     q_np = s.q()
+    tq = tk = fr = None
+    if wl.rotate_k == 2:  # the caller's dual transform pair
+        tq, tk = synth.dual_pair(rep.seed(wl), wl.Hkv)
+    if wl.bucket:  # the model's rotary frequencies
+        fr = synth.rope_inv_freq(wl.rope_base)
     cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev,
-                            rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent)
+                            rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent,
+                            t_query=None if tq is None else torch.from_numpy(tq).to(dev),
+                            t_key=None if tk is None else torch.from_numpy(tk).to(dev),
+                            bucket_tokens=wl.bucket, rope_inv_freq=None if fr is None else torch.from_numpy(fr).to(dev))
+    chunk = wl.bucket or wl.T  # an append stays inside one bucket
     for b in range(wl.B):  # one sequence at a time keeps host memory small
         kd = up(np.stack([s.k_slice(b, h) for h in range(wl.Hkv)]))
         vd = up(np.stack([s.v_slice(b, h) for h in range(wl.Hkv)]))
-        cache.append_sequence(b, kd, vd, wl.offset)
+        for t0 in range(0, wl.T, chunk):
+            cache.append_sequence(b, kd[:, t0:t0 + chunk].contiguous(), vd[:, t0:t0 + chunk].contiguous(),
+                                  wl.offset + t0)
         torch.cuda.synchronize()
         del kd, vd
     qd = up(q_np)
@@ -373,7 +400,8 @@ def run_kvq(args):
     max_len = int(wl.T if wl.len_range is None else wl.capacity)
     scale = 1.0 / math.sqrt(128)
     keep = wl.keep_groups
-    mask = torch.full((wl.B, wl.Hkv), -1, dtype=torch.int32, device=dev)
+    mask = torch.full((wl.B, cache.n_buckets, wl.Hkv) if wl.bucket else (wl.B, wl.Hkv), -1, dtype=torch.int32,
+                      device=dev)
     ws = torch.empty(cache.workspace_bytes(wl.Hq, max_len), dtype=torch.uint8, device=dev)
     out = torch.empty((wl.B, wl.Hq, 128), dtype=torch.float32, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -384,7 +412,9 @@ def run_kvq(args):
         flush.zero_()
         if ev is not None:
             ev[0].record(stream)
-        if keep < 32:
+        if keep < 32 and wl.bucket:
+            cache.select_at(qd, lens, keep, mask)
+        elif keep < 32:
             cache.select(qd, keep, mask)
         if ev is not None:
             ev[1].record(stream)
@@ -398,7 +428,7 @@ def run_kvq(args):
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
-    masks_np = mask.cpu().numpy().view(np.uint32) if keep < 32 else np.full((wl.B, wl.Hkv), 0xFFFFFFFF, np.uint32)
+    masks_np = mask.cpu().numpy().view(np.uint32) if keep < 32 else np.full(tuple(mask.shape), 0xFFFFFFFF, np.uint32)
     abytes = algorithmic_bytes(wl, masks_np, lens_np)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -443,7 +473,7 @@ def run_kvq(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        leg = OracleLeg(wl, s, q_np, n_seqs=1)
+        leg = OracleLeg(wl, s, q_np, n_seqs=1, tq=tq, tk=tk, fr=fr)
         rate, done, dt = oracle_rate(leg, args.cpu_seconds)
         cpu = {"value": rate, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                "sample": f"{done} decode steps of sequence 0 (all {wl.Hq} query heads over "
@@ -467,7 +497,8 @@ def run_kvq(args):
             "e2e": {"value": rep.whole_job(wl.B, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": int(q_pin.numel() * q_pin.element_size()),
                     "d2h_bytes_per_step": int(out_pin.numel() * 4)},
-            "gpu_launches": args.steps * (2 + (1 if keep < 32 else 0) + (1 if wl.sink + wl.recent else 0)),
+            "gpu_launches": args.steps * (2 + (1 if keep < 32 else 0) + (1 if wl.sink + wl.recent else 0) +
+                                          (1 if wl.rotate_k == 2 or wl.bucket else 0)),
             "roofline": {"bound": "hbm", "kernel": "decode split (kvq_decode_partials)", "achieved": achieved,
                          "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": abytes["split_kernel"], "peak_source": peak_src,

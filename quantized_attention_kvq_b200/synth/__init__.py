@@ -69,6 +69,26 @@ def normals(key: int, first: int, count: int, fmt: str = "f32", scale: np.ndarra
     return out
 
 
+def dual_pair(key: int, H: int, d: int = 128, spread: float = 0.35) -> tuple:
+    """Caller inputs of the dual transform pair: per kv head an anisotropic
+    invertible T = I + spread * N / sqrt(d) with its first d/2 columns doubled,
+    and T's inverse transpose, both fp32 [H][d][d] (seeded normals N)."""
+    z = normals(stream_key(key, 0x7A17), 0, H * d * d).astype(np.float64).reshape(H, d, d)
+    tq = np.empty((H, d, d), np.float32)
+    tk = np.empty((H, d, d), np.float32)
+    for h in range(H):
+        t = np.eye(d) + spread * z[h] / np.sqrt(d)
+        t[:, : d // 2] *= 2.0
+        tq[h] = t
+        tk[h] = np.linalg.inv(t).T
+    return tq, tk
+
+
+def rope_inv_freq(base: float, d: int = 128) -> np.ndarray:
+    """A model's rotary inverse frequencies base^(-2i/d), i < d/2, fp32."""
+    return (base ** (-np.arange(0, d, 2, dtype=np.float64) / d)).astype(np.float32)
+
+
 def channel_scales(key: int, d: int, sigma: float = 0.5, n_outliers: int = 4, mult: float = 10.0) -> np.ndarray:
     out = np.empty(d, dtype=np.float64)
     _load().kvqgen_chscale(key, d, sigma, n_outliers, mult, _ptr(out))

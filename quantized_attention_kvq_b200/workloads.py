@@ -31,6 +31,8 @@ class Workload:
     kind: str = "decode"  # what bench.py times: "decode" or "append"
     sink: int = 0       # bf16 window: the first tokens of each sequence
     recent: int = 0     # bf16 window: the most recent tokens of each sequence
+    bucket: int = 0     # bucket-relative RoPE bucket width (0 = none); keys and queries drawn before RoPE
+    rope_base: float = 1.0e6  # rotary base of the inverse frequencies (the Qwen3 value)
 
     @property
     def G(self) -> int:
@@ -53,6 +55,11 @@ WORKLOADS = [
     # and the first 64 and most recent 256 tokens kept in bf16 (Dual-QK Sec. 3.3)
     Workload(7, "dualqk_int2_vrot_win64x256_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16", 2,
              2, 1, 1, 19, rotate_v=1, v_clip=0.92, sink=64, recent=256),
+    # a caller-supplied dual transform pair on queries and keys (Dual-QK Sec. 3.1)
+    # with bucket-relative RoPE at w = 2048 (Sec. 3.4); bf16 windows are not
+    # combined with buckets on the CUDA path
+    Workload(8, "dualqk_int2_pair_bucket2048_vrot_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16",
+             2, 2, 2, 1, 19, rotate_v=1, v_clip=0.92, bucket=2048),
 ]
 
 BASE_SEED = 0

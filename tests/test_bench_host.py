@@ -65,3 +65,29 @@ def test_decode_bytes_with_bf16_windows():
     split = sum((int(n) - w) * per_code for n, w in zip(lens, windowed)) * wl.Hkv
     assert got["split_kernel"] == split + wl.B * wl.Hq * 128 * 2
     assert got["window"] == sum(windowed) * wl.Hkv * 2 * 128 * 2
+
+
+def test_decode_bytes_with_rope_buckets():
+    # each 2048-token bucket counts with its own mask; the split decode reads
+    # one fp32 query row per (bucket holding tokens, query head)
+    wl = workloads.by_id(8)
+    nb = wl.capacity // wl.bucket
+    keep = (1 << 19) - 1
+    other = 0xFFFFFFFF ^ 1
+    masks = np.zeros((wl.B, nb, wl.Hkv), np.uint32)
+    masks[:, 0::2, :] = keep
+    masks[:, 1::2, :] = other
+    lens = np.array([wl.T, 2048, 2049, 1], np.int32)
+    got = bench.algorithmic_bytes(wl, masks, lens)
+    per = {keep: 19 * 4 * 2 // 8 + 3 * 4 + 2 + 128 * 2 // 8 + 4 * 4,
+           other: 31 * 4 * 2 // 8 + 4 * 4 + 128 * 2 // 8 + 4 * 4}
+    want = 0
+    rows = 0
+    for n in lens:
+        used = -(-int(n) // wl.bucket)
+        rows += used * wl.Hq
+        for k in range(used):
+            nk = min(int(n) - k * wl.bucket, wl.bucket)
+            want += nk * wl.Hkv * per[keep if k % 2 == 0 else other]
+    assert got["split_kernel"] == want + rows * 128 * 4
+    assert got["window"] == 0
