@@ -309,6 +309,17 @@ class Replicas:
 
 
 # ------------------------------------------------------------------ main arms
+def option_inputs(wl: workloads.Workload, seed: int):
+    """The caller inputs of the workload's options: (t_query, t_key, inv_freq),
+    None where the option is off."""
+    tq = tk = fr = None
+    if wl.rotate_k == 2:  # the caller's dual transform pair
+        tq, tk = synth.dual_pair(seed, wl.Hkv)
+    if wl.bucket:  # the model's rotary frequencies
+        fr = synth.rope_inv_freq(wl.rope_base)
+    return tq, tk, fr
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -319,7 +330,8 @@ def run_reference(args):
         leg, per_step, unit, metric = OracleAppendLeg(wl, s), wl.T, "appended tokens/s", APPEND_METRIC
         sample = f"the {wl.T} new tokens of sequence 0 ({wl.Hkv} kv heads) appended per step"
     else:
-        leg, per_step, unit, metric = OracleLeg(wl, s, s.q(), n_seqs=1), 1, "tokens/s", METRIC
+        tq, tk, fr = option_inputs(wl, workloads.BASE_SEED + wl.id)
+        leg, per_step, unit, metric = OracleLeg(wl, s, s.q(), 1, tq, tk, fr), 1, "tokens/s", METRIC
         sample = f"all {wl.Hq} query heads of sequence 0 over its {int(s.lens[0])} cached tokens per step"
     for i in range(args.warmup):
         leg.step(i)
@@ -375,11 +387,7 @@ def run_kvq(args):
 
     # -- resident cache (built by the append kernel, not timed here)
     q_np = s.q()
-    tq = tk = fr = None
-    if wl.rotate_k == 2:  # the caller's dual transform pair
-        tq, tk = synth.dual_pair(rep.seed(wl), wl.Hkv)
-    if wl.bucket:  # the model's rotary frequencies
-        fr = synth.rope_inv_freq(wl.rope_base)
+    tq, tk, fr = option_inputs(wl, rep.seed(wl))
     cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev,
                             rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent,
                             t_query=None if tq is None else torch.from_numpy(tq).to(dev),
