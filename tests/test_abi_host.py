@@ -162,6 +162,10 @@ def test_bucket_rope_host_checks(L):
         native.KVQ_ERR_INVALID_ARG
     assert L.kvq_select_channels_at(ctypes.byref(d), FAKE, native.KVQ_BF16, 8, None, 4, FAKE, None) == \
         native.KVQ_ERR_INVALID_ARG
+    many = desc(B=300, cap=128 * 256, bucket_tokens=128)  # 300 x 256 bucket rows
+    many.rope_inv_freq = FAKE
+    assert L.kvq_quantize_append(ctypes.byref(many), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
+        native.KVQ_ERR_UNSUPPORTED
     odd = desc(cap=512, bucket_tokens=384)
     odd.rope_inv_freq = FAKE
     assert L.kvq_quantize_append(ctypes.byref(odd), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
