@@ -54,3 +54,24 @@ def test_lengths_in_range():
     s = synth.Synth(9, 64, 64, 8, 128, 16384, "bf16", (1024, 16384))
     assert s.lens.min() >= 1024 and s.lens.max() <= 16384
     assert len(set(s.lens.tolist())) > 50
+
+
+def test_dual_pair_inputs_are_seeded_inverse_transposes():
+    tq, tk = synth.dual_pair(8, 3)
+    tq2, tk2 = synth.dual_pair(8, 3)
+    assert np.array_equal(tq, tq2) and np.array_equal(tk, tk2)  # same seed, same matrices
+    assert not np.array_equal(tq, synth.dual_pair(9, 3)[0])
+    assert tq.dtype == np.float32 and tq.shape == (3, 128, 128)
+    for h in range(3):
+        t = tq[h].astype(np.float64)
+        # T^T T^-T = I up to the fp32 rounding of T^-T
+        assert np.abs(t.T @ tk[h].astype(np.float64) - np.eye(128)).max() < 1e-5
+        assert not np.allclose(t, t.T)  # a general pair, not an orthogonal one
+        assert np.linalg.cond(t) < 20
+
+
+def test_rope_frequencies():
+    f = synth.rope_inv_freq(1.0e6)
+    assert f.dtype == np.float32 and f.shape == (64,)
+    assert f[0] == 1.0 and np.all(np.diff(f) < 0)
+    np.testing.assert_allclose(f[32], 1.0e6 ** -0.5, rtol=1e-7)
