@@ -184,7 +184,7 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
       if (v.max_len > 0 && (st = cuda_status(launch_decode(v, s))) != KVQ_OK) return st;
     }
     if (parts & kRunCombine)
-      return cuda_status(launch_bucket_merge(v, nb, decode_slots(0, 0, G) / decode_groups(G), out, s));
+      return cuda_status(launch_bucket_merge(v, nb, decode_slots(0, 0, G) / decode_groups(G), decode_groups(G), out, s));
     return KVQ_OK;
   }
   DecodeArgs a;

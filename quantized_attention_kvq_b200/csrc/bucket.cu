@@ -42,9 +42,11 @@ __device__ __forceinline__ int bucket_tiles(const DecodeArgs& v, int vb) {
 // split decode left, for bucket unit u = vb * H + h of n_t tiles starting at
 // tile t_u of the flattened tile list, one partial per CTA c in
 // [t_u / per, (t_u + n_t - 1) / per] (per = ceil(total tiles / ctas)) in slot
-// u + c, row slot * G + the head's index in its group; an empty one has max
-// -inf.  Maxima and sums are in the log2 domain of the decode.
-__global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb, int ctas, float* __restrict__ out) {
+// (u + c) * ngrp + e for each of its ngrp epilogue groups e, row slot * G +
+// the head's index in its group; an empty one has max -inf.  Maxima and sums
+// are in the log2 domain of the decode.
+__global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb, int ctas, int ngrp,
+                                                           float* __restrict__ out) {
   const int row = blockIdx.x;  // b * Hq + query head
   const int b = row / v.Hq, hq = row - b * v.Hq;
   const int G = v.Hq / v.c.H;
@@ -63,7 +65,7 @@ __global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb,
       const int vb = b * nb + k, nt = bucket_tiles(v, vb);
       if (nt > 0) {
         const int u = vb * v.c.H + h, tu = t0 + h * nt;
-        for (int sl = u + tu / per; sl <= u + (tu + nt - 1) / per; ++sl)
+        for (int sl = (u + tu / per) * ngrp; sl < (u + (tu + nt - 1) / per + 1) * ngrp; ++sl)
           M = fmaxf(M, v.part_ml[(size_t)sl * G + hl].x);
       }
       t0 += v.c.H * nt;
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb,
       const int vb = b * nb + k, nt = bucket_tiles(v, vb);
       if (nt > 0) {
         const int u = vb * v.c.H + h, tu = t0 + h * nt;
-        for (int sl = u + tu / per; sl <= u + (tu + nt - 1) / per; ++sl) {
+        for (int sl = (u + tu / per) * ngrp; sl < (u + (tu + nt - 1) / per + 1) * ngrp; ++sl) {
           const size_t r = (size_t)sl * G + hl;
           const float2 ml = v.part_ml[r];
           if (ml.x == NEG_INF) continue;
@@ -130,8 +132,8 @@ cudaError_t launch_bucket_queries(const void* q, int dtype, int rotate, const fl
   return cudaGetLastError();
 }
 
-cudaError_t launch_bucket_merge(const DecodeArgs& v, int nb, int ctas, float* out, cudaStream_t s) {
-  k_bucket_merge<<<(v.c.B / nb) * v.Hq, kHeadDim, 0, s>>>(v, nb, ctas, out);
+cudaError_t launch_bucket_merge(const DecodeArgs& v, int nb, int ctas, int ngrp, float* out, cudaStream_t s) {
+  k_bucket_merge<<<(v.c.B / nb) * v.Hq, kHeadDim, 0, s>>>(v, nb, ctas, ngrp, out);
   return cudaGetLastError();
 }
 

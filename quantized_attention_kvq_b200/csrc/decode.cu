@@ -1,5 +1,5 @@
-// Split decode over the packed cache on the tcgen05 tensor cores, with both
-// MMA A-operands (key codes, value codes) built in tensor memory.
+// Split decode over the packed cache on the tcgen05 tensor cores: scores and
+// the value sums are both integer MMAs straight from the codes.
 //
 // Work split ("stream-K"): every (sequence b, kv head h) unit contributes
 // ceil(len_b / 128) tiles of 128 tokens; the tiles of all units, in (b, h)
@@ -10,17 +10,18 @@
 // touch at their ends.  The combine pass merges a unit's slots into one
 // softmax over the whole sequence (Dual-QK summary Sec. 3.4).
 //
-// A tcgen05.mma costs about the same whatever its N (up to 256), so the
-// schedule minimises MMA instructions per tile and keeps dependent ones apart:
-//   scores: 4 MMAs of kind::i8 (K = 32 = one quantization group each): key
-//           codes as u8 in tensor memory x the rotated query as two exact s8
-//           pieces (q = delta * (128 q1 + q2)), one s32 accumulator per group,
-//           so the per-token group scale applies exactly afterwards;
-//   PV:     8 MMAs of kind::f16 (K = 16 tokens each): value codes centred as
-//           c - L/2 (exact f16) in tensor memory x P' = p * value scale, spread
-//           over independent partial accumulators that stay in tensor memory
-//           for a whole segment (one accumulator set per segment parity); the
-//           zero point, with the L/2 steps folded in, is summed in registers.
+// Per 128-token tile, 8 MMAs:
+//   scores: 4 of kind::i8 (K = 32 = one quantization group each): key codes
+//           as u8 in tensor memory x the rotated query as two exact s8 pieces
+//           (q = delta * (128 q1 + q2)), one s32 accumulator per group, so the
+//           per-token group scale applies exactly afterwards;
+//   PV:     4 of kind::i8 (K = 32 tokens each): value codes as u8 in tensor
+//           memory x P' as three u8 bytes of a 23-bit integer, P' = p * value
+//           scale normalized per tile by the tile's largest p (per head) and
+//           largest value scale (per group) to [0, 2^23 - 1], so the s32 sums
+//           are exact and P' can neither overflow nor lose precision at the
+//           ends of any float range; each tile's sums are read back and added,
+//           with the tile's scale, into fp32 accumulators held in registers.
 //
 // Roles inside a CTA, pipelined over tiles with mbarriers:
 //   producer warp   : 1-D bulk async copies of a tile's kept key-code rows
@@ -31,17 +32,15 @@
 //                     memory (lane = token); at a segment start also the
 //                     query operand (dropped channel groups zeroed), its
 //                     per-head step and its per-group sums;
-//   value warps (4) : thread = channel: the channel's 128 value codes -> f16
+//   value warps (4) : thread = channel: the channel's 128 value codes -> u8
 //                     -> tensor memory (lane = channel);
 //   UMMA warp       : the score MMAs one tile ahead, then the PV MMAs;
 //   epilogue warps  : thread = (token, heads): score = delta * sum_g s_g S_g +
-//                     sum_g z_g sum(q_g) (+ q_0 k_0), online softmax with a
-//                     lazily raised max, P' into shared memory, the value
-//                     zero-point terms sum_t p_t z_t in registers; when the max
-//                     rises inside a segment, thread = (channel, heads) rescales
-//                     the segment's PV accumulator in tensor memory; two tiles
-//                     after a segment ends, the accumulator is read out into
-//                     the segment's partial.
+//                     sum_g z_g sum(q_g) (+ q_0 k_0), the tile's maxima, the
+//                     online softmax with a lazily raised running max, P' into
+//                     shared memory, the value zero-point terms sum_t p_t z_t;
+//                     thread = (channel, heads): the PV sums of the tile before
+//                     last into the fp32 accumulators.
 // Scores come straight from the codes; no dequantized key is ever formed
 // (tq-kv abstract; Dual-QK summary Sec. 3.2, 3.3).  Every mbarrier wait is
 // bounded; after a give-up all waits fall through and the CTA writes NaN
@@ -60,36 +59,36 @@ constexpr float kLazyMax = 8.0f;  // the running max is raised only when a score
 constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr float kQSteps = 16000.0f;  // |q| / delta <= 16000: pieces q1 in [-125, 125], q2 in [-64, 63]
+constexpr float kPSteps = 8388607.0f;  // P' integer range: 2^23 - 1, three u8 bytes
 
 template <int G, int KB, int VB, bool CH0>
 struct Shape {
   static constexpr int TPT = G > 4 ? 2 : 1;  // epilogue threads per token (head parts)
   static constexpr int HH = G / TPT;         // heads per epilogue thread: 1, 2, 4 or 8
-  static constexpr int NGRP = 1;  // epilogue groups, group g taking tiles t with t % NGRP == g (2 measured no faster)
-  static constexpr int EPI_WARPS = 4 * TPT * NGRP;
+  static constexpr int EPI_WARPS = 4 * TPT;
   static constexpr int EPI_THREADS = 32 * EPI_WARPS;
   static constexpr int MMA_WARP = 8 + EPI_WARPS;
   static constexpr int PROD_WARP = MMA_WARP + 1;
   static constexpr int THREADS = 32 * (PROD_WARP + 1);
   static constexpr int NS = 2 * G < 16 ? 16 : 2 * G;  // score columns per group: q1 rows, then q2 rows
-  static constexpr int NO = 4 * G < 16 ? 16 : 4 * G;  // PV columns: (value group, head)
+  static constexpr int PH = 4 * G;  // P' columns per byte: (value group, head)
+  // PV columns: low, middle, high bytes, padded to a power of two (>= 16)
+  static constexpr int NPV = 3 * PH <= 16 ? 16 : (3 * PH <= 32 ? 32 : (3 * PH <= 64 ? 64 : (3 * PH <= 128 ? 128 : 256)));
   static constexpr int KST = G > 8 ? 1 : 2;  // key operand stages in tensor memory
-  static constexpr int VST = G > 8 ? 1 : 2;  // value operand stages in tensor memory
-  static constexpr int SB = 2;               // score accumulator buffers
+  static constexpr int VST = 2;              // value operand stages in tensor memory
+  static constexpr int SB = G > 8 ? 1 : 2;   // score accumulator buffers
   static constexpr int LA = SB - 1;          // score MMAs are issued LA tiles ahead of the PV MMAs
   static constexpr int NKR = KST > 1 ? KST : 2;  // key-ready barriers
-  static constexpr int OB = 2;                        // PV accumulator sets: one per segment parity
-  static constexpr int PP = G > 8 ? 1 : 2;  // partial accumulators per PV (independent chains)
   // tensor-memory columns; every accumulator starts at a multiple of its width
-  static constexpr int TM_AK = 0;                                  // KST key stages x 32 columns (128 u8 codes)
-  static constexpr int TM_AV = 32 * KST;                           // VST value stages x 64 columns (128 f16 codes)
-  static constexpr int TM_S = (TM_AV + 64 * VST + 63) / 64 * 64;   // SB score buffers x 4 groups x NS
-  static constexpr int TM_O = TM_S + SB * 4 * NS;                  // NGRP x 2 PV sets x PP partials x NO
+  static constexpr int TM_AK = 0;             // KST key stages x 32 columns (128 u8 codes)
+  static constexpr int TM_AV = 32 * KST;      // VST value stages x 32 columns (128 u8 codes)
+  static constexpr int TM_S = 128;            // SB score buffers x 4 groups x NS
+  static constexpr int TM_D = 256;            // DB PV buffers x NPV
   static constexpr int TMEM_COLS = 512;
-  static_assert(TM_AK + 32 * KST <= TM_AV && TM_AV + 64 * VST <= TM_S, "operand columns");
-  static_assert(SB >= LA + 1 && KST >= 1 && VST <= 2, "stage counts");
-  static_assert(TM_O + NGRP * OB * PP * NO <= TMEM_COLS, "tensor memory");
-  static_assert(TM_S % NS == 0 && TM_O % NO == 0, "accumulator alignment");
+  static constexpr int DB = TM_D + 2 * NPV <= TMEM_COLS ? 2 : 1;  // PV buffers: read back 2 or 1 tiles later
+  static_assert(TM_AV + 32 * VST <= TM_S && TM_S + SB * 4 * NS <= TM_D, "operand columns");
+  static_assert(TM_D + DB * NPV <= TMEM_COLS, "tensor memory");
+  static_assert(TM_S % NS == 0 && TM_D % NPV == 0, "accumulator alignment");
   // one ring stage: key-code rows, value-code rows, key (scale, zero) rows,
   // value (scale, zero) per token, channel 0
   static constexpr int KROW = kTile * (KB == 4 ? 2 : 1);  // bytes of one key row (4 channels)
@@ -102,7 +101,7 @@ struct Shape {
   static constexpr int STAGE = (R_K0 + (CH0 ? kTile * 2 : 0) + 127) / 128 * 128;
   // fixed region behind the ring
   static constexpr int BQ_BYTES = NS * kHeadDim;     // s8 query operand: NS rows x 128 channels
-  static constexpr int BP_BYTES = NO * kTile * 2;    // one f16 P' operand
+  static constexpr int BP_BYTES = NPV * kTile;       // one u8 P' operand: NPV columns x 128 tokens
   // query data per segment, double-buffered by segment parity
   static constexpr int QV = (G * 4 + 15) / 16 * 16;  // bytes of G floats, rounded to 16
   static constexpr int F_BQ = 0;                     // [2] query operands
@@ -110,10 +109,9 @@ struct Shape {
   static constexpr int F_QS = F_BP + 2 * BP_BYTES;   // [2][G][4] f32: per-group sums of the kept q
   static constexpr int F_Q0 = F_QS + 2 * G * 16;     // [2][G] f32: q_0 (channel 0 kept in bf16)
   static constexpr int F_QD = F_Q0 + 2 * QV;         // [2][G] f32: delta of the query pieces
-  static constexpr int F_RED = F_QD + 2 * QV;        // [2 tiles][TPT][4 warps][16] f32
-  static constexpr int F_RED2 = F_RED + 2 * TPT * 4 * 16 * 4;         // [NGRP][TPT][4 warps][16] f32
-  static constexpr int F_PEND = F_RED2 + NGRP * TPT * 4 * 16 * 4;     // [NGRP][2 segment parities][TPT][6 HH] f32
-  static constexpr int F_BAR = (F_PEND + NGRP * 2 * TPT * 6 * HH * 4 + 15) / 16 * 16;
+  static constexpr int F_RED = F_QD + 2 * QV;        // [2 tiles][TPT][4 warps][16] s32: warp maxima
+  static constexpr int F_RED2 = F_RED + 2 * TPT * 4 * 16 * 4;  // [TPT][4 warps][16] f32: segment sums
+  static constexpr int F_BAR = (F_RED2 + TPT * 4 * 16 * 4 + 15) / 16 * 16;
   // kready[3] vready[2] pready[2] sdone[3] pvdone[2] qready[2] qfree[2]
   static constexpr int NBAR_FIXED = 16;
   static constexpr int F_REST_NO_RING = F_BAR + NBAR_FIXED * 8 + 16;  // + tmem slot, error flag
@@ -136,21 +134,29 @@ __device__ __forceinline__ int kpos_of(int r) {
   if (BITS == 4) return (r & 1) * 4 + (r >> 1);
   return 4 * (r & 3) + (r >> 2);
 }
-// K position of code i of an 8-token (INT4) or 16-token (INT2) block in the
-// f16 value operand: the f16 conversion pairs code i with code i + 4 (i + 8).
+// K position (byte) of token j of a tile in the u8 value operand: the INT4
+// unpacking puts the even tokens of each 8-token word first, the INT2
+// unpacking crumb m of every byte of a 16-token word together.
 template <int BITS>
-__device__ __forceinline__ int vpos_of(int i) {
-  if (BITS == 4) return i < 4 ? 2 * i : 2 * (i - 4) + 1;
-  return i < 8 ? 2 * i : 2 * (i - 8) + 1;
+__device__ __forceinline__ int vpos_of(int j) {
+  if (BITS == 4) return (j & ~7) + 4 * (j & 1) + ((j & 7) >> 1);
+  return (j & ~15) + 4 * (j & 3) + ((j & 15) >> 2);
 }
 // byte offset of element (row r, byte k) in a K-major 8-bit operand with 128 K bytes
 __device__ __forceinline__ uint32_t kmajor8(int r, int k) {
   return (r & 7) * 16 + (k & 15) + (k >> 4) * 128 + (r >> 3) * 1024;
 }
-// byte offset of element (mn, k) in an MN-major f16 operand with 128 K elements
-__device__ __forceinline__ uint32_t mnmajor(int mn, int k) {
-  return (mn & 7) * 2 + (k & 7) * 16 + (mn >> 3) * 2048 + (k >> 3) * 128;
+// byte offset of element (n, k) in an MN-major 8-bit operand with 128 K elements
+__device__ __forceinline__ uint32_t mnmajor8(int n, int k) {
+  return (n & 15) + (k & 7) * 16 + (n >> 4) * 2048 + (k >> 3) * 128;
 }
+// Order-preserving map of a float onto int32 (and back: it is its own inverse),
+// so that a warp's float maximum is one integer reduction.
+__device__ __forceinline__ int ord_of(float x) {
+  const int i = __float_as_int(x);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float float_of_ord(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF); }
 
 __device__ __forceinline__ int tiles_of(const DecodeArgs& a, int b) {
   const int len = min(max(a.seq_lens[b], 0), a.max_len);
@@ -229,19 +235,6 @@ __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile 
 __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
-// named barrier that also ORs a predicate over the participating threads
-__device__ __forceinline__ bool named_sync_or(int id, int threads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(threads)
-      : "memory");
-  return r != 0;
-}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -249,7 +242,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 template <int G, int KB, int VB, bool CH0, typename In>
 __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(DecodeArgs a) {
   using S = Shape<G, KB, VB, CH0>;
-  constexpr int HH = S::HH, ST = S::STAGES, OB = S::OB, PP = S::PP;
+  constexpr int HH = S::HH, ST = S::STAGES;
   extern __shared__ __align__(1024) uint8_t smem[];
   const CacheView& c = a.c;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -281,16 +274,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(FULL(s), 1);
-      mbar_init(EMPTY(s), 256 + S::EPI_THREADS / S::NGRP);  // key, value and the tile's epilogue group
+      mbar_init(EMPTY(s), 256 + S::EPI_THREADS);  // key, value and epilogue threads
     }
     for (int k = 0; k < S::NKR; ++k) mbar_init(KREADY(k), 128);
     for (int k = 0; k < S::SB; ++k) mbar_init(SDONE(k), 1);
     for (int k = 0; k < 2; ++k) {
       mbar_init(VREADY(k), 128);
-      mbar_init(PREADY(k), S::EPI_THREADS / S::NGRP);
-    }
-    for (int k = 0; k < 2; ++k) mbar_init(PVDONE(k), 1);
-    for (int k = 0; k < 2; ++k) {
+      mbar_init(PREADY(k), S::EPI_THREADS);
+      mbar_init(PVDONE(k), 1);
       mbar_init(QREADY(k), 128);
       mbar_init(QFREE(k), S::EPI_THREADS);
     }
@@ -344,19 +335,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   } else if (warp == S::MMA_WARP) {
     // ================================================================ UMMA issue
     const uint32_t idesc_s = idesc_u8s8_s32(kTile, S::NS);
-    const uint32_t idesc_o = idesc_f16_f32(kTile, S::NO, 0, 1);
+    const uint32_t idesc_o = idesc_u8u8_s32_bmn(kTile, S::NPV);
     const uint32_t bp = smem_addr(fix + S::F_BP);
-    int sseg = -1;    // segment of the tile being scored
-    int sstart = 0;   // its first tile
-    // bit (t & 3): tile t is its epilogue group's first of the segment / the segment's parity
-    uint32_t firstbits = 0, setbits = 0;
+    int sseg = -1;  // segment of the tile being scored
     auto score = [&](int t) {
-      if (it.first) {
-        ++sseg;
-        sstart = t;
-      }
-      firstbits = (firstbits & ~(1u << (t & 3))) | ((t - sstart < S::NGRP ? 1u : 0u) << (t & 3));
-      setbits = (setbits & ~(1u << (t & 3))) | ((uint32_t)(sseg & 1) << (t & 3));
+      if (it.first) ++sseg;
       const uint32_t bq = smem_addr(fix + S::F_BQ + (sseg & 1) * S::BQ_BYTES);
       it.next(a);
       ws_wait(KREADY(t % S::NKR), (t / S::NKR) & 1, err);
@@ -383,18 +366,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       ws_wait(VREADY(t & 1), (t >> 1) & 1, err);
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a0 = tmem + S::TM_AV + (t % S::VST) * 64;
+        // 32 tokens per MMA: u8 value codes (8 tensor-memory columns) x the
+        // tile's P' bytes; each tile's sums start afresh in PV buffer t & 1
+        const uint32_t a0 = tmem + S::TM_AV + (t % S::VST) * 32;
         const uint32_t b0 = bp + (t & 1) * S::BP_BYTES;
-        // accumulator set: (epilogue group of tile t, segment parity)
-        const uint32_t set = (S::NGRP == 2 ? (uint32_t)(t & 1) * OB : 0u) + ((setbits >> (t & 3)) & 1u);
-        const uint32_t d0 = tmem + S::TM_O + set * PP * S::NO;
-        const bool fresh = (firstbits >> (t & 3)) & 1u;  // the group's first tile of the segment starts its sums
-        // 16 tokens per MMA; K step s accumulates into partial s % PP, so
-        // consecutive MMAs of one accumulator are PP issues apart
+        const uint32_t d0 = tmem + S::TM_D + (t % S::DB) * S::NPV;
 #pragma unroll
-        for (int s = 0; s < kTile / 16; ++s)
-          umma_f16_tmem_a(d0 + (s % PP) * S::NO, a0 + s * 8, smem_desc(b0 + s * 256, 128, 2048), idesc_o,
-                          (fresh && s < PP) ? 0u : 1u);
+        for (int s = 0; s < kTile / 32; ++s)
+          umma_i8_tmem_a(d0, a0 + s * 8, smem_desc(b0 + s * 512, 128, 2048), idesc_o, s > 0 ? 1u : 0u);
         umma_commit(PVDONE(t & 1));
       }
       __syncwarp();
@@ -507,37 +486,32 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       // this value stage was read by the PV UMMAs of tile t - VST
       if (t >= S::VST) ws_wait(PVDONE((t - S::VST) & 1), ((t - S::VST) >> 1) & 1, err);
       tc_fence_after();
-      const uint32_t col = tl + S::TM_AV + (t % S::VST) * 64;
-      constexpr int CHUNKS = S::VROW / 16;  // 4 (INT4: 32 tokens each) or 2 (INT2: 64 tokens each)
+      uint32_t r[32];  // 128 u8 codes in the order vpos_of gives
+      if (VB == 4) {
 #pragma unroll
-      for (int k = 0; k < CHUNKS; ++k) {
-        const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * (k ^ swz));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-        if (VB == 4) {
-          uint32_t rr[16];
+        for (int k = 0; k < 4; ++k) {  // 16-byte chunk k: tokens 32k .. 32k+31, 8 per word
+          const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * (k ^ swz));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            uint32_t c4[4];
-            codes4_to_f16(ws[i], c4);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) rr[4 * i + m] = c4[m];
-          }
-          tmem_st16(col + 16 * k, rr);
-        } else {
-#pragma unroll
-          for (int hlf = 0; hlf < 2; ++hlf) {
-            uint32_t rr[16];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              uint32_t c8[8];
-              codes2_to_f16(ws[2 * hlf + i], c8);
-#pragma unroll
-              for (int m = 0; m < 8; ++m) rr[8 * i + m] = c8[m];
-            }
-            tmem_st16(col + 32 * k + 16 * hlf, rr);
+            r[8 * k + 2 * i] = ws[i] & 0x0F0F0F0Fu;             // even tokens
+            r[8 * k + 2 * i + 1] = (ws[i] >> 4) & 0x0F0F0F0Fu;  // odd tokens
           }
         }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {  // 16-byte chunk k: tokens 64k .. 64k+63, 16 per word
+          const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * (k ^ swz));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int m = 0; m < 4; ++m) r[16 * k + 4 * i + m] = (ws[i] >> (2 * m)) & 0x03030303u;
+        }
       }
+      const uint32_t col = tl + S::TM_AV + (t % S::VST) * 32;
+      tmem_st16(col, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
+      tmem_st16(col + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(VREADY(t & 1));
@@ -545,117 +519,65 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     }
   } else if (warp < 8 + S::EPI_WARPS) {
     // ================================================================ epilogue
-    // With NGRP epilogue groups, group g takes the tiles t with t % NGRP == g,
-    // so one tile's chain of waits and latencies can overlap another's; each
-    // group keeps its own online softmax and PV accumulator sets per segment and
-    // leaves its own partial, which the combine merges like any other split.
-    // (Two groups measured no faster than one at G = 4, so NGRP is 1.)
-    const int e = tid - 256;                  // 0 .. EPI_THREADS-1
-    const int grp = e / (128 * S::TPT);       // epilogue group
-    const int j = e & 127;                    // token (score phase) == tensor-memory lane == channel (PV phase)
-    const int part = (e >> 7) % S::TPT;       // head part: heads part*HH .. part*HH + HH - 1
-    const int wq = warp & 3;                  // lane quarter == value group in the PV phase
-    const int bar_id = 1 + grp * S::TPT + part;
+    const int e = tid - 256;             // 0 .. EPI_THREADS-1
+    const int j = e & 127;               // token (score phase) == tensor-memory lane == channel (PV phase)
+    const int part = e >> 7;             // head part: heads part*HH .. part*HH + HH - 1
+    const int wq = warp & 3;             // lane quarter == value group of channel j
+    const int bar_id = 1 + part;
     const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
-    // K position of token j in the P' operand (the value conversion's pairing)
-    const int pos = VB == 4 ? (j & ~7) + vpos_of<4>(j & 7) : (j & ~15) + vpos_of<2>(j & 15);
-    float* red = reinterpret_cast<float*>(fix + S::F_RED);      // [2][TPT][4][16]
-    float* red2 = reinterpret_cast<float*>(fix + S::F_RED2) + grp * S::TPT * 64;         // [TPT][4][16]
-    float* pend = reinterpret_cast<float*>(fix + S::F_PEND) + grp * 2 * S::TPT * 6 * HH;  // [2][TPT][6 HH]
+    const int pos = vpos_of<VB>(j);      // K position of token j in the P' operand
+    int* rmax = reinterpret_cast<int*>(fix + S::F_RED);                      // [2][TPT][4][16]
+    float* red2 = reinterpret_cast<float*>(fix + S::F_RED2) + part * 64;      // [4][16]
     const float NEG_INF = -__int_as_float(0x7f800000);
+    // P' columns of this part: (byte, part, group, head), 4 HH per part and byte
+    constexpr int NC = 4 * HH;
+    const int n0 = part * NC;
 
     float m_run[HH], l_acc[HH], zacc[kGroups][HH];
+    float acc[HH];  // PV sums of channel j for this part's heads, scaled to m_run
+    // PV sums of the last tile (ds1) and, with two PV buffers, the tile before
+    // (ds2) still to be read back, with their scales for channel j's group; a
+    // tile's sums are read back RD tiles later, before the PV MMAs that reuse
+    // its buffer are issued
+    constexpr int RD = S::DB;
+    float ds1[HH] = {}, ds2[HH] = {};
+    bool have1 = false, have2 = false;
     // this segment's query data for the thread's heads (per-group sums of the
     // kept q, q_0, the step of the query pieces), held in registers when one
     // thread takes a token's heads, else read from shared memory per tile
     constexpr bool QREG = S::TPT == 1;
     float qsg[QREG ? HH : 1][kGroups], q0r[QREG ? HH : 1], qdr[QREG ? HH : 1];
-    int nseg = 0;       // segments begun so far
-    int qb = 0;         // query buffer and PV accumulator set of the current segment (its parity)
-    int seg_tiles = 0;  // tiles of the current segment this group has taken
-    int last_own = 0;   // the last tile this group took
-    // segments waiting for their read-out: last tile into the set, set, partial slot
-    int pn = 0, p0_tile = 0, p0_set = 0, p0_slot = 0, p1_tile = 0, p1_set = 0, p1_slot = 0;
+    int nseg = 0;  // segments begun so far
+    int qb = 0;    // query buffer of the current segment (its parity)
     bool ok = true;
-#pragma unroll
-    for (int i = 0; i < HH; ++i) {
-      m_run[i] = NEG_INF;
-      l_acc[i] = 0.0f;
-#pragma unroll
-      for (int g = 0; g < kGroups; ++g) zacc[g][i] = 0.0f;
-    }
 
-    // this thread's PV accumulator columns (channel j, its HH heads) of partial 0 of set os
-    auto obase = [&](int os) {
-      return tmem + lane_base + S::TM_O + (grp * OB + os) * PP * S::NO + wq * G + part * HH;
-    };
-    // sum of the PP partials of set os (after the last PV into it completed)
-    auto load_out = [&](int os, float (&d)[HH]) {
-      const uint32_t base = obase(os);
-      if constexpr (PP == 4) {
-        uint32_t r[4][HH];
-        tmem_ld4_wait<HH>(base, S::NO, r);
-#pragma unroll
-        for (int i = 0; i < HH; ++i)
-          d[i] = (__uint_as_float(r[0][i]) + __uint_as_float(r[1][i])) +
-                 (__uint_as_float(r[2][i]) + __uint_as_float(r[3][i]));
-      } else if constexpr (PP == 2) {
-        uint32_t r0[HH], r1[HH];
-        tmem_ld_wait<HH>(base, r0);
-        tmem_ld_wait<HH>(base + S::NO, r1);
-#pragma unroll
-        for (int i = 0; i < HH; ++i) d[i] = __uint_as_float(r0[i]) + __uint_as_float(r1[i]);
-      } else {
-        uint32_t r0[HH];
-        tmem_ld_wait<HH>(base, r0);
-#pragma unroll
-        for (int i = 0; i < HH; ++i) d[i] = __uint_as_float(r0[i]);
-      }
-    };
-    // a segment that ended at tile tp: its PV output (plus the group's value
-    // zero-point term) and its running max and sum into partial slot `slot`
-    auto readout = [&](int tp, int os, int slot) {
-      ok &= ws_wait(PVDONE(tp & 1), (tp >> 1) & 1, err);
-      tc_fence_after();
-      float d[HH];
-      load_out(os, d);
-      tc_fence_before();
-      const float nan = __int_as_float(0x7fc00000);
-      const bool good = ok && !*err;
-      const float* pd = pend + (os * S::TPT + part) * 6 * HH;
+    // add the PV sums of tile tp (buffer tp % DB) times its scale into acc:
+    // the sums of the low, middle and high bytes of P' (each exact in fp32)
+    auto read_pv = [&](int tp, const float (&ds)[HH]) {
+      const uint32_t base = tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * HH;
+      uint32_t lo[HH], mi[HH], hi[HH];
+      tmem_ld_wait<HH>(base, lo);
+      tmem_ld_wait<HH>(base + S::PH, mi);
+      tmem_ld_wait<HH>(base + 2 * S::PH, hi);
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        const size_t row = (size_t)slot * G + part * HH + i;
-        a.part_acc[row * kHeadDim + j] = good ? d[i] + pd[(2 + wq) * HH + i] : nan;
-        if (j == 0) a.part_ml[row] = good ? make_float2(pd[i], pd[HH + i]) : make_float2(nan, nan);
-      }
-    };
-
-    // Read out the pending segments whose last PV tile is at least two tiles
-    // before tile u.  A set is next written by the group's first tile of the
-    // segment after next, at or after u, whose PV follows this tile's P'.
-    auto drain = [&](int u) {
-      while (pn > 0 && u >= p0_tile + 2) {
-        readout(p0_tile, p0_set, p0_slot);
-        p0_tile = p1_tile;
-        p0_set = p1_set;
-        p0_slot = p1_slot;
-        --pn;
+        const float v = fmaf((float)(int)hi[i], 65536.0f, fmaf((float)(int)mi[i], 256.0f, (float)(int)lo[i]));
+        acc[i] = fmaf(v, ds[i], acc[i]);
       }
     };
 
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int k = t & 1;
-      const bool own = S::NGRP == 1 || k == grp;
       if (it.first) {
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           m_run[i] = NEG_INF;
           l_acc[i] = 0.0f;
+          acc[i] = 0.0f;
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) zacc[g][i] = 0.0f;
         }
-        seg_tiles = 0;
+        have1 = have2 = false;
         qb = nseg & 1;  // this segment's query data
         ok &= ws_wait(QREADY(qb), (nseg >> 1) & 1, err);
         ++nseg;
@@ -674,8 +596,6 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           qdr[i] = qds[hh];
         }
       }
-      if (own) {
-      drain(t);
       // tokens past the end, and the bf16 window tokens (scored by k_window), take no part
       const int tok = it.i * kTile + j;  // token position in the sequence
       const bool valid = tok < it.len && !in_window(c.sink, c.recent, tok, it.len);
@@ -702,10 +622,6 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         for (int g = 0; g < kGroups; ++g) ksz[g] = vsz[g] = make_float2(0.0f, 0.0f);
         k0v = 0.0f;
       }
-      // the value operand holds c - L/2, so the zero point carries the L/2 steps
-      constexpr float kHalfL = ((1 << VB) - 1) * 0.5f;
-#pragma unroll
-      for (int g = 0; g < kGroups; ++g) vsz[g].y = fmaf(kHalfL, vsz[g].x, vsz[g].y);
 
       ok &= ws_wait(SDONE(t % S::SB), (t / S::SB) & 1, err);
       tc_fence_after();
@@ -748,166 +664,171 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             dot = fmaf(ksz[g].x, (float)dg, dot);
             zt = fmaf(ksz[g].y, qg[g], zt);
           }
-          sc[i] = fmaf(dot, qd, zt);
+          sc[i] = valid ? fmaf(dot, qd, zt) * a.scale_log2 : NEG_INF;
         }
       }
       tc_fence_before();
       if (it.last) mbar_arrive(QFREE(qb));  // done with this segment's query data and score UMMAs
-      // lazy running max: raise it (part-wide) only if some score exceeds it by 2^kLazyMax
-      bool exceed = false;
+
+      // The tile's largest score per head and largest value scale per group
+      // (warp maxima, then the part's four warps through shared memory).
+      int* rk = rmax + (k * S::TPT + part) * 64;
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        sc[i] = valid ? sc[i] * a.scale_log2 : NEG_INF;
-        exceed |= sc[i] > m_run[i] + kLazyMax;
+        const int m = __reduce_max_sync(kFull, ord_of(sc[i]));
+        if (lane == 0) rk[wq * 16 + i] = m;
       }
-      float* rt = red + (k * S::TPT + part) * 64;
-      const bool raise = named_sync_or(bar_id, 128, exceed);
-      if (raise) {  // uniform across the part
-        float alpha[HH];
-        float m_new[HH];
 #pragma unroll
-        for (int i = 0; i < HH; ++i) {
-          const float mx = warp_max(sc[i]);
-          if (lane == 0) rt[wq * 16 + i] = mx;
-        }
-        named_sync(bar_id, 128);
+      for (int g = 0; g < kGroups; ++g) {  // scales are >= 0: their bits order like the values
+        const unsigned m = __reduce_max_sync(kFull, __float_as_uint(vsz[g].x));
+        if (lane == 0) rk[wq * 16 + HH + g] = (int)m;
+      }
+      named_sync(bar_id, 128);
+      float smax[HH], vmax[kGroups];
 #pragma unroll
-        for (int i = 0; i < HH; ++i) {
-          m_new[i] = fmaxf(m_run[i], fmaxf(fmaxf(rt[i], rt[16 + i]), fmaxf(rt[32 + i], rt[48 + i])));
-          alpha[i] = exp2f(m_run[i] - m_new[i]);
-          m_run[i] = m_new[i];
-          l_acc[i] *= alpha[i];
+      for (int i = 0; i < HH; ++i)
+        smax[i] = float_of_ord(max(max(rk[i], rk[16 + i]), max(rk[32 + i], rk[48 + i])));
 #pragma unroll
-          for (int g = 0; g < kGroups; ++g) zacc[g][i] *= alpha[i];
-        }
-        if (seg_tiles > 0) {
-          // rescale the group's PV sums of the segment so far (this thread: channel
-          // j, its heads) once the PV of its previous tile has landed; tile t's PV
-          // adds after PREADY below
-          ok &= ws_wait(PVDONE(last_own & 1), (last_own >> 1) & 1, err);
+      for (int g = 0; g < kGroups; ++g)
+        vmax[g] = __uint_as_float((unsigned)max(max(rk[HH + g], rk[16 + HH + g]), max(rk[32 + HH + g], rk[48 + HH + g])));
+
+      // P' buffer k was read by the PV UMMAs of tile t - 2; the sums of tile
+      // t - RD (of this segment) are read back now, before the running max can
+      // move (the UMMAs of one thread complete in order, so PV t - 1 done
+      // implies PV t - 2 done)
+      if (t >= RD) {
+        ok &= ws_wait(PVDONE((t - RD) & 1), ((t - RD) >> 1) & 1, err);
+        if (RD == 2 ? have2 : have1) {
           tc_fence_after();
-          const uint32_t base = obase(qb);
-#pragma unroll
-          for (int pp = 0; pp < PP; ++pp) {
-            uint32_t r[HH];
-            tmem_ld_wait<HH>(base + pp * S::NO, r);
-#pragma unroll
-            for (int i = 0; i < HH; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha[i]);
-            tmem_st_n<HH>(base + pp * S::NO, r);
-          }
-          tmem_wait_st();
+          read_pv(t - RD, RD == 2 ? ds2 : ds1);
           tc_fence_before();
         }
       }
-      float p[HH];
+      // lazy running max: raised (uniformly across the part) only when the
+      // tile's maximum exceeds it by 2^kLazyMax
+      bool raise = false;
 #pragma unroll
-      for (int i = 0; i < HH; ++i) {
-        p[i] = valid ? exp2f(sc[i] - m_run[i]) : 0.0f;
-        l_acc[i] += p[i];
+      for (int i = 0; i < HH; ++i) raise |= smax[i] > m_run[i] + kLazyMax;
+      if (raise) {
 #pragma unroll
-        for (int g = 0; g < kGroups; ++g) zacc[g][i] = fmaf(p[i], vsz[g].y, zacc[g][i]);
-      }
-      // P' = p * value scale into the MN-major operand: column (group g, head),
-      // K position pos.  This buffer was last read by the PV UMMAs of tile t-2.
-      if (t >= 2) ok &= ws_wait(PVDONE(k), ((t - 2) >> 1) & 1, err);
-      uint8_t* BP = fix + S::F_BP + k * S::BP_BYTES;
-      if constexpr (G == 1) {
-        // one head: columns 0..3 = groups 0..3, one 8-byte store
-        const __half2 a01 = __floats2half2_rn(p[0] * vsz[0].x, p[0] * vsz[1].x);
-        const __half2 a23 = __floats2half2_rn(p[0] * vsz[2].x, p[0] * vsz[3].x);
-        *reinterpret_cast<uint2*>(BP + mnmajor(0, pos)) =
-            make_uint2(*reinterpret_cast<const uint32_t*>(&a01), *reinterpret_cast<const uint32_t*>(&a23));
-      } else if constexpr (S::TPT == 1) {
-        // columns g*G + i, 0 .. 4G-1, contiguous: 8 per 16-byte store
-        uint32_t pk[2 * G];
+        for (int i = 0; i < HH; ++i) {
+          const float m_new = fmaxf(m_run[i], smax[i]);
+          const float alpha = exp2f(m_run[i] - m_new);
+          m_run[i] = m_new;
+          l_acc[i] *= alpha;
+          acc[i] *= alpha;
+          ds1[i] *= alpha;
 #pragma unroll
-        for (int g = 0; g < kGroups; ++g)
-#pragma unroll
-          for (int i = 0; i < HH; i += 2) {
-            const __half2 h2 = __floats2half2_rn(p[i] * vsz[g].x, p[i + 1] * vsz[g].x);
-            pk[(g * HH + i) / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-#pragma unroll
-        for (int n = 0; n < 4 * G; n += 8)
-          *reinterpret_cast<uint4*>(BP + mnmajor(n, pos)) =
-              make_uint4(pk[n / 2], pk[n / 2 + 1], pk[n / 2 + 2], pk[n / 2 + 3]);
-      } else {
-        // HH consecutive columns g*G + part*HH .. per group
-#pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          uint32_t pk[HH / 2];
-#pragma unroll
-          for (int i = 0; i < HH; i += 2) {
-            const __half2 h2 = __floats2half2_rn(p[i] * vsz[g].x, p[i + 1] * vsz[g].x);
-            pk[i / 2] = *reinterpret_cast<const uint32_t*>(&h2);
-          }
-          uint8_t* dst = BP + mnmajor(g * G + part * HH, pos);
-          if constexpr (HH == 2) *reinterpret_cast<uint32_t*>(dst) = pk[0];
-          if constexpr (HH == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
-          if constexpr (HH == 8) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          for (int g = 0; g < kGroups; ++g) zacc[g][i] *= alpha;
         }
       }
+      // p = 2^(s - m_run) = pn * pmax with pn = 2^(s - smax) in [0, 1];
+      // P' = pn * scale * ((2^23 - 1) / vmax) rounded to an integer in
+      // [0, 2^23 - 1] (the fma with 2^23 rounds it into the low 23 bits of the float)
+      float pmax[HH], kv[kGroups];
+#pragma unroll
+      for (int i = 0; i < HH; ++i) pmax[i] = smax[i] == NEG_INF ? 0.0f : exp2f(smax[i] - m_run[i]);
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) kv[g] = vmax[g] > 0.0f ? __fdividef(kPSteps, vmax[g]) : 0.0f;
+      uint32_t xb[kGroups * HH];  // column order: group, then head
+#pragma unroll
+      for (int i = 0; i < HH; ++i) {
+        const float pn = valid ? exp2f(sc[i] - smax[i]) : 0.0f;
+        const float p = pn * pmax[i];
+        l_acc[i] += p;
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) {
+          zacc[g][i] = fmaf(p, vsz[g].y, zacc[g][i]);
+          xb[g * HH + i] = __float_as_uint(fmaf(pn, vsz[g].x * kv[g], 8388608.0f));
+        }
+      }
+      // the tile's PV sums (read back RD tiles later) carry pmax * vmax / (2^23 - 1)
+      // for channel j's group
+      float ds0[HH];
+#pragma unroll
+      for (int i = 0; i < HH; ++i) ds0[i] = pmax[i] * (vmax[wq] * (1.0f / kPSteps));
+      // low, middle and high bytes of four consecutive columns per 32-bit word
+      uint32_t by[3][NC / 4];
+#pragma unroll
+      for (int w = 0; w < NC / 4; ++w) {
+        const uint32_t t01 = __byte_perm(xb[4 * w], xb[4 * w + 1], 0x5140);      // x0.b0 x1.b0 x0.b1 x1.b1
+        const uint32_t t23 = __byte_perm(xb[4 * w + 2], xb[4 * w + 3], 0x5140);
+        const uint32_t u01 = __byte_perm(xb[4 * w], xb[4 * w + 1], 0x0062);      // x0.b2 x1.b2
+        const uint32_t u23 = __byte_perm(xb[4 * w + 2], xb[4 * w + 3], 0x0062);
+        by[0][w] = __byte_perm(t01, t23, 0x5410);
+        by[1][w] = __byte_perm(t01, t23, 0x7632);
+        by[2][w] = __byte_perm(u01, u23, 0x5410);
+      }
+      uint8_t* BP = fix + S::F_BP + k * S::BP_BYTES;
+#pragma unroll
+      for (int b = 0; b < 3; ++b)
+#pragma unroll
+        for (int w = 0; w < NC / 4; w += (NC >= 16 ? 4 : 1)) {
+          uint8_t* dst = BP + mnmajor8(b * S::PH + n0 + 4 * w, pos);
+          if constexpr (NC >= 16)
+            *reinterpret_cast<uint4*>(dst) = make_uint4(by[b][w], by[b][w + 1], by[b][w + 2], by[b][w + 3]);
+          else
+            *reinterpret_cast<uint32_t*>(dst) = by[b][w];
+        }
       fence_proxy_async();
       mbar_arrive(PREADY(k));
-      ++seg_tiles;
-      last_own = t;
-      } else if (it.last) {
-        mbar_arrive(QFREE(qb));  // done with this segment's query data
-      }
-
-      if (it.last && seg_tiles == 0) {
-        // no tile of this segment fell to this group: an empty partial (the combine skips it)
-        const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
-        if (j == 0)
 #pragma unroll
-          for (int i = 0; i < HH; ++i) a.part_ml[(size_t)slot * G + part * HH + i] = make_float2(NEG_INF, 0.0f);
-      } else if (it.last) {
-        // segment totals over this part's 128 tokens (max, sum, value zero-point terms),
-        // parked in shared memory until the segment's output is read out
-        float* r2 = red2 + part * 64;
-        float* pd = pend + (qb * S::TPT + part) * 6 * HH;
+      for (int i = 0; i < HH; ++i) {
+        ds2[i] = ds1[i];
+        ds1[i] = ds0[i];
+      }
+      have2 = RD == 2 && have1;
+      have1 = true;
+
+      if (it.last) {
+        // the segment's last two tiles' PV sums, then its totals over the
+        // tokens (max, sum, value zero-point terms) into partial slot u + CTA
+        if (RD == 2 && have2) {
+          ok &= ws_wait(PVDONE((t - 1) & 1), ((t - 1) >> 1) & 1, err);
+          tc_fence_after();
+          read_pv(t - 1, ds2);
+        }
+        ok &= ws_wait(PVDONE(k), (t >> 1) & 1, err);
+        tc_fence_after();
+        read_pv(t, ds1);
+        tc_fence_before();
+        have1 = have2 = false;
+        const int slot = (int)it.bh(a) + blockIdx.x;
+        const float nan = __int_as_float(0x7fc00000);
+        const bool good = ok && !*err;
+        float lsum[HH];
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           const float sm = warp_sum(l_acc[i]);
-          if (lane == 0) r2[wq * 16 + i] = sm;
+          if (lane == 0) red2[wq * 16 + i] = sm;
         }
         named_sync(bar_id, 128);
-        if (j == 0) {
 #pragma unroll
-          for (int i = 0; i < HH; ++i) {
-            pd[i] = m_run[i];
-            pd[HH + i] = r2[i] + r2[16 + i] + r2[32 + i] + r2[48 + i];
-          }
-        }
+        for (int i = 0; i < HH; ++i) lsum[i] = red2[i] + red2[16 + i] + red2[32 + i] + red2[48 + i];
+        float zown[HH];  // sum over the tokens of p * zero of channel j's group
 #pragma unroll
         for (int g = 0; g < kGroups; ++g) {
           named_sync(bar_id, 128);
 #pragma unroll
           for (int i = 0; i < HH; ++i) {
             const float sm = warp_sum(zacc[g][i]);
-            if (lane == 0) r2[wq * 16 + i] = sm;
+            if (lane == 0) red2[wq * 16 + i] = sm;
           }
           named_sync(bar_id, 128);
-          if (j == 0) {
+          if (g == wq) {
 #pragma unroll
-            for (int i = 0; i < HH; ++i) pd[(2 + g) * HH + i] = r2[i] + r2[16 + i] + r2[32 + i] + r2[48 + i];
+            for (int i = 0; i < HH; ++i) zown[i] = red2[i] + red2[16 + i] + red2[32 + i] + red2[48 + i];
           }
         }
         named_sync(bar_id, 128);
-        const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
-        if (pn == 0) {
-          p0_tile = last_own;
-          p0_set = qb;
-          p0_slot = slot;
-        } else {
-          p1_tile = last_own;
-          p1_set = qb;
-          p1_slot = slot;
+#pragma unroll
+        for (int i = 0; i < HH; ++i) {
+          const size_t row = (size_t)slot * G + part * HH + i;
+          a.part_acc[row * kHeadDim + j] = good ? acc[i] + zown[i] : nan;
+          if (j == 0) a.part_ml[row] = good ? make_float2(m_run[i], lsum[i]) : make_float2(nan, nan);
         }
-        ++pn;
       }
     }
-    drain(ntiles + 2);
   }
   tc_fence_before();
   __syncthreads();

@@ -141,6 +141,16 @@ __host__ __device__ constexpr uint32_t idesc_u8s8_s32(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor for kind::i8: unsigned 8-bit A (K-major) and B
+// (MN-major), s32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_u8u8_s32_bmn(int M, int N) {
+  return (2u << 4)                        // D format: s32
+         | (0u << 7) | (0u << 10)         // A, B: unsigned 8-bit
+         | (1u << 16)                     // B stored MN-major
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T on 8-bit integers (K = 32 per instruction), issued by one thread.
 __device__ __forceinline__ void umma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                                uint32_t accumulate) {

@@ -80,7 +80,7 @@ cudaError_t launch_bucket_queries(const void* q, int dtype, int rotate, const fl
 // One softmax over every bucket: merges the split decode's partials of the
 // nb bucket units of each sequence (v: the decode's arguments over the
 // bucket batch) into out [B][Hq][128], rotated back when v.c.rotate_v.
-cudaError_t launch_bucket_merge(const DecodeArgs& v, int nb, int ctas, float* out, cudaStream_t s);
+cudaError_t launch_bucket_merge(const DecodeArgs& v, int nb, int ctas, int ngrp, float* out, cudaStream_t s);
 // out[b][j] = tq[j / G] q[b][j] as fp32 rows, G = Hq / H, for the decode.
 cudaError_t launch_transform_q(const void* q, int dtype, const float* tq, int B, int Hq, int H, float* out,
                                cudaStream_t s);
