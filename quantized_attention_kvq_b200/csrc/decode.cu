@@ -60,16 +60,23 @@ constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr float kQSteps = 16000.0f;  // |q| / delta <= 16000: pieces q1 in [-125, 125], q2 in [-64, 63]
 constexpr float kPSteps = 8388607.0f;  // P' integer range: 2^23 - 1, three u8 bytes
+constexpr int kProducers = 2;
 
 template <int G, int KB, int VB, bool CH0>
 struct Shape {
   static constexpr int TPT = G > 4 ? 2 : 1;  // epilogue threads per token (head parts)
+  // epilogue groups: group g takes the tiles t with t % NGRP == g, so two
+  // tiles' chains of waits and latencies overlap (as many as 16 warps allow)
+  static constexpr int NGRP = TPT == 1 ? 2 : 1;
   static constexpr int HH = G / TPT;         // heads per epilogue thread: 1, 2, 4 or 8
-  static constexpr int EPI_WARPS = 4 * TPT;
+  static constexpr int EPI_WARPS = 4 * TPT * NGRP;
   static constexpr int EPI_THREADS = 32 * EPI_WARPS;
-  static constexpr int MMA_WARP = 8 + EPI_WARPS;
+  static constexpr int MMA_WARP = 4 + EPI_WARPS;
+  // ring fillers: producer p issues the copies of the tiles t with t % NPROD == p
+  // (a pruned tile takes one copy per run of kept channel groups)
+  static constexpr int NPROD = kProducers;
   static constexpr int PROD_WARP = MMA_WARP + 1;
-  static constexpr int THREADS = 32 * (PROD_WARP + 1);
+  static constexpr int THREADS = 32 * (PROD_WARP + NPROD);
   static constexpr int NS = 2 * G < 16 ? 16 : 2 * G;  // score columns per group: q1 rows, then q2 rows
   static constexpr int PH = 4 * G;  // P' columns per byte: (value group, head)
   // PV columns: low, middle, high bytes, padded to a power of two (>= 16)
@@ -109,9 +116,9 @@ struct Shape {
   static constexpr int F_QS = F_BP + 2 * BP_BYTES;   // [2][G][4] f32: per-group sums of the kept q
   static constexpr int F_Q0 = F_QS + 2 * G * 16;     // [2][G] f32: q_0 (channel 0 kept in bf16)
   static constexpr int F_QD = F_Q0 + 2 * QV;         // [2][G] f32: delta of the query pieces
-  static constexpr int F_RED = F_QD + 2 * QV;        // [2 tiles][TPT][4 warps][16] s32: warp maxima
-  static constexpr int F_RED2 = F_RED + 2 * TPT * 4 * 16 * 4;  // [TPT][4 warps][16] f32: segment sums
-  static constexpr int F_BAR = (F_RED2 + TPT * 4 * 16 * 4 + 15) / 16 * 16;
+  static constexpr int F_RED = F_QD + 2 * QV;  // [2 own tiles][NGRP][TPT][4 warps][16] s32: warp maxima
+  static constexpr int F_RED2 = F_RED + 2 * NGRP * TPT * 4 * 16 * 4;  // [NGRP][TPT][4 warps][16] f32: segment sums
+  static constexpr int F_BAR = (F_RED2 + NGRP * TPT * 4 * 16 * 4 + 15) / 16 * 16;
   // kready[3] vready[2] pready[2] sdone[3] pvdone[2] qready[2] qfree[2]
   static constexpr int NBAR_FIXED = 16;
   static constexpr int F_REST_NO_RING = F_BAR + NBAR_FIXED * 8 + 16;  // + tmem slot, error flag
@@ -274,13 +281,13 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(FULL(s), 1);
-      mbar_init(EMPTY(s), 256 + S::EPI_THREADS);  // key, value and epilogue threads
+      mbar_init(EMPTY(s), 128 + S::EPI_THREADS / S::NGRP);  // code conversion and the tile's epilogue group
     }
     for (int k = 0; k < S::NKR; ++k) mbar_init(KREADY(k), 128);
     for (int k = 0; k < S::SB; ++k) mbar_init(SDONE(k), 1);
     for (int k = 0; k < 2; ++k) {
       mbar_init(VREADY(k), 128);
-      mbar_init(PREADY(k), S::EPI_THREADS);
+      mbar_init(PREADY(k), S::EPI_THREADS / S::NGRP);
       mbar_init(PVDONE(k), 1);
       mbar_init(QREADY(k), 128);
       mbar_init(QFREE(k), S::EPI_THREADS);
@@ -304,10 +311,12 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   TileIter it;
   it.init(a, g0, g1);
 
-  if (warp == S::PROD_WARP) {
-    // ================================================================ producer
+  if (warp >= S::PROD_WARP) {
+    // ================================================================ producers
     const int nblk = c.cap / kTile;
+    const int pw = warp - S::PROD_WARP;
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
+      if (t % S::NPROD != pw) continue;
       const int s = t % ST;
       if (t >= ST) ws_wait(EMPTY(s), ((t / ST) - 1) & 1, err);
       const size_t bh = it.bh(a);
@@ -379,9 +388,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       __syncwarp();
     }
   } else if (warp < 4) {
-    // ================================================================ key codes -> tensor memory
-    const int j = tid;  // token of the tile == tensor-memory lane
+    // ================================================================ codes -> tensor memory
+    // Per tile, first the key codes (thread = token), then the value codes
+    // (thread = channel); both land in this warp's lane quarter.
+    const int j = tid;  // token of the tile == tensor-memory lane; then channel
     const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+    // the 16-byte chunks of a channel's value row are stored rotated by
+    // channel, so the rows of 8 consecutive channels hit 8 different bank groups
+    const int swz = VB == 4 ? (j >> 1) & 3 : (j >> 2) & 1;
     int kseg = 0;  // segments begun so far
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int s = t % ST;
@@ -470,23 +484,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       fence_proxy_async();  // query operand (generic writes) -> tensor core
       tc_fence_before();
       mbar_arrive(KREADY(t % S::NKR));
-      mbar_arrive(EMPTY(s));
-    }
-  } else if (warp < 8) {
-    // ================================================================ value codes -> tensor memory
-    const int ch = tid - 128;  // channel == tensor-memory lane
-    const uint32_t tl = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
-    // the 16-byte chunks of a channel's row are stored rotated by channel, so
-    // the rows of 8 consecutive channels hit 8 different bank groups
-    const int swz = VB == 4 ? (ch >> 1) & 3 : (ch >> 2) & 1;
-    for (int t = 0; t < ntiles; ++t) {
-      const int s = t % ST;
-      const uint8_t* row = smem + s * S::STAGE + S::R_VC + ch * S::VROW;
-      ws_wait(FULL(s), (t / ST) & 1, err);
-      // this value stage was read by the PV UMMAs of tile t - VST
+
+      // value codes of channel j: this value stage was read by the PV UMMAs of tile t - VST
       if (t >= S::VST) ws_wait(PVDONE((t - S::VST) & 1), ((t - S::VST) >> 1) & 1, err);
       tc_fence_after();
-      uint32_t r[32];  // 128 u8 codes in the order vpos_of gives
+      const uint8_t* row = smem + s * S::STAGE + S::R_VC + j * S::VROW;
       if (VB == 4) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {  // 16-byte chunk k: tokens 32k .. 32k+31, 8 per word
@@ -509,25 +511,29 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             for (int m = 0; m < 4; ++m) r[16 * k + 4 * i + m] = (ws[i] >> (2 * m)) & 0x03030303u;
         }
       }
-      const uint32_t col = tl + S::TM_AV + (t % S::VST) * 32;
-      tmem_st16(col, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
-      tmem_st16(col + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
+      const uint32_t vcol = tl + S::TM_AV + (t % S::VST) * 32;  // 128 u8 codes in the order vpos_of gives
+      tmem_st16(vcol, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
+      tmem_st16(vcol + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(VREADY(t & 1));
       mbar_arrive(EMPTY(s));
     }
-  } else if (warp < 8 + S::EPI_WARPS) {
+  } else if (warp < 4 + S::EPI_WARPS) {
     // ================================================================ epilogue
-    const int e = tid - 256;             // 0 .. EPI_THREADS-1
+    // With NGRP epilogue groups, group g takes the tiles t with t % NGRP == g;
+    // each keeps its own online softmax and accumulators per segment and
+    // leaves its own partial, which the combine merges like any other split.
+    const int e = tid - 128;             // 0 .. EPI_THREADS-1
+    const int grp = e / (128 * S::TPT);  // epilogue group
     const int j = e & 127;               // token (score phase) == tensor-memory lane == channel (PV phase)
-    const int part = e >> 7;             // head part: heads part*HH .. part*HH + HH - 1
+    const int part = (e >> 7) % S::TPT;  // head part: heads part*HH .. part*HH + HH - 1
     const int wq = warp & 3;             // lane quarter == value group of channel j
-    const int bar_id = 1 + part;
+    const int bar_id = 1 + grp * S::TPT + part;
     const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
     const int pos = vpos_of<VB>(j);      // K position of token j in the P' operand
     int* rmax = reinterpret_cast<int*>(fix + S::F_RED);                      // [2][TPT][4][16]
-    float* red2 = reinterpret_cast<float*>(fix + S::F_RED2) + part * 64;      // [4][16]
+    float* red2 = reinterpret_cast<float*>(fix + S::F_RED2) + (grp * S::TPT + part) * 64;  // [4][16]
     const float NEG_INF = -__int_as_float(0x7f800000);
     // P' columns of this part: (byte, part, group, head), 4 HH per part and byte
     constexpr int NC = 4 * HH;
@@ -535,11 +541,12 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
     float m_run[HH], l_acc[HH], zacc[kGroups][HH];
     float acc[HH];  // PV sums of channel j for this part's heads, scaled to m_run
-    // PV sums of the last tile (ds1) and, with two PV buffers, the tile before
-    // (ds2) still to be read back, with their scales for channel j's group; a
-    // tile's sums are read back RD tiles later, before the PV MMAs that reuse
-    // its buffer are issued
-    constexpr int RD = S::DB;
+    // PV sums of this group's last tile (ds1) and, when two of its tiles can be
+    // in flight, the one before (ds2) still to be read back, with their scales
+    // for channel j's group; tile t's sums sit in PV buffer t % DB and are read
+    // back at tile t + DB, before the PV MMAs that reuse the buffer are issued
+    constexpr int RD = S::DB;                // in tiles
+    constexpr int PLEN = S::DB / S::NGRP;    // in this group's tiles: 1 or 2
     float ds1[HH] = {}, ds2[HH] = {};
     bool have1 = false, have2 = false;
     // this segment's query data for the thread's heads (per-group sums of the
@@ -547,8 +554,10 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     // thread takes a token's heads, else read from shared memory per tile
     constexpr bool QREG = S::TPT == 1;
     float qsg[QREG ? HH : 1][kGroups], q0r[QREG ? HH : 1], qdr[QREG ? HH : 1];
-    int nseg = 0;  // segments begun so far
-    int qb = 0;    // query buffer of the current segment (its parity)
+    int nseg = 0;       // segments begun so far
+    int qb = 0;         // query buffer of the current segment (its parity)
+    int seg_tiles = 0;  // tiles of the current segment this group has taken
+    int last_own = 0;   // the last tile this group took
     bool ok = true;
 
     // add the PV sums of tile tp (buffer tp % DB) times its scale into acc:
@@ -578,6 +587,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           for (int g = 0; g < kGroups; ++g) zacc[g][i] = 0.0f;
         }
         have1 = have2 = false;
+        seg_tiles = 0;
         qb = nseg & 1;  // this segment's query data
         ok &= ws_wait(QREADY(qb), (nseg >> 1) & 1, err);
         ++nseg;
@@ -596,6 +606,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           qdr[i] = qds[hh];
         }
       }
+      if (t % S::NGRP != grp) {
+        if (it.last) mbar_arrive(QFREE(qb));  // done with this segment's query data
+      } else {
       // tokens past the end, and the bf16 window tokens (scored by k_window), take no part
       const int tok = it.i * kTile + j;  // token position in the sequence
       const bool valid = tok < it.len && !in_window(c.sink, c.recent, tok, it.len);
@@ -672,7 +685,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
       // The tile's largest score per head and largest value scale per group
       // (warp maxima, then the part's four warps through shared memory).
-      int* rk = rmax + (k * S::TPT + part) * 64;
+      int* rk = rmax + ((((t / S::NGRP) & 1) * S::NGRP + grp) * S::TPT + part) * 64;
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
         const int m = __reduce_max_sync(kFull, ord_of(sc[i]));
@@ -698,9 +711,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       // implies PV t - 2 done)
       if (t >= RD) {
         ok &= ws_wait(PVDONE((t - RD) & 1), ((t - RD) >> 1) & 1, err);
-        if (RD == 2 ? have2 : have1) {
+        if (PLEN == 2 ? have2 : have1) {
           tc_fence_after();
-          read_pv(t - RD, RD == 2 ? ds2 : ds1);
+          read_pv(t - RD, PLEN == 2 ? ds2 : ds1);
           tc_fence_before();
         }
       }
@@ -777,23 +790,33 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         ds2[i] = ds1[i];
         ds1[i] = ds0[i];
       }
-      have2 = RD == 2 && have1;
+      have2 = PLEN == 2 && have1;
       have1 = true;
+      ++seg_tiles;
+      last_own = t;
+      }  // own tile
 
-      if (it.last) {
-        // the segment's last two tiles' PV sums, then its totals over the
-        // tokens (max, sum, value zero-point terms) into partial slot u + CTA
-        if (RD == 2 && have2) {
-          ok &= ws_wait(PVDONE((t - 1) & 1), ((t - 1) >> 1) & 1, err);
+      if (it.last && seg_tiles == 0) {
+        // no tile of this segment fell to this group: an empty partial (the combine skips it)
+        const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
+        if (j == 0)
+#pragma unroll
+          for (int i = 0; i < HH; ++i) a.part_ml[(size_t)slot * G + part * HH + i] = make_float2(NEG_INF, 0.0f);
+      } else if (it.last) {
+        // this group's pending PV sums of the segment, then its totals over the
+        // tokens (max, sum, value zero-point terms) into its partial slot
+        const int tl1 = last_own, tl2 = last_own - S::NGRP;  // its last tile, and the one before
+        if (PLEN == 2 && have2) {
+          ok &= ws_wait(PVDONE(tl2 & 1), (tl2 >> 1) & 1, err);
           tc_fence_after();
-          read_pv(t - 1, ds2);
+          read_pv(tl2, ds2);
         }
-        ok &= ws_wait(PVDONE(k), (t >> 1) & 1, err);
+        ok &= ws_wait(PVDONE(tl1 & 1), (tl1 >> 1) & 1, err);
         tc_fence_after();
-        read_pv(t, ds1);
+        read_pv(tl1, ds1);
         tc_fence_before();
         have1 = have2 = false;
-        const int slot = (int)it.bh(a) + blockIdx.x;
+        const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
         const float nan = __int_as_float(0x7fc00000);
         const bool good = ok && !*err;
         float lsum[HH];
@@ -933,7 +956,7 @@ cudaError_t launch_bits(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool decode_g_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
-int decode_groups(int) { return 1; }
+int decode_groups(int G) { return G <= 4 ? 2 : 1; }
 int decode_slots(int B, int H, int G) { return (B * H + kCtas) * decode_groups(G); }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {

@@ -246,11 +246,14 @@ def test_decode_step_host_argument_checks(L):
                                            (16, 8, 2, 12288), (2, 2, 16, 100), (1, 1, 1, 0), (3, 7, 8, 4096)])
 def test_decode_workspace_holds_one_partial_per_slot_and_head(L, B, H, G, max_len):
     # the decode spreads all tiles over 148 persistent CTAs; a (sequence, kv head)
-    # unit leaves at most one partial per CTA its tiles touch, and consecutive
-    # units share at most one CTA, so B*H + 148 slots of G partial rows suffice
+    # unit leaves at most one partial per CTA its tiles touch and per epilogue
+    # group of that CTA (two groups taking alternate tiles when G <= 4, else
+    # one), and consecutive units share at most one CTA, so B*H + 148 slots of
+    # groups * G partial rows suffice
     d = native.describe(B, H, max(128, (max_len + 127) // 128 * 128), 4, 4)
     ws = L.kvq_decode_workspace_bytes(ctypes.byref(d), H * G, max_len)
-    rows = (B * H + 148) * G
+    groups = 2 if G <= 4 else 1
+    rows = (B * H + 148) * groups * G
     assert ws >= rows * (128 * 4 + 8)
     assert ws <= rows * (128 * 4 + 8) + 512  # two 256-byte aligned regions
 
