@@ -532,11 +532,12 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     const int bar_id = 1 + grp * S::TPT + part;
     const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
     const int pos = vpos_of<VB>(j);      // K position of token j in the P' operand
-    int* rmax = reinterpret_cast<int*>(fix + S::F_RED);                      // [2][TPT][4][16]
+    int* rmax = reinterpret_cast<int*>(fix + S::F_RED);  // [2][NGRP][TPT][16][4 warps]
     float* red2 = reinterpret_cast<float*>(fix + S::F_RED2) + (grp * S::TPT + part) * 64;  // [4][16]
     const float NEG_INF = -__int_as_float(0x7f800000);
-    // P' columns of this part: (byte, part, group, head), 4 HH per part and byte
-    constexpr int NC = 4 * HH;
+    // P' columns: (part, group, head, byte), 12 HH per part; the three bytes of
+    // one P' integer sit in adjacent columns
+    constexpr int NC = 12 * HH;
     const int n0 = part * NC;
 
     float m_run[HH], l_acc[HH], zacc[kGroups][HH];
@@ -562,15 +563,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
     // add the PV sums of tile tp (buffer tp % DB) times its scale into acc:
     // the sums of the low, middle and high bytes of P' (each exact in fp32)
+    constexpr int NRD = HH == 1 ? 4 : (HH == 2 ? 8 : (HH == 4 ? 16 : 32));  // >= 3 HH columns per load
     auto read_pv = [&](int tp, const float (&ds)[HH]) {
-      const uint32_t base = tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * HH;
-      uint32_t lo[HH], mi[HH], hi[HH];
-      tmem_ld_wait<HH>(base, lo);
-      tmem_ld_wait<HH>(base + S::PH, mi);
-      tmem_ld_wait<HH>(base + 2 * S::PH, hi);
+      uint32_t r[NRD];  // (head, byte) of channel j's group; the columns past 3 HH are not used
+      tmem_ld_wait<NRD>(tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * 3 * HH, r);
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        const float v = fmaf((float)(int)hi[i], 65536.0f, fmaf((float)(int)mi[i], 256.0f, (float)(int)lo[i]));
+        const float v =
+            fmaf((float)(int)r[3 * i + 2], 65536.0f, fmaf((float)(int)r[3 * i + 1], 256.0f, (float)(int)r[3 * i]));
         acc[i] = fmaf(v, ds[i], acc[i]);
       }
     };
@@ -670,14 +670,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             q0 = CH0 ? q0s[hh] : 0.0f;
             qd = qds[hh];
           }
-          float dot = 0.0f, zt = CH0 ? q0 * k0v : 0.0f;
+          // dot and zero-point sums over the groups as one paired fma each
+          float2 dz = make_float2(0.0f, CH0 ? q0 * k0v : 0.0f);
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) {
             const int dg = (int)d1[g][i] * 128 + (int)d2[g][i];  // exact: |dg| < 2^23
-            dot = fmaf(ksz[g].x, (float)dg, dot);
-            zt = fmaf(ksz[g].y, qg[g], zt);
+            dz = ffma2(ksz[g], make_float2((float)dg, qg[g]), dz);
           }
-          sc[i] = valid ? fmaf(dot, qd, zt) * a.scale_log2 : NEG_INF;
+          sc[i] = valid ? fmaf(dz.x, qd, dz.y) * a.scale_log2 : NEG_INF;
         }
       }
       tc_fence_before();
@@ -689,21 +689,25 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
         const int m = __reduce_max_sync(kFull, ord_of(sc[i]));
-        if (lane == 0) rk[wq * 16 + i] = m;
+        if (lane == 0) rk[4 * i + wq] = m;
       }
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) {  // scales are >= 0: their bits order like the values
         const unsigned m = __reduce_max_sync(kFull, __float_as_uint(vsz[g].x));
-        if (lane == 0) rk[wq * 16 + HH + g] = (int)m;
+        if (lane == 0) rk[4 * (HH + g) + wq] = (int)m;
       }
       named_sync(bar_id, 128);
       float smax[HH], vmax[kGroups];
 #pragma unroll
-      for (int i = 0; i < HH; ++i)
-        smax[i] = float_of_ord(max(max(rk[i], rk[16 + i]), max(rk[32 + i], rk[48 + i])));
+      for (int i = 0; i < HH; ++i) {
+        const int4 w = reinterpret_cast<const int4*>(rk)[i];
+        smax[i] = float_of_ord(max(max(w.x, w.y), max(w.z, w.w)));
+      }
 #pragma unroll
-      for (int g = 0; g < kGroups; ++g)
-        vmax[g] = __uint_as_float((unsigned)max(max(rk[HH + g], rk[16 + HH + g]), max(rk[32 + HH + g], rk[48 + HH + g])));
+      for (int g = 0; g < kGroups; ++g) {
+        const int4 w = reinterpret_cast<const int4*>(rk)[HH + g];
+        vmax[g] = __uint_as_float((unsigned)max(max(w.x, w.y), max(w.z, w.w)));
+      }
 
       // P' buffer k was read by the PV UMMAs of tile t - 2; the sums of tile
       // t - RD (of this segment) are read back now, before the running max can
@@ -743,16 +747,31 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       for (int i = 0; i < HH; ++i) pmax[i] = smax[i] == NEG_INF ? 0.0f : exp2f(smax[i] - m_run[i]);
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) kv[g] = vmax[g] > 0.0f ? __fdividef(kPSteps, vmax[g]) : 0.0f;
-      uint32_t xb[kGroups * HH];  // column order: group, then head
+      float pn[HH], p[HH];
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        const float pn = valid ? exp2f(sc[i] - smax[i]) : 0.0f;
-        const float p = pn * pmax[i];
-        l_acc[i] += p;
+        pn[i] = valid ? exp2f(sc[i] - smax[i]) : 0.0f;
+        p[i] = pn[i] * pmax[i];
+        l_acc[i] += p[i];
+      }
+      uint32_t xb[kGroups * HH + 1];  // column order: group, then head (one spare for odd HH)
 #pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          zacc[g][i] = fmaf(p, vsz[g].y, zacc[g][i]);
-          xb[g * HH + i] = __float_as_uint(fmaf(pn, vsz[g].x * kv[g], 8388608.0f));
+      for (int g = 0; g < kGroups; ++g) {
+        const float vk = vsz[g].x * kv[g];
+        if constexpr (HH == 1) {
+          zacc[g][0] = fmaf(p[0], vsz[g].y, zacc[g][0]);
+          xb[g] = __float_as_uint(fmaf(pn[0], vk, 8388608.0f));
+        } else {
+#pragma unroll
+          for (int i = 0; i < HH; i += 2) {  // heads in pairs: one paired fma per pair
+            const float2 z = ffma2(make_float2(p[i], p[i + 1]), make_float2(vsz[g].y, vsz[g].y),
+                                   make_float2(zacc[g][i], zacc[g][i + 1]));
+            zacc[g][i] = z.x;
+            zacc[g][i + 1] = z.y;
+            const float2 x = ffma2(make_float2(pn[i], pn[i + 1]), make_float2(vk, vk), make_float2(8388608.0f, 8388608.0f));
+            xb[g * HH + i] = __float_as_uint(x.x);
+            xb[g * HH + i + 1] = __float_as_uint(x.y);
+          }
         }
       }
       // the tile's PV sums (read back RD tiles later) carry pmax * vmax / (2^23 - 1)
@@ -760,29 +779,29 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       float ds0[HH];
 #pragma unroll
       for (int i = 0; i < HH; ++i) ds0[i] = pmax[i] * (vmax[wq] * (1.0f / kPSteps));
-      // low, middle and high bytes of four consecutive columns per 32-bit word
-      uint32_t by[3][NC / 4];
+      // the low three bytes of each P' integer, in column order, four per word:
+      // three words per four integers
+      uint32_t by[NC / 4];
 #pragma unroll
-      for (int w = 0; w < NC / 4; ++w) {
-        const uint32_t t01 = __byte_perm(xb[4 * w], xb[4 * w + 1], 0x5140);      // x0.b0 x1.b0 x0.b1 x1.b1
-        const uint32_t t23 = __byte_perm(xb[4 * w + 2], xb[4 * w + 3], 0x5140);
-        const uint32_t u01 = __byte_perm(xb[4 * w], xb[4 * w + 1], 0x0062);      // x0.b2 x1.b2
-        const uint32_t u23 = __byte_perm(xb[4 * w + 2], xb[4 * w + 3], 0x0062);
-        by[0][w] = __byte_perm(t01, t23, 0x5410);
-        by[1][w] = __byte_perm(t01, t23, 0x7632);
-        by[2][w] = __byte_perm(u01, u23, 0x5410);
+      for (int w = 0; w < kGroups * HH / 4; ++w) {
+        by[3 * w] = __byte_perm(xb[4 * w], xb[4 * w + 1], 0x4210);          // x0.b0 x0.b1 x0.b2 x1.b0
+        by[3 * w + 1] = __byte_perm(xb[4 * w + 1], xb[4 * w + 2], 0x5421);  // x1.b1 x1.b2 x2.b0 x2.b1
+        by[3 * w + 2] = __byte_perm(xb[4 * w + 2], xb[4 * w + 3], 0x6542);  // x2.b2 x3.b0 x3.b1 x3.b2
       }
       uint8_t* BP = fix + S::F_BP + k * S::BP_BYTES;
 #pragma unroll
-      for (int b = 0; b < 3; ++b)
-#pragma unroll
-        for (int w = 0; w < NC / 4; w += (NC >= 16 ? 4 : 1)) {
-          uint8_t* dst = BP + mnmajor8(b * S::PH + n0 + 4 * w, pos);
-          if constexpr (NC >= 16)
-            *reinterpret_cast<uint4*>(dst) = make_uint4(by[b][w], by[b][w + 1], by[b][w + 2], by[b][w + 3]);
-          else
-            *reinterpret_cast<uint32_t*>(dst) = by[b][w];
-        }
+      for (int w = 0; w < NC / 4; w += 4) {  // 16 columns (one 16-byte row) at a time, or what is left
+        uint8_t* dst = BP + mnmajor8(n0 + 4 * w, pos);
+        if (NC / 4 - w >= 4)
+          *reinterpret_cast<uint4*>(dst) = make_uint4(by[w], by[w + 1], by[w + 2], by[w + 3]);
+        else if (NC / 4 - w == 3) {
+          *reinterpret_cast<uint2*>(dst) = make_uint2(by[w], by[w + 1]);
+          *reinterpret_cast<uint32_t*>(dst + 8) = by[w + 2];
+        } else if (NC / 4 - w == 2)
+          *reinterpret_cast<uint2*>(dst) = make_uint2(by[w], by[w + 1]);
+        else
+          *reinterpret_cast<uint32_t*>(dst) = by[w];
+      }
       fence_proxy_async();
       mbar_arrive(PREADY(k));
 #pragma unroll
