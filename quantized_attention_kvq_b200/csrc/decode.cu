@@ -24,23 +24,26 @@
 //           with the tile's scale, into fp32 accumulators held in registers.
 //
 // Roles inside a CTA, pipelined over tiles with mbarriers:
-//   producer warp   : 1-D bulk async copies of a tile's kept key-code rows
+//   producer warps (2): 1-D bulk async copies of a tile's kept key-code rows
 //                     (Dual-QK Sec. 3.3: channel-major rows, read selectively),
 //                     value-code rows, key and value scale/zero pairs and
 //                     channel 0 into one stage of a deep shared-memory ring;
-//   key warps (4)   : thread = token: the token's key codes -> u8 -> tensor
+//                     the two take alternate tiles;
+//   code warps (4)  : thread = token: the token's key codes -> u8 -> tensor
 //                     memory (lane = token); at a segment start also the
 //                     query operand (dropped channel groups zeroed), its
-//                     per-head step and its per-group sums;
-//   value warps (4) : thread = channel: the channel's 128 value codes -> u8
-//                     -> tensor memory (lane = channel);
-//   UMMA warp       : the score MMAs one tile ahead, then the PV MMAs;
+//                     per-head step and its per-group sums; then, one tile
+//                     behind, thread = channel: the channel's 128 value codes
+//                     -> u8 -> tensor memory (lane = channel);
+//   score warp      : the score MMAs, as far ahead as the score buffers allow;
+//   PV warp         : the PV MMAs of each tile once its P' is written;
 //   epilogue warps  : thread = (token, heads): score = delta * sum_g s_g S_g +
 //                     sum_g z_g sum(q_g) (+ q_0 k_0), the tile's maxima, the
 //                     online softmax with a lazily raised running max, P' into
 //                     shared memory, the value zero-point terms sum_t p_t z_t;
-//                     thread = (channel, heads): the PV sums of the tile before
-//                     last into the fp32 accumulators.
+//                     thread = (channel, heads): the PV sums of an earlier
+//                     tile into the fp32 accumulators.  Two epilogue groups
+//                     take alternate tiles when the heads fit one thread.
 // Scores come straight from the codes; no dequantized key is ever formed
 // (tq-kv abstract; Dual-QK summary Sec. 3.2, 3.3).  Every mbarrier wait is
 // bounded; after a give-up all waits fall through and the CTA writes NaN
@@ -71,31 +74,37 @@ struct Shape {
   static constexpr int HH = G / TPT;         // heads per epilogue thread: 1, 2, 4 or 8
   static constexpr int EPI_WARPS = 4 * TPT * NGRP;
   static constexpr int EPI_THREADS = 32 * EPI_WARPS;
-  static constexpr int MMA_WARP = 4 + EPI_WARPS;
+  // two UMMA issuers: one thread can only have about one MMA in its issue
+  // stage at a time (some 150 cycles each, whatever the shape), so the score
+  // and the PV MMAs come from two warps and overlap
+  static constexpr int MMA_WARP = 4 + EPI_WARPS;  // score MMAs
+  static constexpr int PV_WARP = MMA_WARP + 1;    // PV MMAs
   // ring fillers: producer p issues the copies of the tiles t with t % NPROD == p
   // (a pruned tile takes one copy per run of kept channel groups)
   static constexpr int NPROD = kProducers;
-  static constexpr int PROD_WARP = MMA_WARP + 1;
+  static constexpr int PROD_WARP = PV_WARP + 1;
   static constexpr int THREADS = 32 * (PROD_WARP + NPROD);
   static constexpr int NS = 2 * G < 16 ? 16 : 2 * G;  // score columns per group: q1 rows, then q2 rows
   static constexpr int PH = 4 * G;  // P' columns per byte: (value group, head)
-  // PV columns: low, middle, high bytes, padded to a power of two (>= 16)
-  static constexpr int NPV = 3 * PH <= 16 ? 16 : (3 * PH <= 32 ? 32 : (3 * PH <= 64 ? 64 : (3 * PH <= 128 ? 128 : 256)));
   static constexpr int KST = G > 8 ? 1 : 2;  // key operand stages in tensor memory
   static constexpr int VST = 2;              // value operand stages in tensor memory
-  static constexpr int SB = G > 8 ? 1 : 2;   // score accumulator buffers
-  static constexpr int LA = SB - 1;          // score MMAs are issued LA tiles ahead of the PV MMAs
+  static constexpr int SB = G > 8 ? 1 : 3;   // score accumulator buffers
   static constexpr int NKR = KST > 1 ? KST : 2;  // key-ready barriers
-  // tensor-memory columns; every accumulator starts at a multiple of its width
-  static constexpr int TM_AK = 0;             // KST key stages x 32 columns (128 u8 codes)
-  static constexpr int TM_AV = 32 * KST;      // VST value stages x 32 columns (128 u8 codes)
-  static constexpr int TM_S = 128;            // SB score buffers x 4 groups x NS
-  static constexpr int TM_D = 256;            // DB PV buffers x NPV
+  // tensor-memory columns
   static constexpr int TMEM_COLS = 512;
+  static constexpr int TM_AK = 0;                 // KST key stages x 32 columns (128 u8 codes)
+  static constexpr int TM_AV = 32 * KST;          // VST value stages x 32 columns (128 u8 codes)
+  static constexpr int TM_S = 128;                // SB score buffers x 4 groups x NS
+  static constexpr int TM_D = TM_S + SB * 4 * NS;  // DB PV buffers x NPV
+  // PV columns: low, middle, high bytes, padded to a power of two (>= 16), or
+  // to a multiple of 32 where two power-of-two buffers do not fit
+  static constexpr int NPV_P2 = 3 * PH <= 16 ? 16 : (3 * PH <= 32 ? 32 : (3 * PH <= 64 ? 64 : (3 * PH <= 128 ? 128 : 256)));
+  static constexpr int NPV_32 = (3 * PH + 31) / 32 * 32;
+  static constexpr int NPV = TM_D + 2 * NPV_P2 <= TMEM_COLS ? NPV_P2 : (TM_D + 2 * NPV_32 <= TMEM_COLS ? NPV_32 : NPV_P2);
   static constexpr int DB = TM_D + 2 * NPV <= TMEM_COLS ? 2 : 1;  // PV buffers: read back 2 or 1 tiles later
-  static_assert(TM_AV + 32 * VST <= TM_S && TM_S + SB * 4 * NS <= TM_D, "operand columns");
+  static_assert(TM_AV + 32 * VST <= TM_S, "operand columns");
   static_assert(TM_D + DB * NPV <= TMEM_COLS, "tensor memory");
-  static_assert(TM_S % NS == 0 && TM_D % NPV == 0, "accumulator alignment");
+  static_assert(TM_S % NS == 0 && TM_D % 16 == 0 && NPV % 16 == 0, "accumulator alignment");
   // one ring stage: key-code rows, value-code rows, key (scale, zero) rows,
   // value (scale, zero) per token, channel 0
   static constexpr int KROW = kTile * (KB == 4 ? 2 : 1);  // bytes of one key row (4 channels)
@@ -119,8 +128,8 @@ struct Shape {
   static constexpr int F_RED = F_QD + 2 * QV;  // [2 own tiles][NGRP][TPT][4 warps][16] s32: warp maxima
   static constexpr int F_RED2 = F_RED + 2 * NGRP * TPT * 4 * 16 * 4;  // [NGRP][TPT][4 warps][16] f32: segment sums
   static constexpr int F_BAR = (F_RED2 + NGRP * TPT * 4 * 16 * 4 + 15) / 16 * 16;
-  // kready[3] vready[2] pready[2] sdone[3] pvdone[2] qready[2] qfree[2]
-  static constexpr int NBAR_FIXED = 16;
+  // kready[3] vready[2] pready[2] sdone[3] pvdone[2] qready[2] qfree[2] sfree[3]
+  static constexpr int NBAR_FIXED = 19;
   static constexpr int F_REST_NO_RING = F_BAR + NBAR_FIXED * 8 + 16;  // + tmem slot, error flag
   static constexpr int STAGES_FIT = (kSmemLimit - F_REST_NO_RING - 2 * kMaxStages * 8) / STAGE;
   static constexpr int STAGES = STAGES_FIT < kMaxStages ? STAGES_FIT : kMaxStages;
@@ -273,6 +282,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   auto PVDONE = [&](int k) { return bar0 + 8 * (10 + k); };  // PV UMMAs of tiles of parity k
   auto QREADY = [&](int k) { return bar0 + 8 * (12 + k); };  // a segment's query data is in buffer k
   auto QFREE = [&](int k) { return bar0 + 8 * (14 + k); };   // the epilogue is done with buffer k
+  auto SFREE = [&](int k) { return bar0 + 8 * (16 + k); };   // the epilogue has read score buffer k
   auto FULL = [&](int s) { return bar0 + 8 * (S::NBAR_FIXED + s); };
   auto EMPTY = [&](int s) { return bar0 + 8 * (S::NBAR_FIXED + ST + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fix + S::F_SLOT);
@@ -284,7 +294,10 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       mbar_init(EMPTY(s), 128 + S::EPI_THREADS / S::NGRP);  // code conversion and the tile's epilogue group
     }
     for (int k = 0; k < S::NKR; ++k) mbar_init(KREADY(k), 128);
-    for (int k = 0; k < S::SB; ++k) mbar_init(SDONE(k), 1);
+    for (int k = 0; k < S::SB; ++k) {
+      mbar_init(SDONE(k), 1);
+      mbar_init(SFREE(k), S::EPI_THREADS / S::NGRP);
+    }
     for (int k = 0; k < 2; ++k) {
       mbar_init(VREADY(k), 128);
       mbar_init(PREADY(k), S::EPI_THREADS / S::NGRP);
@@ -342,15 +355,16 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       if (k0 && lane == 3) bulk_g2s(dst + S::R_K0, c.k0 + bh * c.cap + n0, kTile * 2, FULL(s));
     }
   } else if (warp == S::MMA_WARP) {
-    // ================================================================ UMMA issue
+    // ================================================================ score UMMAs
+    // As far ahead as the SB score buffers allow: buffer t % SB was last read
+    // by the epilogue of tile t - SB, which frees it (SFREE) once its scores are
+    // in registers.
     const uint32_t idesc_s = idesc_u8s8_s32(kTile, S::NS);
-    const uint32_t idesc_o = idesc_u8u8_s32_bmn(kTile, S::NPV);
-    const uint32_t bp = smem_addr(fix + S::F_BP);
     int sseg = -1;  // segment of the tile being scored
-    auto score = [&](int t) {
+    for (int t = 0; t < ntiles; ++t, it.next(a)) {
       if (it.first) ++sseg;
       const uint32_t bq = smem_addr(fix + S::F_BQ + (sseg & 1) * S::BQ_BYTES);
-      it.next(a);
+      if (t >= S::SB) ws_wait(SFREE(t % S::SB), ((t - S::SB) / S::SB) & 1, err);
       ws_wait(KREADY(t % S::NKR), (t / S::NKR) & 1, err);
       tc_fence_after();
       if (lane == 0) {
@@ -363,20 +377,18 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         umma_commit(SDONE(t % S::SB));
       }
       __syncwarp();
-    };
-    // The score MMAs of tile t + LA go ahead of the PV MMAs of tile t, so the
-    // epilogue finds tile t + 1's scores done while it works on tile t.  Score
-    // buffer (t + LA) % SB was last read by the epilogue of tile t + LA - SB
-    // <= t - 1, whose P' (PREADY) was waited for in the previous iteration.
-    for (int u = 0; u < S::LA && u < ntiles; ++u) score(u);
+    }
+  } else if (warp == S::PV_WARP) {
+    // ================================================================ PV UMMAs
+    const uint32_t idesc_o = idesc_u8u8_s32_bmn(kTile, S::NPV);
+    const uint32_t bp = smem_addr(fix + S::F_BP);
     for (int t = 0; t < ntiles; ++t) {
-      if (t + S::LA < ntiles) score(t + S::LA);
       ws_wait(PREADY(t & 1), (t >> 1) & 1, err);
       ws_wait(VREADY(t & 1), (t >> 1) & 1, err);
       tc_fence_after();
       if (lane == 0) {
         // 32 tokens per MMA: u8 value codes (8 tensor-memory columns) x the
-        // tile's P' bytes; each tile's sums start afresh in PV buffer t & 1
+        // tile's P' bytes; each tile's sums start afresh in PV buffer t % DB
         const uint32_t a0 = tmem + S::TM_AV + (t % S::VST) * 32;
         const uint32_t b0 = bp + (t & 1) * S::BP_BYTES;
         const uint32_t d0 = tmem + S::TM_D + (t % S::DB) * S::NPV;
@@ -389,105 +401,115 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     }
   } else if (warp < 4) {
     // ================================================================ codes -> tensor memory
-    // Per tile, first the key codes (thread = token), then the value codes
-    // (thread = channel); both land in this warp's lane quarter.
+    // The key codes (thread = token) run one tile ahead of the value codes
+    // (thread = channel): step t converts the keys of tile t, then the values
+    // of tile t - 1, so the score MMAs of a tile never wait for the value
+    // conversion of the tile before it.  Both land in this warp's lane quarter.
     const int j = tid;  // token of the tile == tensor-memory lane; then channel
     const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
     // the 16-byte chunks of a channel's value row are stored rotated by
     // channel, so the rows of 8 consecutive channels hit 8 different bank groups
     const int swz = VB == 4 ? (j >> 1) & 3 : (j >> 2) & 1;
     int kseg = 0;  // segments begun so far
-    for (int t = 0; t < ntiles; ++t, it.next(a)) {
-      const int s = t % ST;
-      const uint8_t* raw = smem + s * S::STAGE + S::R_KC;
-      ws_wait(FULL(s), (t / ST) & 1, err);
-      // this key stage was read by the score UMMAs of tile t - KST
-      if (t >= S::KST) ws_wait(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err);
-      tc_fence_after();
-      if (it.first) {
-        // query data of segment kseg into buffer kseg & 1: per head, delta =
-        // max|q| / 16000 and q = delta * (128 q1 + q2) exactly, q1 in row h, q2 in
-        // row G + h; dropped channel groups (and channel 0 when it is kept in bf16)
-        // are zero.  The buffer was last used by segment kseg - 2, which the
-        // epilogue (and so its score UMMAs) finished before freeing it.  Each
-        // buffer's two barriers see one phase per use, in order, so no parity wait
-        // can pass on a later or an earlier phase.
-        const int qb = kseg & 1;
-        if (kseg >= 2) ws_wait(QFREE(qb), ((kseg - 2) >> 1) & 1, err);
-        uint8_t* BQ = fix + S::F_BQ + qb * S::BQ_BYTES;
-        float* qsum = reinterpret_cast<float*>(fix + S::F_QS + qb * G * 16);
-        float* q0s = reinterpret_cast<float*>(fix + S::F_Q0 + qb * S::QV);
-        float* qds = reinterpret_cast<float*>(fix + S::F_QD + qb * S::QV);
-        const uint32_t msk = it.msk;
-        for (int hq = warp; hq < G; hq += 4) {
-          const In* qrow = static_cast<const In*>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.h * G + hq) * kHeadDim;
-          float x[4];
-          load_row_warp(qrow, c.rotate != 0, a.inv_sqrt_d, lane, x);
-          const bool sel = (msk >> lane) & 1u;
-          float v[4], part = 0.0f, amax = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            v[i] = sel ? x[i] : 0.0f;
-            if (CH0 && lane == 0 && i == 0) v[i] = 0.0f;
-            part += v[i];
-            amax = fmaxf(amax, fabsf(v[i]));
+    for (int t = 0; t <= ntiles; ++t) {
+      if (t < ntiles) {
+        const int s = t % ST;
+        const uint8_t* raw = smem + s * S::STAGE + S::R_KC;
+        ws_wait(FULL(s), (t / ST) & 1, err);
+        // this key stage was read by the score UMMAs of tile t - KST
+        if (t >= S::KST) ws_wait(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err);
+        tc_fence_after();
+        if (it.first) {
+          // query data of segment kseg into buffer kseg & 1: per head, delta =
+          // max|q| / 16000 and q = delta * (128 q1 + q2) exactly, q1 in row h, q2 in
+          // row G + h; dropped channel groups (and channel 0 when it is kept in bf16)
+          // are zero.  The buffer was last used by segment kseg - 2, which the
+          // epilogue (and so its score UMMAs) finished before freeing it.  Each
+          // buffer's two barriers see one phase per use, in order, so no parity wait
+          // can pass on a later or an earlier phase.
+          const int qb = kseg & 1;
+          if (kseg >= 2) ws_wait(QFREE(qb), ((kseg - 2) >> 1) & 1, err);
+          uint8_t* BQ = fix + S::F_BQ + qb * S::BQ_BYTES;
+          float* qsum = reinterpret_cast<float*>(fix + S::F_QS + qb * G * 16);
+          float* q0s = reinterpret_cast<float*>(fix + S::F_Q0 + qb * S::QV);
+          float* qds = reinterpret_cast<float*>(fix + S::F_QD + qb * S::QV);
+          const uint32_t msk = it.msk;
+          for (int hq = warp; hq < G; hq += 4) {
+            const In* qrow = static_cast<const In*>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.h * G + hq) * kHeadDim;
+            float x[4];
+            load_row_warp(qrow, c.rotate != 0, a.inv_sqrt_d, lane, x);
+            const bool sel = (msk >> lane) & 1u;
+            float v[4], part = 0.0f, amax = 0.0f;
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              v[i] = sel ? x[i] : 0.0f;
+              if (CH0 && lane == 0 && i == 0) v[i] = 0.0f;
+              part += v[i];
+              amax = fmaxf(amax, fabsf(v[i]));
+            }
+            amax = warp_max(amax);
+            const float delta = amax > 0.0f ? amax / kQSteps : 1.0f;
+  #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int ch = 4 * lane + i;
+              const int qi = __float2int_rn(v[i] / delta);  // |qi| <= 16000
+              const int q1 = (qi + 64) >> 7;                // nearest multiple of 128 below qi + 64
+              const int q2 = qi - 128 * q1;                 // in [-64, 63]
+              constexpr int blk = KB == 4 ? 8 : 16;
+              const int p = (ch / blk) * blk + kpos_of<KB>(ch % blk);
+              BQ[kmajor8(hq, p)] = (uint8_t)(int8_t)q1;
+              BQ[kmajor8(G + hq, p)] = (uint8_t)(int8_t)q2;
+            }
+  #pragma unroll
+            for (int m = 1; m < 8; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
+            if ((lane & 7) == 0) qsum[hq * kGroups + (lane >> 3)] = part;
+            if (lane == 0) {
+              q0s[hq] = (CH0 && sel) ? x[0] : 0.0f;
+              qds[hq] = delta;
+            }
           }
-          amax = warp_max(amax);
-          const float delta = amax > 0.0f ? amax / kQSteps : 1.0f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int ch = 4 * lane + i;
-            const int qi = __float2int_rn(v[i] / delta);  // |qi| <= 16000
-            const int q1 = (qi + 64) >> 7;                // nearest multiple of 128 below qi + 64
-            const int q2 = qi - 128 * q1;                 // in [-64, 63]
-            constexpr int blk = KB == 4 ? 8 : 16;
-            const int p = (ch / blk) * blk + kpos_of<KB>(ch % blk);
-            BQ[kmajor8(hq, p)] = (uint8_t)(int8_t)q1;
-            BQ[kmajor8(G + hq, p)] = (uint8_t)(int8_t)q2;
+          mbar_arrive(QREADY(qb));  // release: the epilogue reads the data after waiting on it
+          ++kseg;
+        }
+        // every key row is converted: rows of dropped channel groups hold stale
+        // codes, which meet zeros in the query operand
+        uint32_t r[32];
+        if (KB == 4) {
+          const uint16_t* kc = reinterpret_cast<const uint16_t*>(raw) + j;
+  #pragma unroll
+          for (int q = 0; q < 16; ++q) {  // channels 8q .. 8q+7: even ones, then odd ones
+            const uint32_t x = (uint32_t)kc[(2 * q) * kTile] | ((uint32_t)kc[(2 * q + 1) * kTile] << 16);
+            r[2 * q] = x & 0x0F0F0F0Fu;
+            r[2 * q + 1] = (x >> 4) & 0x0F0F0F0Fu;
           }
-#pragma unroll
-          for (int m = 1; m < 8; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
-          if ((lane & 7) == 0) qsum[hq * kGroups + (lane >> 3)] = part;
-          if (lane == 0) {
-            q0s[hq] = (CH0 && sel) ? x[0] : 0.0f;
-            qds[hq] = delta;
+        } else {
+          const uint8_t* kc = raw + j;
+  #pragma unroll
+          for (int q = 0; q < 8; ++q) {  // channels 16q .. 16q+15: crumb k of every byte together
+            const uint32_t x = (uint32_t)kc[(4 * q) * kTile] | ((uint32_t)kc[(4 * q + 1) * kTile] << 8) |
+                               ((uint32_t)kc[(4 * q + 2) * kTile] << 16) | ((uint32_t)kc[(4 * q + 3) * kTile] << 24);
+  #pragma unroll
+            for (int k = 0; k < 4; ++k) r[4 * q + k] = (x >> (2 * k)) & 0x03030303u;
           }
         }
-        mbar_arrive(QREADY(qb));  // release: the epilogue reads the data after waiting on it
-        ++kseg;
+        const uint32_t col = tl + S::TM_AK + (t % S::KST) * 32;
+        tmem_st16(col, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
+        tmem_st16(col + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
+        tmem_wait_st();
+        fence_proxy_async();  // query operand (generic writes) -> tensor core
+        tc_fence_before();
+        mbar_arrive(KREADY(t % S::NKR));
+        it.next(a);
       }
-      // every key row is converted: rows of dropped channel groups hold stale
-      // codes, which meet zeros in the query operand
-      uint32_t r[32];
-      if (KB == 4) {
-        const uint16_t* kc = reinterpret_cast<const uint16_t*>(raw) + j;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {  // channels 8q .. 8q+7: even ones, then odd ones
-          const uint32_t x = (uint32_t)kc[(2 * q) * kTile] | ((uint32_t)kc[(2 * q + 1) * kTile] << 16);
-          r[2 * q] = x & 0x0F0F0F0Fu;
-          r[2 * q + 1] = (x >> 4) & 0x0F0F0F0Fu;
-        }
-      } else {
-        const uint8_t* kc = raw + j;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {  // channels 16q .. 16q+15: crumb k of every byte together
-          const uint32_t x = (uint32_t)kc[(4 * q) * kTile] | ((uint32_t)kc[(4 * q + 1) * kTile] << 8) |
-                             ((uint32_t)kc[(4 * q + 2) * kTile] << 16) | ((uint32_t)kc[(4 * q + 3) * kTile] << 24);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) r[4 * q + k] = (x >> (2 * k)) & 0x03030303u;
-        }
-      }
-      const uint32_t col = tl + S::TM_AK + (t % S::KST) * 32;
-      tmem_st16(col, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
-      tmem_st16(col + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
-      tmem_wait_st();
-      fence_proxy_async();  // query operand (generic writes) -> tensor core
-      tc_fence_before();
-      mbar_arrive(KREADY(t % S::NKR));
+      if (t == 0) continue;
 
-      // value codes of channel j: this value stage was read by the PV UMMAs of tile t - VST
-      if (t >= S::VST) ws_wait(PVDONE((t - S::VST) & 1), ((t - S::VST) >> 1) & 1, err);
+      // value codes of channel j of tile tv: this value stage was read by the
+      // PV UMMAs of tile tv - VST
+      const int tv = t - 1;
+      const int s = tv % ST;
+      if (tv >= S::VST) ws_wait(PVDONE((tv - S::VST) & 1), ((tv - S::VST) >> 1) & 1, err);
       tc_fence_after();
+      uint32_t r[32];
       const uint8_t* row = smem + s * S::STAGE + S::R_VC + j * S::VROW;
       if (VB == 4) {
 #pragma unroll
@@ -511,12 +533,12 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             for (int m = 0; m < 4; ++m) r[16 * k + 4 * i + m] = (ws[i] >> (2 * m)) & 0x03030303u;
         }
       }
-      const uint32_t vcol = tl + S::TM_AV + (t % S::VST) * 32;  // 128 u8 codes in the order vpos_of gives
+      const uint32_t vcol = tl + S::TM_AV + (tv % S::VST) * 32;  // 128 u8 codes in the order vpos_of gives
       tmem_st16(vcol, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
       tmem_st16(vcol + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(VREADY(t & 1));
+      mbar_arrive(VREADY(tv & 1));
       mbar_arrive(EMPTY(s));
     }
   } else if (warp < 4 + S::EPI_WARPS) {
@@ -563,10 +585,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
     // add the PV sums of tile tp (buffer tp % DB) times its scale into acc:
     // the sums of the low, middle and high bytes of P' (each exact in fp32)
-    constexpr int NRD = HH == 1 ? 4 : (HH == 2 ? 8 : (HH == 4 ? 16 : 32));  // >= 3 HH columns per load
     auto read_pv = [&](int tp, const float (&ds)[HH]) {
-      uint32_t r[NRD];  // (head, byte) of channel j's group; the columns past 3 HH are not used
-      tmem_ld_wait<NRD>(tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * 3 * HH, r);
+      uint32_t r[3 * HH];  // (head, byte) of channel j's group
+      tmem_ld_wait<3 * HH>(tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * 3 * HH, r);
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
         const float v =
@@ -681,6 +702,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         }
       }
       tc_fence_before();
+      mbar_arrive(SFREE(t % S::SB));        // the score buffer may take tile t + SB
       if (it.last) mbar_arrive(QFREE(qb));  // done with this segment's query data and score UMMAs
 
       // The tile's largest score per head and largest value scale per group

@@ -267,6 +267,52 @@ __device__ __forceinline__ void tmem_ld_wait<32>(uint32_t taddr, uint32_t (&r)[3
       : "r"(taddr)
       : "memory");
 }
+// 3, 6, 12 or 24 consecutive columns as two loads (2+1, 4+2, 8+4, 16+8), so
+// that no column past the last one is touched.
+template <>
+__device__ __forceinline__ void tmem_ld_wait<3>(uint32_t taddr, uint32_t (&r)[3]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%3];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%2}, [%4];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2])
+      : "r"(taddr), "r"(taddr + 2)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_wait<6>(uint32_t taddr, uint32_t (&r)[6]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%6];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%4, %5}, [%7];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5])
+      : "r"(taddr), "r"(taddr + 4)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_wait<12>(uint32_t taddr, uint32_t (&r)[12]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%12];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [%13];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11])
+      : "r"(taddr), "r"(taddr + 8)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_wait<24>(uint32_t taddr, uint32_t (&r)[24]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%24];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16, %17, %18, %19, %20, %21, %22, %23}, [%25];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23])
+      : "r"(taddr), "r"(taddr + 16)
+      : "memory");
+}
 // Four runs of N columns at taddr + k * stride (k = 0..3), one wait for all.
 template <int N>
 __device__ __forceinline__ void tmem_ld4_wait(uint32_t taddr, uint32_t stride, uint32_t (&r)[4][N]);
