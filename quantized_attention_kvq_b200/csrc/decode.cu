@@ -16,12 +16,13 @@
 //           (q = delta * (128 q1 + q2)), one s32 accumulator per group, so the
 //           per-token group scale applies exactly afterwards;
 //   PV:     4 of kind::i8 (K = 32 tokens each): value codes as u8 in tensor
-//           memory x P' as three u8 bytes of a 23-bit integer, P' = p * value
-//           scale normalized per tile by the tile's largest p (per head) and
-//           largest value scale (per group) to [0, 2^23 - 1], so the s32 sums
-//           are exact and P' can neither overflow nor lose precision at the
-//           ends of any float range; each tile's sums are read back and added,
-//           with the tile's scale, into fp32 accumulators held in registers.
+//           memory x P' as four u8 bytes of an integer up to 2^31, P' = p *
+//           value scale normalized by running bounds (p relative to a lazily
+//           raised running max, the scale relative to the running maximum
+//           scale of its group), so the s32 sums are exact, P' never
+//           overflows and keeps the 24 significant bits of the float it is
+//           rounded from; each tile's sums are read back and added, with the
+//           tile's scale, into fp32 accumulators held in registers.
 //
 // Roles inside a CTA, pipelined over tiles with mbarriers:
 //   producer warps (2): 1-D bulk async copies of a tile's kept key-code rows
@@ -58,11 +59,13 @@ using namespace sm100;
 
 constexpr int kCtas = 148;  // one persistent CTA per SM
 constexpr int kTile = 128;
-constexpr float kLazyMax = 8.0f;  // the running max is raised only when a score exceeds it by 2^8
+constexpr float kLazyMax = 8.0f;  // the running max is raised only when a score exceeds it by 2^8 (log2 units)
 constexpr int kMaxStages = 12;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr float kQSteps = 16000.0f;  // |q| / delta <= 16000: pieces q1 in [-125, 125], q2 in [-64, 63]
-constexpr float kPSteps = 8388607.0f;  // P' integer range: 2^23 - 1, three u8 bytes
+// P' = p * value scale * 2^23 / vmr with p <= 2^kLazyMax and scale <= vmr, so
+// P' <= 2^31: four u8 bytes, rounded from a float (24 significant bits)
+constexpr float kPUnit = 8388608.0f;  // 2^23
 constexpr int kProducers = 2;
 
 template <int G, int KB, int VB, bool CH0>
@@ -84,11 +87,26 @@ struct Shape {
   static constexpr int NPROD = kProducers;
   static constexpr int PROD_WARP = PV_WARP + 1;
   static constexpr int THREADS = 32 * (PROD_WARP + NPROD);
+  // registers per thread: the block is launched with 65536 / THREADS; the
+  // code warps and the issue/producer warpgroup give some back to the
+  // epilogue warpgroups (the shares add up to at most the launch total)
+  static constexpr int REG_LAUNCH = 65536 / THREADS / 8 * 8;
+  static constexpr int REG_CODE = 80;
+  static constexpr int REG_ISSUE = 56;
+  static constexpr int REG_EPI = (REG_LAUNCH * THREADS - 128 * (REG_CODE + REG_ISSUE)) / EPI_THREADS / 8 * 8 > 248
+                                     ? 248
+                                     : (REG_LAUNCH * THREADS - 128 * (REG_CODE + REG_ISSUE)) / EPI_THREADS / 8 * 8;
+  static_assert(THREADS == 128 + EPI_THREADS + 128, "warpgroups: code, epilogue, issue + producers");
+  static_assert(128 * (REG_CODE + REG_ISSUE) + EPI_THREADS * REG_EPI <= REG_LAUNCH * THREADS, "register split");
+  static_assert(REG_EPI >= REG_LAUNCH, "register split");
   static constexpr int NS = 2 * G < 16 ? 16 : 2 * G;  // score columns per group: q1 rows, then q2 rows
   static constexpr int PH = 4 * G;  // P' columns per byte: (value group, head)
   static constexpr int KST = G > 8 ? 1 : 2;  // key operand stages in tensor memory
   static constexpr int VST = 2;              // value operand stages in tensor memory
-  static constexpr int SB = G > 8 ? 1 : 3;   // score accumulator buffers
+  // PV columns: four bytes x (value group, head)
+  static constexpr int NPV = 4 * PH;
+  // score accumulator buffers: as many (up to 3) as leave room for two PV buffers
+  static constexpr int SB = 128 + 3 * 4 * NS + 2 * NPV <= 512 ? 3 : (128 + 2 * 4 * NS + 2 * NPV <= 512 ? 2 : 1);
   static constexpr int NKR = KST > 1 ? KST : 2;  // key-ready barriers
   // tensor-memory columns
   static constexpr int TMEM_COLS = 512;
@@ -96,15 +114,10 @@ struct Shape {
   static constexpr int TM_AV = 32 * KST;          // VST value stages x 32 columns (128 u8 codes)
   static constexpr int TM_S = 128;                // SB score buffers x 4 groups x NS
   static constexpr int TM_D = TM_S + SB * 4 * NS;  // DB PV buffers x NPV
-  // PV columns: low, middle, high bytes, padded to a power of two (>= 16), or
-  // to a multiple of 32 where two power-of-two buffers do not fit
-  static constexpr int NPV_P2 = 3 * PH <= 16 ? 16 : (3 * PH <= 32 ? 32 : (3 * PH <= 64 ? 64 : (3 * PH <= 128 ? 128 : 256)));
-  static constexpr int NPV_32 = (3 * PH + 31) / 32 * 32;
-  static constexpr int NPV = TM_D + 2 * NPV_P2 <= TMEM_COLS ? NPV_P2 : (TM_D + 2 * NPV_32 <= TMEM_COLS ? NPV_32 : NPV_P2);
   static constexpr int DB = TM_D + 2 * NPV <= TMEM_COLS ? 2 : 1;  // PV buffers: read back 2 or 1 tiles later
   static_assert(TM_AV + 32 * VST <= TM_S, "operand columns");
   static_assert(TM_D + DB * NPV <= TMEM_COLS, "tensor memory");
-  static_assert(TM_S % NS == 0 && TM_D % 16 == 0 && NPV % 16 == 0, "accumulator alignment");
+  static_assert(TM_S % NS == 0 && TM_D % NPV == 0, "accumulator alignment");
   // one ring stage: key-code rows, value-code rows, key (scale, zero) rows,
   // value (scale, zero) per token, channel 0
   static constexpr int KROW = kTile * (KB == 4 ? 2 : 1);  // bytes of one key row (4 channels)
@@ -251,6 +264,19 @@ __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile 
 __device__ __forceinline__ void named_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Named barrier that also returns whether any participating thread passed true.
+__device__ __forceinline__ bool bar_any(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -323,83 +349,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
   TileIter it;
   it.init(a, g0, g1);
-
-  if (warp >= S::PROD_WARP) {
-    // ================================================================ producers
-    const int nblk = c.cap / kTile;
-    const int pw = warp - S::PROD_WARP;
-    for (int t = 0; t < ntiles; ++t, it.next(a)) {
-      if (t % S::NPROD != pw) continue;
-      const int s = t % ST;
-      if (t >= ST) ws_wait(EMPTY(s), ((t / ST) - 1) & 1, err);
-      const size_t bh = it.bh(a);
-      const uint32_t msk = it.msk;
-      const int n0 = it.i * kTile;
-      const size_t blk = bh * nblk + it.i;
-      const uint32_t dst = smem_addr(smem + s * S::STAGE);
-      const bool k0 = CH0 && (msk & 1u);
-      if (lane == 0)
-        mbar_arrive_expect_tx(FULL(s), (uint32_t)(__popc(msk) * S::KROW + kHeadDim * S::VROW + 2 * kGroups * kTile * 4 +
-                                                  (k0 ? kTile * 2 : 0)));
-      __syncwarp();
-      // one copy per run of adjacent kept channel groups (their rows are adjacent in the block)
-      const bool run_start = ((msk >> lane) & 1u) && (lane == 0 || !((msk >> (lane - 1)) & 1u));
-      if (run_start) {
-        const int run = __ffsll((long long)~((unsigned long long)msk >> lane)) - 1;
-        bulk_g2s(dst + S::R_KC + lane * S::KROW, c.kc + key_word_index(bh, c.cap, lane, n0) * (KB == 4 ? 2 : 1),
-                 run * S::KROW, FULL(s));
-      }
-      if (lane == 0) bulk_g2s(dst + S::R_VC, c.vc + blk * kHeadDim * S::VROW, kHeadDim * S::VROW, FULL(s));
-      if (lane == 1) bulk_g2s(dst + S::R_KS, c.ks + key_scale_index(bh, c.cap, 0, n0), kGroups * kTile * 4, FULL(s));
-      if (lane == 2) bulk_g2s(dst + S::R_VS, c.vs + (bh * c.cap + n0) * kGroups, kTile * kGroups * 4, FULL(s));
-      if (k0 && lane == 3) bulk_g2s(dst + S::R_K0, c.k0 + bh * c.cap + n0, kTile * 2, FULL(s));
-    }
-  } else if (warp == S::MMA_WARP) {
-    // ================================================================ score UMMAs
-    // As far ahead as the SB score buffers allow: buffer t % SB was last read
-    // by the epilogue of tile t - SB, which frees it (SFREE) once its scores are
-    // in registers.
-    const uint32_t idesc_s = idesc_u8s8_s32(kTile, S::NS);
-    int sseg = -1;  // segment of the tile being scored
-    for (int t = 0; t < ntiles; ++t, it.next(a)) {
-      if (it.first) ++sseg;
-      const uint32_t bq = smem_addr(fix + S::F_BQ + (sseg & 1) * S::BQ_BYTES);
-      if (t >= S::SB) ws_wait(SFREE(t % S::SB), ((t - S::SB) / S::SB) & 1, err);
-      ws_wait(KREADY(t % S::NKR), (t / S::NKR) & 1, err);
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t a0 = tmem + S::TM_AK + (t % S::KST) * 32;
-        const uint32_t d0 = tmem + S::TM_S + (t % S::SB) * 4 * S::NS;
-        // one MMA per 32-channel group (8 columns of u8 codes, 32 query bytes), all independent
-#pragma unroll
-        for (int g = 0; g < kGroups; ++g)
-          umma_i8_tmem_a(d0 + g * S::NS, a0 + g * 8, smem_desc(bq + g * 256, 128, 1024), idesc_s, 0u);
-        umma_commit(SDONE(t % S::SB));
-      }
-      __syncwarp();
-    }
-  } else if (warp == S::PV_WARP) {
-    // ================================================================ PV UMMAs
-    const uint32_t idesc_o = idesc_u8u8_s32_bmn(kTile, S::NPV);
-    const uint32_t bp = smem_addr(fix + S::F_BP);
-    for (int t = 0; t < ntiles; ++t) {
-      ws_wait(PREADY(t & 1), (t >> 1) & 1, err);
-      ws_wait(VREADY(t & 1), (t >> 1) & 1, err);
-      tc_fence_after();
-      if (lane == 0) {
-        // 32 tokens per MMA: u8 value codes (8 tensor-memory columns) x the
-        // tile's P' bytes; each tile's sums start afresh in PV buffer t % DB
-        const uint32_t a0 = tmem + S::TM_AV + (t % S::VST) * 32;
-        const uint32_t b0 = bp + (t & 1) * S::BP_BYTES;
-        const uint32_t d0 = tmem + S::TM_D + (t % S::DB) * S::NPV;
-#pragma unroll
-        for (int s = 0; s < kTile / 32; ++s)
-          umma_i8_tmem_a(d0, a0 + s * 8, smem_desc(b0 + s * 512, 128, 2048), idesc_o, s > 0 ? 1u : 0u);
-        umma_commit(PVDONE(t & 1));
-      }
-      __syncwarp();
-    }
-  } else if (warp < 4) {
+  // Each warpgroup first sets its register budget (the code warps and the
+  // issue/producer warpgroup give registers back to the epilogue), then
+  // takes its role.
+  if (warp < 4) {
+    setmaxnreg_dec<S::REG_CODE>();
     // ================================================================ codes -> tensor memory
     // The key codes (thread = token) run one tile ahead of the value codes
     // (thread = channel): step t converts the keys of tile t, then the values
@@ -542,6 +496,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       mbar_arrive(EMPTY(s));
     }
   } else if (warp < 4 + S::EPI_WARPS) {
+    setmaxnreg_inc<S::REG_EPI>();
     // ================================================================ epilogue
     // With NGRP epilogue groups, group g takes the tiles t with t % NGRP == g;
     // each keeps its own online softmax and accumulators per segment and
@@ -557,12 +512,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     int* rmax = reinterpret_cast<int*>(fix + S::F_RED);  // [2][NGRP][TPT][16][4 warps]
     float* red2 = reinterpret_cast<float*>(fix + S::F_RED2) + (grp * S::TPT + part) * 64;  // [4][16]
     const float NEG_INF = -__int_as_float(0x7f800000);
-    // P' columns: (part, group, head, byte), 12 HH per part; the three bytes of
-    // one P' integer sit in adjacent columns
-    constexpr int NC = 12 * HH;
+    // P' columns: (part, group, head, byte), 16 HH per part; the four bytes of
+    // one P' integer sit in adjacent columns, so a P' integer is one 32-bit word
+    constexpr int NC = 16 * HH;
     const int n0 = part * NC;
 
     float m_run[HH], l_acc[HH], zacc[kGroups][HH];
+    // running maximum of the value scales per group this segment, and 2^23 / it
+    float vmr[kGroups], kvr[kGroups];
     float acc[HH];  // PV sums of channel j for this part's heads, scaled to m_run
     // PV sums of this group's last tile (ds1) and, when two of its tiles can be
     // in flight, the one before (ds2) still to be read back, with their scales
@@ -584,14 +541,16 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     bool ok = true;
 
     // add the PV sums of tile tp (buffer tp % DB) times its scale into acc:
-    // the sums of the low, middle and high bytes of P' (each exact in fp32)
+    // the sums of the four bytes of P' (each exact in fp32)
     auto read_pv = [&](int tp, const float (&ds)[HH]) {
-      uint32_t r[3 * HH];  // (head, byte) of channel j's group
-      tmem_ld_wait<3 * HH>(tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * 3 * HH, r);
+      uint32_t r[4 * HH];  // (head, byte) of channel j's group
+      tmem_ld_wait<4 * HH>(tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * 4 * HH, r);
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        const float v =
-            fmaf((float)(int)r[3 * i + 2], 65536.0f, fmaf((float)(int)r[3 * i + 1], 256.0f, (float)(int)r[3 * i]));
+        float v = (float)(int)r[4 * i + 3];
+        v = fmaf(v, 256.0f, (float)(int)r[4 * i + 2]);
+        v = fmaf(v, 256.0f, (float)(int)r[4 * i + 1]);
+        v = fmaf(v, 256.0f, (float)(int)r[4 * i]);
         acc[i] = fmaf(v, ds[i], acc[i]);
       }
     };
@@ -607,6 +566,8 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) zacc[g][i] = 0.0f;
         }
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) vmr[g] = kvr[g] = 0.0f;
         have1 = have2 = false;
         seg_tiles = 0;
         qb = nseg & 1;  // this segment's query data
@@ -705,30 +666,47 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       mbar_arrive(SFREE(t % S::SB));        // the score buffer may take tile t + SB
       if (it.last) mbar_arrive(QFREE(qb));  // done with this segment's query data and score UMMAs
 
-      // The tile's largest score per head and largest value scale per group
-      // (warp maxima, then the part's four warps through shared memory).
-      int* rk = rmax + ((((t / S::NGRP) & 1) * S::NGRP + grp) * S::TPT + part) * 64;
+      // P' is normalized by running bounds, not by the tile's own maxima:
+      // scores count from the running max m_run, raised only when a score
+      // passes it by 2^kLazyMax, and value scales from the running maximum vmr
+      // of their group.  One barrier with an OR tells the part whether any of
+      // its tokens passes a bound; only then are the tile's maxima reduced.
+      bool pass = false;
 #pragma unroll
-      for (int i = 0; i < HH; ++i) {
-        const int m = __reduce_max_sync(kFull, ord_of(sc[i]));
-        if (lane == 0) rk[4 * i + wq] = m;
-      }
+      for (int i = 0; i < HH; ++i) pass |= sc[i] > m_run[i] + kLazyMax;
 #pragma unroll
-      for (int g = 0; g < kGroups; ++g) {  // scales are >= 0: their bits order like the values
-        const unsigned m = __reduce_max_sync(kFull, __float_as_uint(vsz[g].x));
-        if (lane == 0) rk[4 * (HH + g) + wq] = (int)m;
-      }
-      named_sync(bar_id, 128);
-      float smax[HH], vmax[kGroups];
+      for (int g = 0; g < kGroups; ++g) pass |= vsz[g].x > vmr[g];
+      const bool raise = bar_any(bar_id, 128, pass);
+      float alpha[HH];
+      if (raise) {
+        // the tile's largest score per head and largest value scale per group
+        // (warp maxima, then the part's four warps through shared memory)
+        int* rk = rmax + ((((t / S::NGRP) & 1) * S::NGRP + grp) * S::TPT + part) * 64;
 #pragma unroll
-      for (int i = 0; i < HH; ++i) {
-        const int4 w = reinterpret_cast<const int4*>(rk)[i];
-        smax[i] = float_of_ord(max(max(w.x, w.y), max(w.z, w.w)));
-      }
+        for (int i = 0; i < HH; ++i) {
+          const int m = __reduce_max_sync(kFull, ord_of(sc[i]));
+          if (lane == 0) rk[4 * i + wq] = m;
+        }
 #pragma unroll
-      for (int g = 0; g < kGroups; ++g) {
-        const int4 w = reinterpret_cast<const int4*>(rk)[HH + g];
-        vmax[g] = __uint_as_float((unsigned)max(max(w.x, w.y), max(w.z, w.w)));
+        for (int g = 0; g < kGroups; ++g) {  // scales are >= 0: their bits order like the values
+          const unsigned m = __reduce_max_sync(kFull, __float_as_uint(vsz[g].x));
+          if (lane == 0) rk[4 * (HH + g) + wq] = (int)m;
+        }
+        named_sync(bar_id, 128);
+#pragma unroll
+        for (int i = 0; i < HH; ++i) {
+          const int4 w = reinterpret_cast<const int4*>(rk)[i];
+          const float smax = float_of_ord(max(max(w.x, w.y), max(w.z, w.w)));
+          const float m_new = fmaxf(m_run[i], smax);
+          alpha[i] = m_new == NEG_INF ? 1.0f : exp2f(m_run[i] - m_new);
+          m_run[i] = m_new;
+        }
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) {
+          const int4 w = reinterpret_cast<const int4*>(rk)[HH + g];
+          vmr[g] = fmaxf(vmr[g], __uint_as_float((unsigned)max(max(w.x, w.y), max(w.z, w.w))));
+          kvr[g] = vmr[g] > 0.0f ? __fdividef(kPUnit, vmr[g]) : 0.0f;
+        }
       }
 
       // P' buffer k was read by the PV UMMAs of tile t - 2; the sums of tile
@@ -743,87 +721,54 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           tc_fence_before();
         }
       }
-      // lazy running max: raised (uniformly across the part) only when the
-      // tile's maximum exceeds it by 2^kLazyMax
-      bool raise = false;
-#pragma unroll
-      for (int i = 0; i < HH; ++i) raise |= smax[i] > m_run[i] + kLazyMax;
       if (raise) {
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
-          const float m_new = fmaxf(m_run[i], smax[i]);
-          const float alpha = exp2f(m_run[i] - m_new);
-          m_run[i] = m_new;
-          l_acc[i] *= alpha;
-          acc[i] *= alpha;
-          ds1[i] *= alpha;
+          l_acc[i] *= alpha[i];
+          acc[i] *= alpha[i];
+          ds1[i] *= alpha[i];
 #pragma unroll
-          for (int g = 0; g < kGroups; ++g) zacc[g][i] *= alpha;
+          for (int g = 0; g < kGroups; ++g) zacc[g][i] *= alpha[i];
         }
       }
-      // p = 2^(s - m_run) = pn * pmax with pn = 2^(s - smax) in [0, 1];
-      // P' = pn * scale * ((2^23 - 1) / vmax) rounded to an integer in
-      // [0, 2^23 - 1] (the fma with 2^23 rounds it into the low 23 bits of the float)
-      float pmax[HH], kv[kGroups];
-#pragma unroll
-      for (int i = 0; i < HH; ++i) pmax[i] = smax[i] == NEG_INF ? 0.0f : exp2f(smax[i] - m_run[i]);
-#pragma unroll
-      for (int g = 0; g < kGroups; ++g) kv[g] = vmax[g] > 0.0f ? __fdividef(kPSteps, vmax[g]) : 0.0f;
-      float pn[HH], p[HH];
+      // p = 2^(s - m_run) in [0, 2^kLazyMax]; P' = p * scale * 2^23 / vmr rounded
+      // to an integer in [0, 2^31]
+      float pn[HH];
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
-        pn[i] = valid ? exp2f(sc[i] - smax[i]) : 0.0f;
-        p[i] = pn[i] * pmax[i];
-        l_acc[i] += p[i];
+        pn[i] = valid ? exp2f(sc[i] - m_run[i]) : 0.0f;
+        l_acc[i] += pn[i];
       }
-      uint32_t xb[kGroups * HH + 1];  // column order: group, then head (one spare for odd HH)
+      uint32_t xw[kGroups * HH];  // column order: group, then head
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) {
-        const float vk = vsz[g].x * kv[g];
+        const float vk = vsz[g].x * kvr[g];
         if constexpr (HH == 1) {
-          zacc[g][0] = fmaf(p[0], vsz[g].y, zacc[g][0]);
-          xb[g] = __float_as_uint(fmaf(pn[0], vk, 8388608.0f));
+          zacc[g][0] = fmaf(pn[0], vsz[g].y, zacc[g][0]);
+          xw[g] = __float2uint_rn(pn[0] * vk);
         } else {
 #pragma unroll
           for (int i = 0; i < HH; i += 2) {  // heads in pairs: one paired fma per pair
-            const float2 z = ffma2(make_float2(p[i], p[i + 1]), make_float2(vsz[g].y, vsz[g].y),
+            const float2 z = ffma2(make_float2(pn[i], pn[i + 1]), make_float2(vsz[g].y, vsz[g].y),
                                    make_float2(zacc[g][i], zacc[g][i + 1]));
             zacc[g][i] = z.x;
             zacc[g][i + 1] = z.y;
-            const float2 x = ffma2(make_float2(pn[i], pn[i + 1]), make_float2(vk, vk), make_float2(8388608.0f, 8388608.0f));
-            xb[g * HH + i] = __float_as_uint(x.x);
-            xb[g * HH + i + 1] = __float_as_uint(x.y);
+            xw[g * HH + i] = __float2uint_rn(pn[i] * vk);
+            xw[g * HH + i + 1] = __float2uint_rn(pn[i + 1] * vk);
           }
         }
       }
-      // the tile's PV sums (read back RD tiles later) carry pmax * vmax / (2^23 - 1)
-      // for channel j's group
+      // the tile's PV sums (read back RD tiles later) carry vmr / 2^23 for
+      // channel j's group
       float ds0[HH];
 #pragma unroll
-      for (int i = 0; i < HH; ++i) ds0[i] = pmax[i] * (vmax[wq] * (1.0f / kPSteps));
-      // the low three bytes of each P' integer, in column order, four per word:
-      // three words per four integers
-      uint32_t by[NC / 4];
-#pragma unroll
-      for (int w = 0; w < kGroups * HH / 4; ++w) {
-        by[3 * w] = __byte_perm(xb[4 * w], xb[4 * w + 1], 0x4210);          // x0.b0 x0.b1 x0.b2 x1.b0
-        by[3 * w + 1] = __byte_perm(xb[4 * w + 1], xb[4 * w + 2], 0x5421);  // x1.b1 x1.b2 x2.b0 x2.b1
-        by[3 * w + 2] = __byte_perm(xb[4 * w + 2], xb[4 * w + 3], 0x6542);  // x2.b2 x3.b0 x3.b1 x3.b2
-      }
+      for (int i = 0; i < HH; ++i) ds0[i] = vmr[wq] * (1.0f / kPUnit);
+      // four P' words (16 columns, one 16-byte row of the operand) per store
       uint8_t* BP = fix + S::F_BP + k * S::BP_BYTES;
 #pragma unroll
-      for (int w = 0; w < NC / 4; w += 4) {  // 16 columns (one 16-byte row) at a time, or what is left
-        uint8_t* dst = BP + mnmajor8(n0 + 4 * w, pos);
-        if (NC / 4 - w >= 4)
-          *reinterpret_cast<uint4*>(dst) = make_uint4(by[w], by[w + 1], by[w + 2], by[w + 3]);
-        else if (NC / 4 - w == 3) {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(by[w], by[w + 1]);
-          *reinterpret_cast<uint32_t*>(dst + 8) = by[w + 2];
-        } else if (NC / 4 - w == 2)
-          *reinterpret_cast<uint2*>(dst) = make_uint2(by[w], by[w + 1]);
-        else
-          *reinterpret_cast<uint32_t*>(dst) = by[w];
-      }
+      for (int w = 0; w < kGroups * HH / 4; ++w)
+        *reinterpret_cast<uint4*>(BP + mnmajor8(n0 + 16 * w, pos)) =
+            make_uint4(xw[4 * w], xw[4 * w + 1], xw[4 * w + 2], xw[4 * w + 3]);
       fence_proxy_async();
       mbar_arrive(PREADY(k));
 #pragma unroll
@@ -891,6 +836,84 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           a.part_acc[row * kHeadDim + j] = good ? acc[i] + zown[i] : nan;
           if (j == 0) a.part_ml[row] = good ? make_float2(m_run[i], lsum[i]) : make_float2(nan, nan);
         }
+      }
+    }
+  } else {
+    setmaxnreg_dec<S::REG_ISSUE>();
+    if (warp == S::MMA_WARP) {
+      // ================================================================ score UMMAs
+      // As far ahead as the SB score buffers allow: buffer t % SB was last read
+      // by the epilogue of tile t - SB, which frees it (SFREE) once its scores are
+      // in registers.
+      const uint32_t idesc_s = idesc_u8s8_s32(kTile, S::NS);
+      int sseg = -1;  // segment of the tile being scored
+      for (int t = 0; t < ntiles; ++t, it.next(a)) {
+        if (it.first) ++sseg;
+        const uint32_t bq = smem_addr(fix + S::F_BQ + (sseg & 1) * S::BQ_BYTES);
+        if (t >= S::SB) ws_wait(SFREE(t % S::SB), ((t - S::SB) / S::SB) & 1, err);
+        ws_wait(KREADY(t % S::NKR), (t / S::NKR) & 1, err);
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = tmem + S::TM_AK + (t % S::KST) * 32;
+          const uint32_t d0 = tmem + S::TM_S + (t % S::SB) * 4 * S::NS;
+          // one MMA per 32-channel group (8 columns of u8 codes, 32 query bytes), all independent
+  #pragma unroll
+          for (int g = 0; g < kGroups; ++g)
+            umma_i8_tmem_a(d0 + g * S::NS, a0 + g * 8, smem_desc(bq + g * 256, 128, 1024), idesc_s, 0u);
+          umma_commit(SDONE(t % S::SB));
+        }
+        __syncwarp();
+      }
+    } else if (warp == S::PV_WARP) {
+      // ================================================================ PV UMMAs
+      const uint32_t idesc_o = idesc_u8u8_s32_bmn(kTile, S::NPV);
+      const uint32_t bp = smem_addr(fix + S::F_BP);
+      for (int t = 0; t < ntiles; ++t) {
+        ws_wait(PREADY(t & 1), (t >> 1) & 1, err);
+        ws_wait(VREADY(t & 1), (t >> 1) & 1, err);
+        tc_fence_after();
+        if (lane == 0) {
+          // 32 tokens per MMA: u8 value codes (8 tensor-memory columns) x the
+          // tile's P' bytes; each tile's sums start afresh in PV buffer t % DB
+          const uint32_t a0 = tmem + S::TM_AV + (t % S::VST) * 32;
+          const uint32_t b0 = bp + (t & 1) * S::BP_BYTES;
+          const uint32_t d0 = tmem + S::TM_D + (t % S::DB) * S::NPV;
+  #pragma unroll
+          for (int s = 0; s < kTile / 32; ++s)
+            umma_i8_tmem_a(d0, a0 + s * 8, smem_desc(b0 + s * 512, 128, 2048), idesc_o, s > 0 ? 1u : 0u);
+          umma_commit(PVDONE(t & 1));
+        }
+        __syncwarp();
+      }
+    } else {
+      // ================================================================ producers
+      const int nblk = c.cap / kTile;
+      const int pw = warp - S::PROD_WARP;
+      for (int t = 0; t < ntiles; ++t, it.next(a)) {
+        if (t % S::NPROD != pw) continue;
+        const int s = t % ST;
+        if (t >= ST) ws_wait(EMPTY(s), ((t / ST) - 1) & 1, err);
+        const size_t bh = it.bh(a);
+        const uint32_t msk = it.msk;
+        const int n0 = it.i * kTile;
+        const size_t blk = bh * nblk + it.i;
+        const uint32_t dst = smem_addr(smem + s * S::STAGE);
+        const bool k0 = CH0 && (msk & 1u);
+        if (lane == 0)
+          mbar_arrive_expect_tx(FULL(s), (uint32_t)(__popc(msk) * S::KROW + kHeadDim * S::VROW + 2 * kGroups * kTile * 4 +
+                                                    (k0 ? kTile * 2 : 0)));
+        __syncwarp();
+        // one copy per run of adjacent kept channel groups (their rows are adjacent in the block)
+        const bool run_start = ((msk >> lane) & 1u) && (lane == 0 || !((msk >> (lane - 1)) & 1u));
+        if (run_start) {
+          const int run = __ffsll((long long)~((unsigned long long)msk >> lane)) - 1;
+          bulk_g2s(dst + S::R_KC + lane * S::KROW, c.kc + key_word_index(bh, c.cap, lane, n0) * (KB == 4 ? 2 : 1),
+                   run * S::KROW, FULL(s));
+        }
+        if (lane == 0) bulk_g2s(dst + S::R_VC, c.vc + blk * kHeadDim * S::VROW, kHeadDim * S::VROW, FULL(s));
+        if (lane == 1) bulk_g2s(dst + S::R_KS, c.ks + key_scale_index(bh, c.cap, 0, n0), kGroups * kTile * 4, FULL(s));
+        if (lane == 2) bulk_g2s(dst + S::R_VS, c.vs + (bh * c.cap + n0) * kGroups, kTile * kGroups * 4, FULL(s));
+        if (k0 && lane == 3) bulk_g2s(dst + S::R_K0, c.k0 + bh * c.cap + n0, kTile * 2, FULL(s));
       }
     }
   }
