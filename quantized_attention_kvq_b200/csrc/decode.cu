@@ -80,7 +80,7 @@ struct Shape {
   // two UMMA issuers: one thread can only have about one MMA in its issue
   // stage at a time (some 150 cycles each, whatever the shape), so the score
   // and the PV MMAs come from two warps and overlap
-  static constexpr int MMA_WARP = 4 + EPI_WARPS;  // score MMAs
+  static constexpr int MMA_WARP = 8 + EPI_WARPS;  // score MMAs
   static constexpr int PV_WARP = MMA_WARP + 1;    // PV MMAs
   // ring fillers: producer p issues the copies of the tiles t with t % NPROD == p
   // (a pruned tile takes one copy per run of kept channel groups)
@@ -88,16 +88,17 @@ struct Shape {
   static constexpr int PROD_WARP = PV_WARP + 1;
   static constexpr int THREADS = 32 * (PROD_WARP + NPROD);
   // registers per thread: the block is launched with 65536 / THREADS; the
-  // code warps and the issue/producer warpgroup give some back to the
+  // code warpgroups and the issue/producer warpgroup give some back to the
   // epilogue warpgroups (the shares add up to at most the launch total)
   static constexpr int REG_LAUNCH = 65536 / THREADS / 8 * 8;
-  static constexpr int REG_CODE = 80;
+  static constexpr int REG_KCODE = 80;
+  static constexpr int REG_VCODE = 56;
   static constexpr int REG_ISSUE = 56;
-  static constexpr int REG_EPI = (REG_LAUNCH * THREADS - 128 * (REG_CODE + REG_ISSUE)) / EPI_THREADS / 8 * 8 > 248
-                                     ? 248
-                                     : (REG_LAUNCH * THREADS - 128 * (REG_CODE + REG_ISSUE)) / EPI_THREADS / 8 * 8;
-  static_assert(THREADS == 128 + EPI_THREADS + 128, "warpgroups: code, epilogue, issue + producers");
-  static_assert(128 * (REG_CODE + REG_ISSUE) + EPI_THREADS * REG_EPI <= REG_LAUNCH * THREADS, "register split");
+  static constexpr int REG_REST = 128 * (REG_KCODE + REG_VCODE + REG_ISSUE);
+  static constexpr int REG_EPI_FIT = (REG_LAUNCH * THREADS - REG_REST) / EPI_THREADS / 8 * 8;
+  static constexpr int REG_EPI = REG_EPI_FIT > 248 ? 248 : REG_EPI_FIT;
+  static_assert(THREADS == 256 + EPI_THREADS + 128, "warpgroups: key codes, value codes, epilogue, issue + producers");
+  static_assert(REG_REST + EPI_THREADS * REG_EPI <= REG_LAUNCH * THREADS, "register split");
   static_assert(REG_EPI >= REG_LAUNCH, "register split");
   static constexpr int NS = 2 * G < 16 ? 16 : 2 * G;  // score columns per group: q1 rows, then q2 rows
   static constexpr int PH = 4 * G;  // P' columns per byte: (value group, head)
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   if (tid == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(FULL(s), 1);
-      mbar_init(EMPTY(s), 128 + S::EPI_THREADS / S::NGRP);  // code conversion and the tile's epilogue group
+      mbar_init(EMPTY(s), 256 + S::EPI_THREADS / S::NGRP);  // key and value conversion, the tile's epilogue group
     }
     for (int k = 0; k < S::NKR; ++k) mbar_init(KREADY(k), 128);
     for (int k = 0; k < S::SB; ++k) {
@@ -353,115 +354,115 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   // issue/producer warpgroup give registers back to the epilogue), then
   // takes its role.
   if (warp < 4) {
-    setmaxnreg_dec<S::REG_CODE>();
-    // ================================================================ codes -> tensor memory
-    // The key codes (thread = token) run one tile ahead of the value codes
-    // (thread = channel): step t converts the keys of tile t, then the values
-    // of tile t - 1, so the score MMAs of a tile never wait for the value
-    // conversion of the tile before it.  Both land in this warp's lane quarter.
-    const int j = tid;  // token of the tile == tensor-memory lane; then channel
+    setmaxnreg_dec<S::REG_KCODE>();
+    // ================================================================ key codes -> tensor memory
+    // thread = token of the tile == tensor-memory lane of this warp's quarter
+    const int j = tid;
     const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+    int kseg = 0;  // segments begun so far
+    for (int t = 0; t < ntiles; ++t, it.next(a)) {
+      const int s = t % ST;
+      const uint8_t* raw = smem + s * S::STAGE + S::R_KC;
+      ws_wait(FULL(s), (t / ST) & 1, err);
+      // this key stage was read by the score UMMAs of tile t - KST
+      if (t >= S::KST) ws_wait(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err);
+      tc_fence_after();
+      if (it.first) {
+        // query data of segment kseg into buffer kseg & 1: per head, delta =
+        // max|q| / 16000 and q = delta * (128 q1 + q2) exactly, q1 in row h, q2 in
+        // row G + h; dropped channel groups (and channel 0 when it is kept in bf16)
+        // are zero.  The buffer was last used by segment kseg - 2, which the
+        // epilogue (and so its score UMMAs) finished before freeing it.  Each
+        // buffer's two barriers see one phase per use, in order, so no parity wait
+        // can pass on a later or an earlier phase.
+        const int qb = kseg & 1;
+        if (kseg >= 2) ws_wait(QFREE(qb), ((kseg - 2) >> 1) & 1, err);
+        uint8_t* BQ = fix + S::F_BQ + qb * S::BQ_BYTES;
+        float* qsum = reinterpret_cast<float*>(fix + S::F_QS + qb * G * 16);
+        float* q0s = reinterpret_cast<float*>(fix + S::F_Q0 + qb * S::QV);
+        float* qds = reinterpret_cast<float*>(fix + S::F_QD + qb * S::QV);
+        const uint32_t msk = it.msk;
+        for (int hq = warp; hq < G; hq += 4) {
+          const In* qrow = static_cast<const In*>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.h * G + hq) * kHeadDim;
+          float x[4];
+          load_row_warp(qrow, c.rotate != 0, a.inv_sqrt_d, lane, x);
+          const bool sel = (msk >> lane) & 1u;
+          float v[4], part = 0.0f, amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            v[i] = sel ? x[i] : 0.0f;
+            if (CH0 && lane == 0 && i == 0) v[i] = 0.0f;
+            part += v[i];
+            amax = fmaxf(amax, fabsf(v[i]));
+          }
+          amax = warp_max(amax);
+          const float delta = amax > 0.0f ? amax / kQSteps : 1.0f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int ch = 4 * lane + i;
+            const int qi = __float2int_rn(v[i] / delta);  // |qi| <= 16000
+            const int q1 = (qi + 64) >> 7;                // nearest multiple of 128 below qi + 64
+            const int q2 = qi - 128 * q1;                 // in [-64, 63]
+            constexpr int blk = KB == 4 ? 8 : 16;
+            const int p = (ch / blk) * blk + kpos_of<KB>(ch % blk);
+            BQ[kmajor8(hq, p)] = (uint8_t)(int8_t)q1;
+            BQ[kmajor8(G + hq, p)] = (uint8_t)(int8_t)q2;
+          }
+#pragma unroll
+          for (int m = 1; m < 8; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
+          if ((lane & 7) == 0) qsum[hq * kGroups + (lane >> 3)] = part;
+          if (lane == 0) {
+            q0s[hq] = (CH0 && sel) ? x[0] : 0.0f;
+            qds[hq] = delta;
+          }
+        }
+        fence_proxy_async();      // query operand (generic writes) -> tensor core
+        mbar_arrive(QREADY(qb));  // release: the epilogue reads the data after waiting on it
+        ++kseg;
+      }
+      // every key row is converted: rows of dropped channel groups hold stale
+      // codes, which meet zeros in the query operand
+      uint32_t r[32];
+      if (KB == 4) {
+        const uint16_t* kc = reinterpret_cast<const uint16_t*>(raw) + j;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {  // channels 8q .. 8q+7: even ones, then odd ones
+          const uint32_t x = (uint32_t)kc[(2 * q) * kTile] | ((uint32_t)kc[(2 * q + 1) * kTile] << 16);
+          r[2 * q] = x & 0x0F0F0F0Fu;
+          r[2 * q + 1] = (x >> 4) & 0x0F0F0F0Fu;
+        }
+      } else {
+        const uint8_t* kc = raw + j;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // channels 16q .. 16q+15: crumb k of every byte together
+          const uint32_t x = (uint32_t)kc[(4 * q) * kTile] | ((uint32_t)kc[(4 * q + 1) * kTile] << 8) |
+                             ((uint32_t)kc[(4 * q + 2) * kTile] << 16) | ((uint32_t)kc[(4 * q + 3) * kTile] << 24);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) r[4 * q + k] = (x >> (2 * k)) & 0x03030303u;
+        }
+      }
+      const uint32_t col = tl + S::TM_AK + (t % S::KST) * 32;
+      tmem_st16(col, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
+      tmem_st16(col + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(KREADY(t % S::NKR));
+      mbar_arrive(EMPTY(t % ST));
+    }
+  } else if (warp < 8) {
+    setmaxnreg_dec<S::REG_VCODE>();
+    // ================================================================ value codes -> tensor memory
+    // thread = channel == tensor-memory lane of this warp's quarter
+    const int j = tid - 128;
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     // the 16-byte chunks of a channel's value row are stored rotated by
     // channel, so the rows of 8 consecutive channels hit 8 different bank groups
     const int swz = VB == 4 ? (j >> 1) & 3 : (j >> 2) & 1;
-    int kseg = 0;  // segments begun so far
-    for (int t = 0; t <= ntiles; ++t) {
-      if (t < ntiles) {
-        const int s = t % ST;
-        const uint8_t* raw = smem + s * S::STAGE + S::R_KC;
-        ws_wait(FULL(s), (t / ST) & 1, err);
-        // this key stage was read by the score UMMAs of tile t - KST
-        if (t >= S::KST) ws_wait(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err);
-        tc_fence_after();
-        if (it.first) {
-          // query data of segment kseg into buffer kseg & 1: per head, delta =
-          // max|q| / 16000 and q = delta * (128 q1 + q2) exactly, q1 in row h, q2 in
-          // row G + h; dropped channel groups (and channel 0 when it is kept in bf16)
-          // are zero.  The buffer was last used by segment kseg - 2, which the
-          // epilogue (and so its score UMMAs) finished before freeing it.  Each
-          // buffer's two barriers see one phase per use, in order, so no parity wait
-          // can pass on a later or an earlier phase.
-          const int qb = kseg & 1;
-          if (kseg >= 2) ws_wait(QFREE(qb), ((kseg - 2) >> 1) & 1, err);
-          uint8_t* BQ = fix + S::F_BQ + qb * S::BQ_BYTES;
-          float* qsum = reinterpret_cast<float*>(fix + S::F_QS + qb * G * 16);
-          float* q0s = reinterpret_cast<float*>(fix + S::F_Q0 + qb * S::QV);
-          float* qds = reinterpret_cast<float*>(fix + S::F_QD + qb * S::QV);
-          const uint32_t msk = it.msk;
-          for (int hq = warp; hq < G; hq += 4) {
-            const In* qrow = static_cast<const In*>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.h * G + hq) * kHeadDim;
-            float x[4];
-            load_row_warp(qrow, c.rotate != 0, a.inv_sqrt_d, lane, x);
-            const bool sel = (msk >> lane) & 1u;
-            float v[4], part = 0.0f, amax = 0.0f;
-  #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              v[i] = sel ? x[i] : 0.0f;
-              if (CH0 && lane == 0 && i == 0) v[i] = 0.0f;
-              part += v[i];
-              amax = fmaxf(amax, fabsf(v[i]));
-            }
-            amax = warp_max(amax);
-            const float delta = amax > 0.0f ? amax / kQSteps : 1.0f;
-  #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int ch = 4 * lane + i;
-              const int qi = __float2int_rn(v[i] / delta);  // |qi| <= 16000
-              const int q1 = (qi + 64) >> 7;                // nearest multiple of 128 below qi + 64
-              const int q2 = qi - 128 * q1;                 // in [-64, 63]
-              constexpr int blk = KB == 4 ? 8 : 16;
-              const int p = (ch / blk) * blk + kpos_of<KB>(ch % blk);
-              BQ[kmajor8(hq, p)] = (uint8_t)(int8_t)q1;
-              BQ[kmajor8(G + hq, p)] = (uint8_t)(int8_t)q2;
-            }
-  #pragma unroll
-            for (int m = 1; m < 8; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
-            if ((lane & 7) == 0) qsum[hq * kGroups + (lane >> 3)] = part;
-            if (lane == 0) {
-              q0s[hq] = (CH0 && sel) ? x[0] : 0.0f;
-              qds[hq] = delta;
-            }
-          }
-          mbar_arrive(QREADY(qb));  // release: the epilogue reads the data after waiting on it
-          ++kseg;
-        }
-        // every key row is converted: rows of dropped channel groups hold stale
-        // codes, which meet zeros in the query operand
-        uint32_t r[32];
-        if (KB == 4) {
-          const uint16_t* kc = reinterpret_cast<const uint16_t*>(raw) + j;
-  #pragma unroll
-          for (int q = 0; q < 16; ++q) {  // channels 8q .. 8q+7: even ones, then odd ones
-            const uint32_t x = (uint32_t)kc[(2 * q) * kTile] | ((uint32_t)kc[(2 * q + 1) * kTile] << 16);
-            r[2 * q] = x & 0x0F0F0F0Fu;
-            r[2 * q + 1] = (x >> 4) & 0x0F0F0F0Fu;
-          }
-        } else {
-          const uint8_t* kc = raw + j;
-  #pragma unroll
-          for (int q = 0; q < 8; ++q) {  // channels 16q .. 16q+15: crumb k of every byte together
-            const uint32_t x = (uint32_t)kc[(4 * q) * kTile] | ((uint32_t)kc[(4 * q + 1) * kTile] << 8) |
-                               ((uint32_t)kc[(4 * q + 2) * kTile] << 16) | ((uint32_t)kc[(4 * q + 3) * kTile] << 24);
-  #pragma unroll
-            for (int k = 0; k < 4; ++k) r[4 * q + k] = (x >> (2 * k)) & 0x03030303u;
-          }
-        }
-        const uint32_t col = tl + S::TM_AK + (t % S::KST) * 32;
-        tmem_st16(col, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
-        tmem_st16(col + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
-        tmem_wait_st();
-        fence_proxy_async();  // query operand (generic writes) -> tensor core
-        tc_fence_before();
-        mbar_arrive(KREADY(t % S::NKR));
-        it.next(a);
-      }
-      if (t == 0) continue;
-
-      // value codes of channel j of tile tv: this value stage was read by the
-      // PV UMMAs of tile tv - VST
-      const int tv = t - 1;
-      const int s = tv % ST;
-      if (tv >= S::VST) ws_wait(PVDONE((tv - S::VST) & 1), ((tv - S::VST) >> 1) & 1, err);
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % ST;
+      ws_wait(FULL(s), (t / ST) & 1, err);
+      // this value stage was read by the PV UMMAs of tile t - VST
+      if (t >= S::VST) ws_wait(PVDONE((t - S::VST) & 1), ((t - S::VST) >> 1) & 1, err);
       tc_fence_after();
       uint32_t r[32];
       const uint8_t* row = smem + s * S::STAGE + S::R_VC + j * S::VROW;
@@ -487,21 +488,21 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             for (int m = 0; m < 4; ++m) r[16 * k + 4 * i + m] = (ws[i] >> (2 * m)) & 0x03030303u;
         }
       }
-      const uint32_t vcol = tl + S::TM_AV + (tv % S::VST) * 32;  // 128 u8 codes in the order vpos_of gives
+      const uint32_t vcol = tl + S::TM_AV + (t % S::VST) * 32;  // 128 u8 codes in the order vpos_of gives
       tmem_st16(vcol, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
       tmem_st16(vcol + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(VREADY(tv & 1));
+      mbar_arrive(VREADY(t & 1));
       mbar_arrive(EMPTY(s));
     }
-  } else if (warp < 4 + S::EPI_WARPS) {
+  } else if (warp < 8 + S::EPI_WARPS) {
     setmaxnreg_inc<S::REG_EPI>();
     // ================================================================ epilogue
     // With NGRP epilogue groups, group g takes the tiles t with t % NGRP == g;
     // each keeps its own online softmax and accumulators per segment and
     // leaves its own partial, which the combine merges like any other split.
-    const int e = tid - 128;             // 0 .. EPI_THREADS-1
+    const int e = tid - 256;             // 0 .. EPI_THREADS-1
     const int grp = e / (128 * S::TPT);  // epilogue group
     const int j = e & 127;               // token (score phase) == tensor-memory lane == channel (PV phase)
     const int part = (e >> 7) % S::TPT;  // head part: heads part*HH .. part*HH + HH - 1
@@ -1036,3 +1037,4 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
 }
 
 }  // namespace kvq
+
