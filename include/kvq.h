@@ -273,7 +273,10 @@ KVQ_API kvq_status kvq_decode_combine(const kvq_cache* cache, int32_t q_heads, c
  * kvq_decode_workspace_bytes exceeds 16 MiB, returns KVQ_ERR_WORKSPACE and
  * enqueues nothing.  The call allocates nothing.  The first call on a device
  * looks up that array's device address (with the device current) and caches
- * it, so make that first call before any stream capture.  Every call shares
+ * it, so make that first call before any stream capture.  The cached address
+ * belongs to the device's context of that first call: after cudaDeviceReset,
+ * or any other teardown and re-creation of the context, it is stale, and this
+ * entry point must not be called again in the process.  Every call shares
  * the array: calls that run concurrently on the GPU (different streams, or
  * different host threads, without ordering between them) race on it and give
  * undefined results.  Nothing in the array needs to start at zero: each call

@@ -32,8 +32,10 @@ kvq_status check_shape(const kvq_cache* c) {
   if (c->bucket_tokens > 0 && (c->bucket_tokens % kKeyBlock != 0 || c->capacity % c->bucket_tokens != 0 ||
                                c->sink_tokens + c->recent_tokens > 0))
     return KVQ_ERR_UNSUPPORTED;
-  // the per-bucket selection runs one grid row per (sequence, bucket)
-  if (c->bucket_tokens > 0 && (int64_t)c->batch * (c->capacity / c->bucket_tokens) > 65535) return KVQ_ERR_UNSUPPORTED;
+  // the selection runs one grid row per (sequence, bucket), the append one grid
+  // layer per sequence: both at most 65535
+  const int64_t rows = (int64_t)c->batch * (c->bucket_tokens > 0 ? c->capacity / c->bucket_tokens : 1);
+  if (rows > 65535) return KVQ_ERR_UNSUPPORTED;
   return KVQ_OK;
 }
 

@@ -166,6 +166,14 @@ def test_bucket_rope_host_checks(L):
     many.rope_inv_freq = FAKE
     assert L.kvq_quantize_append(ctypes.byref(many), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
         native.KVQ_ERR_UNSUPPORTED
+    # without buckets the batch alone is the grid row count
+    wide = desc(B=65536, cap=128)
+    assert L.kvq_quantize_append(ctypes.byref(wide), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
+        native.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_select_channels(ctypes.byref(wide), FAKE, native.KVQ_BF16, 8, 4, FAKE, None) == \
+        native.KVQ_ERR_UNSUPPORTED
+    edge = desc(B=65535, cap=128)
+    assert L.kvq_cache_sizes(ctypes.byref(edge), (ctypes.c_size_t * 5)()) == native.KVQ_OK
     odd = desc(cap=512, bucket_tokens=384)
     odd.rope_inv_freq = FAKE
     assert L.kvq_quantize_append(ctypes.byref(odd), FAKE, FAKE, native.KVQ_BF16, 8, 0, None) == \
