@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 from quantized_attention_kvq_b200 import synth, workloads  # noqa: E402
 
-DEFAULT_WORKLOAD = 1  # GQA INT4 decode, batch 8, 32/8 heads, 32768 cached tokens
+DEFAULT_WORKLOAD = 4  # the largest decode: 64 ragged sequences (1K-16K tokens), 64/8 heads, INT4 keys pruned to 24/32, INT2 values
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SOURCES = ("decode.cu", "common.cuh", "sm100.cuh")
 APPEND_SOURCES = ("append.cu", "common.cuh")
@@ -109,11 +109,11 @@ def source_sha(names=DECODE_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name: str, summary: str = "decode_split_traffic.md", sources=DECODE_SOURCES):
-    """DRAM bytes per launch of a kernel from its committed ncu summary, or None
-    when the summary is missing, covers another workload, or the kernel source
-    changed since."""
-    p = os.path.join(ROOT, "profiles", summary)
+def recorded_traffic(workload_name: str, kernel: str = "k_decode", sources=DECODE_SOURCES):
+    """DRAM bytes per launch of a kernel on a workload from its committed ncu
+    summary (profiles/<kernel>_traffic_<workload>.md), or None when the summary
+    is missing, covers another workload, or the kernel source changed since."""
+    p = os.path.join(ROOT, "profiles", f"{kernel}_traffic_{workload_name}.md")
     if not os.path.exists(p):
         return None
     fields = {}
@@ -617,7 +617,7 @@ def run_append(args):
             "gpu_launches": args.steps,
             "roofline": {"bound": "hbm", "kernel": "quantize-append (kvq_quantize_append)", "achieved": achieved,
                          "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": recorded_traffic(wl.name, "append_traffic.md", APPEND_SOURCES),
+                         "traffic": recorded_traffic(wl.name, "k_quantize_append", APPEND_SOURCES),
                          "algorithmic_bytes_per_launch": abytes, "peak_source": peak_src, "kernel_ms": ms},
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
