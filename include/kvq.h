@@ -42,7 +42,8 @@ typedef enum {
   KVQ_ERR_UNSUPPORTED = 2, /* a valid configuration this build does not implement          */
   KVQ_ERR_CAPACITY = 3,    /* offset + n_new > capacity, or max_len > capacity             */
   KVQ_ERR_WORKSPACE = 4,   /* workspace smaller than the matching *_workspace_bytes query */
-  KVQ_ERR_CUDA = 5         /* the CUDA runtime reported an error when enqueuing            */
+  KVQ_ERR_CUDA = 5,        /* the CUDA runtime reported an error when enqueuing            */
+  KVQ_ERR_TIMEOUT = 6      /* a bounded wait inside a kernel gave up (kvq_decode_status)   */
 } kvq_status;
 
 typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1, KVQ_F16 = 2 } kvq_dtype;
@@ -202,6 +203,30 @@ KVQ_API kvq_status kvq_select_channels(const kvq_cache* cache, const void* q, kv
 KVQ_API kvq_status kvq_select_channels_at(const kvq_cache* cache, const void* q, kvq_dtype dtype, int32_t q_heads,
                                           const int32_t* seq_lens, int32_t keep_groups, uint32_t* mask_out,
                                           void* stream);
+
+/*
+ * The status of the last split decode (kvq_decode_attention or
+ * kvq_decode_partials) that used `workspace`: KVQ_OK, or KVQ_ERR_TIMEOUT when
+ * one of its bounded waits gave up.  The split decode's roles hand tiles to
+ * one another through shared-memory barriers, and every wait on one is
+ * bounded (about a second); after a give-up the CTA lets its work in flight
+ * land, writes NaN partials (so the affected outputs are NaN), sets a status
+ * word in the workspace and returns, and the context stays usable.  Each
+ * split decode clears the word before it starts.  This call copies the word
+ * back on `stream` and synchronizes that stream.  q_heads and workspace_bytes
+ * as given to the decode.
+ */
+KVQ_API kvq_status kvq_decode_status(const kvq_cache* cache, int32_t q_heads, const void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/*
+ * Test hook for the give-up path: the next split decode enqueued from the
+ * calling host thread leaves tile `tile` of its first CTA unfilled (its ring
+ * stage never completes), so the waits on that tile give up after about a
+ * second and kvq_decode_status reports KVQ_ERR_TIMEOUT.  A negative tile
+ * clears the hook.  Not for production use.
+ */
+KVQ_API void kvq_test_withhold_tile(int32_t tile);
 
 /* Device workspace bytes kvq_decode_attention needs for these sizes (0 on bad arguments). */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_heads, int32_t max_len);

@@ -124,7 +124,7 @@ CacheView bucket_sequence_view(const kvq_cache* c, size_t vb) {
 // max and sum) per (slot, query head of the GQA group), decode_slots slots;
 // with the caller's transform pair, then the transformed fp32 query rows.
 struct DecodePlan {
-  size_t acc_bytes, ml_offset, tq_offset, qb_offset, vl_offset, bytes;
+  size_t acc_bytes, ml_offset, tq_offset, qb_offset, vl_offset, status_offset, bytes;
 };
 
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
@@ -143,7 +143,18 @@ DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   if (c->bucket_tokens > 0) p.bytes += round_up((size_t)Bv * q_heads * kHeadDim * sizeof(float), kAlign);
   p.vl_offset = p.bytes;
   if (c->bucket_tokens > 0) p.bytes += round_up((size_t)Bv * sizeof(int32_t), kAlign);
+  // the split decode's status word (a wait gave up), cleared by each split
+  p.status_offset = p.bytes;
+  p.bytes += kAlign;
   return p;
+}
+
+// test hook: the tile the next split decode of this host thread withholds
+thread_local int g_withheld_tile = -1;
+int take_withheld_tile() {
+  const int t = g_withheld_tile;
+  g_withheld_tile = -1;
+  return t;
 }
 
 kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
@@ -177,7 +188,12 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
     v.part_acc = reinterpret_cast<float*>(ws);
     v.part_ml = reinterpret_cast<float2*>(ws + plan.ml_offset);
     v.out = nullptr;
+    v.status = reinterpret_cast<int*>(ws + plan.status_offset);
+    v.withheld_tile = -1;
     if (parts & kRunSplit) {
+      v.withheld_tile = take_withheld_tile();
+      kvq_status st0 = cuda_status(cudaMemsetAsync(v.status, 0, sizeof(int), s));
+      if (st0 != KVQ_OK) return st0;
       kvq_status st = cuda_status(launch_bucket_queries(
           q, dtype, c->rotate_k, c->t_query, c->rope_inv_freq, seq_lens, max_len, c->batch, q_heads, c->kv_heads,
           c->bucket_tokens, nb, inv_sqrt_d(), reinterpret_cast<float*>(ws + plan.qb_offset),
@@ -203,6 +219,13 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.part_acc = static_cast<float*>(workspace);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
+  a.status = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan.status_offset);
+  a.withheld_tile = -1;
+  if (parts & kRunSplit) {
+    a.withheld_tile = take_withheld_tile();
+    kvq_status st = cuda_status(cudaMemsetAsync(a.status, 0, sizeof(int), s));
+    if (st != KVQ_OK) return st;
+  }
   if ((parts & kRunSplit) && c->rotate_k == 2) {
     // the kernels below read the transformed rows as untransformed fp32 queries
     float* qt = reinterpret_cast<float*>(static_cast<char*>(workspace) + plan.tq_offset);
@@ -346,6 +369,24 @@ KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dt
   return kvq_select_channels_at(c, q, dtype, q_heads, nullptr, keep_groups, mask_out, stream);
 }
 
+KVQ_API kvq_status kvq_decode_status(const kvq_cache* c, int32_t q_heads, const void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK || !workspace || !aligned16(workspace))
+    return KVQ_ERR_INVALID_ARG;
+  if (!decode_g_supported(q_heads / c->kv_heads)) return KVQ_ERR_UNSUPPORTED;
+  const DecodePlan plan = plan_decode(c, q_heads);
+  if (workspace_bytes < plan.bytes) return KVQ_ERR_WORKSPACE;
+  int word = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&word, static_cast<const char*>(workspace) + plan.status_offset, sizeof(int),
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  return word ? KVQ_ERR_TIMEOUT : KVQ_OK;
+}
+
+KVQ_API void kvq_test_withhold_tile(int32_t tile) { kvq::g_withheld_tile = tile < 0 ? -1 : tile; }
+
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
   if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK) return 0;
   if (max_len < 0 || max_len > c->capacity) return 0;
@@ -437,6 +478,7 @@ KVQ_API const char* kvq_status_string(kvq_status s) {
     case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
     case KVQ_ERR_WORKSPACE: return "workspace too small";
     case KVQ_ERR_CUDA: return "CUDA runtime error";
+    case KVQ_ERR_TIMEOUT: return "a bounded wait in a kernel gave up";
   }
   return "unknown status";
 }

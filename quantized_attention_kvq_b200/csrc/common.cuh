@@ -168,6 +168,8 @@ struct DecodeArgs {
   float* part_acc;  // [decode_slots][G][128] unnormalized accumulators
   float2* part_ml;  // [decode_slots][G] (running max, running sum)
   float* out;       // [B][Hq][128]
+  int* status;      // device word: bit 0 set when a bounded wait of the split decode gave up
+  int withheld_tile;  // test hook: CTA 0 never fills this tile's ring stage (-1: none)
 };
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);

@@ -252,7 +252,7 @@ struct TileIter {
 // slots.  Gives up after about a second, or at once after any earlier give-up
 // in the CTA, and reports false.
 __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile int* err) {
-  if (mbar_test_wait(bar, parity)) return true;
+  if (__builtin_expect(mbar_test_wait(bar, parity), 1)) return true;
 #pragma unroll 1
   for (uint32_t it = 0; it < (1u << 21); ++it) {
     if (mbar_try_wait_sleep(bar, parity, 500u)) return true;
@@ -367,11 +367,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       // this key stage was read by the score UMMAs of tile t - KST
       if (t >= S::KST) ws_wait(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err);
       tc_fence_after();
-      if (it.first) {
+      if (__builtin_expect(it.first, 0)) {
         // query data of segment kseg into buffer kseg & 1: per head, delta =
-        // max|q| / 16000 and q = delta * (128 q1 + q2) exactly, q1 in row h, q2 in
-        // row G + h; dropped channel groups (and channel 0 when it is kept in bf16)
-        // are zero.  The buffer was last used by segment kseg - 2, which the
+        // max|q| / 16000 and q = delta * (128 q1 + q2) exactly; the rows of each
+        // epilogue head part are its heads' q1 pieces, then their q2 pieces;
+        // dropped channel groups (and channel 0 when it is kept in bf16) are zero.  The buffer was last used by segment kseg - 2, which the
         // epilogue (and so its score UMMAs) finished before freeing it.  Each
         // buffer's two barriers see one phase per use, in order, so no parity wait
         // can pass on a later or an earlier phase.
@@ -405,8 +405,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             const int q2 = qi - 128 * q1;                 // in [-64, 63]
             constexpr int blk = KB == 4 ? 8 : 16;
             const int p = (ch / blk) * blk + kpos_of<KB>(ch % blk);
-            BQ[kmajor8(hq, p)] = (uint8_t)(int8_t)q1;
-            BQ[kmajor8(G + hq, p)] = (uint8_t)(int8_t)q2;
+            const int r1 = (hq / S::HH) * 2 * S::HH + hq % S::HH;
+            BQ[kmajor8(r1, p)] = (uint8_t)(int8_t)q1;
+            BQ[kmajor8(r1 + S::HH, p)] = (uint8_t)(int8_t)q2;
           }
 #pragma unroll
           for (int m = 1; m < 8; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
@@ -543,9 +544,8 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 
     // add the PV sums of tile tp (buffer tp % DB) times its scale into acc:
     // the sums of the four bytes of P' (each exact in fp32)
-    auto read_pv = [&](int tp, const float (&ds)[HH]) {
-      uint32_t r[4 * HH];  // (head, byte) of channel j's group
-      tmem_ld_wait<4 * HH>(tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * 4 * HH, r);
+    auto pv_addr = [&](int tp) { return tmem + lane_base + S::TM_D + (tp % S::DB) * S::NPV + n0 + wq * 4 * HH; };
+    auto add_pv = [&](const uint32_t (&r)[4 * HH], const float (&ds)[HH]) {
 #pragma unroll
       for (int i = 0; i < HH; ++i) {
         float v = (float)(int)r[4 * i + 3];
@@ -555,10 +555,15 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         acc[i] = fmaf(v, ds[i], acc[i]);
       }
     };
+    auto read_pv = [&](int tp, const float (&ds)[HH]) {
+      uint32_t r[4 * HH];  // (head, byte) of channel j's group
+      tmem_ld_wait<4 * HH>(pv_addr(tp), r);
+      add_pv(r, ds);
+    };
 
     for (int t = 0; t < ntiles; ++t, it.next(a)) {
       const int k = t & 1;
-      if (it.first) {
+      if (__builtin_expect(it.first, 0)) {
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           m_run[i] = NEG_INF;
@@ -619,19 +624,45 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         k0v = 0.0f;
       }
 
+      // The P' buffer k was read by the PV UMMAs of tile t - 2 (the UMMAs of
+      // one thread complete in order, so PV t - 1 done implies PV t - 2 done),
+      // whose sums, this group's when it has one in this segment, are read back
+      // before the running max can move.  With one epilogue group, tile t - 2
+      // is two tiles back and long done: its sums come in the same
+      // tensor-memory round trip as the scores.  With two, it is this group's
+      // previous tile, still in flight: they come after the scores.
+      constexpr bool MERGED = HH <= 4 && S::NGRP == 1;
       ok &= ws_wait(SDONE(t % S::SB), (t / S::SB) & 1, err);
+      if (MERGED && t >= RD) ok &= ws_wait(PVDONE((t - RD) & 1), ((t - RD) >> 1) & 1, err);
+      const bool rdp = t >= RD && (PLEN == 2 ? have2 : have1);
       tc_fence_after();
+      // S_g = sum_c u8 code * (128 q1 + q2): q1 in column 2 HH part + h, q2 in
+      // column 2 HH part + HH + h of group g
+      uint32_t sd[kGroups][2 * HH];
+      const uint32_t sbase = tmem + lane_base + S::TM_S + (t % S::SB) * 4 * S::NS + part * 2 * HH;
+      if constexpr (MERGED) {
+        uint32_t pv[4 * HH];
+        tmem_ld_sc_pv<HH>(sbase, S::NS, pv_addr(t), sd, pv);
+        tc_fence_before();
+        if (rdp) add_pv(pv, PLEN == 2 ? ds2 : ds1);
+      } else if constexpr (HH <= 4) {
+        tmem_ld4_wait<2 * HH>(sbase, S::NS, sd);
+        tc_fence_before();
+      } else {
+        uint32_t d1[kGroups][HH], d2[kGroups][HH];
+        tmem_ld4_wait<HH>(sbase, S::NS, d1);
+        tmem_ld4_wait<HH>(sbase + HH, S::NS, d2);
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g)
+#pragma unroll
+          for (int i = 0; i < HH; ++i) {
+            sd[g][i] = d1[g][i];
+            sd[g][HH + i] = d2[g][i];
+          }
+        tc_fence_before();
+      }
       float sc[HH];
       {
-        // S_g = sum_c u8 code * (128 q1 + q2): q1 in column h, q2 in column G + h of group g
-        uint32_t d1[kGroups][HH], d2[kGroups][HH];
-        const uint32_t sbase = tmem + lane_base + S::TM_S + (t % S::SB) * 4 * S::NS + part * HH;
-        if constexpr (HH == 2 || HH == 4) {
-          tmem_ld8_wait<HH>(sbase, S::NS, G, d1, d2);
-        } else {
-          tmem_ld4_wait<HH>(sbase, S::NS, d1);
-          tmem_ld4_wait<HH>(sbase + G, S::NS, d2);
-        }
         const float* qsum = reinterpret_cast<const float*>(fix + S::F_QS + qb * G * 16);
         const float* q0s = reinterpret_cast<const float*>(fix + S::F_Q0 + qb * S::QV);
         const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * S::QV);
@@ -657,13 +688,12 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           float2 dz = make_float2(0.0f, CH0 ? q0 * k0v : 0.0f);
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) {
-            const int dg = (int)d1[g][i] * 128 + (int)d2[g][i];  // exact: |dg| < 2^23
+            const int dg = (int)sd[g][i] * 128 + (int)sd[g][HH + i];  // exact: |dg| < 2^23
             dz = ffma2(ksz[g], make_float2((float)dg, qg[g]), dz);
           }
           sc[i] = valid ? fmaf(dz.x, qd, dz.y) * a.scale_log2 : NEG_INF;
         }
       }
-      tc_fence_before();
       mbar_arrive(SFREE(t % S::SB));        // the score buffer may take tile t + SB
       if (it.last) mbar_arrive(QFREE(qb));  // done with this segment's query data and score UMMAs
 
@@ -679,7 +709,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       for (int g = 0; g < kGroups; ++g) pass |= vsz[g].x > vmr[g];
       const bool raise = bar_any(bar_id, 128, pass);
       float alpha[HH];
-      if (raise) {
+      if (__builtin_expect(raise, 0)) {
         // the tile's largest score per head and largest value scale per group
         // (warp maxima, then the part's four warps through shared memory)
         int* rk = rmax + ((((t / S::NGRP) & 1) * S::NGRP + grp) * S::TPT + part) * 64;
@@ -710,19 +740,15 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         }
       }
 
-      // P' buffer k was read by the PV UMMAs of tile t - 2; the sums of tile
-      // t - RD (of this segment) are read back now, before the running max can
-      // move (the UMMAs of one thread complete in order, so PV t - 1 done
-      // implies PV t - 2 done)
-      if (t >= RD) {
+      if (!MERGED && t >= RD) {
         ok &= ws_wait(PVDONE((t - RD) & 1), ((t - RD) >> 1) & 1, err);
-        if (PLEN == 2 ? have2 : have1) {
+        if (rdp) {
           tc_fence_after();
-          read_pv(t - RD, PLEN == 2 ? ds2 : ds1);
+          read_pv(t, PLEN == 2 ? ds2 : ds1);  // tile t - RD, in PV buffer (t - RD) % DB = t % DB
           tc_fence_before();
         }
       }
-      if (raise) {
+      if (__builtin_expect(raise, 0)) {
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           l_acc[i] *= alpha[i];
@@ -783,13 +809,13 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       last_own = t;
       }  // own tile
 
-      if (it.last && seg_tiles == 0) {
+      if (__builtin_expect(it.last && seg_tiles == 0, 0)) {
         // no tile of this segment fell to this group: an empty partial (the combine skips it)
         const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
         if (j == 0)
 #pragma unroll
           for (int i = 0; i < HH; ++i) a.part_ml[(size_t)slot * G + part * HH + i] = make_float2(NEG_INF, 0.0f);
-      } else if (it.last) {
+      } else if (__builtin_expect(it.last, 0)) {
         // this group's pending PV sums of the segment, then its totals over the
         // tokens (max, sum, value zero-point terms) into its partial slot
         const int tl1 = last_own, tl2 = last_own - S::NGRP;  // its last tile, and the one before
@@ -892,6 +918,8 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       const int pw = warp - S::PROD_WARP;
       for (int t = 0; t < ntiles; ++t, it.next(a)) {
         if (t % S::NPROD != pw) continue;
+        // test hook: leave this tile's stage unfilled, so that the waits on it give up
+        if (blockIdx.x == 0 && t == a.withheld_tile) continue;
         const int s = t % ST;
         if (t >= ST) ws_wait(EMPTY(s), ((t / ST) - 1) & 1, err);
         const size_t bh = it.bh(a);
@@ -920,6 +948,14 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
   }
   tc_fence_before();
   __syncthreads();
+  if (*err) {
+    // a wait gave up: copies and MMAs issued before it may still be in flight;
+    // let them land (they take microseconds) before the tensor memory is freed
+    // and the CTA exits, and report the give-up to the host
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i) __nanosleep(1000);
+    if (tid == 0 && a.status) atomicOr(a.status, 1);
+  }
   if (warp == S::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, S::TMEM_COLS);

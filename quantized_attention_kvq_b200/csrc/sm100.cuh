@@ -325,6 +325,69 @@ __device__ __forceinline__ void tmem_ld_wait<24>(uint32_t taddr, uint32_t (&r)[2
       : "r"(taddr), "r"(taddr + 16)
       : "memory");
 }
+// Scores and PV sums of an epilogue tile in one round trip: four runs of
+// 2 HH columns at taddr + g * stride (g = 0..3) and one run of 4 HH columns at
+// paddr, then one wait for all of them.
+template <int HH>
+__device__ __forceinline__ void tmem_ld_sc_pv(uint32_t taddr, uint32_t stride, uint32_t paddr, uint32_t (&s)[4][2 * HH],
+                                              uint32_t (&p)[4 * HH]);
+template <>
+__device__ __forceinline__ void tmem_ld_sc_pv<1>(uint32_t taddr, uint32_t stride, uint32_t paddr,
+                                                   uint32_t (&s)[4][2], uint32_t (&p)[4]) {
+  asm volatile(
+      "{\n\t.reg .b32 a;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%12];\n\t"
+      "mov.u32 a, %12;\n\t"
+      "add.u32 a, a, %13;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%2, %3}, [a];\n\t"
+      "add.u32 a, a, %13;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%4, %5}, [a];\n\t"
+      "add.u32 a, a, %13;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%6, %7}, [a];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [%14];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(s[0][0]), "=r"(s[0][1]), "=r"(s[1][0]), "=r"(s[1][1]), "=r"(s[2][0]), "=r"(s[2][1]), "=r"(s[3][0]), "=r"(s[3][1]), "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3])
+      : "r"(taddr), "r"(stride), "r"(paddr)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_sc_pv<2>(uint32_t taddr, uint32_t stride, uint32_t paddr,
+                                                   uint32_t (&s)[4][4], uint32_t (&p)[8]) {
+  asm volatile(
+      "{\n\t.reg .b32 a;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%24];\n\t"
+      "mov.u32 a, %24;\n\t"
+      "add.u32 a, a, %25;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [a];\n\t"
+      "add.u32 a, a, %25;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [a];\n\t"
+      "add.u32 a, a, %25;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%12, %13, %14, %15}, [a];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16, %17, %18, %19, %20, %21, %22, %23}, [%26];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(s[0][0]), "=r"(s[0][1]), "=r"(s[0][2]), "=r"(s[0][3]), "=r"(s[1][0]), "=r"(s[1][1]), "=r"(s[1][2]), "=r"(s[1][3]), "=r"(s[2][0]), "=r"(s[2][1]), "=r"(s[2][2]), "=r"(s[2][3]), "=r"(s[3][0]), "=r"(s[3][1]), "=r"(s[3][2]), "=r"(s[3][3]), "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3]), "=r"(p[4]), "=r"(p[5]), "=r"(p[6]), "=r"(p[7])
+      : "r"(taddr), "r"(stride), "r"(paddr)
+      : "memory");
+}
+template <>
+__device__ __forceinline__ void tmem_ld_sc_pv<4>(uint32_t taddr, uint32_t stride, uint32_t paddr,
+                                                   uint32_t (&s)[4][8], uint32_t (&p)[16]) {
+  asm volatile(
+      "{\n\t.reg .b32 a;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%48];\n\t"
+      "mov.u32 a, %48;\n\t"
+      "add.u32 a, a, %49;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [a];\n\t"
+      "add.u32 a, a, %49;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16, %17, %18, %19, %20, %21, %22, %23}, [a];\n\t"
+      "add.u32 a, a, %49;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%24, %25, %26, %27, %28, %29, %30, %31}, [a];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%50];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : "=r"(s[0][0]), "=r"(s[0][1]), "=r"(s[0][2]), "=r"(s[0][3]), "=r"(s[0][4]), "=r"(s[0][5]), "=r"(s[0][6]), "=r"(s[0][7]), "=r"(s[1][0]), "=r"(s[1][1]), "=r"(s[1][2]), "=r"(s[1][3]), "=r"(s[1][4]), "=r"(s[1][5]), "=r"(s[1][6]), "=r"(s[1][7]), "=r"(s[2][0]), "=r"(s[2][1]), "=r"(s[2][2]), "=r"(s[2][3]), "=r"(s[2][4]), "=r"(s[2][5]), "=r"(s[2][6]), "=r"(s[2][7]), "=r"(s[3][0]), "=r"(s[3][1]), "=r"(s[3][2]), "=r"(s[3][3]), "=r"(s[3][4]), "=r"(s[3][5]), "=r"(s[3][6]), "=r"(s[3][7]), "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3]), "=r"(p[4]), "=r"(p[5]), "=r"(p[6]), "=r"(p[7]), "=r"(p[8]), "=r"(p[9]), "=r"(p[10]), "=r"(p[11]), "=r"(p[12]), "=r"(p[13]), "=r"(p[14]), "=r"(p[15])
+      : "r"(taddr), "r"(stride), "r"(paddr)
+      : "memory");
+}
 // Four runs of N columns at taddr + k * stride (k = 0..3), one wait for all.
 template <int N>
 __device__ __forceinline__ void tmem_ld4_wait(uint32_t taddr, uint32_t stride, uint32_t (&r)[4][N]);

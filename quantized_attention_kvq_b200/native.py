@@ -14,14 +14,15 @@ import torch
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libkvq.so")
 
-KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA = range(6)
+KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA, KVQ_ERR_TIMEOUT = range(7)
 KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 
 # every exported symbol the header declares
 SYMBOLS = ("kvq_cache_sizes", "kvq_window_bytes", "kvq_quantize_append", "kvq_select_channels",
            "kvq_select_channels_at", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
            "kvq_decode_step_workspace_bytes",
-           "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_status_string")
+           "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_decode_status", "kvq_test_withhold_tile",
+           "kvq_status_string")
 
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -79,6 +80,10 @@ def lib():
         L.kvq_decode_step_host.restype = ctypes.c_int
         L.kvq_decode_attention_static.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _P, ctypes.c_float, _P, _P]
         L.kvq_decode_attention_static.restype = ctypes.c_int
+        L.kvq_decode_status.argtypes = [C, _I32, _P, ctypes.c_size_t, _P]
+        L.kvq_decode_status.restype = ctypes.c_int
+        L.kvq_test_withhold_tile.argtypes = [_I32]
+        L.kvq_test_withhold_tile.restype = None
         L.kvq_status_string.argtypes = [ctypes.c_int]
         L.kvq_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -264,6 +269,12 @@ class KVQCache:
         _check(lib().kvq_decode_combine(ctypes.byref(self.desc), q_heads, _dev_ptr(seq_lens), max_len,
                                         _dev_ptr(out), _dev_ptr(workspace), workspace.numel(), _stream(stream)),
                "kvq_decode_combine")
+
+    def decode_status(self, q_heads: int, workspace: torch.Tensor, stream=None) -> int:
+        """Status of the last split decode that used `workspace`: KVQ_OK or KVQ_ERR_TIMEOUT
+        (synchronizes the stream)."""
+        return lib().kvq_decode_status(ctypes.byref(self.desc), q_heads, _dev_ptr(workspace), workspace.numel(),
+                                       _stream(stream))
 
     def step_workspace_bytes(self, dtype: torch.dtype, q_heads: int, max_len: int) -> int:
         return lib().kvq_decode_step_workspace_bytes(ctypes.byref(self.desc), torch_dtype_code(dtype), q_heads,

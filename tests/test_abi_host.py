@@ -267,6 +267,19 @@ def test_decode_workspace_holds_one_partial_per_slot_and_head(L, B, H, G, max_le
 
 
 def test_status_strings(L):
-    for s in range(6):
+    for s in range(7):
         assert native.status_string(s)
     assert "workspace" in native.status_string(native.KVQ_ERR_WORKSPACE)
+    assert "gave up" in native.status_string(native.KVQ_ERR_TIMEOUT)
+
+
+def test_decode_status_argument_checks(L):
+    d = desc(cap=512)
+    need = L.kvq_decode_workspace_bytes(ctypes.byref(d), 8, 512)
+    assert need > 0
+    assert L.kvq_decode_status(None, 8, FAKE, need, None) == native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_status(ctypes.byref(d), 8, None, need, None) == native.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_status(ctypes.byref(d), 6, FAKE, need, None) == native.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_decode_status(ctypes.byref(d), 8, FAKE, need - 1, None) == native.KVQ_ERR_WORKSPACE
+    # the hook only arms the next split decode of this thread; clearing it is harmless
+    L.kvq_test_withhold_tile(-1)
