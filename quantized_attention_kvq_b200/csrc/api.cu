@@ -4,10 +4,22 @@
 #include <cmath>
 #include <cstdint>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "transform.cuh"
 
 namespace kvq {
 namespace {
+
+// One NVTX range per enqueueing ABI call (named after it), so that a
+// timeline profiler shows which call enqueued which kernels.  NVTX is
+// header-only and costs a branch when no tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr size_t kAlign = 256;
 
@@ -297,6 +309,7 @@ KVQ_API size_t kvq_window_bytes(const kvq_cache* c) {
 
 KVQ_API kvq_status kvq_quantize_append(const kvq_cache* c, const void* k_new, const void* v_new, kvq_dtype dtype,
                                        int32_t n_new, int32_t offset, void* stream) {
+  NvtxRange range("kvq_quantize_append");
   kvq_status st = check_cache(c);
   if (st != KVQ_OK) return st;
   if (!dtype_ok(dtype) || n_new < 0 || offset < 0) return KVQ_ERR_INVALID_ARG;
@@ -337,6 +350,7 @@ KVQ_API kvq_status kvq_quantize_append(const kvq_cache* c, const void* k_new, co
 KVQ_API kvq_status kvq_select_channels_at(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
                                           const int32_t* seq_lens, int32_t keep_groups, uint32_t* mask_out,
                                           void* stream) {
+  NvtxRange range("kvq_select_channels_at");
   kvq_status st = check_shape(c);
   if (st != KVQ_OK) return st;
   if ((st = check_heads(c, q_heads)) != KVQ_OK) return st;
@@ -364,6 +378,7 @@ KVQ_API kvq_status kvq_select_channels_at(const kvq_cache* c, const void* q, kvq
 
 KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
                                        int32_t keep_groups, uint32_t* mask_out, void* stream) {
+  NvtxRange range("kvq_select_channels");
   // bucket-relative RoPE needs the queries' positions: kvq_select_channels_at
   if (c && c->bucket_tokens != 0) return KVQ_ERR_INVALID_ARG;
   return kvq_select_channels_at(c, q, dtype, q_heads, nullptr, keep_groups, mask_out, stream);
@@ -371,6 +386,7 @@ KVQ_API kvq_status kvq_select_channels(const kvq_cache* c, const void* q, kvq_dt
 
 KVQ_API kvq_status kvq_decode_status(const kvq_cache* c, int32_t q_heads, const void* workspace,
                                      size_t workspace_bytes, void* stream) {
+  NvtxRange range("kvq_decode_status");
   if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK || !workspace || !aligned16(workspace))
     return KVQ_ERR_INVALID_ARG;
   if (!decode_g_supported(q_heads / c->kv_heads)) return KVQ_ERR_UNSUPPORTED;
@@ -397,6 +413,7 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_d
                                         const int32_t* seq_lens, int32_t max_len, const uint32_t* mask,
                                         float softmax_scale, float* out, void* workspace, size_t workspace_bytes,
                                         void* stream) {
+  NvtxRange range("kvq_decode_attention");
   kvq_status st = check_decode(c, q, dtype, q_heads, seq_lens, max_len, softmax_scale, out, workspace,
                                workspace_bytes, true);
   if (st != KVQ_OK) return st;
@@ -407,6 +424,7 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache* c, const void* q, kvq_d
 KVQ_API kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
                                        const int32_t* seq_lens, int32_t max_len, const uint32_t* mask,
                                        float softmax_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange range("kvq_decode_partials");
   kvq_status st = check_decode(c, q, dtype, q_heads, seq_lens, max_len, softmax_scale, workspace, workspace,
                                workspace_bytes, true);
   if (st != KVQ_OK) return st;
@@ -416,6 +434,7 @@ KVQ_API kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dt
 
 KVQ_API kvq_status kvq_decode_combine(const kvq_cache* c, int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
                                       float* out, const void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange range("kvq_decode_combine");
   kvq_status st = check_decode(c, nullptr, KVQ_F32, q_heads, seq_lens, max_len, 1.0f, out, workspace,
                                workspace_bytes, false);
   if (st != KVQ_OK) return st;
@@ -438,6 +457,7 @@ KVQ_API kvq_status kvq_decode_step_host(const kvq_cache* c, const void* q_host, 
                                         const int32_t* seq_lens, int32_t max_len, int32_t keep_groups,
                                         float softmax_scale, float* out_host, void* workspace,
                                         size_t workspace_bytes, void* stream) {
+  NvtxRange range("kvq_decode_step_host");
   kvq_status st = check_cache(c);
   if (st != KVQ_OK) return st;
   if ((st = check_heads(c, q_heads)) != KVQ_OK) return st;

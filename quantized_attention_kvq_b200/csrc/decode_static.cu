@@ -13,6 +13,7 @@
 // use the symbol's name as a device address; the address is looked up once
 // per device with cudaGetSymbolAddress, with that device current, on the
 // first call made on it.
+#include <nvtx3/nvToolsExt.h>
 #include <mutex>
 
 #include "common.cuh"
@@ -49,6 +50,10 @@ extern "C" KVQ_API kvq_status kvq_decode_attention_static(const kvq_cache* cache
                                                           int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
                                                           const uint32_t* mask, float softmax_scale, float* out,
                                                           void* stream) {
+  struct Range {  // NVTX range named after the call (header-only; a branch when no tool is attached)
+    Range() { nvtxRangePushA("kvq_decode_attention_static"); }
+    ~Range() { nvtxRangePop(); }
+  } range;
   void* scratch = nullptr;
   kvq_status st = kvq::scratch_for_current_device(&scratch);
   if (st != KVQ_OK) return st;
