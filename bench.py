@@ -420,13 +420,15 @@ def run_kvq(args):
         flush.zero_()
         if ev is not None:
             ev[0].record(stream)
-        if keep < 32 and wl.bucket:
-            cache.select_at(qd, lens, keep, mask)
-        elif keep < 32:
+        if keep < 32 and not wl.bucket:
             cache.select(qd, keep, mask)
         if ev is not None:
             ev[1].record(stream)
-        cache.decode_partials(qd, lens, max_len, mask if keep < 32 else None, scale, ws)
+        if keep < 32 and wl.bucket:
+            # the selection runs inside the split half, on the bucket query rows it prepares
+            cache.decode_partials_select(qd, lens, max_len, keep, scale, ws)
+        else:
+            cache.decode_partials(qd, lens, max_len, mask if keep < 32 else None, scale, ws)
         if ev is not None:
             ev[2].record(stream)
         cache.decode_combine(wl.Hq, lens, max_len, out, ws)
@@ -435,6 +437,8 @@ def run_kvq(args):
 
     for _ in range(max(args.warmup, 3)):
         step()
+    if keep < 32 and wl.bucket:
+        cache.select_at(qd, lens, keep, mask)  # the same masks, for the byte count
     torch.cuda.synchronize()
     masks_np = mask.cpu().numpy().view(np.uint32) if keep < 32 else np.full(tuple(mask.shape), 0xFFFFFFFF, np.uint32)
     abytes = algorithmic_bytes(wl, masks_np, lens_np)
@@ -554,8 +558,11 @@ def run_append(args):
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
     kd, vd = up(s.k_full()), up(s.v_full())
+    tq, tk, _ = option_inputs(wl, rep.seed(wl))
     cache = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, device=dev,
-                            rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent)
+                            rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent,
+                            t_query=None if tq is None else torch.from_numpy(tq).to(dev),
+                            t_key=None if tk is None else torch.from_numpy(tk).to(dev))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()

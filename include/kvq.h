@@ -284,6 +284,28 @@ KVQ_API kvq_status kvq_decode_combine(const kvq_cache* cache, int32_t q_heads, c
                                       void* stream);
 
 /*
+ * kvq_decode_attention with the query-channel selection of
+ * kvq_select_channels (kvq_select_channels_at with bucket-relative RoPE) done
+ * inside the call, keeping `keep_groups` (1..32) channel groups per (sequence,
+ * kv head) [DQK Sec. 3.2, App. C.2].  The selection reads the query rows the
+ * decode prepares anyway: with bucket-relative RoPE each bucket's embedded and
+ * transformed rows, with the caller's pair the transformed rows, so they are
+ * computed once.  Masks and outputs are those of the two calls in sequence.
+ * The masks stay in `workspace` (kvq_decode_workspace_bytes covers them).
+ * keep_groups outside 1..32: KVQ_ERR_INVALID_ARG; the other rules are those of
+ * kvq_decode_attention.  kvq_decode_partials_select is its split half (its
+ * partials are combined by kvq_decode_combine).
+ */
+KVQ_API kvq_status kvq_decode_attention_select(const kvq_cache* cache, const void* q, kvq_dtype dtype,
+                                               int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
+                                               int32_t keep_groups, float softmax_scale, float* out,
+                                               void* workspace, size_t workspace_bytes, void* stream);
+KVQ_API kvq_status kvq_decode_partials_select(const kvq_cache* cache, const void* q, kvq_dtype dtype,
+                                              int32_t q_heads, const int32_t* seq_lens, int32_t max_len,
+                                              int32_t keep_groups, float softmax_scale, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
+/*
  * kvq_decode_attention without a workspace argument, for callers that cannot
  * allocate device memory: an engine that owns every byte of device memory in
  * its own pool and has no allocator to lend across this C boundary, or a

@@ -136,7 +136,7 @@ CacheView bucket_sequence_view(const kvq_cache* c, size_t vb) {
 // max and sum) per (slot, query head of the GQA group), decode_slots slots;
 // with the caller's transform pair, then the transformed fp32 query rows.
 struct DecodePlan {
-  size_t acc_bytes, ml_offset, tq_offset, qb_offset, vl_offset, status_offset, bytes;
+  size_t acc_bytes, ml_offset, tq_offset, qb_offset, vl_offset, mask_offset, status_offset, bytes;
 };
 
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
@@ -155,6 +155,9 @@ DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   if (c->bucket_tokens > 0) p.bytes += round_up((size_t)Bv * q_heads * kHeadDim * sizeof(float), kAlign);
   p.vl_offset = p.bytes;
   if (c->bucket_tokens > 0) p.bytes += round_up((size_t)Bv * sizeof(int32_t), kAlign);
+  // the kept-group masks of a decode that selects channels itself
+  p.mask_offset = p.bytes;
+  p.bytes += round_up((size_t)Bv * c->kv_heads * sizeof(uint32_t), kAlign);
   // the split decode's status word (a wait gave up), cleared by each split
   p.status_offset = p.bytes;
   p.bytes += kAlign;
@@ -174,10 +177,30 @@ kvq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_E
 // which halves of the decode to enqueue
 enum { kRunSplit = 1, kRunCombine = 2 };
 
+// The kept-group masks of a decode that selects its channels itself, from the
+// query rows the decode prepares anyway: rows already transformed (fp32, no
+// further rotation) when `rows` is not NULL, else the caller's queries.
+kvq_status enqueue_select(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads, int32_t B,
+                          const float* rows, int32_t keep_groups, uint32_t* mask, cudaStream_t s) {
+  SelectArgs a;
+  a.q = rows ? static_cast<const void*>(rows) : q;
+  a.dtype = rows ? KVQ_F32 : dtype;
+  a.B = B;
+  a.Hq = q_heads;
+  a.H = c->kv_heads;
+  a.rotate = rows ? 0 : c->rotate_k;
+  a.keep = keep_groups;
+  a.inv_sqrt_d = inv_sqrt_d();
+  a.mask = mask;
+  return cuda_status(launch_select_pair(a, rows ? nullptr : c->t_query, s));
+}
+
 kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
                           const int32_t* seq_lens, int32_t max_len, const uint32_t* mask, float softmax_scale,
                           float* out, void* workspace, const DecodePlan& plan, cudaStream_t s,
-                          int parts = kRunSplit | kRunCombine) {
+                          int parts = kRunSplit | kRunCombine, int32_t keep_groups = kPruneGroups) {
+  uint32_t* own_mask = reinterpret_cast<uint32_t*>(static_cast<char*>(workspace) + plan.mask_offset);
+  const bool select = keep_groups < kPruneGroups;
   if (c->bucket_tokens > 0) {
     // every bucket is a sequence of the split decode, with its own query and
     // length; the merge makes one softmax of them
@@ -211,6 +234,13 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
           c->bucket_tokens, nb, inv_sqrt_d(), reinterpret_cast<float*>(ws + plan.qb_offset),
           reinterpret_cast<int32_t*>(ws + plan.vl_offset), s));
       if (st != KVQ_OK) return st;
+      if (select) {
+        // every bucket's query rows are embedded and transformed already
+        st = enqueue_select(c, nullptr, KVQ_F32, q_heads, v.c.B, reinterpret_cast<const float*>(ws + plan.qb_offset),
+                            keep_groups, own_mask, s);
+        if (st != KVQ_OK) return st;
+        v.mask = own_mask;
+      }
       if (v.max_len > 0 && (st = cuda_status(launch_decode(v, s))) != KVQ_OK) return st;
     }
     if (parts & kRunCombine)
@@ -246,6 +276,12 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
     a.q = qt;
     a.dtype = KVQ_F32;
     a.c.rotate = 0;
+  }
+  if ((parts & kRunSplit) && select) {
+    kvq_status st = enqueue_select(c, q, dtype, q_heads, c->batch,
+                                   c->rotate_k == 2 ? static_cast<const float*>(a.q) : nullptr, keep_groups, own_mask, s);
+    if (st != KVQ_OK) return st;
+    a.mask = own_mask;
   }
   if ((parts & kRunSplit) && max_len > 0) {
     kvq_status st = cuda_status(launch_decode(a, s));
@@ -430,6 +466,33 @@ KVQ_API kvq_status kvq_decode_partials(const kvq_cache* c, const void* q, kvq_dt
   if (st != KVQ_OK) return st;
   return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, mask, softmax_scale, nullptr, workspace,
                         plan_decode(c, q_heads), static_cast<cudaStream_t>(stream), kRunSplit);
+}
+
+KVQ_API kvq_status kvq_decode_attention_select(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                               const int32_t* seq_lens, int32_t max_len, int32_t keep_groups,
+                                               float softmax_scale, float* out, void* workspace,
+                                               size_t workspace_bytes, void* stream) {
+  NvtxRange range("kvq_decode_attention_select");
+  kvq_status st = check_decode(c, q, dtype, q_heads, seq_lens, max_len, softmax_scale, out, workspace,
+                               workspace_bytes, true);
+  if (st != KVQ_OK) return st;
+  if (keep_groups < 1 || keep_groups > kPruneGroups) return KVQ_ERR_INVALID_ARG;
+  return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, nullptr, softmax_scale, out, workspace,
+                        plan_decode(c, q_heads), static_cast<cudaStream_t>(stream), kRunSplit | kRunCombine,
+                        keep_groups);
+}
+
+KVQ_API kvq_status kvq_decode_partials_select(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
+                                              const int32_t* seq_lens, int32_t max_len, int32_t keep_groups,
+                                              float softmax_scale, void* workspace, size_t workspace_bytes,
+                                              void* stream) {
+  NvtxRange range("kvq_decode_partials_select");
+  kvq_status st = check_decode(c, q, dtype, q_heads, seq_lens, max_len, softmax_scale, workspace, workspace,
+                               workspace_bytes, true);
+  if (st != KVQ_OK) return st;
+  if (keep_groups < 1 || keep_groups > kPruneGroups) return KVQ_ERR_INVALID_ARG;
+  return enqueue_decode(c, q, dtype, q_heads, seq_lens, max_len, nullptr, softmax_scale, nullptr, workspace,
+                        plan_decode(c, q_heads), static_cast<cudaStream_t>(stream), kRunSplit, keep_groups);
 }
 
 KVQ_API kvq_status kvq_decode_combine(const kvq_cache* c, int32_t q_heads, const int32_t* seq_lens, int32_t max_len,

@@ -52,13 +52,13 @@ __global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb,
   const int G = v.Hq / v.c.H;
   const int h = hq / G, hl = hq - h * G;
   const int chn = threadIdx.x;
-  int total = 0;
-  for (int vb = 0; vb < v.c.B; ++vb) total += v.c.H * bucket_tiles(v, vb);
+  // tiles of the whole bucket batch and of the buckets before sequence b
+  // (block-wide sums, each thread taking every 128th bucket sequence)
+  const int2 tp = block_tile_prefix(v.c.B, b * nb, v.c.H, [&](int vb) { return bucket_tiles(v, vb); });
+  const int total = tp.x, tb = tp.y;
   const int per = (total + ctas - 1) / ctas;
   const float NEG_INF = -__int_as_float(0x7f800000);
   float M = NEG_INF;
-  int tb = 0;
-  for (int vb = 0; vb < b * nb; ++vb) tb += v.c.H * bucket_tiles(v, vb);
   {
     int t0 = tb;
     for (int k = 0; k < nb; ++k) {

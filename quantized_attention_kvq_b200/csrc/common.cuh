@@ -81,6 +81,34 @@ __device__ __forceinline__ float warp_max(float v) {
   for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
   return v;
 }
+// Tile counts over sequences [0, n) of a batch, by a 128-thread block:
+// thread t takes sequences t, t + 128, ...; returns (sum over all, sum over
+// sequences < before), each times `mult`, in every thread.
+template <typename TilesOf>
+__device__ __forceinline__ int2 block_tile_prefix(int n, int before, int mult, TilesOf tiles_of_seq) {
+  __shared__ int red[2][4];
+  int all = 0, pre = 0;
+  for (int i = threadIdx.x; i < n; i += 128) {
+    const int t = tiles_of_seq(i);
+    all += t;
+    if (i < before) pre += t;
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) {
+    all += __shfl_xor_sync(0xFFFFFFFFu, all, m);
+    pre += __shfl_xor_sync(0xFFFFFFFFu, pre, m);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = all;
+    red[1][threadIdx.x >> 5] = pre;
+  }
+  __syncthreads();
+  const int2 r = make_int2(mult * (red[0][0] + red[0][1] + red[0][2] + red[0][3]),
+                           mult * (red[1][0] + red[1][1] + red[1][2] + red[1][3]));
+  __syncthreads();
+  return r;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(kFull, v, m);

@@ -970,11 +970,9 @@ __global__ void __launch_bounds__(kHeadDim) k_combine(DecodeArgs a, int G, int n
   const int b = row / a.Hq, hq = row - b * a.Hq;
   const int h = hq / G, hl = hq - h * G;
   const int chn = threadIdx.x;
-  int total = 0, tb = 0;
-  for (int bb = 0; bb < a.c.B; ++bb) {
-    if (bb == b) tb = total;
-    total += a.c.H * tiles_of(a, bb);
-  }
+  // tiles of the whole batch and of the sequences before b (block-wide sums)
+  const int2 tp = block_tile_prefix(a.c.B, b, a.c.H, [&](int bb) { return tiles_of(a, bb); });
+  const int total = tp.x, tb = tp.y;
   const int nt = tiles_of(a, b);
   float out = 0.0f;
   if (nt > 0) {

@@ -21,7 +21,8 @@ KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
 SYMBOLS = ("kvq_cache_sizes", "kvq_window_bytes", "kvq_quantize_append", "kvq_select_channels",
            "kvq_select_channels_at", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
            "kvq_decode_step_workspace_bytes",
-           "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_decode_status", "kvq_test_withhold_tile",
+           "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_decode_attention_select",
+           "kvq_decode_partials_select", "kvq_decode_status", "kvq_test_withhold_tile",
            "kvq_status_string")
 
 _P = ctypes.c_void_p
@@ -80,6 +81,12 @@ def lib():
         L.kvq_decode_step_host.restype = ctypes.c_int
         L.kvq_decode_attention_static.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _P, ctypes.c_float, _P, _P]
         L.kvq_decode_attention_static.restype = ctypes.c_int
+        L.kvq_decode_attention_select.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _I32, ctypes.c_float, _P,
+                                                  _P, ctypes.c_size_t, _P]
+        L.kvq_decode_attention_select.restype = ctypes.c_int
+        L.kvq_decode_partials_select.argtypes = [C, _P, ctypes.c_int, _I32, _P, _I32, _I32, ctypes.c_float, _P,
+                                                 ctypes.c_size_t, _P]
+        L.kvq_decode_partials_select.restype = ctypes.c_int
         L.kvq_decode_status.argtypes = [C, _I32, _P, ctypes.c_size_t, _P]
         L.kvq_decode_status.restype = ctypes.c_int
         L.kvq_test_withhold_tile.argtypes = [_I32]
@@ -263,6 +270,32 @@ class KVQCache:
                                          _dev_ptr(seq_lens), max_len, _dev_ptr(mask), float(softmax_scale),
                                          _dev_ptr(workspace), workspace.numel(), _stream(stream)),
                "kvq_decode_partials")
+
+    def decode_select(self, q: torch.Tensor, seq_lens: torch.Tensor, max_len: int, keep_groups: int,
+                      softmax_scale: float | None = None, out: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """decode() with the channel selection done inside the call (kvq_decode_attention_select)."""
+        Hq = q.shape[1]
+        if softmax_scale is None:
+            softmax_scale = 1.0 / math.sqrt(128)
+        if out is None:
+            out = torch.empty((self.B, Hq, 128), dtype=torch.float32, device=q.device)
+        if workspace is None:
+            workspace = torch.empty(max(self.workspace_bytes(Hq, max_len), 256), dtype=torch.uint8, device=q.device)
+        _check(lib().kvq_decode_attention_select(ctypes.byref(self.desc), _dev_ptr(q), torch_dtype_code(q.dtype), Hq,
+                                                 _dev_ptr(seq_lens), max_len, keep_groups, float(softmax_scale),
+                                                 _dev_ptr(out), _dev_ptr(workspace), workspace.numel(),
+                                                 _stream(stream)),
+               "kvq_decode_attention_select")
+        return out
+
+    def decode_partials_select(self, q: torch.Tensor, seq_lens: torch.Tensor, max_len: int, keep_groups: int,
+                               softmax_scale: float, workspace: torch.Tensor, stream=None):
+        _check(lib().kvq_decode_partials_select(ctypes.byref(self.desc), _dev_ptr(q), torch_dtype_code(q.dtype),
+                                                q.shape[1], _dev_ptr(seq_lens), max_len, keep_groups,
+                                                float(softmax_scale), _dev_ptr(workspace), workspace.numel(),
+                                                _stream(stream)),
+               "kvq_decode_partials_select")
 
     def decode_combine(self, q_heads: int, seq_lens: torch.Tensor, max_len: int, out: torch.Tensor,
                        workspace: torch.Tensor, stream=None):

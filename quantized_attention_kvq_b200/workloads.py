@@ -60,6 +60,10 @@ WORKLOADS = [
     # combined with buckets on the CUDA path
     Workload(8, "dualqk_int2_pair_bucket2048_vrot_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16",
              2, 2, 2, 1, 19, rotate_v=1, v_clip=0.92, bucket=2048),
+    # the append through a caller-supplied dual transform pair (Dual-QK Sec. 3.1):
+    # each key row taken through its kv head's 128 x 128 key matrix
+    Workload(9, "append_pair_b16_h8_t4096_at8192", 16, 8, 8, 128, 4096, 12288, 8192, "bf16", 4, 2, 2, 0, 32,
+             kind="append"),
 ]
 
 BASE_SEED = 0
