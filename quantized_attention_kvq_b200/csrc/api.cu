@@ -3,6 +3,7 @@
 // leaves this file.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -195,6 +196,47 @@ kvq_status enqueue_select(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   return cuda_status(launch_select_pair(a, rows ? nullptr : c->t_query, s));
 }
 
+// Per device: a non-blocking side stream and two events for forking the
+// window kernel off the caller's stream (created on first use, never freed).
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+SideStream g_side[kMaxSideDevices];
+std::mutex g_side_mutex;
+
+kvq_status side_stream(SideStream** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return KVQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_side_mutex);
+  SideStream& ss = g_side[dev];
+  if (!ss.stream) {
+    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return KVQ_ERR_CUDA;
+  }
+  *out = &ss;
+  return KVQ_OK;
+}
+
+// The window attention on the side stream: after everything enqueued on s so
+// far, and before everything enqueued on s afterwards.  One fork at a time
+// per device (the events are reused), which the mutex above orders.
+kvq_status fork_window(const DecodeArgs& a, cudaStream_t s) {
+  SideStream* ss = nullptr;
+  kvq_status st = side_stream(&ss);
+  if (st != KVQ_OK) return st;
+  std::lock_guard<std::mutex> lock(g_side_mutex);
+  if (cudaEventRecord(ss->fork, s) != cudaSuccess || cudaStreamWaitEvent(ss->stream, ss->fork, 0) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  if ((st = cuda_status(launch_window(a, ss->stream))) != KVQ_OK) return st;
+  if (cudaEventRecord(ss->join, ss->stream) != cudaSuccess || cudaStreamWaitEvent(s, ss->join, 0) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
 kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, int32_t q_heads,
                           const int32_t* seq_lens, int32_t max_len, const uint32_t* mask, float softmax_scale,
                           float* out, void* workspace, const DecodePlan& plan, cudaStream_t s,
@@ -288,7 +330,10 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
     if (st != KVQ_OK) return st;
   }
   if ((parts & kRunSplit) && c->sink_tokens + c->recent_tokens > 0) {
-    kvq_status st = cuda_status(launch_window(a, s));
+    // the bf16 window attention is independent of the split decode: it runs on
+    // a side stream forked after the split, so its CTAs take SMs as the split's
+    // CTAs finish, and joins before the combine
+    kvq_status st = fork_window(a, s);
     if (st != KVQ_OK) return st;
   }
   if (parts & kRunCombine) return cuda_status(launch_combine(a, s));

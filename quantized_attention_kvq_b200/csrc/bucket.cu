@@ -12,6 +12,8 @@ namespace {
 
 constexpr int kBucketWarps = 4;
 constexpr int kDecodeTile = 128;  // tokens per tile of the split decode
+constexpr int kMergeSlots = 1024;  // slots listed at once by the merge (a chunk of 128 buckets needs fewer)
+constexpr int kMergeBatch = 16;   // slots whose loads the merge issues together
 
 template <typename In>
 __global__ void __launch_bounds__(kBucketWarps * 32)
@@ -45,50 +47,142 @@ __device__ __forceinline__ int bucket_tiles(const DecodeArgs& v, int vb) {
 // (u + c) * ngrp + e for each of its ngrp epilogue groups e, row slot * G +
 // the head's index in its group; an empty one has max -inf.  Maxima and sums
 // are in the log2 domain of the decode.
+//
+// The sequence's buckets are taken 128 at a time, thread k taking bucket k
+// of the chunk: its tile count, then (block scan) its first tile, then its
+// first and last slot and the max over them.  With the maximum of the whole
+// sequence known, every thread walks the chunk's slot ranges from shared
+// memory, so its loads do not wait on one another.
 __global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb, int ctas, int ngrp,
                                                            float* __restrict__ out) {
   const int row = blockIdx.x;  // b * Hq + query head
   const int b = row / v.Hq, hq = row - b * v.Hq;
   const int G = v.Hq / v.c.H;
   const int h = hq / G, hl = hq - h * G;
-  const int chn = threadIdx.x;
+  const int chn = threadIdx.x, lane = chn & 31, warp = chn >> 5;
   // tiles of the whole bucket batch and of the buckets before sequence b
   // (block-wide sums, each thread taking every 128th bucket sequence)
   const int2 tp = block_tile_prefix(v.c.B, b * nb, v.c.H, [&](int vb) { return bucket_tiles(v, vb); });
-  const int total = tp.x, tb = tp.y;
+  const int total = tp.x;
   const int per = (total + ctas - 1) / ctas;
   const float NEG_INF = -__int_as_float(0x7f800000);
+  __shared__ int s_first[kHeadDim], s_last[kHeadDim];  // slot range of each bucket of the chunk
+  __shared__ int s_scan[4];
+  __shared__ float s_max[4];
+
+  // pass 1: the maximum over every slot of the sequence
   float M = NEG_INF;
-  {
-    int t0 = tb;
-    for (int k = 0; k < nb; ++k) {
-      const int vb = b * nb + k, nt = bucket_tiles(v, vb);
-      if (nt > 0) {
-        const int u = vb * v.c.H + h, tu = t0 + h * nt;
-        for (int sl = (u + tu / per) * ngrp; sl < (u + (tu + nt - 1) / per + 1) * ngrp; ++sl)
-          M = fmaxf(M, v.part_ml[(size_t)sl * G + hl].x);
-      }
-      t0 += v.c.H * nt;
+  int t0 = tp.y;  // first tile of the chunk's first bucket sequence (its kv head 0 unit)
+  for (int k0 = 0; k0 < nb; k0 += kHeadDim) {
+    const int k = k0 + chn;
+    const int vb = b * nb + k;
+    const int nt = k < nb ? bucket_tiles(v, vb) : 0;
+    // exclusive scan of H * nt over the chunk
+    int x = v.c.H * nt;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, m);
+      if (lane >= m) x += y;
     }
+    if (lane == 31) s_scan[warp] = x;
+    __syncthreads();
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += s_scan[w];
+    const int incl = x + before;
+    const int chunk_sum = s_scan[0] + s_scan[1] + s_scan[2] + s_scan[3];
+    const int tk = t0 + incl - v.c.H * nt;  // first tile of bucket sequence vb
+    int f = 0, l = -1;
+    float mk = NEG_INF;
+    if (nt > 0) {
+      const int u = vb * v.c.H + h, tu = tk + h * nt;
+      f = (u + tu / per) * ngrp;
+      l = (u + (tu + nt - 1) / per + 1) * ngrp - 1;
+      for (int sl = f; sl <= l; ++sl) mk = fmaxf(mk, v.part_ml[(size_t)sl * G + hl].x);
+    }
+    s_first[chn] = f;
+    s_last[chn] = l;
+    mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, 16));
+    mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, 8));
+    mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, 4));
+    mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, 2));
+    mk = fmaxf(mk, __shfl_xor_sync(kFull, mk, 1));
+    if (lane == 0) s_max[warp] = mk;
+    __syncthreads();
+    M = fmaxf(M, fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3])));
+    t0 += chunk_sum;
   }
+  // pass 2: every slot's weight 2^(m - M), its sum and its channel.  A
+  // chunk's slots are listed in shared memory first (at most 2 per CTA range
+  // end per bucket plus one per `per` tiles, so under 1024), then walked
+  // kMergeBatch at a time with their loads issued together.
+  __shared__ int s_slot[kMergeSlots];
   float l = 0.0f, o = 0.0f;
-  {
-    int t0 = tb;
-    for (int k = 0; k < nb; ++k) {
-      const int vb = b * nb + k, nt = bucket_tiles(v, vb);
-      if (nt > 0) {
-        const int u = vb * v.c.H + h, tu = t0 + h * nt;
-        for (int sl = (u + tu / per) * ngrp; sl < (u + (tu + nt - 1) / per + 1) * ngrp; ++sl) {
-          const size_t r = (size_t)sl * G + hl;
-          const float2 ml = v.part_ml[r];
-          if (ml.x == NEG_INF) continue;
-          const float e = exp2f(ml.x - M);
-          l = fmaf(e, ml.y, l);
-          o = fmaf(e, v.part_acc[r * kHeadDim + chn], o);
-        }
+  const int nchunks = (nb + kHeadDim - 1) / kHeadDim;
+  t0 = tp.y;
+  for (int c = 0; c < nchunks; ++c) {
+    const int k = c * kHeadDim + chn;
+    const int vb = b * nb + k;
+    int f = 0, ll = -1;
+    if (nchunks > 1) {
+      // this chunk's slot ranges again (pass 1 kept only the last chunk's)
+      const int nt = k < nb ? bucket_tiles(v, vb) : 0;
+      int x = v.c.H * nt;
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, m);
+        if (lane >= m) x += y;
       }
-      t0 += v.c.H * nt;
+      __syncthreads();
+      if (lane == 31) s_scan[warp] = x;
+      __syncthreads();
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += s_scan[w];
+      const int tk = t0 + x + before - v.c.H * nt;
+      t0 += s_scan[0] + s_scan[1] + s_scan[2] + s_scan[3];
+      if (nt > 0) {
+        const int u = vb * v.c.H + h, tu = tk + h * nt;
+        f = (u + tu / per) * ngrp;
+        ll = (u + (tu + nt - 1) / per + 1) * ngrp - 1;
+      }
+    } else {
+      f = s_first[chn];
+      ll = s_last[chn];
     }
+    // list the chunk's slots: exclusive scan of the per-bucket counts
+    const int cnt = ll - f + 1;
+    int x = cnt;
+#pragma unroll
+    for (int m = 1; m < 32; m <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, m);
+      if (lane >= m) x += y;
+    }
+    __syncthreads();
+    if (lane == 31) s_scan[warp] = x;
+    __syncthreads();
+    int base = x - cnt;
+    for (int w = 0; w < warp; ++w) base += s_scan[w];
+    const int n = min(s_scan[0] + s_scan[1] + s_scan[2] + s_scan[3], kMergeSlots);
+    for (int i = 0; i < cnt && base + i < kMergeSlots; ++i) s_slot[base + i] = f + i;
+    __syncthreads();
+    for (int i0 = 0; i0 < n; i0 += kMergeBatch) {
+      float2 ml[kMergeBatch];
+      float ac[kMergeBatch];
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const int i = min(i0 + j, n - 1);
+        const size_t r = (size_t)s_slot[i] * G + hl;
+        ml[j] = v.part_ml[r];
+        ac[j] = v.part_acc[r * kHeadDim + chn];  // an empty slot's is not used
+      }
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const bool use = i0 + j < n && ml[j].x != NEG_INF;
+        const float e = use ? exp2f(ml[j].x - M) : 0.0f;
+        l = fmaf(e, use ? ml[j].y : 0.0f, l);
+        o = use ? fmaf(e, ac[j], o) : o;
+      }
+    }
+    __syncthreads();
   }
   float res = l > 0.0f ? o / l : 0.0f;
   if (v.c.rotate_v) {
