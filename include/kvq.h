@@ -228,6 +228,16 @@ KVQ_API kvq_status kvq_decode_status(const kvq_cache* cache, int32_t q_heads, co
  */
 KVQ_API void kvq_test_withhold_tile(int32_t tile);
 
+/*
+ * Bounds-checked debug build (libkvq_checked.so, compiled with
+ * -DKVQ_BOUNDS_CHECK): the kernels compare the range of every cache-array,
+ * partial and window access they check with the array's extent, skip an
+ * access out of bounds and count it.  This call synchronizes the device and
+ * returns the count since the last reset (clearing it when `reset` is not
+ * 0); in the regular library it returns UINT32_MAX (no checks compiled in).
+ */
+KVQ_API uint32_t kvq_bounds_violations(int32_t reset);
+
 /* Device workspace bytes kvq_decode_attention needs for these sizes (0 on bad arguments). */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* cache, int32_t q_heads, int32_t max_len);
 

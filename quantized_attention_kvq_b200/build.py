@@ -1,6 +1,9 @@
 """Build the package's native libraries in-tree.
 
 * ``lib/libkvq.so``    -- the C-ABI library (CUDA, sm_100a only), from ``csrc/*.cu``.
+* ``lib/libkvq_checked.so`` -- the same with -DKVQ_BOUNDS_CHECK: every checked
+  cache, partial and window access compares its range with the array's extent,
+  skips and counts an access out of bounds (``kvq_bounds_violations``).
 * ``lib/libkvqgen.so`` -- the seeded input generator (plain C + OpenMP).
 
 The quantizer inside libkvq relies on IEEE-rounded fp32 subtract/divide and
@@ -43,19 +46,21 @@ def build_gen(force: bool = False) -> str:
     return so
 
 
-def build_kvq(force: bool = False, verbose_ptxas: bool = False) -> str:
+def build_kvq(force: bool = False, verbose_ptxas: bool = False, checked: bool = False) -> str:
     os.makedirs(LIB_DIR, exist_ok=True)
-    os.makedirs(BUILD_DIR, exist_ok=True)
-    so = os.path.join(LIB_DIR, "libkvq.so")
+    build_dir = BUILD_DIR + ("_checked" if checked else "")
+    os.makedirs(build_dir, exist_ok=True)
+    so = os.path.join(LIB_DIR, "libkvq_checked.so" if checked else "libkvq.so")
+    extra = ["-DKVQ_BOUNDS_CHECK"] if checked else []
     cus = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h")))
     objs = []
     jobs = []
     for cu in cus:
-        obj = os.path.join(BUILD_DIR, os.path.basename(cu) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(cu) + ".o")
         objs.append(obj)
         if force or _newer(obj, [cu] + hdrs):
-            cmd = [NVCC, *ARCH, *NVCC_FLAGS, "-c", cu, "-o", obj]
+            cmd = [NVCC, *ARCH, *NVCC_FLAGS, *extra, "-c", cu, "-o", obj]
             if verbose_ptxas:
                 cmd[1:1] = ["-Xptxas", "-v"]
             jobs.append(cmd)
@@ -72,6 +77,7 @@ def build_kvq(force: bool = False, verbose_ptxas: bool = False) -> str:
 def build_all(force: bool = False) -> None:
     build_gen(force)
     build_kvq(force)
+    build_kvq(force, checked=True)
 
 
 if __name__ == "__main__":

@@ -137,7 +137,7 @@ CacheView bucket_sequence_view(const kvq_cache* c, size_t vb) {
 // max and sum) per (slot, query head of the GQA group), decode_slots slots;
 // with the caller's transform pair, then the transformed fp32 query rows.
 struct DecodePlan {
-  size_t acc_bytes, ml_offset, tq_offset, qb_offset, vl_offset, mask_offset, status_offset, bytes;
+  size_t rows, acc_bytes, ml_offset, tq_offset, qb_offset, vl_offset, mask_offset, status_offset, bytes;
 };
 
 DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
@@ -146,6 +146,7 @@ DecodePlan plan_decode(const kvq_cache* c, int32_t q_heads) {
   const bool win = c->sink_tokens + c->recent_tokens > 0;  // one more partial per unit for the windows
   const int Bv = c->batch * n_buckets(c);  // the split decode runs over every bucket as a sequence
   const size_t rows = ((size_t)decode_slots(Bv, c->kv_heads, G) + (win ? c->batch * c->kv_heads : 0)) * G;
+  p.rows = rows;
   p.acc_bytes = rows * kHeadDim * sizeof(float);
   p.ml_offset = round_up(p.acc_bytes, kAlign);
   p.tq_offset = p.ml_offset + round_up(rows * sizeof(float2), kAlign);
@@ -265,6 +266,7 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
     v.part_acc = reinterpret_cast<float*>(ws);
     v.part_ml = reinterpret_cast<float2*>(ws + plan.ml_offset);
     v.out = nullptr;
+    v.part_rows = plan.rows;
     v.status = reinterpret_cast<int*>(ws + plan.status_offset);
     v.withheld_tile = -1;
     if (parts & kRunSplit) {
@@ -303,6 +305,7 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.part_acc = static_cast<float*>(workspace);
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
+  a.part_rows = plan.rows;
   a.status = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan.status_offset);
   a.withheld_tile = -1;
   if (parts & kRunSplit) {
@@ -483,6 +486,17 @@ KVQ_API kvq_status kvq_decode_status(const kvq_cache* c, int32_t q_heads, const 
 }
 
 KVQ_API void kvq_test_withhold_tile(int32_t tile) { kvq::g_withheld_tile = tile < 0 ? -1 : tile; }
+
+KVQ_API uint32_t kvq_bounds_violations(int32_t reset) {
+#ifdef KVQ_BOUNDS_CHECK
+  if (cudaDeviceSynchronize() != cudaSuccess) return UINT32_MAX;
+  const bool r = reset != 0;
+  return kvq::bounds_append(r) + kvq::bounds_decode(r) + kvq::bounds_window(r);
+#else
+  (void)reset;
+  return UINT32_MAX;  // this build has no bounds checks
+#endif
+}
 
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache* c, int32_t q_heads, int32_t max_len) {
   if (check_shape(c) != KVQ_OK || check_heads(c, q_heads) != KVQ_OK) return 0;

@@ -332,7 +332,9 @@ __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
   const int wn = w0 + tt;
   const int wslot = active && (wn < c.sink || wn >= a.offset + a.n_new - c.recent)
                         ? window_slot(c.sink, c.recent, wn) : -1;
-  if (wslot >= 0) store_bf16_32(c.kwin + (bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, kx);
+  if (wslot >= 0 &&
+      kvq_in_bounds((bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, 32, c.win_elems()))
+    store_bf16_32(c.kwin + (bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, kx);
   uint32_t code[8];
   {
     const bool skip0 = CH0 && g == 0;
@@ -340,8 +342,9 @@ __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
 #pragma unroll
     for (int p = 0; p < 8; ++p) kw[8 * g + p][tt] = (uint16_t)compress_codes<KB>(code[p]);
     if (active) {
-      c.ks[(unit_blk * kGroups + g) * kKeyBlock + tb0 + tt] = sz;
-      if (skip0) c.k0[bh * c.cap + w0 + tt] = __float2bfloat16_rn(kx[0]);
+      const size_t ksi = (unit_blk * kGroups + g) * kKeyBlock + tb0 + tt;
+      if (kvq_in_bounds(ksi, 1, c.ks_pairs())) c.ks[ksi] = sz;
+      if (skip0 && kvq_in_bounds(bh * c.cap + w0 + tt, 1, c.rows())) c.k0[bh * c.cap + w0 + tt] = __float2bfloat16_rn(kx[0]);
     }
   }
   // ---- value row: optionally rotated, the same quantizer with the clipping
@@ -350,12 +353,14 @@ __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
     float vx[32];
     widen(vraw, vx);
     if (ROTV) rotate_row_4lanes(vx, g, a.inv_sqrt_d);
-    if (wslot >= 0) store_bf16_32(c.vwin + (bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, vx);
+    if (wslot >= 0 &&
+        kvq_in_bounds((bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, 32, c.win_elems()))
+      store_bf16_32(c.vwin + (bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, vx);
     const __half2 sz = quantize_group32<VB>(vx, false, c.v_clip, code);
     if (!active) {
 #pragma unroll
       for (int p = 0; p < 8; ++p) code[p] = 0;  // tokens outside the append contribute zero bits
-    } else {
+    } else if (kvq_in_bounds((bh * c.cap + w0 + tt) * kGroups + g, 1, c.ks_pairs())) {
       c.vs[(bh * c.cap + w0 + tt) * kGroups + g] = sz;
     }
     *reinterpret_cast<uint4*>(&vcode[tt][32 * g]) = make_uint4(code[0], code[1], code[2], code[3]);
@@ -370,6 +375,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
     for (int pg = warp; pg < kPruneGroups; pg += kAppendWarps) {
       const size_t idx = (unit_blk * kPruneGroups + pg) * kKeyBlock + tb0 + t;
       const uint32_t w2 = *reinterpret_cast<const uint32_t*>(&kw[pg][t]);  // token t in the low half
+      if (!kvq_in_bounds(idx * (KB == 4 ? 2 : 1), KB == 4 ? 4 : 2, c.kc_bytes())) continue;
       if (KB == 4) {
         uint16_t* dst = reinterpret_cast<uint16_t*>(c.kc) + idx;
         if (a0 && a1)
@@ -420,6 +426,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
     const int chunk = (tb / TPC) ^ v_chunk_swizzle(VB, ch);
     uint32_t* dst =
         reinterpret_cast<uint32_t*>(vblk + ch * (kKeyBlock * VB / 8) + chunk * 16 + (tb % TPC) / (8 / VB));
+    if (!kvq_in_bounds((size_t)(reinterpret_cast<uint8_t*>(dst) - c.vc), 4, c.vc_bytes())) continue;
     uint32_t word = vword[w][ch];
     if (a0 > 0 || a1 < TPW) {
       const uint32_t keep_lo = a0 * VB >= 32 ? ~0u : ((1u << (a0 * VB)) - 1u);
@@ -477,5 +484,7 @@ cudaError_t launch_append_ext(const AppendArgs& a, const float* tk, const float*
 }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) { return launch_append_ext(a, nullptr, nullptr, s); }
+
+KVQ_BOUNDS_COUNTER(bounds_append)
 
 }  // namespace kvq

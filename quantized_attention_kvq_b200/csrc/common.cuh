@@ -166,7 +166,47 @@ struct CacheView {
   __nv_bfloat16* k0;
   uint8_t* vc;
   __half2* vs;
+  // extents of the arrays (what kvq_cache_sizes reports), for the bounds checks
+  __host__ __device__ size_t rows() const { return (size_t)B * H * cap; }
+  __host__ __device__ size_t kc_bytes() const { return rows() * kPruneGroups * (k_bits == 4 ? 2 : 1); }
+  __host__ __device__ size_t ks_pairs() const { return rows() * kGroups; }
+  __host__ __device__ size_t vc_bytes() const { return rows() * (kHeadDim * v_bits / 8); }
+  __host__ __device__ size_t win_elems() const { return (size_t)B * H * (sink + recent) * kHeadDim; }
 };
+
+// Debug build (-DKVQ_BOUNDS_CHECK): a checked access first compares its
+// element range [idx, idx + n) with its buffer's extent; an access out of
+// bounds is skipped and counted in this translation unit's counter, which the
+// host reads through kvq_bounds_violations.  Without the flag the checks
+// compile to nothing.
+#ifdef KVQ_BOUNDS_CHECK
+namespace {
+__device__ unsigned int g_kvq_oob = 0;
+}
+__device__ __forceinline__ bool kvq_in_bounds(size_t idx, size_t n, size_t extent) {
+  if (idx + n <= extent) return true;
+  atomicAdd(&g_kvq_oob, 1u);
+  return false;
+}
+#define KVQ_BOUNDS_COUNTER(fn)                                                          \
+  unsigned fn(bool reset) {                                                             \
+    unsigned v = 0;                                                                     \
+    cudaMemcpyFromSymbol(&v, g_kvq_oob, sizeof(v));                                    \
+    if (reset) {                                                                        \
+      const unsigned z = 0;                                                             \
+      cudaMemcpyToSymbol(g_kvq_oob, &z, sizeof(z));                                     \
+    }                                                                                   \
+    return v;                                                                           \
+  }
+#else
+__device__ __forceinline__ bool kvq_in_bounds(size_t, size_t, size_t) { return true; }
+#define KVQ_BOUNDS_COUNTER(fn) \
+  unsigned fn(bool) { return 0; }
+#endif
+// per translation unit: its count of skipped accesses (optionally cleared)
+unsigned bounds_append(bool reset);
+unsigned bounds_decode(bool reset);
+unsigned bounds_window(bool reset);
 
 struct AppendArgs {
   CacheView c;
@@ -196,6 +236,7 @@ struct DecodeArgs {
   float* part_acc;  // [decode_slots][G][128] unnormalized accumulators
   float2* part_ml;  // [decode_slots][G] (running max, running sum)
   float* out;       // [B][Hq][128]
+  size_t part_rows;  // rows of part_acc / part_ml (for the bounds checks)
   int* status;      // device word: bit 0 set when a bounded wait of the split decode gave up
   int withheld_tile;  // test hook: CTA 0 never fills this tile's ring stage (-1: none)
 };

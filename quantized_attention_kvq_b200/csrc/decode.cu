@@ -814,7 +814,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         const int slot = ((int)it.bh(a) + blockIdx.x) * S::NGRP + grp;
         if (j == 0)
 #pragma unroll
-          for (int i = 0; i < HH; ++i) a.part_ml[(size_t)slot * G + part * HH + i] = make_float2(NEG_INF, 0.0f);
+          for (int i = 0; i < HH; ++i)
+            if (kvq_in_bounds((size_t)slot * G + part * HH + i, 1, a.part_rows))
+              a.part_ml[(size_t)slot * G + part * HH + i] = make_float2(NEG_INF, 0.0f);
       } else if (__builtin_expect(it.last, 0)) {
         // this group's pending PV sums of the segment, then its totals over the
         // tokens (max, sum, value zero-point terms) into its partial slot
@@ -860,6 +862,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           const size_t row = (size_t)slot * G + part * HH + i;
+          if (!kvq_in_bounds(row, 1, a.part_rows)) continue;
           a.part_acc[row * kHeadDim + j] = good ? acc[i] + zown[i] : nan;
           if (j == 0) a.part_ml[row] = good ? make_float2(m_run[i], lsum[i]) : make_float2(nan, nan);
         }
@@ -934,15 +937,21 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         __syncwarp();
         // one copy per run of adjacent kept channel groups (their rows are adjacent in the block)
         const bool run_start = ((msk >> lane) & 1u) && (lane == 0 || !((msk >> (lane - 1)) & 1u));
+        // (a copy the bounds checks refuse leaves its stage short: its waits give up)
         if (run_start) {
           const int run = __ffsll((long long)~((unsigned long long)msk >> lane)) - 1;
-          bulk_g2s(dst + S::R_KC + lane * S::KROW, c.kc + key_word_index(bh, c.cap, lane, n0) * (KB == 4 ? 2 : 1),
-                   run * S::KROW, FULL(s));
+          const size_t off = key_word_index(bh, c.cap, lane, n0) * (KB == 4 ? 2 : 1);
+          if (kvq_in_bounds(off, run * S::KROW, c.kc_bytes()))
+            bulk_g2s(dst + S::R_KC + lane * S::KROW, c.kc + off, run * S::KROW, FULL(s));
         }
-        if (lane == 0) bulk_g2s(dst + S::R_VC, c.vc + blk * kHeadDim * S::VROW, kHeadDim * S::VROW, FULL(s));
-        if (lane == 1) bulk_g2s(dst + S::R_KS, c.ks + key_scale_index(bh, c.cap, 0, n0), kGroups * kTile * 4, FULL(s));
-        if (lane == 2) bulk_g2s(dst + S::R_VS, c.vs + (bh * c.cap + n0) * kGroups, kTile * kGroups * 4, FULL(s));
-        if (k0 && lane == 3) bulk_g2s(dst + S::R_K0, c.k0 + bh * c.cap + n0, kTile * 2, FULL(s));
+        if (lane == 0 && kvq_in_bounds(blk * kHeadDim * S::VROW, kHeadDim * S::VROW, c.vc_bytes()))
+          bulk_g2s(dst + S::R_VC, c.vc + blk * kHeadDim * S::VROW, kHeadDim * S::VROW, FULL(s));
+        if (lane == 1 && kvq_in_bounds(key_scale_index(bh, c.cap, 0, n0), kGroups * kTile, c.ks_pairs()))
+          bulk_g2s(dst + S::R_KS, c.ks + key_scale_index(bh, c.cap, 0, n0), kGroups * kTile * 4, FULL(s));
+        if (lane == 2 && kvq_in_bounds((bh * c.cap + n0) * kGroups, kTile * kGroups, c.ks_pairs()))
+          bulk_g2s(dst + S::R_VS, c.vs + (bh * c.cap + n0) * kGroups, kTile * kGroups * 4, FULL(s));
+        if (k0 && lane == 3 && kvq_in_bounds(bh * c.cap + n0, kTile, c.rows()))
+          bulk_g2s(dst + S::R_K0, c.k0 + bh * c.cap + n0, kTile * 2, FULL(s));
       }
     }
   }
@@ -983,14 +992,16 @@ __global__ void __launch_bounds__(kHeadDim) k_combine(DecodeArgs a, int G, int n
     // slots (u + CTA) * ngrp + epilogue group; an empty one has max -inf and is skipped
     const float NEG_INF = -__int_as_float(0x7f800000);
     float M = NEG_INF;
-    for (int sl = (u + c0) * ngrp; sl < (u + c1 + 1) * ngrp; ++sl) M = fmaxf(M, a.part_ml[(size_t)sl * G + hl].x);
+    for (int sl = (u + c0) * ngrp; sl < (u + c1 + 1) * ngrp; ++sl)
+      if (kvq_in_bounds((size_t)sl * G + hl, 1, a.part_rows)) M = fmaxf(M, a.part_ml[(size_t)sl * G + hl].x);
     // the bf16 window tokens' partial, when the cache has windows
     const bool win = a.c.sink + a.c.recent > 0;
     const size_t rw = (size_t)(a.win_base + u) * G + hl;
-    if (win) M = fmaxf(M, a.part_ml[rw].x);
+    if (win && kvq_in_bounds(rw, 1, a.part_rows)) M = fmaxf(M, a.part_ml[rw].x);
     float l = 0.0f, o = 0.0f;
     for (int sl = (u + c0) * ngrp; sl < (u + c1 + 1) * ngrp + (win ? 1 : 0); ++sl) {
       const size_t r = sl < (u + c1 + 1) * ngrp ? (size_t)sl * G + hl : rw;
+      if (!kvq_in_bounds(r, 1, a.part_rows)) continue;
       const float2 v = a.part_ml[r];
       if (v.x == NEG_INF) continue;
       const float w = exp2f(v.x - M);
@@ -1069,6 +1080,8 @@ cudaError_t launch_combine(const DecodeArgs& a, cudaStream_t s) {
   k_combine<<<a.c.B * a.Hq, kHeadDim, 0, s>>>(a, a.Hq / a.c.H, decode_groups(a.Hq / a.c.H));
   return cudaGetLastError();
 }
+
+KVQ_BOUNDS_COUNTER(bounds_decode)
 
 }  // namespace kvq
 

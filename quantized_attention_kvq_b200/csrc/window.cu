@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kWinThreads) k_window(DecodeArgs a) {
       float t = o[g];
       for (int q = 1; q < kWinParts; ++q) t += osum[((q - 1) * G + g) * kHeadDim + ch];
       const size_t r = (size_t)(a.win_base + u) * G + g;
+      if (!kvq_in_bounds(r, 1, a.part_rows)) continue;
       a.part_acc[r * kHeadDim + ch] = t;
       if (ch == 0) {
         float l = 0.0f;
@@ -180,5 +181,7 @@ cudaError_t launch_window(const DecodeArgs& a, cudaStream_t s) {
   }
 }
 
+
+KVQ_BOUNDS_COUNTER(bounds_window)
 
 }  // namespace kvq

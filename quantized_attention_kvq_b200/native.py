@@ -12,7 +12,9 @@ import os
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libkvq.so")
+# KVQ_LIBRARY=checked selects the bounds-checked debug build of the same library
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib",
+                        "libkvq_checked.so" if os.environ.get("KVQ_LIBRARY") == "checked" else "libkvq.so")
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_WORKSPACE, KVQ_ERR_CUDA, KVQ_ERR_TIMEOUT = range(7)
 KVQ_F32, KVQ_BF16, KVQ_F16 = 0, 1, 2
@@ -22,7 +24,7 @@ SYMBOLS = ("kvq_cache_sizes", "kvq_window_bytes", "kvq_quantize_append", "kvq_se
            "kvq_select_channels_at", "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_decode_partials", "kvq_decode_combine",
            "kvq_decode_step_workspace_bytes",
            "kvq_decode_step_host", "kvq_decode_attention_static", "kvq_decode_attention_select",
-           "kvq_decode_partials_select", "kvq_decode_status", "kvq_test_withhold_tile",
+           "kvq_decode_partials_select", "kvq_decode_status", "kvq_test_withhold_tile", "kvq_bounds_violations",
            "kvq_status_string")
 
 _P = ctypes.c_void_p
@@ -89,6 +91,8 @@ def lib():
         L.kvq_decode_partials_select.restype = ctypes.c_int
         L.kvq_decode_status.argtypes = [C, _I32, _P, ctypes.c_size_t, _P]
         L.kvq_decode_status.restype = ctypes.c_int
+        L.kvq_bounds_violations.argtypes = [_I32]
+        L.kvq_bounds_violations.restype = ctypes.c_uint32
         L.kvq_test_withhold_tile.argtypes = [_I32]
         L.kvq_test_withhold_tile.restype = None
         L.kvq_status_string.argtypes = [ctypes.c_int]

@@ -35,6 +35,20 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def test_bounds_checked_build_exports_every_declared_symbol(L):
+    # the debug build of the same sources (-DKVQ_BOUNDS_CHECK), built beside the library
+    path = os.path.join(os.path.dirname(native.LIB_PATH), "libkvq_checked.so")
+    if not os.path.exists(path):
+        from quantized_attention_kvq_b200 import build
+        build.build_kvq(checked=True)
+    C = ctypes.CDLL(path)
+    for name in header_functions():
+        assert hasattr(C, name), name
+    # the regular library has no checks compiled in
+    L.kvq_bounds_violations.restype = ctypes.c_uint32
+    assert L.kvq_bounds_violations(0) == 0xFFFFFFFF
+
+
 def desc(**kw):
     d = native.describe(kw.pop("B", 2), kw.pop("H", 2), kw.pop("cap", 256), kw.pop("kb", 4), kw.pop("vb", 2),
                         kw.pop("rot", 1), kw.pop("ch0", 1))
