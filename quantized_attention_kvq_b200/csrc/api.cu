@@ -42,8 +42,10 @@ kvq_status check_shape(const kvq_cache* c) {
   if ((c->k_bits != 2 && c->k_bits != 4) || (c->v_bits != 2 && c->v_bits != 4)) return KVQ_ERR_UNSUPPORTED;
   if (c->capacity % kKeyBlock != 0) return KVQ_ERR_UNSUPPORTED;
   if (c->bucket_tokens < 0) return KVQ_ERR_INVALID_ARG;
+  // with bucket-relative RoPE the bf16 windows may touch at most three
+  // buckets (the sinks the first, the recent tokens at most two)
   if (c->bucket_tokens > 0 && (c->bucket_tokens % kKeyBlock != 0 || c->capacity % c->bucket_tokens != 0 ||
-                               c->sink_tokens + c->recent_tokens > 0))
+                               c->sink_tokens > c->bucket_tokens || c->recent_tokens > c->bucket_tokens))
     return KVQ_ERR_UNSUPPORTED;
   // the selection runs one grid row per (sequence, bucket), the append one grid
   // layer per sequence: both at most 65535
@@ -92,6 +94,7 @@ CacheView view(const kvq_cache* c) {
   v.v_clip = c->v_clip;
   v.sink = c->sink_tokens;
   v.recent = c->recent_tokens;
+  v.pos_base = 0;
   v.kwin = static_cast<__nv_bfloat16*>(c->k_window);
   v.vwin = static_cast<__nv_bfloat16*>(c->v_window);
   v.kc = static_cast<uint8_t*>(c->k_codes);
@@ -130,6 +133,12 @@ CacheView bucket_sequence_view(const kvq_cache* c, size_t vb) {
   if (v.k0) v.k0 = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(v.k0) + vb * per[2]);
   v.vc = v.vc + vb * per[3];
   v.vs = reinterpret_cast<__half2*>(reinterpret_cast<char*>(v.vs) + vb * per[4]);
+  // the bf16 windows belong to the real sequence vb / nb, at its positions
+  const int nb = n_buckets(c);
+  v.pos_base = (int)(vb % nb) * c->bucket_tokens;
+  const size_t win_seq = (size_t)c->kv_heads * (c->sink_tokens + c->recent_tokens) * kHeadDim;
+  if (v.kwin) v.kwin += (vb / nb) * win_seq;
+  if (v.vwin) v.vwin += (vb / nb) * win_seq;
   return v;
 }
 
@@ -267,6 +276,10 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
     v.part_ml = reinterpret_cast<float2*>(ws + plan.ml_offset);
     v.out = nullptr;
     v.part_rows = plan.rows;
+    v.bucket_nb = nb;
+    v.bucket_w = c->bucket_tokens;
+    v.real_lens = seq_lens;
+    v.real_max_len = max_len;
     v.status = reinterpret_cast<int*>(ws + plan.status_offset);
     v.withheld_tile = -1;
     if (parts & kRunSplit) {
@@ -286,6 +299,18 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
         v.mask = own_mask;
       }
       if (v.max_len > 0 && (st = cuda_status(launch_decode(v, s))) != KVQ_OK) return st;
+      if (c->sink_tokens + c->recent_tokens > 0) {
+        // the bf16 window tokens of each real sequence, scored with the query
+        // rows of the buckets they sit in (already embedded and transformed)
+        DecodeArgs aw = v;
+        aw.c = view(c);
+        aw.c.rotate = 0;
+        aw.q = ws + plan.qb_offset;
+        aw.dtype = KVQ_F32;
+        aw.seq_lens = seq_lens;
+        aw.max_len = max_len;
+        if ((st = fork_window(aw, s)) != KVQ_OK) return st;
+      }
     }
     if (parts & kRunCombine)
       return cuda_status(launch_bucket_merge(v, nb, decode_slots(0, 0, G) / decode_groups(G), decode_groups(G), out, s));
@@ -306,6 +331,10 @@ kvq_status enqueue_decode(const kvq_cache* c, const void* q, kvq_dtype dtype, in
   a.part_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + plan.ml_offset);
   a.out = out;
   a.part_rows = plan.rows;
+  a.bucket_nb = 0;
+  a.bucket_w = 0;
+  a.real_lens = nullptr;
+  a.real_max_len = 0;
   a.status = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan.status_offset);
   a.withheld_tile = -1;
   if (parts & kRunSplit) {

@@ -329,8 +329,10 @@ __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
   // window slot: every sink token, and of the later tokens only this append's
   // last `recent`, the ones that still own their ring slot when it ends (an
   // earlier token of the same append would race with them for the slot)
-  const int wn = w0 + tt;
-  const int wslot = active && (wn < c.sink || wn >= a.offset + a.n_new - c.recent)
+  // (positions count from the view's first token: a bucket's anchor with
+  // bucket-relative RoPE, whose view's window rows are its sequence's)
+  const int wn = c.pos_base + w0 + tt;
+  const int wslot = active && (wn < c.sink || wn >= c.pos_base + a.offset + a.n_new - c.recent)
                         ? window_slot(c.sink, c.recent, wn) : -1;
   if (wslot >= 0 &&
       kvq_in_bounds((bh * (size_t)(c.sink + c.recent) + wslot) * kHeadDim + 32 * g, 32, c.win_elems()))

@@ -111,6 +111,10 @@ __global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb,
     M = fmaxf(M, fmaxf(fmaxf(s_max[0], s_max[1]), fmaxf(s_max[2], s_max[3])));
     t0 += chunk_sum;
   }
+  // the bf16 window tokens' partial of the unit, when the cache has windows
+  const bool win = v.c.sink + v.c.recent > 0;
+  const size_t rw = (size_t)(v.win_base + b * v.c.H + h) * G + hl;
+  if (win) M = fmaxf(M, v.part_ml[rw].x);
   // pass 2: every slot's weight 2^(m - M), its sum and its channel.  A
   // chunk's slots are listed in shared memory first (at most 2 per CTA range
   // end per bucket plus one per `per` tiles, so under 1024), then walked
@@ -183,6 +187,14 @@ __global__ void __launch_bounds__(kHeadDim) k_bucket_merge(DecodeArgs v, int nb,
       }
     }
     __syncthreads();
+  }
+  if (win) {
+    const float2 ml = v.part_ml[rw];
+    if (ml.x != NEG_INF) {
+      const float e = exp2f(ml.x - M);
+      l = fmaf(e, ml.y, l);
+      o = fmaf(e, v.part_acc[rw * kHeadDim + chn], o);
+    }
   }
   float res = l > 0.0f ? o / l : 0.0f;
   if (v.c.rotate_v) {

@@ -159,6 +159,7 @@ struct CacheView {
   int B, H, cap, k_bits, v_bits, rotate, keep_ch0, rotate_v;
   float v_clip;
   int sink, recent;                    // bf16 token windows (0, 0: none)
+  int pos_base;                        // sequence position of the view's token 0 (a bucket's anchor)
   __nv_bfloat16* kwin;                 // [B][H][sink + recent][128]
   __nv_bfloat16* vwin;
   uint8_t* kc;
@@ -238,6 +239,13 @@ struct DecodeArgs {
   float* out;       // [B][Hq][128]
   size_t part_rows;  // rows of part_acc / part_ml (for the bounds checks)
   int* status;      // device word: bit 0 set when a bounded wait of the split decode gave up
+  // bucket-relative RoPE: sequence vb of the decode is bucket vb % bucket_nb of
+  // sequence vb / bucket_nb, whose length is real_lens[] (clamped to
+  // real_max_len); bucket_nb = 0 without buckets.  The bf16 windows are
+  // placed by the real sequence's positions and length.
+  int bucket_nb, bucket_w;
+  const int32_t* real_lens;
+  int real_max_len;
   int withheld_tile;  // test hook: CTA 0 never fills this tile's ring stage (-1: none)
 };
 

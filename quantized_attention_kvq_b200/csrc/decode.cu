@@ -540,6 +540,10 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     int qb = 0;         // query buffer of the current segment (its parity)
     int seg_tiles = 0;  // tiles of the current segment this group has taken
     int last_own = 0;   // the last tile this group took
+    // where the bf16 windows sit for this segment's unit: the sequence position
+    // of its token 0 and the length the windows are placed by (a bucket's
+    // anchor and its sequence's length with bucket-relative RoPE)
+    int wpos0 = 0, wlen = 0;
     bool ok = true;
 
     // add the PV sums of tile tp (buffer tp % DB) times its scale into acc:
@@ -576,6 +580,15 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         for (int g = 0; g < kGroups; ++g) vmr[g] = kvr[g] = 0.0f;
         have1 = have2 = false;
         seg_tiles = 0;
+        if (c.sink + c.recent > 0) {
+          if (a.bucket_nb > 0) {
+            wpos0 = (it.b % a.bucket_nb) * a.bucket_w;
+            wlen = min(max(a.real_lens[it.b / a.bucket_nb], 0), a.real_max_len);
+          } else {
+            wpos0 = 0;
+            wlen = it.len;
+          }
+        }
         qb = nseg & 1;  // this segment's query data
         ok &= ws_wait(QREADY(qb), (nseg >> 1) & 1, err);
         ++nseg;
@@ -599,7 +612,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       } else {
       // tokens past the end, and the bf16 window tokens (scored by k_window), take no part
       const int tok = it.i * kTile + j;  // token position in the sequence
-      const bool valid = tok < it.len && !in_window(c.sink, c.recent, tok, it.len);
+      const bool valid = tok < it.len && !in_window(c.sink, c.recent, wpos0 + tok, wlen);
       // per-token scales, zeros and channel 0 from the ring (zero past the sequence end)
       const int s = t % ST;
       ok &= ws_wait(FULL(s), (t / ST) & 1, err);

@@ -31,21 +31,34 @@ __global__ void __launch_bounds__(kWinThreads) k_window(DecodeArgs a) {
   const int n_sink = min(c.sink, len);
   const int r0 = c.recent > 0 ? max(c.sink, len - c.recent) : len;  // first recent token
   const int W = n_sink + max(len - r0, 0);                            // window tokens
+  // with bucket-relative RoPE the window tokens take the query of the bucket
+  // they sit in: the sinks bucket 0's, the recent tokens one of at most two
+  // buckets' (the recent window is at most a bucket long)
+  const bool bk = a.bucket_nb > 0;
+  const int NQ = bk ? 3 : 1;
+  int kbq[3] = {0, 0, 0};
+  if (bk && len > 0) {
+    kbq[1] = r0 / a.bucket_w;
+    kbq[2] = (len - 1) / a.bucket_w;
+  }
   float* qs = wsm;
-  float* pw = qs + G * kHeadDim;
+  float* pw = qs + NQ * G * kHeadDim;
   float* red = pw + G * WS;
   int* slot = reinterpret_cast<int*>(red + G * kWinWarps);  // window slot of window token w
   float* osum = reinterpret_cast<float*>(slot + WS);
   const size_t row0 = (size_t)u * WS;
   for (int w = tid; w < W; w += kWinThreads)
     slot[w] = window_slot(c.sink, c.recent, w < n_sink ? w : r0 + (w - n_sink));
-  // the query rows, rotated as the keys are, one warp per head
-  for (int g = warp; g < G; g += kWinWarps) {
+  // the query rows, rotated as the keys are (with buckets: each bucket's rows
+  // as the decode prepared them), one warp per head
+  for (int sg = warp; sg < NQ * G; sg += kWinWarps) {
+    const int sq = sg / G, g = sg - sq * G;
+    const size_t qrow = bk ? ((size_t)b * a.bucket_nb + kbq[sq]) * a.Hq + (size_t)h * G + g
+                           : (size_t)b * a.Hq + (size_t)h * G + g;
     float x[4];
-    load_row_warp(static_cast<const In*>(a.q) + ((size_t)b * a.Hq + (size_t)h * G + g) * kHeadDim, c.rotate != 0,
-                  a.inv_sqrt_d, lane, x);
+    load_row_warp(static_cast<const In*>(a.q) + qrow * kHeadDim, c.rotate != 0, a.inv_sqrt_d, lane, x);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) qs[g * kHeadDim + 4 * lane + i] = x[i];
+    for (int i = 0; i < 4; ++i) qs[sg * kHeadDim + 4 * lane + i] = x[i];
   }
   __syncthreads();
   // scores (base-2 units) of every window token, all channels
@@ -61,6 +74,12 @@ __global__ void __launch_bounds__(kWinThreads) k_window(DecodeArgs a) {
     float acc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) acc[g] = 0.0f;
+    int sq = 0;  // the token's query set
+    if (bk) {
+      const int n = w < n_sink ? w : r0 + (w - n_sink);
+      sq = n < c.sink ? 0 : (n / a.bucket_w == kbq[1] ? 1 : 2);
+    }
+    const float* qw = qs + sq * G * kHeadDim;
 #pragma unroll
     for (int i8 = 0; i8 < kHeadDim / 8; ++i8) {
       const uint32_t pr[4] = {raw[i8].x, raw[i8].y, raw[i8].z, raw[i8].w};
@@ -70,7 +89,7 @@ __global__ void __launch_bounds__(kWinThreads) k_window(DecodeArgs a) {
         const float k0 = __uint_as_float(pr[i] << 16), k1 = __uint_as_float(pr[i] & 0xFFFF0000u);
 #pragma unroll
         for (int g = 0; g < G; ++g)
-          acc[g] = fmaf(qs[g * kHeadDim + cc + 1], k1, fmaf(qs[g * kHeadDim + cc], k0, acc[g]));
+          acc[g] = fmaf(qw[g * kHeadDim + cc + 1], k1, fmaf(qw[g * kHeadDim + cc], k0, acc[g]));
       }
     }
 #pragma unroll
@@ -157,8 +176,9 @@ __global__ void __launch_bounds__(kWinThreads) k_window(DecodeArgs a) {
 template <int G>
 cudaError_t launch_window_g(const DecodeArgs& a, cudaStream_t s) {
   const int ws = a.c.sink + a.c.recent;
+  const int nq = a.bucket_nb > 0 ? 3 : 1;  // query sets (bucket-relative RoPE: up to three buckets)
   const size_t smem =
-      (size_t)(G * kHeadDim + G * ws + G * kWinWarps + ws + (kWinParts - 1) * G * kHeadDim) * sizeof(float);
+      (size_t)(nq * G * kHeadDim + G * ws + G * kWinWarps + ws + (kWinParts - 1) * G * kHeadDim) * sizeof(float);
   auto kern = a.dtype == KVQ_F32 ? k_window<G, float> : (a.dtype == KVQ_BF16 ? k_window<G, __nv_bfloat16> : k_window<G, __half>);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

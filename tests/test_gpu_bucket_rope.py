@@ -47,13 +47,13 @@ def bucket_major(a: np.ndarray, B: int, H: int, nb: int) -> np.ndarray:
     return a.reshape(B, H, nb, -1).transpose(0, 2, 1, 3).reshape(-1)
 
 
-def build(B, H, cap, w, kb, vb, rot, ch0, k, v, fmt, fr, tq=None, tk=None, rotv=0, clip=1.0):
+def build(B, H, cap, w, kb, vb, rot, ch0, k, v, fmt, fr, tq=None, tk=None, rotv=0, clip=1.0, sink=0, recent=0):
     nb = cap // w
     gc = native.KVQCache(B, H, cap, kb, vb, rot, ch0, rotate_v=rotv, v_clip=clip, bucket_tokens=w,
-                         rope_inv_freq=torch.from_numpy(fr).cuda(),
+                         rope_inv_freq=torch.from_numpy(fr).cuda(), sink=sink, recent=recent,
                          t_query=None if tq is None else torch.from_numpy(tq).cuda(),
                          t_key=None if tk is None else torch.from_numpy(tk).cuda())
-    oc = orc.Cache(B, H, D, cap, kb, vb, rot, ch0, rotv, clip, 0, 0, tq, tk, bucket_w=w, inv_freq=fr)
+    oc = orc.Cache(B, H, D, cap, kb, vb, rot, ch0, rotv, clip, sink, recent, tq, tk, bucket_w=w, inv_freq=fr)
     T = k.shape[2]
     for t0 in range(0, T, w):  # an append stays inside one bucket
         gc.append(to_device(k[:, :, t0:t0 + w], fmt), to_device(v[:, :, t0:t0 + w], fmt), t0)
@@ -130,3 +130,36 @@ def test_bucket_rope_lengths_at_bucket_edges():
             assert not o_gpu[rows].any()
         else:
             assert_close_output(o_gpu[rows], o_ref[rows], f"sequence {b}")
+
+
+@pytest.mark.parametrize("T,sink,recent,rot,keep", [(700, 64, 200, 1, 19), (1000, 16, 256, 2, 24), (200, 64, 256, 1, 32)])
+def test_bucket_rope_with_bf16_windows_matches_oracle(T, sink, recent, rot, keep):
+    # bf16 sink and recent windows together with bucket-relative RoPE: a window
+    # token is scored over every channel with the query of the bucket it sits
+    # in; the recent window here spans two buckets (Dual-QK Sec. 3.3 and 3.4)
+    B, G, H, w, cap = 2, 4, 2, 256, 1024
+    q, k, v = draw(1900 + T + rot, B, G * H, H, T, "bf16")
+    fr = inv_freq(10000.0)
+    tq, tk = dense_pair(7, H) if rot == 2 else (None, None)
+    gc, oc = build(B, H, cap, w, 4, 2, rot, 1, k, v, "bf16", fr, tq, tk, sink=sink, recent=recent)
+    # the windows are bit-exact (bf16 of the same embedded, transformed rows)
+    assert np.array_equal(gc.k_window.cpu().numpy(), oc.k_win.view(np.uint8))
+    assert np.array_equal(gc.v_window.cpu().numpy(), oc.v_win.view(np.uint8))
+    qd = to_device(q, "bf16")
+    lens_np = np.array([T, T], np.int32)  # the decode length is the tokens appended (the ring holds the last ones)
+    lens_d = torch.from_numpy(lens_np).cuda()
+    if keep < 32:
+        mask_d = gc.select_at(qd, lens_d, keep)
+        ref_mask, _ = oc.select_buckets(host_f32(q, "bf16"), lens_np, keep)
+        np.testing.assert_array_equal(mask_u32(mask_d).reshape(ref_mask.shape), ref_mask)
+    else:
+        mask_d, ref_mask = None, None
+    out = gc.decode(qd, lens_d, cap, mask_d, softmax_scale())
+    sel = gc.decode_select(qd, lens_d, cap, keep, softmax_scale()) if keep < 32 else out
+    torch.cuda.synchronize()
+    assert torch.equal(out, sel)
+    o_ref = oc.attention(host_f32(q, "bf16"), lens_np, ref_mask, softmax_scale())
+    o_gpu = out.cpu().numpy().reshape(-1, D)
+    for b in range(B):
+        rows = slice(b * G * H, (b + 1) * G * H)
+        assert_close_output(o_gpu[rows], o_ref[rows], f"sequence {b}")
