@@ -56,18 +56,24 @@ WORKLOADS = [
     Workload(7, "dualqk_int2_vrot_win64x256_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16", 2,
              2, 1, 1, 19, rotate_v=1, v_clip=0.92, sink=64, recent=256),
     # a caller-supplied dual transform pair on queries and keys (Dual-QK Sec. 3.1)
-    # with bucket-relative RoPE at w = 2048 (Sec. 3.4); bf16 windows are not
-    # combined with buckets on the CUDA path
+    # with bucket-relative RoPE at w = 2048 (Sec. 3.4)
     Workload(8, "dualqk_int2_pair_bucket2048_vrot_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072, 0, "bf16",
              2, 2, 2, 1, 19, rotate_v=1, v_clip=0.92, bucket=2048),
     # the append through a caller-supplied dual transform pair (Dual-QK Sec. 3.1):
     # each key row taken through its kv head's 128 x 128 key matrix
     Workload(9, "append_pair_b16_h8_t4096_at8192", 16, 8, 8, 128, 4096, 12288, 8192, "bf16", 4, 2, 2, 0, 32,
              kind="append"),
+    # the whole Dual-QK recipe: as 8, with the first 64 and the most recent 256
+    # tokens kept in bf16 (Sec. 3.3 with Sec. 3.4)
+    Workload(10, "dualqk_int2_pair_bucket2048_win64x256_vrot_b4_h32x8_n128k_keep19", 4, 32, 8, 128, 131072, 131072,
+             0, "bf16", 2, 2, 2, 1, 19, rotate_v=1, v_clip=0.92, sink=64, recent=256, bucket=2048),
 ]
 
 BASE_SEED = 0
 
 
 def by_id(i: int) -> Workload:
-    return WORKLOADS[i]
+    for w in WORKLOADS:
+        if w.id == i:
+            return w
+    raise KeyError(f"no workload {i}")
