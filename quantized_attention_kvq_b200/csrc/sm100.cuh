@@ -279,52 +279,6 @@ __device__ __forceinline__ void tmem_ld_wait<32>(uint32_t taddr, uint32_t (&r)[3
       : "r"(taddr)
       : "memory");
 }
-// 3, 6, 12 or 24 consecutive columns as two loads (2+1, 4+2, 8+4, 16+8), so
-// that no column past the last one is touched.
-template <>
-__device__ __forceinline__ void tmem_ld_wait<3>(uint32_t taddr, uint32_t (&r)[3]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%3];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%2}, [%4];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2])
-      : "r"(taddr), "r"(taddr + 2)
-      : "memory");
-}
-template <>
-__device__ __forceinline__ void tmem_ld_wait<6>(uint32_t taddr, uint32_t (&r)[6]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%6];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%4, %5}, [%7];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5])
-      : "r"(taddr), "r"(taddr + 4)
-      : "memory");
-}
-template <>
-__device__ __forceinline__ void tmem_ld_wait<12>(uint32_t taddr, uint32_t (&r)[12]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%12];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [%13];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11])
-      : "r"(taddr), "r"(taddr + 8)
-      : "memory");
-}
-template <>
-__device__ __forceinline__ void tmem_ld_wait<24>(uint32_t taddr, uint32_t (&r)[24]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%24];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16, %17, %18, %19, %20, %21, %22, %23}, [%25];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23])
-      : "r"(taddr), "r"(taddr + 16)
-      : "memory");
-}
 // Scores and PV sums of an epilogue tile in one round trip: four runs of
 // 2 HH columns at taddr + g * stride (g = 0..3) and one run of 4 HH columns at
 // paddr, then one wait for all of them.
@@ -463,67 +417,6 @@ __device__ __forceinline__ void tmem_ld4_wait<8>(uint32_t taddr, uint32_t stride
       : "memory");
 }
 
-// Two sets of four runs of N columns (at taddr + k * stride and taddr + off2 +
-// k * stride, k = 0..3), one wait for all eight loads.
-template <int N>
-__device__ __forceinline__ void tmem_ld8_wait(uint32_t taddr, uint32_t stride, uint32_t off2, uint32_t (&r)[4][N],
-                                              uint32_t (&q)[4][N]);
-template <>
-__device__ __forceinline__ void tmem_ld8_wait<2>(uint32_t taddr, uint32_t stride, uint32_t off2, uint32_t (&r)[4][2],
-                                                 uint32_t (&q)[4][2]) {
-  asm volatile(
-      "{\n\t.reg .b32 a, b;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%16];\n\t"
-      "add.u32 b, %16, %18;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%8, %9}, [b];\n\t"
-      "add.u32 a, %16, %17;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%2, %3}, [a];\n\t"
-      "add.u32 b, a, %18;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%10, %11}, [b];\n\t"
-      "add.u32 a, a, %17;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%4, %5}, [a];\n\t"
-      "add.u32 b, a, %18;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%12, %13}, [b];\n\t"
-      "add.u32 a, a, %17;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%6, %7}, [a];\n\t"
-      "add.u32 b, a, %18;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%14, %15}, [b];\n\t"
-      "tcgen05.wait::ld.sync.aligned;\n\t}"
-      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[3][0]),
-        "=r"(r[3][1]), "=r"(q[0][0]), "=r"(q[0][1]), "=r"(q[1][0]), "=r"(q[1][1]), "=r"(q[2][0]), "=r"(q[2][1]),
-        "=r"(q[3][0]), "=r"(q[3][1])
-      : "r"(taddr), "r"(stride), "r"(off2)
-      : "memory");
-}
-template <>
-__device__ __forceinline__ void tmem_ld8_wait<4>(uint32_t taddr, uint32_t stride, uint32_t off2, uint32_t (&r)[4][4],
-                                                 uint32_t (&q)[4][4]) {
-  asm volatile(
-      "{\n\t.reg .b32 a, b;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%32];\n\t"
-      "add.u32 b, %32, %34;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%16, %17, %18, %19}, [b];\n\t"
-      "add.u32 a, %32, %33;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4, %5, %6, %7}, [a];\n\t"
-      "add.u32 b, a, %34;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%20, %21, %22, %23}, [b];\n\t"
-      "add.u32 a, a, %33;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [a];\n\t"
-      "add.u32 b, a, %34;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%24, %25, %26, %27}, [b];\n\t"
-      "add.u32 a, a, %33;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%12, %13, %14, %15}, [a];\n\t"
-      "add.u32 b, a, %34;\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%28, %29, %30, %31}, [b];\n\t"
-      "tcgen05.wait::ld.sync.aligned;\n\t}"
-      : "=r"(r[0][0]), "=r"(r[0][1]), "=r"(r[0][2]), "=r"(r[0][3]), "=r"(r[1][0]), "=r"(r[1][1]), "=r"(r[1][2]),
-        "=r"(r[1][3]), "=r"(r[2][0]), "=r"(r[2][1]), "=r"(r[2][2]), "=r"(r[2][3]), "=r"(r[3][0]), "=r"(r[3][1]),
-        "=r"(r[3][2]), "=r"(r[3][3]), "=r"(q[0][0]), "=r"(q[0][1]), "=r"(q[0][2]), "=r"(q[0][3]), "=r"(q[1][0]),
-        "=r"(q[1][1]), "=r"(q[1][2]), "=r"(q[1][3]), "=r"(q[2][0]), "=r"(q[2][1]), "=r"(q[2][2]), "=r"(q[2][3]),
-        "=r"(q[3][0]), "=r"(q[3][1]), "=r"(q[3][2]), "=r"(q[3][3])
-      : "r"(taddr), "r"(stride), "r"(off2)
-      : "memory");
-}
 
 // Each thread of the warp writes N consecutive 32-bit columns of its own lane.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
