@@ -137,10 +137,13 @@ typedef struct {
      Layout: bucket-major -- every array is laid out as the cache of batch
      B * (capacity / w) and capacity w, bucket k of sequence b being its
      sequence b * (capacity / w) + k (kvq_cache_sizes is unchanged).
+     bf16 token windows combine with buckets: the windows stay per sequence
+     and are placed by sequence positions, and a window token is scored with
+     the query of the bucket it sits in.
      Requires w a multiple of 128 dividing capacity, B * capacity / w <= 65535,
-     and no token windows (otherwise KVQ_ERR_UNSUPPORTED); an append must stay inside one bucket
-     (otherwise KVQ_ERR_INVALID_ARG).  rope_inv_freq: caller-owned device
-     fp32 [d/2], 16-byte aligned. */
+     and sink_tokens, recent_tokens <= w (otherwise KVQ_ERR_UNSUPPORTED); an
+     append must stay inside one bucket (otherwise KVQ_ERR_INVALID_ARG).
+     rope_inv_freq: caller-owned device fp32 [d/2], 16-byte aligned. */
   int32_t bucket_tokens;
   const float* rope_inv_freq;
 } kvq_cache;
