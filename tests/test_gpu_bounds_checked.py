@@ -1,8 +1,9 @@
 """The bounds-checked debug build (libkvq_checked.so, -DKVQ_BOUNDS_CHECK).
 
 Its kernels compare every checked cache, partial and window access with the
-array's extent and count the ones out of bounds.  On the same small append,
-selection and decode (one case with bf16 token windows) it must give the
+array's extent and count the ones out of bounds.  On the same small appends,
+selections and decodes (plain, with bf16 token windows, and with
+bucket-relative RoPE, a dual pair and windows together) it must give the
 regular library's bytes and outputs exactly, with no access out of bounds;
 the regular library reports that it has no checks (UINT32_MAX).
 """
