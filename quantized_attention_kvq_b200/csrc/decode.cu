@@ -653,12 +653,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       // column 2 HH part + HH + h of group g
       uint32_t sd[kGroups][2 * HH];
       const uint32_t sbase = tmem + lane_base + S::TM_S + (t % S::SB) * 4 * S::NS + part * 2 * HH;
-      if constexpr (MERGED) {
-        uint32_t pv[4 * HH];
-        tmem_ld_sc_pv<HH>(sbase, S::NS, pv_addr(t), sd, pv);
-        tc_fence_before();
-        if (rdp) add_pv(pv, PLEN == 2 ? ds2 : ds1);
-      } else if constexpr (HH <= 4) {
+      if constexpr (HH <= 4) {
         tmem_ld4_wait<2 * HH>(sbase, S::NS, sd);
         tc_fence_before();
       } else {
@@ -720,7 +715,19 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       for (int i = 0; i < HH; ++i) pass |= sc[i] > m_run[i] + kLazyMax;
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) pass |= vsz[g].x > vmr[g];
+      // with the sums of tile t - RD long done, their load is in flight while
+      // the part's warps meet at the barrier
+      uint32_t pv[4 * HH];
+      if constexpr (MERGED) {
+        tc_fence_after();
+        tmem_ld_start<4 * HH>(pv_addr(t), pv);
+      }
       const bool raise = bar_any(bar_id, 128, pass);
+      if constexpr (MERGED) {
+        tmem_ld_finish<4 * HH>(pv);
+        tc_fence_before();
+        if (rdp) add_pv(pv, PLEN == 2 ? ds2 : ds1);
+      }
       float alpha[HH];
       if (__builtin_expect(raise, 0)) {
         // the tile's largest score per head and largest value scale per group
