@@ -210,36 +210,88 @@ __device__ __forceinline__ void rotate_row_4lanes(float (&v)[32], int g, double 
   for (int i = 0; i < 32; ++i) v[i] = __double2float_rn(__dmul_rn(x[i], inv_sqrt_d));
 }
 
-// Key row through the kv head's matrix A of the caller's transform pair, held
-// by four lanes as above: channel 32g + r is the fp64 sum over j = 0..127, in
-// order, of A[32g + r][j] x_j (product and sum each rounded once), rounded to
-// fp32; x_j comes from lane j / 32 of the quad by shuffles.  All 32 lanes of
-// the warp take part.
-__device__ __forceinline__ void transform_row_4lanes(float (&v)[32], int g, int lane, const float* __restrict__ A) {
-  const int base = lane & ~3;
-  const float4* rows = reinterpret_cast<const float4*>(A) + (size_t)32 * g * (kHeadDim / 4);
-  double acc[32];
+// Key rows of the window's 64 tokens through the kv head's matrix A of the
+// caller's transform pair, as one 64 x 128 x 128 product: channel i of token t
+// is the fp64 sum over j = 0..127, in order, of A[i][j] x_tj, rounded to fp32.
+// A product of two fp32 numbers is exact in fp64, so a fused multiply-add per
+// step rounds once, as a rounded sum of the rounded product does: the result is
+// that in-order sum bit for bit.  On entry lane (tt, g) holds channels
+// 32g .. 32g+31 of token tt in v; on return the transformed ones.  Every thread
+// of the block takes part.  Dynamic shared memory: A^T in fp64 as [j][i]
+// (128 KB) and X^T in fp64 as [j][t] (64 KB), token t of row j at column
+// (t + 8 (j / 32)) mod 64 so that the four lanes of a token store into
+// distinct banks; the fp32 results then take X^T's space as rows [t][i].
+constexpr int kPairYStride = kHeadDim + 4;  // floats per token row of the results
+constexpr size_t kPairSmemBytes = sizeof(double) * kHeadDim * (kHeadDim + kAppendTile);
+
+__device__ __forceinline__ void transform_rows_block(float (&v)[32], int g, int tt, const float* __restrict__ A,
+                                                     double* __restrict__ sA, double* __restrict__ sX) {
+  static_assert(kAppendWarps * 32 == 256 && kAppendTile == 64, "thread layout of the product");
 #pragma unroll
-  for (int r = 0; r < 32; ++r) acc[r] = 0.0;
+  for (int r = 0; r < 32; ++r) sX[(32 * g + r) * kAppendTile + ((tt + 8 * g) & (kAppendTile - 1))] = (double)v[r];
+  // A^T: thread e converts A[i][4q .. 4q+3], i = e mod 128 (consecutive threads,
+  // consecutive i: conflict-free stores)
+  const float4* A4 = reinterpret_cast<const float4*>(A);
+#pragma unroll 4
+  for (int e = threadIdx.x; e < kHeadDim * kHeadDim / 4; e += 256) {
+    const int i = e & (kHeadDim - 1), q = e >> 7;
+    const float4 m = __ldg(A4 + i * (kHeadDim / 4) + q);
+    double* d = sA + 4 * q * kHeadDim + i;
+    d[0] = (double)m.x;
+    d[kHeadDim] = (double)m.y;
+    d[2 * kHeadDim] = (double)m.z;
+    d[3 * kHeadDim] = (double)m.w;
+  }
+  __syncthreads();
+  // thread: tokens tb + 16 s (s < 4), channels 8 ib .. 8 ib + 7; a warp reads
+  // two A^T addresses (broadcast) and 16 consecutive X^T entries per load
+  const int tb = threadIdx.x & 15, ib = threadIdx.x >> 4;
+  double acc[4][8];
+#pragma unroll
+  for (int s = 0; s < 4; ++s)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[s][r] = 0.0;
 #pragma unroll 1
-  for (int src = 0; src < 4; ++src) {
+  for (int jg = 0; jg < 4; ++jg) {
+    int xo[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      double xs[4];
+    for (int s = 0; s < 4; ++s) xo[s] = (tb + 16 * s + 8 * jg) & (kAppendTile - 1);
+#pragma unroll 4
+    for (int j = 32 * jg; j < 32 * jg + 32; ++j) {
+      const double2* ar = reinterpret_cast<const double2*>(sA + j * kHeadDim + 8 * ib);
+      double a[8], x[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) xs[k] = (double)__shfl_sync(kFull, v[4 * e + k], base + src);
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        const float4 m = __ldg(rows + r * (kHeadDim / 4) + src * 8 + e);  // A[32g + r][32 src + 4e .. + 3]
-        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.x, xs[0]));
-        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.y, xs[1]));
-        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.z, xs[2]));
-        acc[r] = __dadd_rn(acc[r], __dmul_rn((double)m.w, xs[3]));
+      for (int k = 0; k < 4; ++k) {
+        const double2 p = ar[k];
+        a[2 * k] = p.x;
+        a[2 * k + 1] = p.y;
       }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) x[s] = sX[j * kAppendTile + xo[s]];
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[s][r] = __fma_rn(a[r], x[s], acc[s][r]);
     }
   }
+  __syncthreads();  // X^T is read: its space takes the results
+  float* sY = reinterpret_cast<float*>(sX);
 #pragma unroll
-  for (int r = 0; r < 32; ++r) v[r] = __double2float_rn(acc[r]);
+  for (int s = 0; s < 4; ++s)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      *reinterpret_cast<float4*>(sY + (tb + 16 * s) * kPairYStride + 8 * ib + 4 * h) =
+          make_float4(__double2float_rn(acc[s][4 * h]), __double2float_rn(acc[s][4 * h + 1]),
+                      __double2float_rn(acc[s][4 * h + 2]), __double2float_rn(acc[s][4 * h + 3]));
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const float4 o = *reinterpret_cast<const float4*>(sY + tt * kPairYStride + 32 * g + 4 * m);
+    v[4 * m] = o.x;
+    v[4 * m + 1] = o.y;
+    v[4 * m + 2] = o.z;
+    v[4 * m + 3] = o.w;
+  }
 }
 
 // Rotary embedding of one key row held by four lanes as above, at position
@@ -274,8 +326,7 @@ __device__ __forceinline__ void store_bf16_32(__nv_bfloat16* dst, const float (&
 }
 
 // ROT & 3: 0 keys as given, 1 Walsh-Hadamard rotation, 2 the pair's key
-// matrix tk[h] (its fp64 accumulators need the registers of fewer resident
-// blocks); ROT & 4: keys first rotary-embedded at their token index in the
+// matrix tk[h] (192 KB of dynamic shared memory: one resident block); ROT & 4: keys first rotary-embedded at their token index in the
 // view (the offset from their bucket's anchor), frequencies inv_freq
 template <int KB, int VB, int ROT, bool CH0, bool ROTV, typename In>
 __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
@@ -324,7 +375,10 @@ __global__ void __launch_bounds__(kAppendWarps * 32, (ROT & 3) == 2 ? 1 : 3)
   // ---- key row: rotated, then quantized (keys are not clipped)
   if (ROT & 4) rope_row_4lanes(kx, g, w0 + tt, inv_freq);
   if ((ROT & 3) == 1) rotate_row_4lanes(kx, g, a.inv_sqrt_d);
-  if ((ROT & 3) == 2) transform_row_4lanes(kx, g, lane, tk + (size_t)h * kPairElems);
+  if ((ROT & 3) == 2) {
+    extern __shared__ __align__(16) double pair_smem[];
+    transform_rows_block(kx, g, tt, tk + (size_t)h * kPairElems, pair_smem, pair_smem + kHeadDim * kHeadDim);
+  }
   // bf16 window copies (rotated key, then the value below) for tokens with a
   // window slot: every sink token, and of the later tokens only this append's
   // last `recent`, the ones that still own their ring slot when it ends (an
@@ -444,11 +498,15 @@ cudaError_t launch_typed(const AppendArgs& a, const float* tk, const float* fr, 
   const int first = a.offset / kAppendTile, last = (a.offset + a.n_new - 1) / kAppendTile;
   dim3 grid(last - first + 1, a.c.H, a.c.B);
   dim3 block(kAppendWarps * 32);
-  switch (a.dtype) {
-    case KVQ_F32: k_quantize_append<KB, VB, ROT, CH0, ROTV, float><<<grid, block, 0, s>>>(a, tk, fr); break;
-    case KVQ_BF16: k_quantize_append<KB, VB, ROT, CH0, ROTV, __nv_bfloat16><<<grid, block, 0, s>>>(a, tk, fr); break;
-    default: k_quantize_append<KB, VB, ROT, CH0, ROTV, __half><<<grid, block, 0, s>>>(a, tk, fr); break;
+  auto kern = a.dtype == KVQ_F32 ? k_quantize_append<KB, VB, ROT, CH0, ROTV, float>
+                                 : (a.dtype == KVQ_BF16 ? k_quantize_append<KB, VB, ROT, CH0, ROTV, __nv_bfloat16>
+                                                        : k_quantize_append<KB, VB, ROT, CH0, ROTV, __half>);
+  const size_t smem = (ROT & 3) == 2 ? kPairSmemBytes : 0;
+  if (smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
   }
+  kern<<<grid, block, smem, s>>>(a, tk, fr);
   return cudaGetLastError();
 }
 

@@ -41,9 +41,10 @@ def slice_bytes(gc: native.KVQCache, b: int, h: int):
     return {k: v.cpu().numpy() for k, v in out.items()}
 
 
-def oracle_slice(wl, s, b, h):
+def oracle_slice(wl, s, b, h, pair=None):
+    tq, tk = (None, None) if pair is None else (pair[0][h:h + 1], pair[1][h:h + 1])
     c = orc.Cache(1, 1, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v, wl.v_clip,
-                  wl.sink, wl.recent)
+                  wl.sink, wl.recent, tq, tk)
     k = s.k_slice(b, h)[None, None]
     v = s.v_slice(b, h)[None, None]
     st = c.append(host_f32(k, wl.fmt), host_f32(v, wl.fmt), wl.offset, want_exempt=True)
@@ -140,12 +141,14 @@ def test_decode_workload(wid):
     assert not rows, f"identical decode calls differ in {len(rows)} rows, e.g. {rows[:8]}, max {diff.max().item():.3e}"
 
 
-@pytest.mark.parametrize("wid", [3, 6])
+@pytest.mark.parametrize("wid", [3, 6, 9])
 def test_append_workload(wid):
     wl = workloads.by_id(wid)
     s = synth.Synth(workloads.BASE_SEED + wl.id, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt, wl.len_range)
+    pair = synth.dual_pair(workloads.BASE_SEED + wl.id, wl.Hkv) if wl.rotate_k == 2 else None
+    kw = {} if pair is None else dict(t_query=torch.from_numpy(pair[0]).cuda(), t_key=torch.from_numpy(pair[1]).cuda())
     gc = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0,
-                         rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent)
+                         rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent, **kw)
     # one launch over the whole batch, as timed for the append workload
     kd = up(s.k_full(), wl.fmt)
     vd = up(s.v_full(), wl.fmt)
@@ -153,7 +156,7 @@ def test_append_workload(wid):
     torch.cuda.synchronize()
     del kd, vd
     for b, h in sampled_pairs(wl, n=3):
-        c, st = oracle_slice(wl, s, b, h)
+        c, st = oracle_slice(wl, s, b, h, pair)
         check_slice_bytes(slice_bytes(gc, b, h), c, st, wl)
     # nothing before the offset was written
     cap, off = wl.capacity, wl.offset
