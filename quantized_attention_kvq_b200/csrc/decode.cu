@@ -13,8 +13,9 @@
 // Per 128-token tile, 8 MMAs:
 //   scores: 4 of kind::i8 (K = 32 = one quantization group each): key codes
 //           as u8 in tensor memory x the rotated query as two exact s8 pieces
-//           (q = delta * (128 q1 + q2)), one s32 accumulator per group, so the
-//           per-token group scale applies exactly afterwards;
+//           (q = delta_g * (128 q1 + q2), one step delta_g per channel group),
+//           one s32 accumulator per group, so the per-token group scale and
+//           the group's step apply exactly afterwards;
 //   PV:     4 of kind::i8 (K = 32 tokens each): value codes as u8 in tensor
 //           memory x P' as four u8 bytes of an integer up to 2^31, P' = p *
 //           value scale normalized by running bounds (p relative to a lazily
@@ -38,7 +39,7 @@
 //                     -> u8 -> tensor memory (lane = channel);
 //   score warp      : the score MMAs, as far ahead as the score buffers allow;
 //   PV warp         : the PV MMAs of each tile once its P' is written;
-//   epilogue warps  : thread = (token, heads): score = delta * sum_g s_g S_g +
+//   epilogue warps  : thread = (token, heads): score = sum_g delta_g s_g S_g +
 //                     sum_g z_g sum(q_g) (+ q_0 k_0), the tile's maxima, the
 //                     online softmax with a lazily raised running max, P' into
 //                     shared memory, the value zero-point terms sum_t p_t z_t;
@@ -138,8 +139,8 @@ struct Shape {
   static constexpr int F_BP = F_BQ + 2 * BQ_BYTES;   // [2] P' buffers
   static constexpr int F_QS = F_BP + 2 * BP_BYTES;   // [2][G][4] f32: per-group sums of the kept q
   static constexpr int F_Q0 = F_QS + 2 * G * 16;     // [2][G] f32: q_0 (channel 0 kept in bf16)
-  static constexpr int F_QD = F_Q0 + 2 * QV;         // [2][G] f32: delta of the query pieces
-  static constexpr int F_RED = F_QD + 2 * QV;  // [2 own tiles][NGRP][TPT][4 warps][16] s32: warp maxima
+  static constexpr int F_QD = F_Q0 + 2 * QV;         // [2][G][4] f32: step of the query pieces per group
+  static constexpr int F_RED = F_QD + 2 * G * 16;  // [2 own tiles][NGRP][TPT][4 warps][16] s32: warp maxima
   static constexpr int F_RED2 = F_RED + 2 * NGRP * TPT * 4 * 16 * 4;  // [NGRP][TPT][4 warps][16] f32: segment sums
   static constexpr int F_BAR = (F_RED2 + NGRP * TPT * 4 * 16 * 4 + 15) / 16 * 16;
   // kready[3] vready[2] pready[2] sdone[3] pvdone[2] qready[2] qfree[2] sfree[3]
@@ -368,8 +369,10 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       if (t >= S::KST) ws_wait(SDONE((t - S::KST) % S::SB), ((t - S::KST) / S::SB) & 1, err);
       tc_fence_after();
       if (__builtin_expect(it.first, 0)) {
-        // query data of segment kseg into buffer kseg & 1: per head, delta =
-        // max|q| / 16000 and q = delta * (128 q1 + q2) exactly; the rows of each
+        // query data of segment kseg into buffer kseg & 1: per head and
+        // 32-channel group g, delta_g = max|q_g| / 16000 and q = delta_g *
+        // (128 q1 + q2) exactly (a step per group keeps a group of small
+        // channels as fine as its own largest one allows); the rows of each
         // epilogue head part are its heads' q1 pieces, then their q2 pieces;
         // dropped channel groups (and channel 0 when it is kept in bf16) are zero.  The buffer was last used by segment kseg - 2, which the
         // epilogue (and so its score UMMAs) finished before freeing it.  Each
@@ -380,7 +383,7 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         uint8_t* BQ = fix + S::F_BQ + qb * S::BQ_BYTES;
         float* qsum = reinterpret_cast<float*>(fix + S::F_QS + qb * G * 16);
         float* q0s = reinterpret_cast<float*>(fix + S::F_Q0 + qb * S::QV);
-        float* qds = reinterpret_cast<float*>(fix + S::F_QD + qb * S::QV);
+        float* qds = reinterpret_cast<float*>(fix + S::F_QD + qb * G * 16);
         const uint32_t msk = it.msk;
         for (int hq = warp; hq < G; hq += 4) {
           const In* qrow = static_cast<const In*>(a.q) + ((size_t)it.b * a.Hq + (size_t)it.h * G + hq) * kHeadDim;
@@ -395,7 +398,9 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             part += v[i];
             amax = fmaxf(amax, fabsf(v[i]));
           }
-          amax = warp_max(amax);
+          // the group's largest element: lanes 8g .. 8g + 7 hold group g
+#pragma unroll
+          for (int m = 1; m < 8; m <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, m));
           const float delta = amax > 0.0f ? amax / kQSteps : 1.0f;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -411,11 +416,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           }
 #pragma unroll
           for (int m = 1; m < 8; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
-          if ((lane & 7) == 0) qsum[hq * kGroups + (lane >> 3)] = part;
-          if (lane == 0) {
-            q0s[hq] = (CH0 && sel) ? x[0] : 0.0f;
-            qds[hq] = delta;
+          if ((lane & 7) == 0) {
+            qsum[hq * kGroups + (lane >> 3)] = part;
+            qds[hq * kGroups + (lane >> 3)] = delta;
           }
+          if (lane == 0) q0s[hq] = (CH0 && sel) ? x[0] : 0.0f;
         }
         fence_proxy_async();      // query operand (generic writes) -> tensor core
         mbar_arrive(QREADY(qb));  // release: the epilogue reads the data after waiting on it
@@ -532,10 +537,11 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
     float ds1[HH] = {}, ds2[HH] = {};
     bool have1 = false, have2 = false;
     // this segment's query data for the thread's heads (per-group sums of the
-    // kept q, q_0, the step of the query pieces), held in registers when one
-    // thread takes a token's heads, else read from shared memory per tile
+    // kept q, q_0), held in registers when one thread takes a token's heads,
+    // else read from shared memory per tile; the steps of the query pieces are
+    // read from shared memory per tile
     constexpr bool QREG = S::TPT == 1;
-    float qsg[QREG ? HH : 1][kGroups], q0r[QREG ? HH : 1], qdr[QREG ? HH : 1];
+    float qsg[QREG ? HH : 1][kGroups], q0r[QREG ? HH : 1];
     int nseg = 0;       // segments begun so far
     int qb = 0;         // query buffer of the current segment (its parity)
     int seg_tiles = 0;  // tiles of the current segment this group has taken
@@ -594,7 +600,6 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
         ++nseg;
         const float* qsum = reinterpret_cast<const float*>(fix + S::F_QS + qb * G * 16);
         const float* q0s = reinterpret_cast<const float*>(fix + S::F_Q0 + qb * S::QV);
-        const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * S::QV);
 #pragma unroll
         for (int i = 0; i < (QREG ? HH : 0); ++i) {
           const int hh = part * HH + i;
@@ -604,7 +609,6 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
           qsg[i][2] = qs.z;
           qsg[i][3] = qs.w;
           q0r[i] = CH0 ? q0s[hh] : 0.0f;
-          qdr[i] = qds[hh];
         }
       }
       if (t % S::NGRP != grp) {
@@ -673,16 +677,17 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
       {
         const float* qsum = reinterpret_cast<const float*>(fix + S::F_QS + qb * G * 16);
         const float* q0s = reinterpret_cast<const float*>(fix + S::F_Q0 + qb * S::QV);
-        const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * S::QV);
+        const float* qds = reinterpret_cast<const float*>(fix + S::F_QD + qb * G * 16);
 #pragma unroll
         for (int i = 0; i < HH; ++i) {
           const int hh = part * HH + i;
-          float qg[kGroups], q0, qd;
+          float qg[kGroups], q0;
+          const float4 qd = reinterpret_cast<const float4*>(qds)[hh];  // the head's steps per group
+          const float qdg[kGroups] = {qd.x, qd.y, qd.z, qd.w};
           if constexpr (QREG) {
 #pragma unroll
             for (int g = 0; g < kGroups; ++g) qg[g] = qsg[i][g];
             q0 = q0r[i];
-            qd = qdr[i];
           } else {
             const float4 qs = reinterpret_cast<const float4*>(qsum)[hh];
             qg[0] = qs.x;
@@ -690,16 +695,15 @@ __global__ void __launch_bounds__(Shape<G, KB, VB, CH0>::THREADS, 1) k_decode(De
             qg[2] = qs.z;
             qg[3] = qs.w;
             q0 = CH0 ? q0s[hh] : 0.0f;
-            qd = qds[hh];
           }
           // dot and zero-point sums over the groups as one paired fma each
           float2 dz = make_float2(0.0f, CH0 ? q0 * k0v : 0.0f);
 #pragma unroll
           for (int g = 0; g < kGroups; ++g) {
             const int dg = (int)sd[g][i] * 128 + (int)sd[g][HH + i];  // exact: |dg| < 2^23
-            dz = ffma2(ksz[g], make_float2((float)dg, qg[g]), dz);
+            dz = ffma2(ksz[g], make_float2((float)dg * qdg[g], qg[g]), dz);
           }
-          sc[i] = valid ? fmaf(dz.x, qd, dz.y) * a.scale_log2 : NEG_INF;
+          sc[i] = valid ? (dz.x + dz.y) * a.scale_log2 : NEG_INF;
         }
       }
       mbar_arrive(SFREE(t % S::SB));        // the score buffer may take tile t + SB

@@ -166,3 +166,66 @@ def test_append_workload(wid):
     assert kc[:, off // 128:].any().item()
     vc = gc.v_codes.view(wl.B * wl.Hkv, cap, -1)
     assert not vc[:, :off].any().item()
+
+
+@pytest.mark.parametrize("wid", [8, 10])
+def test_decode_bucket_workload(wid):
+    """The whole Dual-QK recipe at 128K (Dual-QK summary Sec. 3.1, 3.3, 3.4): a
+    dual transform pair, bucket-relative RoPE at w = 2048, values rotated and
+    clipped, and for workload 10 the bf16 sink and recent windows.  The cache is
+    built as bench.py builds it (one append per bucket); the decode runs as
+    timed (selection inside the split half) and as selection then decode.
+    Sampled (sequence, kv head) slices: the per-bucket masks bit-exact and the
+    outputs within the bar, against an oracle cache of that slice alone (the
+    bytes of bucket-major caches are compared bit-exactly at small sizes in
+    test_gpu_bucket_rope.py)."""
+    wl = workloads.by_id(wid)
+    seed = workloads.BASE_SEED + wl.id
+    s = synth.Synth(seed, wl.B, wl.Hq, wl.Hkv, wl.d, wl.T, wl.fmt, wl.len_range)
+    tq, tk = synth.dual_pair(seed, wl.Hkv)
+    fr = synth.rope_inv_freq(wl.rope_base)
+    gc = native.KVQCache(wl.B, wl.Hkv, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0,
+                         rotate_v=wl.rotate_v, v_clip=wl.v_clip, sink=wl.sink, recent=wl.recent,
+                         t_query=torch.from_numpy(tq).cuda(), t_key=torch.from_numpy(tk).cuda(),
+                         bucket_tokens=wl.bucket, rope_inv_freq=torch.from_numpy(fr).cuda())
+    for b in range(wl.B):
+        kd = up(np.stack([s.k_slice(b, h) for h in range(wl.Hkv)]), wl.fmt)
+        vd = up(np.stack([s.v_slice(b, h) for h in range(wl.Hkv)]), wl.fmt)
+        for t0 in range(0, wl.T, wl.bucket):  # an append stays inside one bucket
+            gc.append_sequence(b, kd[:, t0:t0 + wl.bucket].contiguous(), vd[:, t0:t0 + wl.bucket].contiguous(),
+                               wl.offset + t0)
+        torch.cuda.synchronize()
+        del kd, vd
+    q = s.q()
+    qd = up(q, wl.fmt)
+    lens = s.lens.astype(np.int32)
+    lens_d = torch.from_numpy(lens).cuda()
+    max_len = wl.T
+    scale = 1.0 / math.sqrt(128)
+    keep = wl.keep_groups
+    ws = torch.empty(gc.workspace_bytes(wl.Hq, max_len), dtype=torch.uint8, device="cuda")
+    out = torch.empty((wl.B, wl.Hq, 128), dtype=torch.float32, device="cuda")
+    gc.decode_partials_select(qd, lens_d, max_len, keep, scale, ws)
+    gc.decode_combine(wl.Hq, lens_d, max_len, out, ws)
+    mask_d = gc.select_at(qd, lens_d, keep)
+    out2 = gc.decode(qd, lens_d, max_len, mask_d, scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2), "selection inside the decode and selection then decode differ"
+    o_gpu = out.cpu().numpy()
+    assert np.isfinite(o_gpu).all()
+    nb = wl.capacity // wl.bucket
+    masks = mask_u32(mask_d).reshape(wl.B, nb, wl.Hkv)
+    G = wl.G
+    qf = host_f32(q, wl.fmt)
+    for b, h in sampled_pairs(wl):
+        c = orc.Cache(1, 1, 128, wl.capacity, wl.k_bits, wl.v_bits, wl.rotate_k, wl.keep_ch0, wl.rotate_v,
+                      wl.v_clip, wl.sink, wl.recent, tq[h:h + 1], tk[h:h + 1], bucket_w=wl.bucket, inv_freq=fr)
+        c.append(host_f32(s.k_slice(b, h)[None, None], wl.fmt), host_f32(s.v_slice(b, h)[None, None], wl.fmt),
+                 wl.offset)
+        qs = qf[b:b + 1, h * G:(h + 1) * G]
+        ref_mask, _ = c.select_buckets(qs, lens[b:b + 1], keep)
+        np.testing.assert_array_equal(masks[b, :, h], ref_mask[0, :, 0], err_msg=f"masks of ({b}, {h})")
+        o_ref = c.attention(qs, lens[b:b + 1], ref_mask, scale)
+        got = o_gpu[b, h * G:(h + 1) * G].astype(np.float64)
+        err = np.abs(got - o_ref).max()
+        assert err <= ATOL_REL * np.abs(o_ref).max(), (wl.name, b, h, err, np.abs(o_ref).max())
